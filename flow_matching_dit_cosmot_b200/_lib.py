@@ -1,0 +1,221 @@
+"""ctypes binding of libcosmot (include/cosmot.h).
+
+Argument marshalling only: every function forwards to the C entry point of the
+same name.  Pointers are plain integers (device addresses, e.g. a torch
+tensor's data_ptr()), streams are cudaStream_t handles as integers.  Nothing
+here computes; if the shared library is missing the import fails loudly.
+"""
+
+from __future__ import annotations
+
+import ctypes
+import os
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libcosmot.so")
+
+COSMOT_OK = 0
+COSMOT_ERR_INVALID_ARG = 1
+COSMOT_ERR_UNSUPPORTED = 2
+COSMOT_ERR_CUDA = 3
+COSMOT_ERR_TIMEOUT = 4
+COSMOT_ERR_WORKSPACE = 5
+
+COSMOT_EPI_NONE = 0
+COSMOT_EPI_RESIDUAL = 1
+COSMOT_EPI_SILU_MUL = 2
+COSMOT_EPI_MROPE = 3
+COSMOT_EPI_EULER = 4
+
+COSMOT_MASK_FULL = 0
+COSMOT_MASK_BLOCK_CAUSAL = 1
+
+c_i32, c_i64, c_f32, c_f64, c_vp = ctypes.c_int32, ctypes.c_int64, ctypes.c_float, ctypes.c_double, ctypes.c_void_p
+
+
+class LayoutSpec(ctypes.Structure):
+    _fields_ = [("n_text", c_i32),
+                ("video_views", c_i32), ("video_grid_h", c_i32), ("video_grid_w", c_i32), ("video_fps", c_i32),
+                ("video_clean_steps", c_i32), ("video_noisy_steps", c_i32),
+                ("audio_clean", c_i32), ("audio_noisy", c_i32), ("audio_rate", c_i32),
+                ("action_clean", c_i32), ("action_noisy", c_i32), ("action_hz", c_i32),
+                ("proprio", c_i32), ("tau_offset", c_i32)]
+
+
+class Segment(ctypes.Structure):
+    _fields_ = [("row_begin", c_i64), ("row_end", c_i64), ("out_row", c_i64),
+                ("weight_set", c_i32), ("reserved", c_i32)]
+
+
+class Epilogue(ctypes.Structure):
+    _fields_ = [("kind", c_i32), ("head_dim", c_i32), ("rope_cols", c_i64), ("rope_cs", c_vp),
+                ("rope_period", c_i64), ("res", c_vp), ("ld_res", c_i64), ("x", c_vp), ("ld_x", c_i64),
+                ("dsigma", c_f32), ("reserved", c_f32)]
+
+
+class AttnDesc(ctypes.Structure):
+    _fields_ = [("n_q", c_i64), ("q_key_offset", c_i64), ("n_keys", c_i64), ("n_ar", c_i64),
+                ("n_heads", c_i32), ("n_kv_heads", c_i32), ("head_dim", c_i32), ("mask_mode", c_i32),
+                ("chunk", c_vp), ("batch", c_i32), ("reserved", c_i32),
+                ("q_batch_stride", c_i64), ("kv_batch_stride", c_i64), ("o_batch_stride", c_i64),
+                ("softmax_scale", c_f32), ("reserved2", c_f32)]
+
+
+class Dims(ctypes.Structure):
+    _fields_ = [("d_model", c_i32), ("n_heads", c_i32), ("n_kv_heads", c_i32), ("head_dim", c_i32),
+                ("ffn", c_i32), ("rope_sections", c_i32 * 3), ("rope_base", c_f64), ("eps", c_f32),
+                ("reserved", c_i32)]
+
+
+class SetWeights(ctypes.Structure):
+    _fields_ = [("g1", c_vp), ("wqkv", c_vp), ("wo", c_vp), ("g2", c_vp), ("wg", c_vp), ("wu", c_vp), ("wd", c_vp)]
+
+
+class LayerWeights(ctypes.Structure):
+    _fields_ = [("set", SetWeights * 2), ("gfin", c_vp), ("wvel", c_vp)]
+
+
+class SeqDesc(ctypes.Structure):
+    _fields_ = [("n_ar", c_i32), ("n_clean", c_i32), ("n_noisy", c_i32), ("batch", c_i32),
+                ("mask_mode", c_i32), ("reserved", c_i32), ("rope_cs", c_vp), ("chunk", c_vp)]
+
+
+_P = ctypes.POINTER
+
+# name -> (restype, argtypes); every entry is declared in include/cosmot.h
+SIGNATURES = {
+    "cosmot_status_string": (ctypes.c_char_p, [c_i32]),
+    "cosmot_version": (c_i32, []),
+    "cosmot_get_device_status": (c_i32, [c_vp, _P(c_i32), _P(c_i32)]),
+    "cosmot_layout_counts": (c_i32, [_P(LayoutSpec), _P(c_i32), _P(c_i32), _P(c_i32), _P(c_i32)]),
+    "cosmot_build_layout": (c_i32, [_P(LayoutSpec), c_vp, c_vp, c_vp, c_vp]),
+    "cosmot_mrope_table": (c_i32, [c_vp, c_i64, c_i32, _P(c_i32), c_f64, c_vp, c_vp]),
+    "cosmot_rmsnorm_routed": (c_i32, [c_vp, c_i64, _P(Segment), c_i32, c_vp, c_vp, c_i64, c_f32, c_vp, c_i64, c_vp]),
+    "cosmot_routed_linear": (c_i32, [c_vp, c_i64, c_i64, _P(Segment), c_i32, c_vp, c_vp, c_vp, c_vp, c_i64, c_vp,
+                                     c_i64, _P(Epilogue), c_vp]),
+    "cosmot_mrope_apply": (c_i32, [c_vp, c_i64, c_i32, c_vp, c_i64, c_i32, c_i64, c_i32, c_vp, c_vp]),
+    "cosmot_mot_attention": (c_i32, [_P(AttnDesc), c_vp, c_i64, c_vp, c_vp, c_i64, c_vp, c_i64, c_vp]),
+    "cosmot_flow_euler_step": (c_i32, [c_vp, c_i64, c_vp, c_i64, c_i64, c_i64, c_i64, c_f64, c_f64, c_vp]),
+    "cosmot_layer_workspace_size": (c_i32, [_P(Dims), _P(SeqDesc), _P(ctypes.c_size_t)]),
+    "cosmot_layer_forward": (c_i32, [_P(Dims), _P(LayerWeights), _P(SeqDesc), c_vp, c_vp, c_f64, c_f64, c_vp,
+                                     ctypes.c_size_t, c_vp]),
+}
+
+_lib = None
+
+
+def lib() -> ctypes.CDLL:
+    """Loads libcosmot.so (built in-tree by flow_matching_dit_cosmot_b200.build)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise ImportError(f"libcosmot.so not built at {LIB_PATH}; run `python -m flow_matching_dit_cosmot_b200.build`")
+        L = ctypes.CDLL(LIB_PATH)
+        for name, (res, args) in SIGNATURES.items():
+            f = getattr(L, name)
+            f.restype = res
+            f.argtypes = args
+        _lib = L
+    return _lib
+
+
+class CosmotError(RuntimeError):
+    def __init__(self, fn, code):
+        super().__init__(f"{fn} failed: {status_string(code)} ({code})")
+        self.code = code
+
+
+def status_string(code: int) -> str:
+    return lib().cosmot_status_string(code).decode()
+
+
+def _check(fn, code):
+    if code != COSMOT_OK:
+        raise CosmotError(fn, code)
+    return code
+
+
+def _call(name, *args, check=True):
+    code = getattr(lib(), name)(*args)
+    return _check(name, code) if check else code
+
+
+# ------------------------------------------------------------------ thin wrappers (same names as the C ABI)
+
+def cosmot_version() -> int:
+    return lib().cosmot_version()
+
+
+def cosmot_get_device_status(stream: int = 0):
+    st, where = c_i32(0), c_i32(0)
+    _call("cosmot_get_device_status", c_vp(stream), ctypes.byref(st), ctypes.byref(where))
+    return st.value, where.value
+
+
+def cosmot_layout_counts(spec: LayoutSpec):
+    n, a, c, z = c_i32(), c_i32(), c_i32(), c_i32()
+    _call("cosmot_layout_counts", ctypes.byref(spec), ctypes.byref(n), ctypes.byref(a), ctypes.byref(c), ctypes.byref(z))
+    return n.value, a.value, c.value, z.value
+
+
+def cosmot_build_layout(spec: LayoutSpec, pos: int, chunk: int, region: int = 0, stream: int = 0, check=True):
+    return _call("cosmot_build_layout", ctypes.byref(spec), c_vp(pos), c_vp(chunk), c_vp(region or None),
+                 c_vp(stream), check=check)
+
+
+def cosmot_mrope_table(pos: int, n_rows: int, head_dim: int, sections, rope_base: float, cs: int, stream: int = 0,
+                       check=True):
+    sec = (c_i32 * 3)(*sections)
+    return _call("cosmot_mrope_table", c_vp(pos), n_rows, head_dim, sec, rope_base, c_vp(cs), c_vp(stream),
+                 check=check)
+
+
+def _segs(segs):
+    arr = (Segment * len(segs))(*[Segment(int(b), int(e), int(o), int(s), 0) for (b, e, o, s) in segs])
+    return arr, len(segs)
+
+
+def cosmot_rmsnorm_routed(h: int, ld_h: int, segs, g0: int, g1: int, d: int, eps: float, out: int, ld_out: int,
+                          stream: int = 0, check=True):
+    arr, n = _segs(segs)
+    return _call("cosmot_rmsnorm_routed", c_vp(h), ld_h, arr, n, c_vp(g0), c_vp(g1), d, eps, c_vp(out), ld_out,
+                 c_vp(stream), check=check)
+
+
+def cosmot_routed_linear(a: int, ld_a: int, k: int, segs, w0: int, w1: int, n_out: int, out: int, ld_out: int,
+                         epi: Epilogue | None = None, w0_up: int = 0, w1_up: int = 0, stream: int = 0, check=True):
+    arr, n = _segs(segs)
+    e = epi if epi is not None else Epilogue(kind=COSMOT_EPI_NONE)
+    return _call("cosmot_routed_linear", c_vp(a), ld_a, k, arr, n, c_vp(w0 or None), c_vp(w1 or None),
+                 c_vp(w0_up or None), c_vp(w1_up or None), n_out, c_vp(out), ld_out, ctypes.byref(e), c_vp(stream),
+                 check=check)
+
+
+def cosmot_mrope_apply(q: int, ld_q: int, n_q_heads: int, k: int, ld_k: int, n_k_heads: int, n_rows: int,
+                       head_dim: int, cs: int, stream: int = 0, check=True):
+    return _call("cosmot_mrope_apply", c_vp(q or None), ld_q, n_q_heads, c_vp(k or None), ld_k, n_k_heads, n_rows,
+                 head_dim, c_vp(cs), c_vp(stream), check=check)
+
+
+def cosmot_mot_attention(desc: AttnDesc, q: int, ld_q: int, k: int, v: int, ld_kv: int, o: int, ld_o: int,
+                         stream: int = 0, check=True):
+    return _call("cosmot_mot_attention", ctypes.byref(desc), c_vp(q), ld_q, c_vp(k), c_vp(v), ld_kv, c_vp(o), ld_o,
+                 c_vp(stream), check=check)
+
+
+def cosmot_flow_euler_step(x: int, ld_x: int, v: int, ld_v: int, row_begin: int, row_end: int, n_cols: int,
+                           sigma: float, sigma_next: float, stream: int = 0, check=True):
+    return _call("cosmot_flow_euler_step", c_vp(x), ld_x, c_vp(v), ld_v, row_begin, row_end, n_cols, sigma,
+                 sigma_next, c_vp(stream), check=check)
+
+
+def cosmot_layer_workspace_size(dims: Dims, seq: SeqDesc) -> int:
+    n = ctypes.c_size_t(0)
+    _call("cosmot_layer_workspace_size", ctypes.byref(dims), ctypes.byref(seq), ctypes.byref(n))
+    return n.value
+
+
+def cosmot_layer_forward(dims: Dims, w: LayerWeights, seq: SeqDesc, h: int, h_out: int, sigma: float,
+                         sigma_next: float, workspace: int, workspace_bytes: int, stream: int = 0, check=True):
+    return _call("cosmot_layer_forward", ctypes.byref(dims), ctypes.byref(w), ctypes.byref(seq), c_vp(h),
+                 c_vp(h_out), sigma, sigma_next, c_vp(workspace), workspace_bytes, c_vp(stream), check=check)

@@ -1,0 +1,111 @@
+"""PyTorch-facing helpers around the C ABI.
+
+PyTorch provides device memory and streams; every step of the layer runs in
+libcosmot's kernels.  These helpers only allocate outputs/workspace with torch
+and translate tensors into the pointers and structs the C entry points take.
+"""
+
+from __future__ import annotations
+
+from dataclasses import dataclass
+from typing import Optional
+
+import torch
+
+from . import _lib as L
+
+L.lib()  # the CUDA library must be present; no fallback
+
+
+def ptr(t: Optional[torch.Tensor]) -> int:
+    return 0 if t is None else t.data_ptr()
+
+
+def stream_handle(stream: Optional[torch.cuda.Stream] = None) -> int:
+    return (stream if stream is not None else torch.cuda.current_stream()).cuda_stream
+
+
+def _need_cuda(*ts):
+    for t in ts:
+        if t is not None and not t.is_cuda:
+            raise ValueError("libcosmot takes CUDA tensors only (no CPU fallback)")
+
+
+def layout_spec(n_text: int, video=None, audio_clean=0, audio_noisy=0, audio_rate=25, action_clean=0,
+                action_noisy=0, action_hz=15, proprio=0, tau_offset=0) -> L.LayoutSpec:
+    """`video` = (views, grid_h, grid_w, fps, clean_steps, noisy_steps) or None."""
+    v = video if video is not None else (0, 0, 0, 0, 0, 0)
+    return L.LayoutSpec(n_text, *[int(x) for x in v], audio_clean, audio_noisy, audio_rate, action_clean,
+                        action_noisy, action_hz, proprio, tau_offset)
+
+
+@dataclass
+class DeviceLayout:
+    pos: torch.Tensor     # float32 [N, 3]
+    chunk: torch.Tensor   # int32 [N]
+    region: torch.Tensor  # int8 [N]
+    n_ar: int
+    n_clean: int
+    n_noisy: int
+
+    @property
+    def n_tokens(self) -> int:
+        return self.n_ar + self.n_clean + self.n_noisy
+
+
+def build_layout(spec: L.LayoutSpec, device="cuda", stream=None) -> DeviceLayout:
+    n, a, c, z = L.cosmot_layout_counts(spec)
+    pos = torch.empty((n, 3), dtype=torch.float32, device=device)
+    chunk = torch.empty((n,), dtype=torch.int32, device=device)
+    region = torch.empty((n,), dtype=torch.int8, device=device)
+    L.cosmot_build_layout(spec, ptr(pos), ptr(chunk), ptr(region), stream_handle(stream))
+    return DeviceLayout(pos, chunk, region, a, c, z)
+
+
+def mrope_table(pos: torch.Tensor, head_dim: int, sections, rope_base: float = 10000.0, stream=None) -> torch.Tensor:
+    _need_cuda(pos)
+    cs = torch.empty((pos.shape[0], head_dim // 2, 2), dtype=torch.float32, device=pos.device)
+    L.cosmot_mrope_table(ptr(pos), pos.shape[0], head_dim, sections, rope_base, ptr(cs), stream_handle(stream))
+    return cs
+
+
+def make_dims(d_model, n_heads, n_kv_heads, head_dim, ffn, rope_sections, rope_base=10000.0, eps=1e-6) -> L.Dims:
+    return L.Dims(d_model, n_heads, n_kv_heads, head_dim, ffn, (L.c_i32 * 3)(*rope_sections), rope_base, eps, 0)
+
+
+class MoTLayer:
+    """One MoT layer: both weight sets resident on the device.
+
+    `weights` maps names to bf16 CUDA tensors: "R.*"/"G.*" for the Reasoner and
+    Generator sets (g1, wqkv, wo, g2, wg, wu, wd), plus "gfin" and "wvel".
+    """
+
+    def __init__(self, dims: L.Dims, weights: dict):
+        self.dims = dims
+        self.weights = weights
+        _need_cuda(*weights.values())
+        sets = []
+        for s in ("R", "G"):
+            sets.append(L.SetWeights(*[ptr(weights[f"{s}.{t}"]) for t in ("g1", "wqkv", "wo", "g2", "wg", "wu", "wd")]))
+        self.cw = L.LayerWeights((L.SetWeights * 2)(*sets), ptr(weights["gfin"]), ptr(weights["wvel"]))
+        self._ws = None
+
+    def seq_desc(self, n_ar, n_clean, n_noisy, batch, rope_cs, chunk=None, mask_mode=L.COSMOT_MASK_FULL) -> L.SeqDesc:
+        return L.SeqDesc(n_ar, n_clean, n_noisy, batch, mask_mode, 0, ptr(rope_cs), ptr(chunk))
+
+    def workspace_bytes(self, seq: L.SeqDesc) -> int:
+        return L.cosmot_layer_workspace_size(self.dims, seq)
+
+    def workspace(self, seq: L.SeqDesc, device="cuda") -> torch.Tensor:
+        n = self.workspace_bytes(seq)
+        if self._ws is None or self._ws.numel() < n:
+            self._ws = torch.empty((n,), dtype=torch.uint8, device=device)
+        return self._ws
+
+    def forward(self, h: torch.Tensor, h_out: torch.Tensor, sigma: float, sigma_next: float, seq: L.SeqDesc,
+                workspace: Optional[torch.Tensor] = None, stream=None):
+        """h [batch, N, d] bf16 (noisy DM rows updated in place to x'); h_out [batch, N, d] bf16."""
+        _need_cuda(h, h_out)
+        ws = workspace if workspace is not None else self.workspace(seq, h.device)
+        L.cosmot_layer_forward(self.dims, self.cw, seq, ptr(h), ptr(h_out), float(sigma), float(sigma_next),
+                               ptr(ws), ws.numel(), stream_handle(stream))

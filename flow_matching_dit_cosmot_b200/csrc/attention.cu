@@ -1,0 +1,463 @@
+// MoT attention on the sm_100a tensor cores (tcgen05 + TMEM + TMA).
+//
+// "Cosmos 3 方法原理全解" §3:
+//     O_AR = Attn_causal(Q_AR, K_AR, V_AR)
+//     O_DM = Attn_full(Q_DM, [K_AR; K_DM], [V_AR; V_DM])
+// plus the time-causal block variant of "流式生成如何工作" (DM keys of later
+// chunks hidden).  Softmax is the usual online (running max / running sum)
+// formulation, exact up to rounding.
+//
+// One CTA per (sequence, head, pair of 128-row query tiles); a pair never
+// mixes AR and DM rows.  320 threads:
+//   warp 0      TMA: both Q tiles once, then K_j and V_j tiles (128 keys x
+//               head_dim, 128-byte swizzle) through a 4-slot ring.
+//   warp 1      owns TMEM and issues the MMAs from one thread:
+//                 S_t = Q_t K_j^T          (M=128, N=128, K=head_dim; SS)
+//                 O_t += P_t V_j           (M=128, N=head_dim, K=128;  A = P in TMEM)
+//               in the order S0 S1 | PV0 S0' PV1 S1' | ..., so the tensor core
+//               works on one tile while the other tile's softmax runs.
+//   warps 2-5   softmax of query tile 0, warps 6-9 of tile 1 (one row per
+//               thread): read S from TMEM, mask, running max, P = 2^(s*c - m)
+//               written back over S as packed bf16, running sum; O is
+//               rescaled in TMEM only when the running max grows by more than
+//               2^8 (the exponent headroom keeps P and O finite meanwhile).
+// TMEM columns: S0 [0,128), S1 [128,256), O0 and O1 after them.
+#include <cuda_bf16.h>
+
+#include <mutex>
+
+#include "cosmot_internal.h"
+#include "ptx.cuh"
+
+namespace cosmot {
+namespace attn {
+
+constexpr int BQ = 128;
+constexpr int BKV = 128;
+constexpr int SLOTS = 4;
+constexpr int BOX_BYTES = 128 * 64 * 2;  // one 128-row x 64-column bf16 box
+constexpr int NUM_THREADS = 320;
+constexpr int TMEM_COLS = 512;
+constexpr float kRescaleThreshold = 8.0f;  // log2 units
+
+template <int HD>
+struct Cfg {
+  static constexpr int NBOX = HD / 64;
+  static constexpr int TILE_BYTES = 128 * HD * 2;
+  static constexpr int SMEM_BYTES = (2 + SLOTS) * TILE_BYTES + 256 + 1024;
+  static constexpr uint32_t IDESC_S = idesc_bf16_f32(BQ, BKV, false, false);
+  static constexpr uint32_t IDESC_O = idesc_bf16_f32(BQ, HD, false, true);
+  __device__ static constexpr uint32_t s_col(int t) { return (uint32_t)t * 128u; }
+  __device__ static constexpr uint32_t o_col(int t) { return 256u + (uint32_t)t * HD; }
+};
+
+struct Params {
+  int64_t n_q, q_key_offset, n_keys, n_ar;
+  int64_t n_q_ar;  // leading query rows that are AR
+  int64_t q_bstride, kv_bstride, o_bstride;
+  int32_t n_heads, group;  // group = n_heads / n_kv_heads
+  int32_t mask_mode;
+  int32_t batch;
+  int32_t dm_pairs, ar_pairs;
+  float scale_log2;
+  const int32_t* chunk;
+  __nv_bfloat16* o;
+  int64_t ld_o;
+  int* status;
+};
+
+struct Work {
+  int32_t b, h;
+  bool is_ar;
+  int64_t row0;     // first query row of tile 0
+  int64_t seg_end;  // query rows >= seg_end are not in this segment
+  int32_t n_kt;     // key tiles to visit
+};
+
+__device__ __forceinline__ Work decode_work(const Params& p) {
+  Work w;
+  int64_t bid = blockIdx.x;
+  const int64_t items_dm = (int64_t)p.batch * p.n_heads * p.dm_pairs;
+  int32_t pairs;
+  if (bid < items_dm) {
+    w.is_ar = false;
+    pairs = p.dm_pairs;
+  } else {
+    bid -= items_dm;
+    w.is_ar = true;
+    pairs = p.ar_pairs;
+  }
+  w.b = (int32_t)(bid / ((int64_t)p.n_heads * pairs));
+  const int64_t r = bid % ((int64_t)p.n_heads * pairs);
+  w.h = (int32_t)(r / pairs);
+  const int64_t pair = r % pairs;
+  if (w.is_ar) {
+    w.row0 = pair * 2 * BQ;
+    w.seg_end = p.n_q_ar;
+    const int64_t last = (w.row0 + 2 * BQ < w.seg_end ? w.row0 + 2 * BQ : w.seg_end) - 1;
+    int64_t kmax = p.q_key_offset + last + 1;
+    if (kmax > p.n_ar) kmax = p.n_ar;
+    w.n_kt = (int32_t)((kmax + BKV - 1) / BKV);
+  } else {
+    w.row0 = p.n_q_ar + pair * 2 * BQ;
+    w.seg_end = p.n_q;
+    w.n_kt = (int32_t)((p.n_keys + BKV - 1) / BKV);
+  }
+  return w;
+}
+
+template <int HD>
+__global__ void __launch_bounds__(NUM_THREADS, 1)
+    mot_attention_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__ CUtensorMap tmap_k,
+                         const __grid_constant__ CUtensorMap tmap_v, const __grid_constant__ Params p) {
+  using C = Cfg<HD>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const uint32_t sQ = smem_u32(smem);
+  const uint32_t sKV = sQ + 2 * C::TILE_BYTES;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + (2 + SLOTS) * C::TILE_BYTES);
+  const uint32_t bar_q = smem_u32(bars);
+  const uint32_t bar_kv_full = bar_q + 8;                // [SLOTS]
+  const uint32_t bar_kv_empty = bar_kv_full + 8 * SLOTS; // [SLOTS]
+  const uint32_t bar_s_full = bar_kv_empty + 8 * SLOTS;  // [2]
+  const uint32_t bar_p_full = bar_s_full + 16;           // [2]
+  const uint32_t bar_o_done = bar_p_full + 16;           // [2]
+  const uint32_t bar_drain = bar_o_done + 16;            // [1]
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 1 + 2 * SLOTS + 7);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const Work w = decode_work(p);
+  const int32_t g = w.h / p.group;
+
+  if (threadIdx.x == 0) {
+    mbar_init(bar_q, 1);
+    for (int s = 0; s < SLOTS; ++s) {
+      mbar_init(bar_kv_full + 8 * s, 1);
+      mbar_init(bar_kv_empty + 8 * s, 1);
+    }
+    for (int t = 0; t < 2; ++t) {
+      mbar_init(bar_s_full + 8 * t, 1);
+      mbar_init(bar_p_full + 8 * t, 128);
+      mbar_init(bar_o_done + 8 * t, 1);
+    }
+    mbar_init(bar_drain, 1);
+    fence_barrier_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_u32(tmem_slot), TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *reinterpret_cast<volatile uint32_t*>(tmem_slot);
+  const int32_t n_kt = w.n_kt;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      tma_prefetch_desc(&tmap_q);
+      tma_prefetch_desc(&tmap_k);
+      tma_prefetch_desc(&tmap_v);
+      mbar_arrive_expect_tx(bar_q, 2 * C::TILE_BYTES);
+      const int qrow = (int)(w.b * p.q_bstride + w.row0);
+      for (int t = 0; t < 2; ++t)
+        for (int bx = 0; bx < C::NBOX; ++bx)
+          tma_load_2d(sQ + t * C::TILE_BYTES + bx * BOX_BYTES, &tmap_q, bar_q, w.h * HD + bx * 64, qrow + t * BQ);
+      uint32_t armed_mask = 0, armed_parity = 0;
+      const int kvrow = (int)(w.b * p.kv_bstride);
+      for (int L = 0; L < 2 * n_kt; ++L) {
+        const int slot = L % SLOTS;
+        const uint32_t par = (L / SLOTS) & 1;
+        if (!mbar_wait(bar_kv_empty + 8 * slot, par ^ 1, p.status, kWhereAttnProducer)) break;
+        const uint32_t fb = bar_kv_full + 8 * slot;
+        mbar_arrive_expect_tx(fb, C::TILE_BYTES);
+        const CUtensorMap* m = (L & 1) ? &tmap_v : &tmap_k;
+        const int krow = kvrow + (L >> 1) * BKV;
+        for (int bx = 0; bx < C::NBOX; ++bx)
+          tma_load_2d(sKV + slot * C::TILE_BYTES + bx * BOX_BYTES, m, fb, g * HD + bx * 64, krow);
+        armed_mask |= 1u << slot;
+        armed_parity = (armed_parity & ~(1u << slot)) | (par << slot);
+      }
+      // Let every bulk copy land before the CTA may exit.
+      const uint64_t t0 = globaltimer_ns();
+      while (!mbar_try_wait(bar_q, 0) && globaltimer_ns() - t0 < kWaitLimitNs) {
+      }
+      for (int s = 0; s < SLOTS; ++s)
+        if (armed_mask & (1u << s)) {
+          const uint32_t par = (armed_parity >> s) & 1u;
+          const uint64_t t1 = globaltimer_ns();
+          while (!mbar_try_wait(bar_kv_full + 8 * s, par) && globaltimer_ns() - t1 < kWaitLimitNs) {
+          }
+        }
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      auto issue_s = [&](int t, int slot) {
+        const uint32_t qa = sQ + t * C::TILE_BYTES;
+        const uint32_t ka = sKV + slot * C::TILE_BYTES;
+#pragma unroll
+        for (int k = 0; k < HD / 16; ++k) {
+          const uint32_t off = (k >> 2) * BOX_BYTES + (k & 3) * 32;
+          umma_ss(tmem_base + C::s_col(t), sw128_desc(qa + off, 16, 1024), sw128_desc(ka + off, 16, 1024),
+                  C::IDESC_S, k > 0 ? 1u : 0u);
+        }
+      };
+      auto issue_pv = [&](int t, int slot, bool acc) {
+        const uint32_t va = sKV + slot * C::TILE_BYTES;
+#pragma unroll
+        for (int k = 0; k < BKV / 16; ++k) {
+          // V rows k*16 .. k*16+15: two 8-row swizzle atoms = 2048 bytes.
+          umma_ts(tmem_base + C::o_col(t), tmem_base + C::s_col(t) + 8 * k, sw128_desc(va + 2048 * k, BOX_BYTES, 1024),
+                  C::IDESC_O, (acc || k > 0) ? 1u : 0u);
+        }
+      };
+      auto kv_wait = [&](int L) -> bool {
+        return mbar_wait(bar_kv_full + 8 * (L % SLOTS), (L / SLOTS) & 1, p.status, kWhereAttnMma);
+      };
+      bool ok = mbar_wait(bar_q, 0, p.status, kWhereAttnMma) && kv_wait(0);
+      if (ok) {
+        tc_fence_after();
+        issue_s(0, 0);
+        umma_commit(bar_s_full);
+        issue_s(1, 0);
+        umma_commit(bar_s_full + 8);
+        umma_commit(bar_kv_empty + 8 * 0);
+      }
+      for (int j = 0; j < n_kt && ok; ++j) {
+        const int LV = 2 * j + 1, LK = 2 * j + 2;
+        const bool has_next = j + 1 < n_kt;
+        const uint32_t par = j & 1;
+        if (!kv_wait(LV) || !mbar_wait(bar_p_full, par, p.status, kWhereAttnMma)) break;
+        tc_fence_after();
+        issue_pv(0, LV % SLOTS, j > 0);
+        if (has_next) {
+          if (!kv_wait(LK)) break;
+          tc_fence_after();
+          issue_s(0, LK % SLOTS);
+          umma_commit(bar_s_full);
+        }
+        if (!mbar_wait(bar_p_full + 8, par, p.status, kWhereAttnMma)) break;
+        tc_fence_after();
+        issue_pv(1, LV % SLOTS, j > 0);
+        umma_commit(bar_kv_empty + 8 * (LV % SLOTS));
+        if (has_next) {
+          issue_s(1, LK % SLOTS);
+          umma_commit(bar_s_full + 8);
+          umma_commit(bar_kv_empty + 8 * (LK % SLOTS));
+        }
+      }
+      umma_commit(bar_o_done);
+      umma_commit(bar_o_done + 8);
+      umma_commit(bar_drain);
+      const uint64_t t0 = globaltimer_ns();
+      while (!mbar_try_wait(bar_drain, 0)) {
+        if (globaltimer_ns() - t0 > kWaitLimitNs) {
+          latch_status(p.status, COSMOT_ERR_TIMEOUT, kWhereAttnDrain);
+          break;
+        }
+      }
+    }
+    __syncwarp();
+  } else {
+    // ------------------------------------------------------------ softmax
+    const int t = (warp - 2) >> 2;           // query tile of this warpgroup
+    const int lane_base = (warp & 3) * 32;   // TMEM lanes this warp may access
+    const int r = lane_base + lane;
+    const int64_t qi = w.row0 + (int64_t)t * BQ + r;
+    const bool valid = qi < w.seg_end;
+    const int64_t qk = p.q_key_offset + qi;  // key index of this query row
+    const bool bc_dm = !w.is_ar && p.mask_mode == COSMOT_MASK_BLOCK_CAUSAL;
+    int64_t klimit = p.n_keys;
+    if (w.is_ar) klimit = qk + 1 < p.n_ar ? qk + 1 : p.n_ar;
+    const int32_t my_chunk = (bc_dm && valid) ? __ldg(p.chunk + qk) : 0;
+    const uint32_t s_addr = tmem_base + ((uint32_t)lane_base << 16) + C::s_col(t);
+    const uint32_t o_addr = tmem_base + ((uint32_t)lane_base << 16) + C::o_col(t);
+    const float sl2 = p.scale_log2;
+    float m = -INFINITY, l = 0.f;
+    bool ok = true;
+    for (int j = 0; j < n_kt; ++j) {
+      if (!mbar_wait(bar_s_full + 8 * t, j & 1, p.status, kWhereAttnSoftmax)) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      uint32_t s[128];
+      tmem_ld32(s_addr + 0, *reinterpret_cast<uint32_t(*)[32]>(&s[0]));
+      tmem_ld32(s_addr + 32, *reinterpret_cast<uint32_t(*)[32]>(&s[32]));
+      tmem_ld32(s_addr + 64, *reinterpret_cast<uint32_t(*)[32]>(&s[64]));
+      tmem_ld32(s_addr + 96, *reinterpret_cast<uint32_t(*)[32]>(&s[96]));
+      tmem_ld_wait();
+      const int64_t kbase = (int64_t)j * BKV;
+      if (kbase + BKV > klimit || (bc_dm && kbase + BKV > p.n_ar)) {
+#pragma unroll
+        for (int c = 0; c < 128; ++c) {
+          const int64_t key = kbase + c;
+          bool vis = key < klimit;
+          if (bc_dm && key >= p.n_ar && vis) vis = __ldg(p.chunk + key) <= my_chunk;
+          if (!vis) s[c] = __float_as_uint(-INFINITY);
+        }
+      }
+      float mt = -INFINITY;
+#pragma unroll
+      for (int c = 0; c < 128; ++c) mt = fmaxf(mt, __uint_as_float(s[c]));
+      const float m_new = fmaxf(m, mt * sl2);
+      const bool first = (m == -INFINITY);
+      const bool need = !first && (m_new > m + kRescaleThreshold);
+      float factor = 1.f;
+      if (first) {
+        m = m_new;
+      } else if (need) {
+        factor = ex2_approx(m - m_new);
+        m = m_new;
+        l *= factor;
+      }
+      if (__any_sync(0xffffffffu, need)) {
+#pragma unroll 1
+        for (int c = 0; c < HD / 32; ++c) {
+          uint32_t ov[32];
+          tmem_ld32(o_addr + 32 * c, ov);
+          tmem_ld_wait();
+#pragma unroll
+          for (int e = 0; e < 32; ++e) ov[e] = __float_as_uint(__uint_as_float(ov[e]) * factor);
+          tmem_st32(o_addr + 32 * c, ov);
+        }
+        tmem_st_wait();
+      }
+      const float mu = (m == -INFINITY) ? 0.f : m;
+      float rs = 0.f;
+#pragma unroll
+      for (int c0 = 0; c0 < 128; c0 += 32) {
+        uint32_t pk[16];
+#pragma unroll
+        for (int e = 0; e < 16; ++e) {
+          const float p0 = ex2_approx(fmaf(__uint_as_float(s[c0 + 2 * e]), sl2, -mu));
+          const float p1 = ex2_approx(fmaf(__uint_as_float(s[c0 + 2 * e + 1]), sl2, -mu));
+          rs += p0 + p1;
+          pk[e] = pack_bf16x2(p0, p1);
+        }
+        tmem_st16(s_addr + (c0 >> 1), pk);
+      }
+      l += rs;
+      tmem_st_wait();
+      tc_fence_before();
+      mbar_arrive(bar_p_full + 8 * t);
+    }
+    if (ok && mbar_wait(bar_o_done + 8 * t, 0, p.status, kWhereAttnSoftmax)) {
+      tc_fence_after();
+      const float inv_l = l > 0.f ? 1.0f / l : 0.f;
+      __nv_bfloat16* dst = p.o + (w.b * p.o_bstride + qi) * p.ld_o + (int64_t)w.h * HD;
+#pragma unroll 1
+      for (int c = 0; c < HD / 32; ++c) {
+        uint32_t ov[32];
+        tmem_ld32(o_addr + 32 * c, ov);
+        tmem_ld_wait();
+        if (valid) {
+#pragma unroll
+          for (int q4 = 0; q4 < 4; ++q4) {
+            uint4 v4;
+            v4.x = pack_bf16x2(__uint_as_float(ov[8 * q4 + 0]) * inv_l, __uint_as_float(ov[8 * q4 + 1]) * inv_l);
+            v4.y = pack_bf16x2(__uint_as_float(ov[8 * q4 + 2]) * inv_l, __uint_as_float(ov[8 * q4 + 3]) * inv_l);
+            v4.z = pack_bf16x2(__uint_as_float(ov[8 * q4 + 4]) * inv_l, __uint_as_float(ov[8 * q4 + 5]) * inv_l);
+            v4.w = pack_bf16x2(__uint_as_float(ov[8 * q4 + 6]) * inv_l, __uint_as_float(ov[8 * q4 + 7]) * inv_l);
+            *reinterpret_cast<uint4*>(dst + 32 * c + 8 * q4) = v4;
+          }
+        }
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 1) tmem_dealloc(tmem_base, TMEM_COLS);
+}
+
+template <int HD>
+cosmot_status launch(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, const Params& p,
+                     unsigned grid, cudaStream_t s) {
+  static std::mutex mu;
+  static uint64_t done_mask = 0;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return COSMOT_ERR_CUDA;
+  {
+    std::lock_guard<std::mutex> lk(mu);
+    if (dev >= 64 || !(done_mask & (1ull << dev))) {
+      if (cudaFuncSetAttribute(mot_attention_kernel<HD>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               Cfg<HD>::SMEM_BYTES) != cudaSuccess)
+        return COSMOT_ERR_CUDA;
+      if (dev < 64) done_mask |= 1ull << dev;
+    }
+  }
+  mot_attention_kernel<HD><<<grid, NUM_THREADS, Cfg<HD>::SMEM_BYTES, s>>>(tq, tk, tv, p);
+  return launch_status();
+}
+
+}  // namespace attn
+}  // namespace cosmot
+
+extern "C" cosmot_status cosmot_mot_attention(const cosmot_attn_desc* d, const void* q, int64_t ld_q, const void* k,
+                                              const void* v, int64_t ld_kv, void* o, int64_t ld_o,
+                                              cosmot_stream_t stream) {
+  using namespace cosmot;
+  using namespace cosmot::attn;
+  if (!d || !q || !k || !v || !o) return COSMOT_ERR_INVALID_ARG;
+  const int hd = d->head_dim;
+  if (hd != 64 && hd != 128) return COSMOT_ERR_UNSUPPORTED;
+  if (d->n_heads < 1 || d->n_kv_heads < 1 || d->n_heads % d->n_kv_heads) return COSMOT_ERR_INVALID_ARG;
+  if (d->n_q < 0 || d->n_keys < 1 || d->n_ar < 0 || d->n_ar > d->n_keys || d->q_key_offset < 0 ||
+      d->q_key_offset + d->n_q > d->n_keys || d->batch < 1)
+    return COSMOT_ERR_INVALID_ARG;
+  if (d->mask_mode != COSMOT_MASK_FULL && d->mask_mode != COSMOT_MASK_BLOCK_CAUSAL) return COSMOT_ERR_INVALID_ARG;
+  if (d->mask_mode == COSMOT_MASK_BLOCK_CAUSAL && !d->chunk) return COSMOT_ERR_INVALID_ARG;
+  const int64_t qcols = (int64_t)d->n_heads * hd, kvcols = (int64_t)d->n_kv_heads * hd;
+  if (ld_q < qcols || ld_kv < kvcols || ld_o < qcols || ld_q % 8 || ld_kv % 8 || ld_o % 8) return COSMOT_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o)) return COSMOT_ERR_INVALID_ARG;
+  if (d->batch > 1 && (d->q_batch_stride < d->n_q || d->kv_batch_stride < d->n_keys || d->o_batch_stride < d->n_q))
+    return COSMOT_ERR_INVALID_ARG;
+  if (d->n_q == 0) return COSMOT_OK;
+
+  Params p{};
+  p.n_q = d->n_q;
+  p.q_key_offset = d->q_key_offset;
+  p.n_keys = d->n_keys;
+  p.n_ar = d->n_ar;
+  int64_t nqar = d->n_ar - d->q_key_offset;
+  p.n_q_ar = nqar < 0 ? 0 : (nqar > d->n_q ? d->n_q : nqar);
+  p.q_bstride = d->batch > 1 ? d->q_batch_stride : 0;
+  p.kv_bstride = d->batch > 1 ? d->kv_batch_stride : 0;
+  p.o_bstride = d->batch > 1 ? d->o_batch_stride : 0;
+  p.n_heads = d->n_heads;
+  p.group = d->n_heads / d->n_kv_heads;
+  p.mask_mode = d->mask_mode;
+  p.batch = d->batch;
+  const int64_t ar_tiles = (p.n_q_ar + BQ - 1) / BQ;
+  const int64_t dm_tiles = (p.n_q - p.n_q_ar + BQ - 1) / BQ;
+  p.ar_pairs = (int32_t)((ar_tiles + 1) / 2);
+  p.dm_pairs = (int32_t)((dm_tiles + 1) / 2);
+  const float scale = d->softmax_scale > 0.f ? d->softmax_scale : 1.0f / sqrtf((float)hd);
+  p.scale_log2 = scale * 1.4426950408889634f;
+  p.chunk = d->chunk;
+  p.o = static_cast<__nv_bfloat16*>(o);
+  p.ld_o = ld_o;
+  p.status = device_status_ptr();
+  if (!p.status) return COSMOT_ERR_CUDA;
+
+  const int64_t grid = (int64_t)d->batch * d->n_heads * (p.ar_pairs + p.dm_pairs);
+  const int64_t q_rows = (d->batch - 1) * p.q_bstride + d->n_q;
+  const int64_t kv_rows = (d->batch - 1) * p.kv_bstride + d->n_keys;
+  if (grid > INT32_MAX || q_rows + 2 * BQ > INT32_MAX || kv_rows + BKV > INT32_MAX) return COSMOT_ERR_UNSUPPORTED;
+
+  CUtensorMap tq, tk, tv;
+  cosmot_status st = make_tmap_bf16_2d(&tq, q, (uint64_t)q_rows, (uint64_t)qcols, (uint64_t)ld_q, BQ, 64);
+  if (st != COSMOT_OK) return st;
+  st = make_tmap_bf16_2d(&tk, k, (uint64_t)kv_rows, (uint64_t)kvcols, (uint64_t)ld_kv, BKV, 64);
+  if (st != COSMOT_OK) return st;
+  st = make_tmap_bf16_2d(&tv, v, (uint64_t)kv_rows, (uint64_t)kvcols, (uint64_t)ld_kv, BKV, 64);
+  if (st != COSMOT_OK) return st;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  return hd == 128 ? launch<128>(tq, tk, tv, p, (unsigned)grid, s) : launch<64>(tq, tk, tv, p, (unsigned)grid, s);
+}

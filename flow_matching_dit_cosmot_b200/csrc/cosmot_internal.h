@@ -1,0 +1,43 @@
+// Internal declarations shared by the libcosmot translation units.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cstdint>
+
+#include "cosmot.h"
+
+namespace cosmot {
+
+// Device status site codes (reported through cosmot_get_device_status).
+enum Where : int {
+  kWhereGemmProducer = 100,
+  kWhereGemmMma = 101,
+  kWhereGemmEpilogue = 102,
+  kWhereGemmDrain = 103,
+  kWhereAttnProducer = 200,
+  kWhereAttnMma = 201,
+  kWhereAttnSoftmax = 202,
+  kWhereAttnDrain = 203,
+};
+
+// Encodes a 2D bf16 tensor map: `rows` x `cols` elements with row pitch
+// `ld` elements, box of box_rows x box_cols (box_cols * 2 == 128 bytes for the
+// 128-byte swizzle), out-of-bounds elements read as zero.
+cosmot_status make_tmap_bf16_2d(CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols, uint64_t ld,
+                                uint32_t box_rows, uint32_t box_cols);
+
+inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+inline cosmot_status launch_status() {
+  cudaError_t e = cudaGetLastError();
+  return e == cudaSuccess ? COSMOT_OK : COSMOT_ERR_CUDA;
+}
+
+int num_sms();
+
+// Per-device address of the status word that kernels latch failures into.
+int* device_status_ptr();
+
+}  // namespace cosmot

@@ -1,0 +1,511 @@
+// Routed projection GEMM on the sm_100a tensor cores (tcgen05 + TMEM + TMA).
+//
+// "Cosmos 3 方法原理全解" §3: a MoT layer holds two weight sets; Reasoner
+// weights act on AR rows and Generator weights on DM rows, with no router.
+// Rows come in segments (a contiguous row range and its weight set); a tile
+// never straddles two segments, so every tile runs one dense contraction
+//     acc[128 x 256] = A[rows, K] . W_set[cols, K]^T
+// on the tensor cores with the fp32 accumulator in tensor memory.
+//
+// Structure (one persistent CTA per SM, 192 threads):
+//   warp 0      TMA producer: A tile 128x64 and B tile 256x64 (bf16, 128-byte
+//               swizzle) per k-block into a 4-stage shared-memory ring.
+//   warp 1      owns TMEM (512 columns = two 128x256 fp32 accumulators) and
+//               issues tcgen05.mma (M=128, N=256, K=16) from one thread;
+//               tcgen05.commit frees ring slots and publishes accumulators.
+//   warps 2-5   epilogue: tcgen05.ld (one row per thread), the fused
+//               epilogue (residual add, SiLU*mul, mRoPE, Euler), bf16 stores.
+// The epilogue of tile i overlaps the mainloop of tile i+1.  Tiles are walked
+// in groups of kGroupM row tiles so that a group's A rows stay in L2 while the
+// weight columns stream past.
+//
+// Every wait is bounded (see ptx.cuh): a stuck pipeline latches
+// COSMOT_ERR_TIMEOUT, drains its outstanding copies and MMAs, frees TMEM and
+// returns.
+#include <cuda_bf16.h>
+
+#include <mutex>
+
+#include "cosmot_internal.h"
+#include "ptx.cuh"
+
+namespace cosmot {
+namespace gemm {
+
+constexpr int BM = 128;
+constexpr int BN = 256;
+constexpr int BK = 64;  // 64 bf16 = 128 bytes = one swizzle row
+constexpr int STAGES = 4;
+constexpr int A_BYTES = BM * BK * 2;
+constexpr int B_BYTES = BN * BK * 2;
+constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+constexpr int NUM_THREADS = 192;
+constexpr int TMEM_COLS = 512;
+constexpr int kMaxSegs = 64;
+constexpr int kGroupM = 16;
+constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 256 + 1024;
+constexpr uint32_t IDESC = idesc_bf16_f32(BM, BN, false, false);
+
+struct Params {
+  int64_t row_begin[kMaxSegs];
+  int64_t row_end[kMaxSegs];
+  int64_t out_row[kMaxSegs];
+  int32_t set[kMaxSegs];
+  int32_t mtile_prefix[kMaxSegs + 1];
+  int32_t n_segs;
+  int32_t num_m_tiles, num_n_tiles, num_tiles;
+  int32_t num_kb;
+  int32_t n_out;
+  int32_t head_dim;
+  int32_t group_m;
+  int64_t rope_cols;
+  const float2* rope_cs;
+  int64_t rope_period;
+  const __nv_bfloat16* res;
+  int64_t ld_res;
+  const __nv_bfloat16* x;
+  int64_t ld_x;
+  float dsigma;
+  __nv_bfloat16* out;
+  int64_t ld_out;
+  int* status;
+};
+
+struct Tile {
+  int32_t set;
+  int32_t n;          // column tile
+  int64_t a_row0;     // first A row
+  int32_t rows;       // valid rows (<= BM)
+  int64_t out_row0;   // output row of a_row0
+};
+
+__device__ __forceinline__ Tile decode_tile(const Params& p, int32_t t) {
+  const int32_t per_group = p.group_m * p.num_n_tiles;
+  const int32_t g = t / per_group;
+  const int32_t first_m = g * p.group_m;
+  const int32_t rem_m = p.num_m_tiles - first_m;
+  const int32_t gm = rem_m < p.group_m ? rem_m : p.group_m;
+  const int32_t in = t - g * per_group;
+  const int32_t m = first_m + in % gm;
+  Tile tl;
+  tl.n = in / gm;
+  int s = 0;
+  while (s + 1 < p.n_segs && m >= p.mtile_prefix[s + 1]) ++s;
+  tl.set = p.set[s];
+  tl.a_row0 = p.row_begin[s] + (int64_t)(m - p.mtile_prefix[s]) * BM;
+  const int64_t left = p.row_end[s] - tl.a_row0;
+  tl.rows = (int32_t)(left < BM ? left : BM);
+  tl.out_row0 = p.out_row[s] + (tl.a_row0 - p.row_begin[s]);
+  return tl;
+}
+
+// Stores 32 consecutive fp32 values of one row as bf16, clipped to n_out.
+__device__ __forceinline__ void store_row32(__nv_bfloat16* dst, int32_t col0, int32_t n_out, const float* v) {
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    if (col0 + 8 * q + 8 <= n_out) {
+      uint4 w;
+      w.x = pack_bf16x2(v[8 * q + 0], v[8 * q + 1]);
+      w.y = pack_bf16x2(v[8 * q + 2], v[8 * q + 3]);
+      w.z = pack_bf16x2(v[8 * q + 4], v[8 * q + 5]);
+      w.w = pack_bf16x2(v[8 * q + 6], v[8 * q + 7]);
+      *reinterpret_cast<uint4*>(dst + 8 * q) = w;
+    }
+  }
+}
+
+// Loads 32 consecutive bf16 of one row as fp32 (zeros past n_out).
+__device__ __forceinline__ void load_row32(const __nv_bfloat16* src, int32_t col0, int32_t n_out, float* v) {
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    if (col0 + 8 * q + 8 <= n_out) {
+      uint4 w = *reinterpret_cast<const uint4*>(src + 8 * q);
+      const uint32_t* u = reinterpret_cast<const uint32_t*>(&w);
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        float2 f = unpack_bf16x2(u[j]);
+        v[8 * q + 2 * j] = f.x;
+        v[8 * q + 2 * j + 1] = f.y;
+      }
+    } else {
+#pragma unroll
+      for (int j = 0; j < 8; ++j) v[8 * q + j] = 0.f;
+    }
+  }
+}
+
+template <int EPI>
+__global__ void __launch_bounds__(NUM_THREADS, 1)
+    routed_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUtensorMap tmap_b0,
+                       const __grid_constant__ CUtensorMap tmap_b1, const __grid_constant__ CUtensorMap tmap_u0,
+                       const __grid_constant__ CUtensorMap tmap_u1, const __grid_constant__ Params p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const uint32_t sbase = smem_u32(smem);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + STAGES * STAGE_BYTES);
+  const uint32_t bar_full = smem_u32(bars);                // [STAGES]
+  const uint32_t bar_empty = bar_full + 8 * STAGES;        // [STAGES]
+  const uint32_t bar_tfull = bar_empty + 8 * STAGES;       // [2]
+  const uint32_t bar_tempty = bar_tfull + 16;              // [2]
+  const uint32_t bar_drain = bar_tempty + 16;              // [1]
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * STAGES + 5);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(bar_full + 8 * s, 1);
+      mbar_init(bar_empty + 8 * s, 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(bar_tfull + 8 * b, 1);
+      mbar_init(bar_tempty + 8 * b, 4 * 32);
+    }
+    mbar_init(bar_drain, 1);
+    fence_barrier_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_u32(tmem_slot), TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *reinterpret_cast<volatile uint32_t*>(tmem_slot);
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      tma_prefetch_desc(&tmap_a);
+      tma_prefetch_desc(&tmap_b0);
+      tma_prefetch_desc(&tmap_b1);
+      if (EPI == COSMOT_EPI_SILU_MUL) {
+        tma_prefetch_desc(&tmap_u0);
+        tma_prefetch_desc(&tmap_u1);
+      }
+      int stage = 0;
+      uint32_t phase = 0;
+      uint32_t armed_mask = 0, armed_parity = 0;
+      bool ok = true;
+      for (int32_t t = blockIdx.x; t < p.num_tiles && ok; t += gridDim.x) {
+        const Tile tl = decode_tile(p, t);
+        const CUtensorMap* mb = tl.set ? &tmap_b1 : &tmap_b0;
+        const CUtensorMap* mu = tl.set ? &tmap_u1 : &tmap_u0;
+        for (int kb = 0; kb < p.num_kb; ++kb) {
+          if (!mbar_wait(bar_empty + 8 * stage, phase ^ 1, p.status, kWhereGemmProducer)) {
+            ok = false;
+            break;
+          }
+          const uint32_t fb = bar_full + 8 * stage;
+          const uint32_t sa = sbase + stage * STAGE_BYTES;
+          const uint32_t sb = sa + A_BYTES;
+          mbar_arrive_expect_tx(fb, STAGE_BYTES);
+          tma_load_2d(sa, &tmap_a, fb, kb * BK, (int)tl.a_row0);
+          if (EPI == COSMOT_EPI_SILU_MUL) {
+            tma_load_2d(sb, mb, fb, kb * BK, tl.n * (BN / 2));
+            tma_load_2d(sb + B_BYTES / 2, mu, fb, kb * BK, tl.n * (BN / 2));
+          } else {
+            tma_load_2d(sb, mb, fb, kb * BK, tl.n * BN);
+          }
+          armed_mask |= 1u << stage;
+          armed_parity = (armed_parity & ~(1u << stage)) | (phase << stage);
+          if (++stage == STAGES) {
+            stage = 0;
+            phase ^= 1;
+          }
+        }
+      }
+      // No bulk copy may still be writing shared memory when the CTA exits.
+      for (int s = 0; s < STAGES; ++s)
+        if (armed_mask & (1u << s)) {
+          const uint32_t par = (armed_parity >> s) & 1u;
+          const uint64_t t0 = globaltimer_ns();
+          while (!mbar_try_wait(bar_full + 8 * s, par) && globaltimer_ns() - t0 < kWaitLimitNs) {
+          }
+        }
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      bool ok = true;
+      uint32_t local = 0;
+      for (int32_t t = blockIdx.x; t < p.num_tiles && ok; t += gridDim.x, ++local) {
+        const uint32_t buf = local & 1;
+        const uint32_t use = local >> 1;
+        if (!mbar_wait(bar_tempty + 8 * buf, (use & 1) ^ 1, p.status, kWhereGemmMma)) break;
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + buf * BN;
+        for (int kb = 0; kb < p.num_kb; ++kb) {
+          if (!mbar_wait(bar_full + 8 * stage, phase, p.status, kWhereGemmMma)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t sa = sbase + stage * STAGE_BYTES;
+          const uint32_t sb = sa + A_BYTES;
+#pragma unroll
+          for (int k = 0; k < BK / 16; ++k) {
+            const uint64_t ad = sw128_desc(sa + 32 * k, 16, 1024);
+            const uint64_t bd = sw128_desc(sb + 32 * k, 16, 1024);
+            umma_ss(d_tmem, ad, bd, IDESC, (kb | k) != 0 ? 1u : 0u);
+          }
+          umma_commit(bar_empty + 8 * stage);
+          if (++stage == STAGES) {
+            stage = 0;
+            phase ^= 1;
+          }
+        }
+        if (!ok) break;
+        umma_commit(bar_tfull + 8 * buf);
+      }
+      // Wait until every MMA issued above has completed before TMEM is freed.
+      umma_commit(bar_drain);
+      const uint64_t t0 = globaltimer_ns();
+      while (!mbar_try_wait(bar_drain, 0)) {
+        if (globaltimer_ns() - t0 > kWaitLimitNs) {
+          latch_status(p.status, COSMOT_ERR_TIMEOUT, kWhereGemmDrain);
+          break;
+        }
+      }
+    }
+    __syncwarp();
+  } else {
+    // ------------------------------------------------------------ epilogue
+    const int lane_base = (warp & 3) * 32;  // TMEM lanes this warp may access
+    const int r = lane_base + lane;          // row within the tile
+    uint32_t local = 0;
+    for (int32_t t = blockIdx.x; t < p.num_tiles; t += gridDim.x, ++local) {
+      const uint32_t buf = local & 1;
+      const uint32_t use = local >> 1;
+      if (!mbar_wait(bar_tfull + 8 * buf, use & 1, p.status, kWhereGemmEpilogue)) break;
+      tc_fence_after();
+      const Tile tl = decode_tile(p, t);
+      const bool valid = r < tl.rows;
+      const int64_t orow = tl.out_row0 + r;
+      const uint32_t tacc = tmem_base + ((uint32_t)lane_base << 16) + buf * BN;
+      uint32_t v[32];
+      float f[32];
+      if (EPI == COSMOT_EPI_SILU_MUL) {
+        const int32_t col_base = tl.n * (BN / 2);
+#pragma unroll 1
+        for (int c = 0; c < 4; ++c) {
+          uint32_t u[32];
+          tmem_ld32(tacc + 32 * c, v);
+          tmem_ld32(tacc + BN / 2 + 32 * c, u);
+          tmem_ld_wait();
+          const int32_t col0 = col_base + 32 * c;
+          if (valid && col0 < p.n_out) {
+#pragma unroll
+            for (int j = 0; j < 32; ++j) {
+              const float g = __uint_as_float(v[j]);
+              const float up = __uint_as_float(u[j]);
+              f[j] = g / (1.0f + __expf(-g)) * up;
+            }
+            store_row32(p.out + orow * p.ld_out + col0, col0, p.n_out, f);
+          }
+        }
+      } else if (EPI == COSMOT_EPI_MROPE) {
+        const int hd = p.head_dim;
+        const int half = hd >> 1;
+        const int64_t trow = p.rope_period > 0 ? orow % p.rope_period : orow;
+        const float2* cs_row = p.rope_cs + trow * half;
+#pragma unroll 1
+        for (int hb = 0; hb < BN / hd; ++hb) {
+          const int32_t hcol = tl.n * BN + hb * hd;
+          const bool rotate = hcol < p.rope_cols;
+#pragma unroll 1
+          for (int i0 = 0; i0 < half; i0 += 32) {
+            uint32_t u[32];
+            tmem_ld32(tacc + hb * hd + i0, v);
+            tmem_ld32(tacc + hb * hd + half + i0, u);
+            tmem_ld_wait();
+            if (valid && hcol < p.n_out) {
+              float lo[32], hi[32];
+              if (rotate) {
+#pragma unroll
+                for (int j = 0; j < 32; j += 2) {
+                  const float4 cs = __ldg(reinterpret_cast<const float4*>(cs_row + i0 + j));
+                  const float a0 = __uint_as_float(v[j]), a1 = __uint_as_float(v[j + 1]);
+                  const float b0 = __uint_as_float(u[j]), b1 = __uint_as_float(u[j + 1]);
+                  lo[j] = a0 * cs.x - b0 * cs.y;
+                  hi[j] = b0 * cs.x + a0 * cs.y;
+                  lo[j + 1] = a1 * cs.z - b1 * cs.w;
+                  hi[j + 1] = b1 * cs.z + a1 * cs.w;
+                }
+              } else {
+#pragma unroll
+                for (int j = 0; j < 32; ++j) {
+                  lo[j] = __uint_as_float(v[j]);
+                  hi[j] = __uint_as_float(u[j]);
+                }
+              }
+              __nv_bfloat16* dst = p.out + orow * p.ld_out + hcol;
+              store_row32(dst + i0, hcol + i0, p.n_out, lo);
+              store_row32(dst + half + i0, hcol + half + i0, p.n_out, hi);
+            }
+          }
+        }
+      } else {
+#pragma unroll 1
+        for (int c = 0; c < BN / 32; ++c) {
+          tmem_ld32(tacc + 32 * c, v);
+          tmem_ld_wait();
+          const int32_t col0 = tl.n * BN + 32 * c;
+          if (valid && col0 < p.n_out) {
+            if (EPI == COSMOT_EPI_RESIDUAL) {
+              float rs[32];
+              load_row32(p.res + orow * p.ld_res + col0, col0, p.n_out, rs);
+#pragma unroll
+              for (int j = 0; j < 32; ++j) f[j] = __uint_as_float(v[j]) + rs[j];
+            } else if (EPI == COSMOT_EPI_EULER) {
+              float xs[32];
+              load_row32(p.x + orow * p.ld_x + col0, col0, p.n_out, xs);
+#pragma unroll
+              for (int j = 0; j < 32; ++j) f[j] = fmaf(p.dsigma, __uint_as_float(v[j]), xs[j]);
+            } else {
+#pragma unroll
+              for (int j = 0; j < 32; ++j) f[j] = __uint_as_float(v[j]);
+            }
+            store_row32(p.out + orow * p.ld_out + col0, col0, p.n_out, f);
+          }
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(bar_tempty + 8 * buf);
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 1) tmem_dealloc(tmem_base, TMEM_COLS);
+}
+
+template <int EPI>
+cosmot_status launch(const CUtensorMap& ta, const CUtensorMap& tb0, const CUtensorMap& tb1, const CUtensorMap& tu0,
+                     const CUtensorMap& tu1, const Params& p, cudaStream_t s) {
+  static std::mutex mu;
+  static uint64_t done_mask = 0;  // devices whose smem limit was raised
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return COSMOT_ERR_CUDA;
+  {
+    std::lock_guard<std::mutex> lk(mu);
+    if (dev >= 64 || !(done_mask & (1ull << dev))) {
+      if (cudaFuncSetAttribute(routed_gemm_kernel<EPI>, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES) !=
+          cudaSuccess)
+        return COSMOT_ERR_CUDA;
+      if (dev < 64) done_mask |= 1ull << dev;
+    }
+  }
+  int grid = num_sms();
+  if (p.num_tiles < grid) grid = p.num_tiles;
+  routed_gemm_kernel<EPI><<<grid, NUM_THREADS, SMEM_BYTES, s>>>(ta, tb0, tb1, tu0, tu1, p);
+  return launch_status();
+}
+
+}  // namespace gemm
+}  // namespace cosmot
+
+extern "C" cosmot_status cosmot_routed_linear(const void* a, int64_t ld_a, int64_t k, const cosmot_segment* segs,
+                                              int32_t n_segs, const void* w0, const void* w1, const void* w0_up,
+                                              const void* w1_up, int64_t n_out, void* out, int64_t ld_out,
+                                              const cosmot_epilogue* epi, cosmot_stream_t stream) {
+  using namespace cosmot;
+  using namespace cosmot::gemm;
+  const int kind = epi ? epi->kind : COSMOT_EPI_NONE;
+  if (!a || !out || !segs || n_segs < 1 || n_segs > kMaxSegs) return COSMOT_ERR_INVALID_ARG;
+  if (k < 8 || k % 8 || n_out < 8 || n_out % 8 || ld_a % 8 || ld_out % 8 || ld_a < k || ld_out < n_out)
+    return COSMOT_ERR_INVALID_ARG;
+  if (!aligned16(a) || !aligned16(out)) return COSMOT_ERR_INVALID_ARG;
+  if (k > INT32_MAX || n_out > INT32_MAX) return COSMOT_ERR_UNSUPPORTED;
+  if (kind < COSMOT_EPI_NONE || kind > COSMOT_EPI_EULER) return COSMOT_ERR_INVALID_ARG;
+
+  Params p{};
+  p.n_segs = n_segs;
+  bool uses[2] = {false, false};
+  int64_t max_row = 0;
+  int32_t mt = 0;
+  for (int i = 0; i < n_segs; ++i) {
+    const cosmot_segment& s = segs[i];
+    if (s.row_begin < 0 || s.row_end < s.row_begin || s.out_row < 0 || (s.weight_set != 0 && s.weight_set != 1))
+      return COSMOT_ERR_INVALID_ARG;
+    p.row_begin[i] = s.row_begin;
+    p.row_end[i] = s.row_end;
+    p.out_row[i] = s.out_row;
+    p.set[i] = s.weight_set;
+    p.mtile_prefix[i] = mt;
+    const int64_t tiles = (s.row_end - s.row_begin + BM - 1) / BM;
+    if ((int64_t)mt + tiles > INT32_MAX / 4) return COSMOT_ERR_UNSUPPORTED;
+    mt += (int32_t)tiles;
+    if (s.row_end > s.row_begin) uses[s.weight_set] = true;
+    if (s.row_end > max_row) max_row = s.row_end;
+  }
+  p.mtile_prefix[n_segs] = mt;
+  p.num_m_tiles = mt;
+  if (mt == 0) return COSMOT_OK;
+  if (max_row > INT32_MAX) return COSMOT_ERR_UNSUPPORTED;
+  const bool silu = kind == COSMOT_EPI_SILU_MUL;
+  p.num_n_tiles = (int32_t)((n_out + (silu ? BN / 2 : BN) - 1) / (silu ? BN / 2 : BN));
+  if ((int64_t)p.num_m_tiles * p.num_n_tiles > INT32_MAX) return COSMOT_ERR_UNSUPPORTED;
+  p.num_tiles = p.num_m_tiles * p.num_n_tiles;
+  p.num_kb = (int32_t)((k + BK - 1) / BK);
+  p.n_out = (int32_t)n_out;
+  p.group_m = kGroupM;
+  p.out = static_cast<__nv_bfloat16*>(out);
+  p.ld_out = ld_out;
+  p.status = device_status_ptr();
+  if (!p.status) return COSMOT_ERR_CUDA;
+
+  if (kind == COSMOT_EPI_RESIDUAL) {
+    if (!epi->res || !aligned16(epi->res) || epi->ld_res % 8 || epi->ld_res < n_out) return COSMOT_ERR_INVALID_ARG;
+    p.res = static_cast<const __nv_bfloat16*>(epi->res);
+    p.ld_res = epi->ld_res;
+  } else if (kind == COSMOT_EPI_EULER) {
+    if (!epi->x || !aligned16(epi->x) || epi->ld_x % 8 || epi->ld_x < n_out) return COSMOT_ERR_INVALID_ARG;
+    p.x = static_cast<const __nv_bfloat16*>(epi->x);
+    p.ld_x = epi->ld_x;
+    p.dsigma = epi->dsigma;
+  } else if (kind == COSMOT_EPI_MROPE) {
+    if (epi->head_dim != 64 && epi->head_dim != 128) return COSMOT_ERR_UNSUPPORTED;
+    if (!epi->rope_cs || !aligned16(epi->rope_cs) || epi->rope_cols < 0 || epi->rope_cols % epi->head_dim ||
+        epi->rope_cols > n_out || epi->rope_period < 0)
+      return COSMOT_ERR_INVALID_ARG;
+    p.head_dim = epi->head_dim;
+    p.rope_cols = epi->rope_cols;
+    p.rope_cs = reinterpret_cast<const float2*>(epi->rope_cs);
+    p.rope_period = epi->rope_period;
+  }
+
+  // Tensor maps: A over all rows the segments touch; B per weight set.
+  CUtensorMap ta, tb[2], tu[2];
+  cosmot_status st = make_tmap_bf16_2d(&ta, a, (uint64_t)max_row, (uint64_t)k, (uint64_t)ld_a, BM, BK);
+  if (st != COSMOT_OK) return st;
+  const void* wb[2] = {w0, w1};
+  const void* wu[2] = {w0_up, w1_up};
+  const uint32_t brows = silu ? BN / 2 : BN;
+  for (int s = 0; s < 2; ++s) {
+    const int src = uses[s] ? s : (uses[0] ? 0 : 1);  // an unused set reuses a valid map
+    if (!wb[src]) return COSMOT_ERR_INVALID_ARG;
+    st = make_tmap_bf16_2d(&tb[s], wb[src], (uint64_t)n_out, (uint64_t)k, (uint64_t)k, brows, BK);
+    if (st != COSMOT_OK) return st;
+    if (silu) {
+      if (!wu[src]) return COSMOT_ERR_INVALID_ARG;
+      st = make_tmap_bf16_2d(&tu[s], wu[src], (uint64_t)n_out, (uint64_t)k, (uint64_t)k, brows, BK);
+      if (st != COSMOT_OK) return st;
+    } else {
+      tu[s] = tb[s];
+    }
+  }
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  switch (kind) {
+    case COSMOT_EPI_NONE: return launch<COSMOT_EPI_NONE>(ta, tb[0], tb[1], tu[0], tu[1], p, s);
+    case COSMOT_EPI_RESIDUAL: return launch<COSMOT_EPI_RESIDUAL>(ta, tb[0], tb[1], tu[0], tu[1], p, s);
+    case COSMOT_EPI_SILU_MUL: return launch<COSMOT_EPI_SILU_MUL>(ta, tb[0], tb[1], tu[0], tu[1], p, s);
+    case COSMOT_EPI_MROPE: return launch<COSMOT_EPI_MROPE>(ta, tb[0], tb[1], tu[0], tu[1], p, s);
+    default: return launch<COSMOT_EPI_EULER>(ta, tb[0], tb[1], tu[0], tu[1], p, s);
+  }
+}

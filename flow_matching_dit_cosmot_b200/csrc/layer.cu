@@ -1,0 +1,191 @@
+// One Mixture-of-Transformers layer forward plus the Euler sampler step.
+//
+// "Cosmos 3 方法原理全解" §3 (two weight sets, one shared attention under the
+// MoT mask) and §7.2 (velocity output, x_next = x + (sigma_next - sigma) v).
+// The driver only sequences kernels on the caller's stream; every step runs in
+// the kernels of this library:
+//   1 routed RMSNorm            h -> a                      (g1 of each set)
+//   2 routed QKV GEMM + mRoPE    a -> qkv
+//   3 MoT attention              qkv -> o
+//   4 routed O GEMM + residual   o, h -> h1
+//   5 routed RMSNorm             h1 -> a                     (g2)
+//   6 routed gate/up + SiLU*mul  a -> u
+//   7 routed down + residual     u, h1 -> h_out
+//   8 RMSNorm (noisy rows)       h_out -> a (packed)         (g_fin)
+//   9 velocity GEMM + Euler      a -> h[noisy rows] in place
+#include "cosmot_internal.h"
+
+namespace cosmot {
+namespace {
+
+constexpr int kMaxBatch = 32;
+
+struct WsLayout {
+  size_t a, qkv, o, h1, u, total;
+};
+
+size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+cosmot_status check_dims(const cosmot_dims* d) {
+  if (!d) return COSMOT_ERR_INVALID_ARG;
+  if (d->d_model <= 0 || d->d_model % 8 || d->ffn <= 0 || d->ffn % 8) return COSMOT_ERR_INVALID_ARG;
+  if (d->n_heads <= 0 || d->n_kv_heads <= 0 || d->n_heads % d->n_kv_heads) return COSMOT_ERR_INVALID_ARG;
+  if (d->head_dim != 64 && d->head_dim != 128) return COSMOT_ERR_UNSUPPORTED;
+  if (d->rope_sections[0] < 0 || d->rope_sections[1] < 0 || d->rope_sections[2] < 0 ||
+      d->rope_sections[0] + d->rope_sections[1] + d->rope_sections[2] != d->head_dim / 2)
+    return COSMOT_ERR_INVALID_ARG;
+  if (!(d->eps >= 0.f) || !(d->rope_base > 0.0)) return COSMOT_ERR_INVALID_ARG;
+  return COSMOT_OK;
+}
+
+cosmot_status check_seq(const cosmot_seq_desc* s) {
+  if (!s) return COSMOT_ERR_INVALID_ARG;
+  if (s->n_ar < 0 || s->n_clean < 0 || s->n_noisy < 0 || s->n_ar + s->n_clean + s->n_noisy < 1)
+    return COSMOT_ERR_INVALID_ARG;
+  if (s->batch < 1 || s->batch > kMaxBatch) return COSMOT_ERR_UNSUPPORTED;
+  if (s->mask_mode != COSMOT_MASK_FULL && s->mask_mode != COSMOT_MASK_BLOCK_CAUSAL) return COSMOT_ERR_INVALID_ARG;
+  if (s->mask_mode == COSMOT_MASK_BLOCK_CAUSAL && !s->chunk) return COSMOT_ERR_INVALID_ARG;
+  if (!s->rope_cs) return COSMOT_ERR_INVALID_ARG;
+  return COSMOT_OK;
+}
+
+WsLayout ws_layout(const cosmot_dims& d, const cosmot_seq_desc& s) {
+  const size_t rows = (size_t)s.batch * (size_t)(s.n_ar + s.n_clean + s.n_noisy);
+  const size_t qkv_cols = (size_t)(d.n_heads + 2 * d.n_kv_heads) * d.head_dim;
+  const size_t q_cols = (size_t)d.n_heads * d.head_dim;
+  WsLayout w;
+  size_t off = 0;
+  w.a = off;   off += align256(rows * d.d_model * 2);
+  w.qkv = off; off += align256(rows * qkv_cols * 2);
+  w.o = off;   off += align256(rows * q_cols * 2);
+  w.h1 = off;  off += align256(rows * d.d_model * 2);
+  w.u = off;   off += align256(rows * d.ffn * 2);
+  w.total = off;
+  return w;
+}
+
+}  // namespace
+}  // namespace cosmot
+
+extern "C" {
+
+cosmot_status cosmot_layer_workspace_size(const cosmot_dims* dims, const cosmot_seq_desc* seq, size_t* bytes) {
+  using namespace cosmot;
+  if (!bytes) return COSMOT_ERR_INVALID_ARG;
+  cosmot_status st = check_dims(dims);
+  if (st != COSMOT_OK) return st;
+  if (!seq || seq->batch < 1 || seq->batch > kMaxBatch || seq->n_ar < 0 || seq->n_clean < 0 || seq->n_noisy < 0)
+    return COSMOT_ERR_INVALID_ARG;
+  *bytes = ws_layout(*dims, *seq).total;
+  return COSMOT_OK;
+}
+
+cosmot_status cosmot_layer_forward(const cosmot_dims* dims, const cosmot_layer_weights* w,
+                                   const cosmot_seq_desc* seq, void* h, void* h_out, double sigma,
+                                   double sigma_next, void* workspace, size_t workspace_bytes,
+                                   cosmot_stream_t stream) {
+  using namespace cosmot;
+  cosmot_status st = check_dims(dims);
+  if (st != COSMOT_OK) return st;
+  st = check_seq(seq);
+  if (st != COSMOT_OK) return st;
+  if (!w || !h || !h_out || !workspace) return COSMOT_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return COSMOT_ERR_INVALID_ARG;
+  const WsLayout L = ws_layout(*dims, *seq);
+  if (workspace_bytes < L.total) return COSMOT_ERR_WORKSPACE;
+
+  const cosmot_dims& D = *dims;
+  const cosmot_seq_desc& S = *seq;
+  const int64_t N = (int64_t)S.n_ar + S.n_clean + S.n_noisy;
+  const int64_t d = D.d_model, F = D.ffn, hd = D.head_dim;
+  const int64_t qc = (int64_t)D.n_heads * hd, kvc = (int64_t)D.n_kv_heads * hd, qkvc = qc + 2 * kvc;
+  const int B = S.batch;
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  void* a = ws + L.a;
+  void* qkv = ws + L.qkv;
+  void* o = ws + L.o;
+  void* h1 = ws + L.h1;
+  void* u = ws + L.u;
+  uint16_t* hb = static_cast<uint16_t*>(h);
+
+  // Row segments: AR rows of every sequence go through set 0, DM rows set 1.
+  cosmot_segment segs[2 * kMaxBatch];
+  int ns = 0;
+  for (int b = 0; b < B; ++b) {
+    const int64_t r0 = b * N;
+    if (S.n_ar > 0) segs[ns++] = cosmot_segment{r0, r0 + S.n_ar, r0, 0, 0};
+    if (N > S.n_ar) segs[ns++] = cosmot_segment{r0 + S.n_ar, r0 + N, r0 + S.n_ar, 1, 0};
+  }
+  const cosmot_set_weights& R = w->set[0];
+  const cosmot_set_weights& G = w->set[1];
+
+  // 1. pre-attention norm
+  st = cosmot_rmsnorm_routed(h, d, segs, ns, R.g1, G.g1, d, D.eps, a, d, stream);
+  if (st != COSMOT_OK) return st;
+  // 2. QKV projection with mRoPE on the Q and K heads
+  cosmot_epilogue e{};
+  e.kind = COSMOT_EPI_MROPE;
+  e.head_dim = D.head_dim;
+  e.rope_cols = qc + kvc;
+  e.rope_cs = S.rope_cs;
+  e.rope_period = N;
+  st = cosmot_routed_linear(a, d, d, segs, ns, R.wqkv, G.wqkv, nullptr, nullptr, qkvc, qkv, qkvc, &e, stream);
+  if (st != COSMOT_OK) return st;
+  // 3. attention
+  cosmot_attn_desc ad{};
+  ad.n_q = N;
+  ad.q_key_offset = 0;
+  ad.n_keys = N;
+  ad.n_ar = S.n_ar;
+  ad.n_heads = D.n_heads;
+  ad.n_kv_heads = D.n_kv_heads;
+  ad.head_dim = D.head_dim;
+  ad.mask_mode = S.mask_mode;
+  ad.chunk = S.chunk;
+  ad.batch = B;
+  ad.q_batch_stride = ad.kv_batch_stride = ad.o_batch_stride = N;
+  uint16_t* qkvp = static_cast<uint16_t*>(qkv);
+  st = cosmot_mot_attention(&ad, qkvp, qkvc, qkvp + qc, qkvp + qc + kvc, qkvc, o, qc, stream);
+  if (st != COSMOT_OK) return st;
+  // 4. output projection + residual
+  e = cosmot_epilogue{};
+  e.kind = COSMOT_EPI_RESIDUAL;
+  e.res = h;
+  e.ld_res = d;
+  st = cosmot_routed_linear(o, qc, qc, segs, ns, R.wo, G.wo, nullptr, nullptr, d, h1, d, &e, stream);
+  if (st != COSMOT_OK) return st;
+  // 5. pre-FFN norm
+  st = cosmot_rmsnorm_routed(h1, d, segs, ns, R.g2, G.g2, d, D.eps, a, d, stream);
+  if (st != COSMOT_OK) return st;
+  // 6. gate/up with SiLU * mul
+  e = cosmot_epilogue{};
+  e.kind = COSMOT_EPI_SILU_MUL;
+  st = cosmot_routed_linear(a, d, d, segs, ns, R.wg, G.wg, R.wu, G.wu, F, u, F, &e, stream);
+  if (st != COSMOT_OK) return st;
+  // 7. down projection + residual
+  e = cosmot_epilogue{};
+  e.kind = COSMOT_EPI_RESIDUAL;
+  e.res = h1;
+  e.ld_res = d;
+  st = cosmot_routed_linear(u, F, F, segs, ns, R.wd, G.wd, nullptr, nullptr, d, h_out, d, &e, stream);
+  if (st != COSMOT_OK) return st;
+  if (S.n_noisy == 0) return COSMOT_OK;
+  // 8. final norm of the noisy rows, packed into a
+  cosmot_segment vs[kMaxBatch], ns_in[kMaxBatch];
+  for (int b = 0; b < B; ++b) {
+    const int64_t z0 = b * N + S.n_ar + S.n_clean;
+    ns_in[b] = cosmot_segment{z0, z0 + S.n_noisy, (int64_t)b * S.n_noisy, 1, 0};
+    vs[b] = cosmot_segment{(int64_t)b * S.n_noisy, (int64_t)(b + 1) * S.n_noisy, z0, 1, 0};
+  }
+  st = cosmot_rmsnorm_routed(h_out, d, ns_in, B, w->gfin, w->gfin, d, D.eps, a, d, stream);
+  if (st != COSMOT_OK) return st;
+  // 9. velocity head with the Euler step, in place on the noisy rows of h
+  e = cosmot_epilogue{};
+  e.kind = COSMOT_EPI_EULER;
+  e.x = h;
+  e.ld_x = d;
+  e.dsigma = (float)(sigma_next - sigma);
+  return cosmot_routed_linear(a, d, d, vs, B, w->wvel, w->wvel, nullptr, nullptr, d, hb, d, &e, stream);
+}
+
+}  // extern "C"

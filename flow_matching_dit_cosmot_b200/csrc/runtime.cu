@@ -1,0 +1,113 @@
+// Status strings, the device status word, tensor-map encoding and device
+// queries shared by every entry point.
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+
+#include "cosmot_internal.h"
+
+namespace cosmot {
+
+__device__ int g_status_word[2];
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+int* g_status_ptr[kMaxDevices] = {};
+int g_sm_count[kMaxDevices] = {};
+std::mutex g_mu;
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+EncodeTiledFn g_encode = nullptr;
+
+EncodeTiledFn encode_fn() {
+  std::lock_guard<std::mutex> lk(g_mu);
+  if (!g_encode) {
+    void* fn = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      g_encode = reinterpret_cast<EncodeTiledFn>(fn);
+  }
+  return g_encode;
+}
+
+}  // namespace
+
+int* device_status_ptr() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+  std::lock_guard<std::mutex> lk(g_mu);
+  if (!g_status_ptr[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_status_word) != cudaSuccess) return nullptr;
+    g_status_ptr[dev] = static_cast<int*>(p);
+  }
+  return g_status_ptr[dev];
+}
+
+int num_sms() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return 148;
+  std::lock_guard<std::mutex> lk(g_mu);
+  if (!g_sm_count[dev]) {
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) n = 148;
+    g_sm_count[dev] = n;
+  }
+  return g_sm_count[dev];
+}
+
+cosmot_status make_tmap_bf16_2d(CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols, uint64_t ld,
+                                uint32_t box_rows, uint32_t box_cols) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return COSMOT_ERR_CUDA;
+  if (!aligned16(base) || (ld * 2) % 16 != 0 || rows == 0 || cols == 0) return COSMOT_ERR_INVALID_ARG;
+  cuuint64_t dims[2] = {cols, rows};
+  cuuint64_t strides[1] = {ld * 2};
+  cuuint32_t box[2] = {box_cols, box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? COSMOT_OK : COSMOT_ERR_INVALID_ARG;
+}
+
+}  // namespace cosmot
+
+extern "C" {
+
+const char* cosmot_status_string(cosmot_status s) {
+  switch (s) {
+    case COSMOT_OK: return "COSMOT_OK";
+    case COSMOT_ERR_INVALID_ARG: return "COSMOT_ERR_INVALID_ARG";
+    case COSMOT_ERR_UNSUPPORTED: return "COSMOT_ERR_UNSUPPORTED";
+    case COSMOT_ERR_CUDA: return "COSMOT_ERR_CUDA";
+    case COSMOT_ERR_TIMEOUT: return "COSMOT_ERR_TIMEOUT";
+    case COSMOT_ERR_WORKSPACE: return "COSMOT_ERR_WORKSPACE";
+    default: return "COSMOT_ERR_UNKNOWN";
+  }
+}
+
+int32_t cosmot_version(void) { return 100; }
+
+cosmot_status cosmot_get_device_status(cosmot_stream_t stream, cosmot_status* out, int32_t* where_out) {
+  if (!out) return COSMOT_ERR_INVALID_ARG;
+  int* p = cosmot::device_status_ptr();
+  if (!p) return COSMOT_ERR_CUDA;
+  int host[2] = {0, 0};
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (cudaMemcpyAsync(host, p, sizeof(host), cudaMemcpyDeviceToHost, s) != cudaSuccess) return COSMOT_ERR_CUDA;
+  if (cudaStreamSynchronize(s) != cudaSuccess) return COSMOT_ERR_CUDA;
+  if (host[0] != 0) {
+    if (cudaMemsetAsync(p, 0, sizeof(host), s) != cudaSuccess) return COSMOT_ERR_CUDA;
+    if (cudaStreamSynchronize(s) != cudaSuccess) return COSMOT_ERR_CUDA;
+  }
+  *out = host[0];
+  if (where_out) *where_out = host[1];
+  return COSMOT_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,299 @@
+/*
+ * libcosmot — the Cosmos 3 Mixture-of-Transformers (MoT) layer hot path on
+ * NVIDIA B200 (sm_100a).  C ABI: plain pointers, sizes and small structs.
+ *
+ * What is computed, and where the pages define it:
+ *   "Cosmos 3 方法原理全解" §2  packed sequence [AR..., EOS, BOG, DM clean..., DM noisy...]
+ *   "Cosmos 3 方法原理全解" §3  two weight sets (Reasoner for AR rows, Generator for DM rows),
+ *                               O_AR = Attn_causal(Q_AR,K_AR,V_AR),
+ *                               O_DM = Attn_full(Q_DM,[K_AR;K_DM],[V_AR;V_DM])
+ *   "Cosmos 3 方法原理全解" §5  unified 3D mRoPE (t,h,w), dt = 6/TPS, AR->DM offset 15000
+ *   "Cosmos 3 方法原理全解" §7.2 Euler step x_next = x + (sigma_next - sigma) * v
+ *   "NVIDIA 发布 Cosmos 3 系列四个开放权重世界模型", "流式生成如何工作":
+ *                               time-causal block attention with a key/value cache
+ *
+ * Conventions for every entry point:
+ *   - All compute runs asynchronously on `stream` (a cudaStream_t; NULL = legacy
+ *     default stream).  Every pointer marked "device" must be device memory
+ *     reachable from the current device.
+ *   - The caller owns every buffer.  The library allocates no device memory on any
+ *     path; scratch comes from the caller (see cosmot_layer_workspace_size).
+ *   - Element types: activations and weights are bf16 (stored as 16-bit words),
+ *     row-major.  Weights are [out_features, in_features] ("K-major").  Leading
+ *     dimensions (`ld*`) count elements, not bytes.
+ *   - Alignment: every bf16 matrix base pointer must be 16-byte aligned and every
+ *     leading dimension a multiple of 8 elements (the 16-byte TMA stride rule).
+ *   - Argument errors are reported synchronously as COSMOT_ERR_INVALID_ARG (or
+ *     COSMOT_ERR_UNSUPPORTED for shapes this build does not handle) and nothing is
+ *     launched.  Launch failures return COSMOT_ERR_CUDA.
+ *   - Device-side failures (a bounded wait that ran out, recorded instead of
+ *     hanging) are latched into a device status word; read and clear it with
+ *     cosmot_get_device_status.
+ *   - Results are deterministic: no atomics in any reduction, no split-K.
+ */
+#ifndef COSMOT_H_
+#define COSMOT_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define COSMOT_API __attribute__((visibility("default")))
+#else
+#define COSMOT_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st* cosmot_stream_t; /* same type as cudaStream_t */
+
+typedef int32_t cosmot_status;
+enum {
+  COSMOT_OK = 0,
+  COSMOT_ERR_INVALID_ARG = 1,
+  COSMOT_ERR_UNSUPPORTED = 2,
+  COSMOT_ERR_CUDA = 3,
+  COSMOT_ERR_TIMEOUT = 4,
+  COSMOT_ERR_WORKSPACE = 5
+};
+
+/* Human-readable name of a status code (static string, never NULL). */
+COSMOT_API const char* cosmot_status_string(cosmot_status s);
+
+/* Library version as MAJOR*10000 + MINOR*100 + PATCH. */
+COSMOT_API int32_t cosmot_version(void);
+
+/*
+ * Reads the device status word on `stream` (synchronising that stream) into *out
+ * and clears it.  COSMOT_OK if no kernel recorded a failure since the last call.
+ * `where_out` (may be NULL) receives an internal site code of the first failure.
+ */
+COSMOT_API cosmot_status cosmot_get_device_status(cosmot_stream_t stream, cosmot_status* out, int32_t* where_out);
+
+/* ===================================================================== layout */
+
+/*
+ * Contents of one packed sequence ("Cosmos 3 方法原理全解" §2): n_text AR text
+ * tokens, then EOS and BOG (both AR), then the clean DM group and the noisy DM
+ * group, each ordered vision, audio, action.  Video: `video_views` views side by
+ * side along w, grid_h x grid_w tokens per view per latent step, clean steps
+ * first, then noisy steps, on one time axis starting at latent step tau_offset.
+ * Proprioception tokens are clean and sit with the clean actions.
+ */
+typedef struct {
+  int32_t n_text;
+  int32_t video_views, video_grid_h, video_grid_w, video_fps;
+  int32_t video_clean_steps, video_noisy_steps;
+  int32_t audio_clean, audio_noisy, audio_rate;   /* audio_rate: tokens per second */
+  int32_t action_clean, action_noisy, action_hz;
+  int32_t proprio;
+  int32_t tau_offset;                             /* first video latent step */
+} cosmot_layout_spec;
+
+/* Token counts of a layout (host only, no launch). */
+COSMOT_API cosmot_status cosmot_layout_counts(const cosmot_layout_spec* spec, int32_t* n_tokens, int32_t* n_ar,
+                                   int32_t* n_clean, int32_t* n_noisy);
+
+/*
+ * Builds the per-token mRoPE coordinates and block ids of one packed sequence
+ * ("Cosmos 3 方法原理全解" §5).  Device outputs, N = n_tokens:
+ *   pos    float32 [N][3]  (t, h, w).  Each value is computed in float64 and
+ *                          rounded once to float32:
+ *                          AR token k -> (k, k, k); T0 = n_ar + 15000;
+ *                          video (step tau, view v, y, x) -> (T0 + tau*dt_v, y, x + v*grid_w),
+ *                          dt_v = 6 / (fps/4); audio k -> (T0 + k*6/rate, 0, 0);
+ *                          action k -> ((T0 + tau_a0*dt_v) + k*6/hz, 0, 0), tau_a0 =
+ *                          first noisy step; proprio -> (T0 + tau_last_clean*dt_v, 0, 0).
+ *   chunk  int32 [N]       -1 on AR rows, else the latent step of the token.
+ *   region int8  [N]       0 AR, 1 clean DM, 2 noisy DM (may be NULL).
+ */
+COSMOT_API cosmot_status cosmot_build_layout(const cosmot_layout_spec* spec, float* pos, int32_t* chunk, int8_t* region,
+                                  cosmot_stream_t stream);
+
+/*
+ * cos/sin table of the unified 3D mRoPE for rows with coordinates `pos`
+ * ([n_rows][3] float32, device).  Pair i in [0, head_dim/2) takes its angle from
+ * axis t, h or w by contiguous sections (sections[0] pairs on t, then
+ * sections[1] on h, then sections[2] on w; their sum is head_dim/2):
+ * theta = pos[axis] * base^(-2i/head_dim), evaluated in float64.
+ * Output cs float32 [n_rows][head_dim/2][2] = (cos theta, sin theta), device.
+ */
+COSMOT_API cosmot_status cosmot_mrope_table(const float* pos, int64_t n_rows, int32_t head_dim, const int32_t sections[3],
+                                 double rope_base, float* cs, cosmot_stream_t stream);
+
+/* ===================================================================== kernels */
+
+/* Row segment of a routed operation: rows [row_begin, row_end) of the input go
+ * through weight set `weight_set` (0 = Reasoner, 1 = Generator); input row r
+ * writes output row out_row + (r - row_begin). */
+typedef struct {
+  int64_t row_begin;
+  int64_t row_end;
+  int64_t out_row;
+  int32_t weight_set;
+  int32_t reserved;
+} cosmot_segment;
+
+/*
+ * Routed RMSNorm ("Cosmos 3 方法原理全解" §3: each room has its own norm).
+ * out[o] = bf16( h[r] * g_s / sqrt(mean(h[r]^2) + eps) ), fp32 arithmetic.
+ * h: [rows, d] (ld_h), out: [rows, d] (ld_out), g0/g1: [d] gains of the two sets.
+ */
+COSMOT_API cosmot_status cosmot_rmsnorm_routed(const void* h, int64_t ld_h, const cosmot_segment* segs, int32_t n_segs,
+                                    const void* g0, const void* g1, int64_t d, float eps, void* out,
+                                    int64_t ld_out, cosmot_stream_t stream);
+
+/* Epilogues of cosmot_routed_linear. */
+enum {
+  COSMOT_EPI_NONE = 0,      /* out = bf16(acc) */
+  COSMOT_EPI_RESIDUAL = 1,  /* out = bf16(acc + res); res may alias out */
+  COSMOT_EPI_SILU_MUL = 2,  /* out[:, j] = bf16(silu(a.Wg_j) * (a.Wu_j)); W = gate, W_up = up */
+  COSMOT_EPI_MROPE = 3,     /* QKV projection: heads in columns [0, rope_cols) rotated by mRoPE */
+  COSMOT_EPI_EULER = 4      /* out = bf16(x + dsigma * acc); x may alias out */
+};
+
+typedef struct {
+  int32_t kind;
+  int32_t head_dim;        /* MROPE: head width (64 or 128) */
+  int64_t rope_cols;       /* MROPE: number of leading output columns rotated (Q and K heads) */
+  const float* rope_cs;    /* MROPE: table of cosmot_mrope_table, row = output row mod rope_period */
+  int64_t rope_period;     /* MROPE: rows per sequence in the table (0 = no wrap) */
+  const void* res;         /* RESIDUAL: [rows, n_out] bf16, indexed by output row */
+  int64_t ld_res;
+  const void* x;           /* EULER: [rows, n_out] bf16, indexed by output row */
+  int64_t ld_x;
+  float dsigma;            /* EULER: sigma_next - sigma */
+  float reserved;
+} cosmot_epilogue;
+
+/*
+ * Routed projection on the 5th-generation tensor cores (tcgen05, fp32 TMEM
+ * accumulation): for every segment s and input row r in it,
+ *     acc[r, j] = sum_k a[r, k] * W_{set(s)}[j, k],   j in [0, n_out)
+ * then the epilogue writes output row out_row(s) + (r - row_begin).
+ *   a      device bf16 [*, k], ld_a            (rows addressed by the segments)
+ *   w0/w1  device bf16 [n_out, k] (Reasoner / Generator); a set no segment uses
+ *          may be NULL
+ *   w0_up/w1_up  SILU_MUL only: the up projections, same shape; NULL otherwise
+ *   out    device bf16 [*, n_out], ld_out
+ * Requires k % 8 == 0, n_out % 8 == 0, ld_a/ld_out % 8 == 0; MROPE needs
+ * head_dim in {64, 128} and rope_cols a multiple of head_dim; 1 <= n_segs <= 64.
+ */
+COSMOT_API cosmot_status cosmot_routed_linear(const void* a, int64_t ld_a, int64_t k, const cosmot_segment* segs,
+                                   int32_t n_segs, const void* w0, const void* w1, const void* w0_up,
+                                   const void* w1_up, int64_t n_out, void* out, int64_t ld_out,
+                                   const cosmot_epilogue* epi, cosmot_stream_t stream);
+
+/*
+ * Standalone mRoPE ("Cosmos 3 方法原理全解" §5), in place on bf16 rows:
+ * for each row r and head, pairs (i, i + head_dim/2) rotate by theta(r, i):
+ *     x_i' = x_i cos - x_{i+hd/2} sin,   x_{i+hd/2}' = x_{i+hd/2} cos + x_i sin
+ * q: [n_rows, ld_q] with n_q_heads heads from column 0; k likewise (may be NULL).
+ * cs: table of cosmot_mrope_table for the same rows.
+ */
+COSMOT_API cosmot_status cosmot_mrope_apply(void* q, int64_t ld_q, int32_t n_q_heads, void* k, int64_t ld_k,
+                                 int32_t n_k_heads, int64_t n_rows, int32_t head_dim, const float* cs,
+                                 cosmot_stream_t stream);
+
+/* Key visibility of cosmot_mot_attention. */
+enum { COSMOT_MASK_FULL = 0, COSMOT_MASK_BLOCK_CAUSAL = 1 };
+
+typedef struct {
+  int64_t n_q;          /* query rows */
+  int64_t q_key_offset; /* query row i is key row q_key_offset + i */
+  int64_t n_keys;       /* key rows: [0, n_ar) AR, the rest DM */
+  int64_t n_ar;
+  int32_t n_heads, n_kv_heads, head_dim;
+  int32_t mask_mode;    /* COSMOT_MASK_* */
+  const int32_t* chunk; /* BLOCK_CAUSAL: device int32 [n_keys] latent step of each key row */
+  int32_t batch;        /* independent sequences */
+  int32_t reserved;
+  int64_t q_batch_stride, kv_batch_stride, o_batch_stride; /* rows between sequences */
+  float softmax_scale;  /* 0 = 1/sqrt(head_dim) */
+  float reserved2;
+} cosmot_attn_desc;
+
+/*
+ * MoT attention ("Cosmos 3 方法原理全解" §3 equations; block-causal variant from
+ * "流式生成如何工作").  Per head h (kv head h / (n_heads/n_kv_heads)):
+ *     o_i = sum_{j visible to i} softmax_j(q_i . k_j * scale) v_j
+ * visible: AR query i sees AR keys j <= i; a DM query sees every AR key and, in
+ * FULL mode, every DM key; in BLOCK_CAUSAL mode the DM keys with
+ * chunk[j] <= chunk[query].  q: [n_q, ld_q] (heads of head_dim from column 0),
+ * k, v: [n_keys, ld_kv], o: [n_q, ld_o], all bf16 device.  head_dim 128 or 64.
+ */
+COSMOT_API cosmot_status cosmot_mot_attention(const cosmot_attn_desc* desc, const void* q, int64_t ld_q, const void* k,
+                                   const void* v, int64_t ld_kv, void* o, int64_t ld_o, cosmot_stream_t stream);
+
+/*
+ * Flow-matching Euler step ("Cosmos 3 方法原理全解" §7.2), in place:
+ *     x[r, c] = bf16( x[r, c] + (sigma_next - sigma) * v[r, c] )  for r in [row_begin, row_end)
+ * Rows outside the range are not touched (clean DM rows pass through bit-exact).
+ * dsigma is formed in float64 and rounded to float32; the update is one fp32 FMA.
+ */
+COSMOT_API cosmot_status cosmot_flow_euler_step(void* x, int64_t ld_x, const void* v, int64_t ld_v, int64_t row_begin,
+                                     int64_t row_end, int64_t n_cols, double sigma, double sigma_next,
+                                     cosmot_stream_t stream);
+
+/* ===================================================================== layer */
+
+typedef struct {
+  int32_t d_model, n_heads, n_kv_heads, head_dim, ffn;
+  int32_t rope_sections[3];
+  double rope_base;
+  float eps;
+  int32_t reserved;
+} cosmot_dims;
+
+typedef struct {
+  const void* g1;   /* [d] pre-attention RMSNorm gain */
+  const void* wqkv; /* [(n_heads + 2 n_kv_heads) head_dim, d]: Q heads, K heads, V heads */
+  const void* wo;   /* [d, n_heads head_dim] */
+  const void* g2;   /* [d] pre-FFN RMSNorm gain */
+  const void* wg;   /* [ffn, d] gate */
+  const void* wu;   /* [ffn, d] up */
+  const void* wd;   /* [d, ffn] down */
+} cosmot_set_weights;
+
+typedef struct {
+  cosmot_set_weights set[2]; /* 0 = Reasoner (AR rows), 1 = Generator (DM rows) */
+  const void* gfin;          /* [d] final RMSNorm gain before the velocity head (noisy rows) */
+  const void* wvel;          /* [d, d] velocity head */
+} cosmot_layer_weights;
+
+typedef struct {
+  int32_t n_ar, n_clean, n_noisy; /* per sequence; N = n_ar + n_clean + n_noisy */
+  int32_t batch;                  /* sequences laid out back to back: [batch][N][d] */
+  int32_t mask_mode;              /* COSMOT_MASK_* among DM rows */
+  int32_t reserved;
+  const float* rope_cs;           /* device table of cosmot_mrope_table for one sequence [N] */
+  const int32_t* chunk;           /* device [N] (BLOCK_CAUSAL only; may be NULL for FULL) */
+} cosmot_seq_desc;
+
+/* Bytes of scratch cosmot_layer_forward needs for these sizes (host only). */
+COSMOT_API cosmot_status cosmot_layer_workspace_size(const cosmot_dims* dims, const cosmot_seq_desc* seq, size_t* bytes);
+
+/*
+ * One MoT layer forward plus the sampler step, for `batch` packed sequences:
+ *   h      device bf16 [batch][N][d], in/out.  Its DM rows are the sampler state x;
+ *          on return the noisy DM rows hold x' = x + (sigma_next - sigma) *
+ *          (RMSNorm(h2; gfin) . Wvel^T).  AR and clean rows are not written.
+ *   h_out  device bf16 [batch][N][d], out: the layer output h2 of every row.
+ * Steps: routed RMSNorm -> routed QKV GEMM with mRoPE epilogue -> MoT attention ->
+ * routed O GEMM + residual -> routed RMSNorm -> routed gate/up GEMM with SiLU*mul
+ * epilogue -> routed down GEMM + residual -> final RMSNorm (noisy rows) ->
+ * velocity GEMM with Euler epilogue.  `workspace` must hold
+ * cosmot_layer_workspace_size bytes (256-byte aligned); it is clobbered.
+ */
+COSMOT_API cosmot_status cosmot_layer_forward(const cosmot_dims* dims, const cosmot_layer_weights* w,
+                                   const cosmot_seq_desc* seq, void* h, void* h_out, double sigma,
+                                   double sigma_next, void* workspace, size_t workspace_bytes,
+                                   cosmot_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* COSMOT_H_ */

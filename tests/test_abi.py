@@ -1,0 +1,112 @@
+"""The C-ABI library builds, loads and exports every declared entry point;
+host-side argument checks and layout counts work without a GPU."""
+
+import ctypes
+import os
+import re
+import subprocess
+
+import numpy as np
+import pytest
+
+import synth
+from oracle import layout as olayout
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "cosmot.h")
+
+
+def _declared():
+    src = open(HEADER).read()
+    return sorted(set(re.findall(r"COSMOT_API\s+[\w\s\*]+?\b(cosmot_\w+)\s*\(", src)))
+
+
+def test_header_declares_the_hot_path_entry_points():
+    names = _declared()
+    for n in ("cosmot_routed_linear", "cosmot_mrope_apply", "cosmot_mot_attention", "cosmot_flow_euler_step",
+              "cosmot_layer_forward", "cosmot_build_layout", "cosmot_get_device_status"):
+        assert n in names
+
+
+def test_library_exports_every_declared_symbol():
+    from flow_matching_dit_cosmot_b200 import _lib as L
+    L.lib()
+    out = subprocess.run(["nm", "-D", "--defined-only", L.LIB_PATH], capture_output=True, text=True, check=True).stdout
+    exported = set(re.findall(r"\sT\s(cosmot_\w+)", out))
+    missing = [n for n in _declared() if n not in exported]
+    assert not missing, missing
+    assert set(_declared()) == set(L.SIGNATURES), "binding and header disagree"
+
+
+def test_status_strings_and_version():
+    from flow_matching_dit_cosmot_b200 import _lib as L
+    assert L.status_string(0) == "COSMOT_OK"
+    assert L.status_string(4) == "COSMOT_ERR_TIMEOUT"
+    assert L.status_string(99) == "COSMOT_ERR_UNKNOWN"
+    assert L.cosmot_version() >= 100
+
+
+@pytest.mark.parametrize("name", sorted(synth.PRESETS))
+def test_layout_counts_match_oracle(name):
+    from flow_matching_dit_cosmot_b200 import api as A
+    from gpu_helpers import layout_spec
+    wl = synth.preset(name)
+    lay = olayout.build_layout(wl.layout)
+    n, a, c, z = A.L.cosmot_layout_counts(layout_spec(A, wl.layout))
+    assert (n, a, c, z) == (lay.n_tokens, lay.n_ar, lay.n_clean, lay.n_noisy)
+
+
+def test_invalid_arguments_are_rejected_before_any_launch():
+    from flow_matching_dit_cosmot_b200 import _lib as L
+    lib = L.lib()
+    seg = (L.Segment * 1)(L.Segment(0, 10, 0, 0, 0))
+    epi = L.Epilogue(kind=0)
+    # null input
+    assert lib.cosmot_routed_linear(None, 64, 64, seg, 1, 16, 16, None, None, 64, 16, 64, ctypes.byref(epi),
+                                    None) == L.COSMOT_ERR_INVALID_ARG
+    # k not a multiple of 8
+    assert lib.cosmot_routed_linear(16, 64, 60, seg, 1, 16, 16, None, None, 64, 16, 64, ctypes.byref(epi),
+                                    None) == L.COSMOT_ERR_INVALID_ARG
+    # misaligned pointer
+    assert lib.cosmot_routed_linear(18, 64, 64, seg, 1, 16, 16, None, None, 64, 16, 64, ctypes.byref(epi),
+                                    None) == L.COSMOT_ERR_INVALID_ARG
+    # bad weight set id
+    bad = (L.Segment * 1)(L.Segment(0, 10, 0, 2, 0))
+    assert lib.cosmot_routed_linear(16, 64, 64, bad, 1, 16, 16, None, None, 64, 16, 64, ctypes.byref(epi),
+                                    None) == L.COSMOT_ERR_INVALID_ARG
+    # attention: heads not divisible by kv heads; unsupported head_dim
+    d = L.AttnDesc(n_q=4, q_key_offset=0, n_keys=4, n_ar=1, n_heads=3, n_kv_heads=2, head_dim=128, batch=1)
+    assert lib.cosmot_mot_attention(ctypes.byref(d), 16, 384, 16, 16, 256, 16, 384, None) == L.COSMOT_ERR_INVALID_ARG
+    d = L.AttnDesc(n_q=4, q_key_offset=0, n_keys=4, n_ar=1, n_heads=2, n_kv_heads=2, head_dim=96, batch=1)
+    assert lib.cosmot_mot_attention(ctypes.byref(d), 16, 192, 16, 16, 192, 16, 192, None) == L.COSMOT_ERR_UNSUPPORTED
+    # queries past the keys
+    d = L.AttnDesc(n_q=5, q_key_offset=0, n_keys=4, n_ar=1, n_heads=2, n_kv_heads=2, head_dim=128, batch=1)
+    assert lib.cosmot_mot_attention(ctypes.byref(d), 16, 256, 16, 16, 256, 16, 256, None) == L.COSMOT_ERR_INVALID_ARG
+    # block-causal without chunk ids
+    d = L.AttnDesc(n_q=4, q_key_offset=0, n_keys=4, n_ar=1, n_heads=2, n_kv_heads=2, head_dim=128, batch=1,
+                   mask_mode=L.COSMOT_MASK_BLOCK_CAUSAL)
+    assert lib.cosmot_mot_attention(ctypes.byref(d), 16, 256, 16, 16, 256, 16, 256, None) == L.COSMOT_ERR_INVALID_ARG
+    # euler: odd column count
+    assert lib.cosmot_flow_euler_step(16, 8, 16, 8, 0, 4, 7, 1.0, 0.9, None) == L.COSMOT_ERR_INVALID_ARG
+    # mrope table: sections do not cover head_dim/2
+    sec = (L.c_i32 * 3)(16, 24, 23)
+    assert lib.cosmot_mrope_table(16, 4, 128, sec, 1e4, 16, None) == L.COSMOT_ERR_INVALID_ARG
+
+
+def test_layer_workspace_and_validation():
+    from flow_matching_dit_cosmot_b200 import api as A
+    wl = synth.preset("t2v480")
+    dm = wl.dims
+    dims = A.make_dims(dm.d_model, dm.n_heads, dm.n_kv_heads, dm.head_dim, dm.ffn, dm.rope_sections)
+    seq = A.L.SeqDesc(258, 0, 18720, 1, 0, 0, 16, 0)
+    n = A.L.cosmot_layer_workspace_size(dims, seq)
+    rows = 18978
+    want = rows * (4096 + 12288 + 4096 + 4096 + 14336) * 2
+    assert want <= n <= want + 5 * 256
+    # the layer rejects a short workspace and bad dims without launching
+    lib = A.L.lib()
+    assert lib.cosmot_layer_forward(ctypes.byref(dims), ctypes.byref(A.L.LayerWeights()), ctypes.byref(seq), 256, 256,
+                                    1.0, 0.97, 256, 1024, None) == A.L.COSMOT_ERR_WORKSPACE
+    bad = A.make_dims(4096, 32, 5, 128, 14336, (16, 24, 24))
+    assert lib.cosmot_layer_forward(ctypes.byref(bad), ctypes.byref(A.L.LayerWeights()), ctypes.byref(seq), 256, 256,
+                                    1.0, 0.97, 256, n, None) == A.L.COSMOT_ERR_INVALID_ARG
