@@ -1,0 +1,475 @@
+#!/usr/bin/env python
+"""Throughput of the Cosmos 3 MoT layer hot path on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload t2v480] [--impl native|reference]
+
+A step is one pass of the whole hot path over one synthetic batch: the layout
+and mRoPE-table build, then one MoT layer forward with the Euler step
+(cosmot_layer_forward: routed norms, QKV + mRoPE, attention, O + residual,
+gate/up + SiLU, down + residual, final norm, velocity + Euler).  Inputs live
+in HBM when the timed region starts; L2 is flushed (256 MiB write) between
+steps outside the timed events.  Rank 0 prints one JSON line.
+
+With N > 1 (torchrun) every rank runs its own sequence: independent replicas,
+no collective on the data path ("scaling": "weak"); the step time is the max
+over ranks.  `--impl reference` times the fp64 CPU oracle instead (rank 0
+only) on a bounded sample of the same workload.
+"""
+
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+
+import synth  # noqa: E402
+
+METRIC = "MoT layer tokens/s and attention+GEMM TFLOP/s (% of B200 bf16 peak), 1 GPU"
+UNIT = "tokens/s"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+# DRAM traffic per launch of the dominant kernel from an ncu capture
+# (dram__bytes_read.sum + dram__bytes_write.sum), keyed by stage, with the
+# sha256 of the kernel source it was taken on; reported only while the source
+# is unchanged.  Summaries live under profiles/.
+NCU_TRAFFIC = {}
+
+
+def parse_args():
+    p = argparse.ArgumentParser()
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=10)
+    p.add_argument("--warmup", type=int, default=3)
+    p.add_argument("--workload", default="t2v480", choices=sorted(synth.PRESETS))
+    p.add_argument("--impl", default="native", choices=["native", "reference"])
+    p.add_argument("--no-e2e", action="store_true")
+    p.add_argument("--no-cpu-baseline", action="store_true")
+    return p.parse_args()
+
+
+# ---------------------------------------------------------------- algorithmic work
+
+class Counts:
+    """Token counts of one packed sequence plus its chunk ids (host copy)."""
+
+    def __init__(self, n_ar, n_clean, n_noisy, chunk=None):
+        self.n_ar, self.n_clean, self.n_noisy = n_ar, n_clean, n_noisy
+        self.n_tokens = n_ar + n_clean + n_noisy
+        self.chunk = chunk
+
+
+def attention_pairs(lay, mode: str) -> int:
+    """Visible (query, key) pairs of one sequence under the MoT mask: causal
+    pairs inside AR, every AR key for each DM row, and every DM key (full) or
+    the DM keys of the same or earlier chunks (block-causal)."""
+    n_ar, n = lay.n_ar, lay.n_tokens
+    n_dm = n - n_ar
+    pairs = n_ar * (n_ar + 1) // 2 + n_dm * n_ar
+    if mode == "full":
+        pairs += n_dm * n_dm
+    else:
+        ch = np.asarray(lay.chunk[n_ar:], dtype=np.int64)
+        pairs += int(np.searchsorted(np.sort(ch), ch, side="right").sum())
+    return int(pairs)
+
+
+def stage_work(wl, lay):
+    """(flops, bytes) per stage per step, algorithmic (no re-reads counted)."""
+    d, B = wl.dims, wl.batch
+    R = B * lay.n_tokens
+    dd, F, hd = d.d_model, d.ffn, d.head_dim
+    qc, qkvc = d.q_cols, d.qkv_cols
+    nz = B * lay.n_noisy
+    pairs = B * attention_pairs(lay, wl.mask_mode)
+    w_set = 2  # bytes per bf16
+    return {
+        "norm1": (0, R * dd * 4),
+        "qkv_mrope": (2 * R * dd * qkvc, (R * dd + 2 * qkvc * dd + R * qkvc) * w_set),
+        "attention": (4 * pairs * d.n_heads * hd, (R * qkvc + R * qc) * w_set),
+        "oproj_residual": (2 * R * qc * dd, (R * qc + 2 * dd * qc + 2 * R * dd) * w_set),
+        "norm2": (0, R * dd * 4),
+        "gateup_silu": (2 * R * dd * 2 * F, (R * dd + 4 * F * dd + R * F) * w_set),
+        "down_residual": (2 * R * F * dd, (R * F + 2 * dd * F + 2 * R * dd) * w_set),
+        "norm_final": (0, nz * dd * 4),
+        "velocity_euler": (2 * nz * dd * dd, (nz * dd * 3 + dd * dd) * w_set),
+    }
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            return json.load(f), "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+# ---------------------------------------------------------------- clocks
+
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, uuid=None):
+        self.uuid = uuid
+        self.proc = None
+        self.out = os.path.join("/tmp", f"cosmot_clocks_{os.getpid()}.csv")
+
+    def start(self):
+        cmd = ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits", "-lms", "200"]
+        if self.uuid:
+            cmd += ["-i", self.uuid]
+        try:
+            self.f = open(self.out, "w")
+            self.proc = subprocess.Popen(cmd, stdout=self.f, stderr=subprocess.DEVNULL)
+        except OSError:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.f.close()
+        sm, smax, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in open(self.out):
+            parts = [x.strip() for x in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                smax.append(float(parts[2]))
+            except ValueError:
+                continue
+            for nm, v in zip(names, parts[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(nm)
+        os.unlink(self.out)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(smax) if smax else None,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ---------------------------------------------------------------- reference arm (fp64 CPU oracle)
+
+def oracle_sample(wl, lay, W, h64, rows_lo=16, rows_hi=48):
+    """Times the oracle on two row samples of the first sequence and extrapolates
+    linearly in query rows to the whole layer (K and V are always formed for
+    every row, so the fixed part is measured, not estimated)."""
+    from oracle import layer as olayer
+    dm0 = lay.n_ar + lay.n_clean
+    s0, s1 = wl.sigmas[0], wl.sigmas[1]
+    t = []
+    for r in (rows_lo, rows_hi):
+        rows = np.arange(dm0, min(lay.n_tokens, dm0 + r))
+        t0 = time.perf_counter()
+        olayer.layer_forward(wl.dims, W, h64, lay.region, lay.pos, lay.chunk, s0, s1, wl.mask_mode, rows=rows)
+        t.append(time.perf_counter() - t0)
+    per_row = max(t[1] - t[0], 0.0) / (rows_hi - rows_lo)
+    fixed = max(t[0] - rows_lo * per_row, 0.0)
+    t_full = (fixed + per_row * lay.n_tokens) * wl.batch
+    return t_full, sum(t)
+
+
+def cpu_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        n = max((i.get("num_threads", 0) for i in threadpool_info()), default=0)
+        if n:
+            return n
+    except Exception:
+        pass
+    return os.cpu_count()
+
+
+def oracle_setup(wl):
+    from oracle import layer as olayer
+    from oracle import layout as olayout
+    lay = olayout.build_layout(wl.layout)
+    W = olayer.weights_from_bits(wl.dims, synth.make_weights(wl.dims, wl.weight_seed))
+    h64 = synth.bf16_to_f64(synth.make_activations(lay.n_tokens, wl.dims.d_model, wl.act_seed(0)))
+    return lay, W, h64
+
+
+def run_reference(args, wl):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    lay, W, h64 = oracle_setup(wl)
+    for _ in range(args.warmup):
+        oracle_sample(wl, lay, W, h64)
+    t_full, t_spent = [], 0.0
+    for _ in range(args.steps):
+        tf, ts = oracle_sample(wl, lay, W, h64)
+        t_full.append(tf)
+        t_spent += ts
+    tokens = wl.batch * lay.n_tokens
+    value = tokens * len(t_full) / sum(t_full)
+    cores = cpu_threads()
+    sample = (f"per step: oracle layer forward on 16 and on 48 noisy query rows of sequence 0 (K/V of all "
+              f"{lay.n_tokens} rows each time), extrapolated linearly to all rows and the batch")
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * statistics.mean(t_full),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic (seeded Philox: activations N(0,1), weights N(0,0.02), gains 1+N(0,0.02))",
+        "config": config_block(wl, lay, args.gpus),
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle", "sample": sample},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+        "wall_s_sampled": t_spent,
+    }
+    print(json.dumps(line), flush=True)
+
+
+def config_block(wl, lay, n_gpus):
+    return {"workload": f"{wl.name}: {wl.description}", "global_batch": wl.batch * n_gpus,
+            "seq_len": lay.n_tokens, "parallelism": f"replicas x{n_gpus}" if n_gpus > 1 else "single GPU",
+            "d_model": wl.dims.d_model, "heads": wl.dims.n_heads, "head_dim": wl.dims.head_dim,
+            "ffn": wl.dims.ffn, "n_ar": lay.n_ar, "n_clean": lay.n_clean, "n_noisy": lay.n_noisy,
+            "mask": wl.mask_mode, "sigma": [wl.sigmas[0], wl.sigmas[1]],
+            "l2": "flushed between steps (256 MiB write, outside the timed events)"}
+
+
+# ---------------------------------------------------------------- native arm
+
+def src_sha(name):
+    p = os.path.join(ROOT, "flow_matching_dit_cosmot_b200", "csrc", name)
+    return hashlib.sha256(open(p, "rb").read()).hexdigest()[:16] if os.path.exists(p) else None
+
+
+def run_native(args, wl):
+    import torch
+    import torch.distributed as dist
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    if world > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=300), device_id=torch.device("cuda", local))
+
+    from flow_matching_dit_cosmot_b200 import _lib as L
+    from flow_matching_dit_cosmot_b200 import api as A
+
+    dims_s = wl.dims
+    dev = torch.device("cuda", local)
+    v = wl.layout.video
+    spec = A.layout_spec(wl.layout.n_text,
+                         None if v is None else (v.views, v.grid_h, v.grid_w, v.fps, v.clean_steps, v.noisy_steps),
+                         wl.layout.audio_clean, wl.layout.audio_noisy, wl.layout.audio_rate, wl.layout.action_clean,
+                         wl.layout.action_noisy, wl.layout.action_hz, wl.layout.proprio)
+    dl = A.build_layout(spec, dev)
+    lay = Counts(dl.n_ar, dl.n_clean, dl.n_noisy, dl.chunk.cpu().numpy())
+    B, N, d = wl.batch, lay.n_tokens, dims_s.d_model
+
+    def to_dev(u16):
+        return torch.from_numpy(np.ascontiguousarray(u16).view(np.int16)).view(torch.bfloat16).to(dev)
+
+    w = {k: to_dev(v) for k, v in synth.make_weights(dims_s, wl.weight_seed).items()}
+    h_host = np.stack([synth.make_activations(N, d, wl.act_seed(rank * B + b)) for b in range(B)])
+    h_src = to_dev(h_host)
+    h = h_src.clone()
+    h_out = torch.empty_like(h)
+    pos = torch.empty((N, 3), dtype=torch.float32, device=dev)
+    chunk = torch.empty((N,), dtype=torch.int32, device=dev)
+    cs = torch.empty((N, dims_s.head_dim // 2, 2), dtype=torch.float32, device=dev)
+    dims = A.make_dims(dims_s.d_model, dims_s.n_heads, dims_s.n_kv_heads, dims_s.head_dim, dims_s.ffn,
+                       dims_s.rope_sections, dims_s.rope_base, dims_s.eps)
+    layer = A.MoTLayer(dims, w)
+    mode = L.COSMOT_MASK_FULL if wl.mask_mode == "full" else L.COSMOT_MASK_BLOCK_CAUSAL
+    seq = layer.seq_desc(lay.n_ar, lay.n_clean, lay.n_noisy, B, cs, chunk, mode)
+    ws = layer.workspace(seq, dev)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream()
+    sh = stream.cuda_stream
+    s0, s1 = wl.sigmas[0], wl.sigmas[1]
+    n_stage = L.COSMOT_LAYER_STAGES
+
+    def new_events(n):
+        evs = [torch.cuda.Event(enable_timing=True) for _ in range(n)]
+        for e in evs:
+            e.record(stream)  # creates the underlying cudaEvent_t
+        return evs
+
+    def step(stage_evs=None):
+        L.cosmot_build_layout(spec, pos.data_ptr(), chunk.data_ptr(), 0, sh)
+        L.cosmot_mrope_table(pos.data_ptr(), N, dims_s.head_dim, dims_s.rope_sections, dims_s.rope_base,
+                             cs.data_ptr(), sh)
+        if stage_evs is None:
+            L.cosmot_layer_forward(dims, layer.cw, seq, h.data_ptr(), h_out.data_ptr(), s0, s1, ws.data_ptr(),
+                                   ws.numel(), sh)
+        else:
+            L.cosmot_layer_forward_timed(dims, layer.cw, seq, h.data_ptr(), h_out.data_ptr(), s0, s1, ws.data_ptr(),
+                                         ws.numel(), sh, [e.cuda_event for e in stage_evs])
+
+    launches_per_step = 2 + (n_stage if lay.n_noisy > 0 else n_stage - 2)
+
+    for _ in range(args.warmup):
+        flush.zero_()
+        step()
+    torch.cuda.synchronize()
+    st, where = L.cosmot_get_device_status(sh)
+    if st:
+        raise RuntimeError(f"device status {L.status_string(st)} at {where}")
+
+    starts, ends = new_events(args.steps), new_events(args.steps)
+    stage_evs = [new_events(n_stage + 1) for _ in range(args.steps)]
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    clocks = ClockSampler(getattr(torch.cuda.get_device_properties(dev), "uuid", None))
+    clocks.start()
+    time.sleep(0.3)
+    for i in range(args.steps):
+        flush.zero_()
+        starts[i].record(stream)
+        step(stage_evs[i])
+        ends[i].record(stream)
+    torch.cuda.synchronize()
+    clk = clocks.stop()
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    st, where = L.cosmot_get_device_status(sh)
+    if st:
+        raise RuntimeError(f"device status {L.status_string(st)} at {where}")
+
+    step_ms = [starts[i].elapsed_time(ends[i]) for i in range(args.steps)]
+    total_ms = sum(step_ms)
+    stage_ms = np.zeros(n_stage)
+    for evs in stage_evs:
+        for j in range(n_stage):
+            stage_ms[j] += evs[j].elapsed_time(evs[j + 1])
+    stage_ms /= args.steps
+
+    # ---------------------------------------------------------------- end to end (host buffers)
+    e2e = None
+    if not args.no_e2e:
+        h_pin = torch.from_numpy(h_host.view(np.int16)).view(torch.bfloat16).pin_memory()
+        z0 = lay.n_ar + lay.n_clean
+        x_pin = torch.empty((B, lay.n_noisy, d), dtype=torch.bfloat16).pin_memory()
+        for _ in range(max(1, args.warmup)):
+            h.copy_(h_pin, non_blocking=True)
+            step()
+            x_pin.copy_(h[:, z0:], non_blocking=True)
+        torch.cuda.synchronize()
+        e_s, e_e = new_events(args.steps), new_events(args.steps)
+        torch.cuda.synchronize()
+        for i in range(args.steps):
+            flush.zero_()
+            e_s[i].record(stream)
+            h.copy_(h_pin, non_blocking=True)
+            step()
+            x_pin.copy_(h[:, z0:], non_blocking=True)
+            e_e[i].record(stream)
+        torch.cuda.synchronize()
+        e2e_ms = sum(e_s[i].elapsed_time(e_e[i]) for i in range(args.steps))
+        if world > 1:
+            t = torch.tensor([e2e_ms], device=dev, dtype=torch.float64)
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            e2e_ms = float(t.item())
+        e2e = {"value": world * B * N * args.steps / (e2e_ms / 1e3), "unit": UNIT,
+               "h2d_bytes_per_step": int(h_pin.numel() * 2), "d2h_bytes_per_step": int(x_pin.numel() * 2),
+               "ms_per_step": e2e_ms / args.steps, "path": "cosmot_build_layout + cosmot_mrope_table + "
+               "cosmot_layer_forward, pinned host h in, x' (noisy rows) out"}
+
+    if world > 1:
+        t = torch.tensor([total_ms], device=dev, dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        total_ms = float(t.item())
+
+    if rank == 0:
+        work = stage_work(wl, lay)
+        names = L.STAGE_NAMES
+        flops_total = sum(f for f, _ in work.values())
+        peaks, peak_src = load_peaks()
+        peak_tf = float(peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"]))
+        peak_tf_burst = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
+        peak_bw = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
+        ms_step = total_ms / args.steps
+        stages = {}
+        for j, nm in enumerate(names):
+            f, b = work[nm]
+            t_s = stage_ms[j] / 1e3
+            ent = {"ms": round(float(stage_ms[j]), 4), "share": round(float(stage_ms[j] / stage_ms.sum()), 4)}
+            if f:
+                ent["tflops"] = round(f / t_s / 1e12, 1) if t_s > 0 else None
+                ent["frac_of_peak"] = round(f / t_s / 1e12 / peak_tf, 3) if t_s > 0 else None
+            else:
+                ent["gbs"] = round(b / t_s / 1e9, 1) if t_s > 0 else None
+                ent["frac_of_hbm"] = round(b / t_s / 1e9 / peak_bw, 3) if t_s > 0 else None
+            stages[nm] = ent
+        dom = max(range(n_stage), key=lambda j: stage_ms[j])
+        dname = names[dom]
+        f, b = work[dname]
+        t_dom = stage_ms[dom] / 1e3
+        src = "attention.cu" if dname == "attention" else ("gemm.cu" if f else "elementwise.cu")
+        traffic = None
+        rec = NCU_TRAFFIC.get(dname)
+        if rec and rec.get("src_sha") == src_sha(src):
+            traffic = rec["bytes_per_launch"]
+        if f:
+            achieved = f / t_dom / 1e12
+            roof = {"bound": "tensor", "kernel": dname, "achieved": round(achieved, 1), "peak": peak_tf,
+                    "unit": "TFLOP/s", "frac": round(achieved / peak_tf, 3), "traffic": traffic,
+                    "algorithmic_flops_per_launch": f, "peak_source": f"{peak_src} bf16_tflops_sustained"}
+        else:
+            achieved = b / t_dom / 1e9
+            roof = {"bound": "hbm", "kernel": dname, "achieved": round(achieved, 1), "peak": peak_bw,
+                    "unit": "GB/s", "frac": round(achieved / peak_bw, 3), "traffic": traffic,
+                    "algorithmic_bytes_per_launch": b, "peak_source": f"{peak_src} hbm_gbs"}
+        tokens = world * B * N * args.steps
+        value = tokens / (total_ms / 1e3)
+        layer_tflops = flops_total / (ms_step / 1e3) / 1e12
+        line = {
+            "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic (seeded Philox: activations N(0,1), weights N(0,0.02), gains 1+N(0,0.02))",
+            "config": config_block(wl, lay, world),
+            "tflops": round(layer_tflops, 1),
+            "tflops_frac_of_peak": round(layer_tflops / peak_tf, 3),
+            "tflops_frac_of_burst_peak": round(layer_tflops / peak_tf_burst, 3),
+            "flops_per_step": flops_total,
+            "clocks": clk, "e2e": e2e, "gpu_launches": launches_per_step * args.steps,
+            "roofline": roof, "stages": stages,
+        }
+        if world == 1 and not args.no_cpu_baseline:
+            lay_o, W, h64 = oracle_setup(wl)
+            t_full, t_spent = oracle_sample(wl, lay_o, W, h64)
+            line["cpu_baseline"] = {
+                "value": B * N / t_full, "unit": UNIT, "cores": cpu_threads(), "kind": "oracle",
+                "sample": f"oracle layer forward on 16 and 48 noisy query rows (K/V of all {N} rows each), "
+                          f"extrapolated linearly to all rows and the batch; {t_spent:.1f} s of CPU wall time"}
+        print(json.dumps(line), flush=True)
+
+    if world > 1:
+        dist.destroy_process_group()
+
+
+def main():
+    args = parse_args()
+    wl = synth.preset(args.workload)
+    if args.impl == "reference":
+        run_reference(args, wl)
+    else:
+        run_native(args, wl)
+
+
+if __name__ == "__main__":
+    main()

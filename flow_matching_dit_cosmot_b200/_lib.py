@@ -99,7 +99,13 @@ SIGNATURES = {
     "cosmot_layer_workspace_size": (c_i32, [_P(Dims), _P(SeqDesc), _P(ctypes.c_size_t)]),
     "cosmot_layer_forward": (c_i32, [_P(Dims), _P(LayerWeights), _P(SeqDesc), c_vp, c_vp, c_f64, c_f64, c_vp,
                                      ctypes.c_size_t, c_vp]),
+    "cosmot_layer_forward_timed": (c_i32, [_P(Dims), _P(LayerWeights), _P(SeqDesc), c_vp, c_vp, c_f64, c_f64, c_vp,
+                                           ctypes.c_size_t, c_vp, _P(c_vp), c_i32]),
 }
+
+COSMOT_LAYER_STAGES = 9
+STAGE_NAMES = ("norm1", "qkv_mrope", "attention", "oproj_residual", "norm2", "gateup_silu", "down_residual",
+               "norm_final", "velocity_euler")
 
 _lib = None
 
@@ -219,3 +225,13 @@ def cosmot_layer_forward(dims: Dims, w: LayerWeights, seq: SeqDesc, h: int, h_ou
                          sigma_next: float, workspace: int, workspace_bytes: int, stream: int = 0, check=True):
     return _call("cosmot_layer_forward", ctypes.byref(dims), ctypes.byref(w), ctypes.byref(seq), c_vp(h),
                  c_vp(h_out), sigma, sigma_next, c_vp(workspace), workspace_bytes, c_vp(stream), check=check)
+
+
+def cosmot_layer_forward_timed(dims: Dims, w: LayerWeights, seq: SeqDesc, h: int, h_out: int, sigma: float,
+                               sigma_next: float, workspace: int, workspace_bytes: int, stream: int, events,
+                               check=True):
+    """`events`: COSMOT_LAYER_STAGES + 1 raw cudaEvent_t handles (ints)."""
+    arr = (c_vp * len(events))(*[c_vp(e) for e in events])
+    return _call("cosmot_layer_forward_timed", ctypes.byref(dims), ctypes.byref(w), ctypes.byref(seq), c_vp(h),
+                 c_vp(h_out), sigma, sigma_next, c_vp(workspace), workspace_bytes, c_vp(stream), arr, len(events),
+                 check=check)

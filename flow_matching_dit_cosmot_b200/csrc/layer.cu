@@ -80,11 +80,25 @@ cosmot_status cosmot_layer_workspace_size(const cosmot_dims* dims, const cosmot_
   return COSMOT_OK;
 }
 
-cosmot_status cosmot_layer_forward(const cosmot_dims* dims, const cosmot_layer_weights* w,
-                                   const cosmot_seq_desc* seq, void* h, void* h_out, double sigma,
-                                   double sigma_next, void* workspace, size_t workspace_bytes,
-                                   cosmot_stream_t stream) {
-  using namespace cosmot;
+}  // extern "C"
+
+namespace cosmot {
+namespace {
+
+// Records ev[i] (when given) on the stream just before stage i starts.
+struct StageMarks {
+  const cudaEvent_t* ev;
+  cudaStream_t s;
+  cosmot_status mark(int i) const {
+    if (!ev) return COSMOT_OK;
+    return cudaEventRecord(ev[i], s) == cudaSuccess ? COSMOT_OK : COSMOT_ERR_CUDA;
+  }
+};
+
+cosmot_status layer_forward_impl(const cosmot_dims* dims, const cosmot_layer_weights* w, const cosmot_seq_desc* seq,
+                                 void* h, void* h_out, double sigma, double sigma_next, void* workspace,
+                                 size_t workspace_bytes, cosmot_stream_t stream, const cudaEvent_t* events) {
+  const StageMarks M{events, reinterpret_cast<cudaStream_t>(stream)};
   cosmot_status st = check_dims(dims);
   if (st != COSMOT_OK) return st;
   st = check_seq(seq);
@@ -119,9 +133,11 @@ cosmot_status cosmot_layer_forward(const cosmot_dims* dims, const cosmot_layer_w
   const cosmot_set_weights& R = w->set[0];
   const cosmot_set_weights& G = w->set[1];
 
+  if ((st = M.mark(0)) != COSMOT_OK) return st;
   // 1. pre-attention norm
   st = cosmot_rmsnorm_routed(h, d, segs, ns, R.g1, G.g1, d, D.eps, a, d, stream);
   if (st != COSMOT_OK) return st;
+  if ((st = M.mark(1)) != COSMOT_OK) return st;
   // 2. QKV projection with mRoPE on the Q and K heads
   cosmot_epilogue e{};
   e.kind = COSMOT_EPI_MROPE;
@@ -131,6 +147,7 @@ cosmot_status cosmot_layer_forward(const cosmot_dims* dims, const cosmot_layer_w
   e.rope_period = N;
   st = cosmot_routed_linear(a, d, d, segs, ns, R.wqkv, G.wqkv, nullptr, nullptr, qkvc, qkv, qkvc, &e, stream);
   if (st != COSMOT_OK) return st;
+  if ((st = M.mark(2)) != COSMOT_OK) return st;
   // 3. attention
   cosmot_attn_desc ad{};
   ad.n_q = N;
@@ -147,6 +164,7 @@ cosmot_status cosmot_layer_forward(const cosmot_dims* dims, const cosmot_layer_w
   uint16_t* qkvp = static_cast<uint16_t*>(qkv);
   st = cosmot_mot_attention(&ad, qkvp, qkvc, qkvp + qc, qkvp + qc + kvc, qkvc, o, qc, stream);
   if (st != COSMOT_OK) return st;
+  if ((st = M.mark(3)) != COSMOT_OK) return st;
   // 4. output projection + residual
   e = cosmot_epilogue{};
   e.kind = COSMOT_EPI_RESIDUAL;
@@ -154,14 +172,17 @@ cosmot_status cosmot_layer_forward(const cosmot_dims* dims, const cosmot_layer_w
   e.ld_res = d;
   st = cosmot_routed_linear(o, qc, qc, segs, ns, R.wo, G.wo, nullptr, nullptr, d, h1, d, &e, stream);
   if (st != COSMOT_OK) return st;
+  if ((st = M.mark(4)) != COSMOT_OK) return st;
   // 5. pre-FFN norm
   st = cosmot_rmsnorm_routed(h1, d, segs, ns, R.g2, G.g2, d, D.eps, a, d, stream);
   if (st != COSMOT_OK) return st;
+  if ((st = M.mark(5)) != COSMOT_OK) return st;
   // 6. gate/up with SiLU * mul
   e = cosmot_epilogue{};
   e.kind = COSMOT_EPI_SILU_MUL;
   st = cosmot_routed_linear(a, d, d, segs, ns, R.wg, G.wg, R.wu, G.wu, F, u, F, &e, stream);
   if (st != COSMOT_OK) return st;
+  if ((st = M.mark(6)) != COSMOT_OK) return st;
   // 7. down projection + residual
   e = cosmot_epilogue{};
   e.kind = COSMOT_EPI_RESIDUAL;
@@ -169,7 +190,11 @@ cosmot_status cosmot_layer_forward(const cosmot_dims* dims, const cosmot_layer_w
   e.ld_res = d;
   st = cosmot_routed_linear(u, F, F, segs, ns, R.wd, G.wd, nullptr, nullptr, d, h_out, d, &e, stream);
   if (st != COSMOT_OK) return st;
-  if (S.n_noisy == 0) return COSMOT_OK;
+  if (S.n_noisy == 0) {
+    if ((st = M.mark(7)) != COSMOT_OK || (st = M.mark(8)) != COSMOT_OK) return st;
+    return M.mark(9);
+  }
+  if ((st = M.mark(7)) != COSMOT_OK) return st;
   // 8. final norm of the noisy rows, packed into a
   cosmot_segment vs[kMaxBatch], ns_in[kMaxBatch];
   for (int b = 0; b < B; ++b) {
@@ -179,13 +204,40 @@ cosmot_status cosmot_layer_forward(const cosmot_dims* dims, const cosmot_layer_w
   }
   st = cosmot_rmsnorm_routed(h_out, d, ns_in, B, w->gfin, w->gfin, d, D.eps, a, d, stream);
   if (st != COSMOT_OK) return st;
+  if ((st = M.mark(8)) != COSMOT_OK) return st;
   // 9. velocity head with the Euler step, in place on the noisy rows of h
   e = cosmot_epilogue{};
   e.kind = COSMOT_EPI_EULER;
   e.x = h;
   e.ld_x = d;
   e.dsigma = (float)(sigma_next - sigma);
-  return cosmot_routed_linear(a, d, d, vs, B, w->wvel, w->wvel, nullptr, nullptr, d, hb, d, &e, stream);
+  st = cosmot_routed_linear(a, d, d, vs, B, w->wvel, w->wvel, nullptr, nullptr, d, hb, d, &e, stream);
+  if (st != COSMOT_OK) return st;
+  return M.mark(9);
+}
+
+}  // namespace
+}  // namespace cosmot
+
+extern "C" {
+
+cosmot_status cosmot_layer_forward(const cosmot_dims* dims, const cosmot_layer_weights* w,
+                                   const cosmot_seq_desc* seq, void* h, void* h_out, double sigma,
+                                   double sigma_next, void* workspace, size_t workspace_bytes,
+                                   cosmot_stream_t stream) {
+  return cosmot::layer_forward_impl(dims, w, seq, h, h_out, sigma, sigma_next, workspace, workspace_bytes, stream,
+                                    nullptr);
+}
+
+cosmot_status cosmot_layer_forward_timed(const cosmot_dims* dims, const cosmot_layer_weights* w,
+                                         const cosmot_seq_desc* seq, void* h, void* h_out, double sigma,
+                                         double sigma_next, void* workspace, size_t workspace_bytes,
+                                         cosmot_stream_t stream, void* const* stage_events, int32_t n_events) {
+  if (!stage_events || n_events != COSMOT_LAYER_STAGES + 1) return COSMOT_ERR_INVALID_ARG;
+  for (int i = 0; i < n_events; ++i)
+    if (!stage_events[i]) return COSMOT_ERR_INVALID_ARG;
+  return cosmot::layer_forward_impl(dims, w, seq, h, h_out, sigma, sigma_next, workspace, workspace_bytes, stream,
+                                    reinterpret_cast<const cudaEvent_t*>(stage_events));
 }
 
 }  // extern "C"

@@ -292,6 +292,34 @@ COSMOT_API cosmot_status cosmot_layer_forward(const cosmot_dims* dims, const cos
                                    double sigma_next, void* workspace, size_t workspace_bytes,
                                    cosmot_stream_t stream);
 
+/* Stages of cosmot_layer_forward, in launch order. */
+enum {
+  COSMOT_STAGE_NORM1 = 0,    /* routed RMSNorm before attention */
+  COSMOT_STAGE_QKV = 1,      /* routed QKV GEMM + mRoPE epilogue */
+  COSMOT_STAGE_ATTN = 2,     /* MoT attention */
+  COSMOT_STAGE_OPROJ = 3,    /* routed O GEMM + residual */
+  COSMOT_STAGE_NORM2 = 4,    /* routed RMSNorm before the FFN */
+  COSMOT_STAGE_GATEUP = 5,   /* routed gate/up GEMM + SiLU*mul */
+  COSMOT_STAGE_DOWN = 6,     /* routed down GEMM + residual */
+  COSMOT_STAGE_NORMFIN = 7,  /* final RMSNorm of the noisy rows */
+  COSMOT_STAGE_VEL = 8,      /* velocity GEMM + Euler step */
+  COSMOT_LAYER_STAGES = 9
+};
+
+/*
+ * cosmot_layer_forward with stage timing: stage_events[i] (i < COSMOT_LAYER_STAGES)
+ * is recorded on `stream` just before stage i and stage_events[COSMOT_LAYER_STAGES]
+ * after the last one, so cudaEventElapsedTime between consecutive events is the
+ * device time of one stage.  The events are cudaEvent_t handles created by the
+ * caller on the current device; n_events must be COSMOT_LAYER_STAGES + 1.  The
+ * computation is identical to cosmot_layer_forward.
+ */
+COSMOT_API cosmot_status cosmot_layer_forward_timed(const cosmot_dims* dims, const cosmot_layer_weights* w,
+                                                    const cosmot_seq_desc* seq, void* h, void* h_out, double sigma,
+                                                    double sigma_next, void* workspace, size_t workspace_bytes,
+                                                    cosmot_stream_t stream, void* const* stage_events,
+                                                    int32_t n_events);
+
 #ifdef __cplusplus
 }
 #endif
