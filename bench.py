@@ -54,6 +54,9 @@ def parse_args():
     p.add_argument("--impl", default="native", choices=["native", "reference"])
     p.add_argument("--no-e2e", action="store_true")
     p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--micro", choices=["attention", "gemm", "mrope", "euler", "rmsnorm"],
+                   help="time one kernel alone on the workload's widths (prints its own JSON line)")
+    p.add_argument("--tokens", type=int, default=0, help="rows for --micro (default: the workload's N)")
     return p.parse_args()
 
 
@@ -121,9 +124,25 @@ class ClockSampler:
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 
     def __init__(self, uuid=None):
-        self.uuid = uuid
+        self.uuid = self._match(uuid)
         self.proc = None
         self.out = os.path.join("/tmp", f"cosmot_clocks_{os.getpid()}.csv")
+
+    @staticmethod
+    def _match(uuid):
+        """nvidia-smi's UUID ("GPU-...") of the torch device, or None."""
+        if uuid is None:
+            return None
+        want = str(uuid).lower().replace("gpu-", "")
+        try:
+            out = subprocess.run(["nvidia-smi", "--query-gpu=uuid", "--format=csv,noheader"], capture_output=True,
+                                 text=True, timeout=30).stdout
+        except (OSError, subprocess.SubprocessError):
+            return None
+        for line in out.split():
+            if line.strip().lower().replace("gpu-", "") == want:
+                return line.strip()
+        return None
 
     def start(self):
         cmd = ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits", "-lms", "200"]
@@ -462,9 +481,109 @@ def run_native(args, wl):
         dist.destroy_process_group()
 
 
+def run_micro(args, wl):
+    """One kernel alone, `--steps` timed launches after `--warmup`, L2 flushed
+    between launches (outside the events).  Burst peaks apply (kernel timed
+    alone)."""
+    import torch
+
+    from flow_matching_dit_cosmot_b200 import _lib as L
+    from flow_matching_dit_cosmot_b200 import api as A
+
+    torch.cuda.set_device(0)
+    dev = torch.device("cuda", 0)
+    dm = wl.dims
+    d, hd, H, Hkv = dm.d_model, dm.head_dim, dm.n_heads, dm.n_kv_heads
+    T = args.tokens or synth.preset(args.workload).layout.n_ar + synth.preset(args.workload).layout.n_dm
+    n_ar = min(wl.layout.n_ar, T)
+    g = torch.Generator(device=dev)
+    g.manual_seed(3000 + wl.config_id)
+
+    def rnd(*shape, std=1.0):
+        return (torch.randn(*shape, generator=g, device=dev, dtype=torch.float32) * std).to(torch.bfloat16)
+
+    sh = torch.cuda.current_stream().cuda_stream
+    peaks, peak_src = load_peaks()
+    qkvc = dm.qkv_cols
+    if args.micro == "attention":
+        qkv = rnd(T, qkvc)
+        o = torch.empty((T, H * hd), dtype=torch.bfloat16, device=dev)
+        desc = L.AttnDesc(n_q=T, q_key_offset=0, n_keys=T, n_ar=n_ar, n_heads=H, n_kv_heads=Hkv, head_dim=hd,
+                          mask_mode=L.COSMOT_MASK_FULL, batch=1)
+        base = qkv.data_ptr()
+
+        def launch():
+            L.cosmot_mot_attention(desc, base, qkvc, base + 2 * H * hd, base + 2 * (H + Hkv) * hd, qkvc,
+                                   o.data_ptr(), H * hd, sh)
+        pairs = n_ar * (n_ar + 1) // 2 + (T - n_ar) * T
+        work, unit, peak = 4 * pairs * H * hd, "TFLOP/s", float(peaks["bf16_tflops"])
+    elif args.micro == "gemm":
+        a = rnd(T, d)
+        w = rnd(qkvc, d, std=0.02)
+        out = torch.empty((T, qkvc), dtype=torch.bfloat16, device=dev)
+        segs = [(0, n_ar, 0, 0), (n_ar, T, n_ar, 1)]
+
+        def launch():
+            L.cosmot_routed_linear(a.data_ptr(), d, d, segs, w.data_ptr(), w.data_ptr(), qkvc, out.data_ptr(), qkvc,
+                                   stream=sh)
+        work, unit, peak = 2 * T * d * qkvc, "TFLOP/s", float(peaks["bf16_tflops"])
+    elif args.micro == "mrope":
+        qkv = rnd(T, qkvc)
+        cs = torch.rand((T, hd // 2, 2), generator=g, device=dev, dtype=torch.float32)
+        base = qkv.data_ptr()
+
+        def launch():
+            L.cosmot_mrope_apply(base, qkvc, H, base + 2 * H * hd, qkvc, Hkv, T, hd, cs.data_ptr(), sh)
+        work, unit, peak = 4 * T * (H + Hkv) * hd + T * (hd // 2) * 8, "GB/s", float(peaks["hbm_gbs"])
+    elif args.micro == "euler":
+        x = rnd(T, d)
+        v = rnd(T, d)
+
+        def launch():
+            L.cosmot_flow_euler_step(x.data_ptr(), d, v.data_ptr(), d, 0, T, d, 1.0, 0.97, sh)
+        work, unit, peak = 6 * T * d, "GB/s", float(peaks["hbm_gbs"])
+    else:
+        h = rnd(T, d)
+        gg = rnd(d, std=0.02) + 1
+        out = torch.empty_like(h)
+        segs = [(0, n_ar, 0, 0), (n_ar, T, n_ar, 1)]
+
+        def launch():
+            L.cosmot_rmsnorm_routed(h.data_ptr(), d, segs, gg.data_ptr(), gg.data_ptr(), d, 1e-6, out.data_ptr(), d,
+                                    sh)
+        work, unit, peak = 4 * T * d, "GB/s", float(peaks["hbm_gbs"])
+
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    for _ in range(args.warmup):
+        flush.zero_()
+        launch()
+    torch.cuda.synchronize()
+    st_ev = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    en_ev = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    for i in range(args.steps):
+        flush.zero_()
+        st_ev[i].record()
+        launch()
+        en_ev[i].record()
+    torch.cuda.synchronize()
+    st, where = L.cosmot_get_device_status(sh)
+    if st:
+        raise RuntimeError(f"device status {L.status_string(st)} at {where}")
+    ms = statistics.mean(st_ev[i].elapsed_time(en_ev[i]) for i in range(args.steps))
+    scale = 1e12 if unit == "TFLOP/s" else 1e9
+    achieved = work / (ms / 1e3) / scale
+    print(json.dumps({"micro": args.micro, "workload": wl.name, "tokens": T, "ms": ms, "achieved": round(achieved, 1),
+                      "unit": unit, "peak": peak, "frac": round(achieved / peak, 3),
+                      "peak_source": f"{peak_src} burst", "algorithmic_per_launch": work,
+                      "steps": args.steps, "warmup": args.warmup}), flush=True)
+
+
 def main():
     args = parse_args()
     wl = synth.preset(args.workload)
+    if args.micro:
+        run_micro(args, wl)
+        return
     if args.impl == "reference":
         run_reference(args, wl)
     else:
