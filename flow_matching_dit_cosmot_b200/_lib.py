@@ -77,7 +77,7 @@ class LayerWeights(ctypes.Structure):
 
 class SeqDesc(ctypes.Structure):
     _fields_ = [("n_ar", c_i32), ("n_clean", c_i32), ("n_noisy", c_i32), ("batch", c_i32),
-                ("mask_mode", c_i32), ("reserved", c_i32), ("rope_cs", c_vp), ("chunk", c_vp)]
+                ("mask_mode", c_i32), ("n_cached", c_i32), ("rope_cs", c_vp), ("chunk", c_vp)]
 
 
 _P = ctypes.POINTER
@@ -99,6 +99,8 @@ SIGNATURES = {
     "cosmot_layer_workspace_size": (c_i32, [_P(Dims), _P(SeqDesc), _P(ctypes.c_size_t)]),
     "cosmot_layer_forward": (c_i32, [_P(Dims), _P(LayerWeights), _P(SeqDesc), c_vp, c_vp, c_f64, c_f64, c_vp,
                                      ctypes.c_size_t, c_vp]),
+    "cosmot_layer_commit_kv": (c_i32, [_P(Dims), _P(LayerWeights), _P(SeqDesc), c_vp, c_i64, c_vp, ctypes.c_size_t,
+                                       c_vp]),
     "cosmot_layer_forward_timed": (c_i32, [_P(Dims), _P(LayerWeights), _P(SeqDesc), c_vp, c_vp, c_f64, c_f64, c_vp,
                                            ctypes.c_size_t, c_vp, _P(c_vp), c_i32]),
 }
@@ -225,6 +227,12 @@ def cosmot_layer_forward(dims: Dims, w: LayerWeights, seq: SeqDesc, h: int, h_ou
                          sigma_next: float, workspace: int, workspace_bytes: int, stream: int = 0, check=True):
     return _call("cosmot_layer_forward", ctypes.byref(dims), ctypes.byref(w), ctypes.byref(seq), c_vp(h),
                  c_vp(h_out), sigma, sigma_next, c_vp(workspace), workspace_bytes, c_vp(stream), check=check)
+
+
+def cosmot_layer_commit_kv(dims: Dims, w: LayerWeights, seq: SeqDesc, h: int, dst_row: int, workspace: int,
+                           workspace_bytes: int, stream: int = 0, check=True):
+    return _call("cosmot_layer_commit_kv", ctypes.byref(dims), ctypes.byref(w), ctypes.byref(seq), c_vp(h), dst_row,
+                 c_vp(workspace), workspace_bytes, c_vp(stream), check=check)
 
 
 def cosmot_layer_forward_timed(dims: Dims, w: LayerWeights, seq: SeqDesc, h: int, h_out: int, sigma: float,

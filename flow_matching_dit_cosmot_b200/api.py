@@ -90,8 +90,9 @@ class MoTLayer:
         self.cw = L.LayerWeights((L.SetWeights * 2)(*sets), ptr(weights["gfin"]), ptr(weights["wvel"]))
         self._ws = None
 
-    def seq_desc(self, n_ar, n_clean, n_noisy, batch, rope_cs, chunk=None, mask_mode=L.COSMOT_MASK_FULL) -> L.SeqDesc:
-        return L.SeqDesc(n_ar, n_clean, n_noisy, batch, mask_mode, 0, ptr(rope_cs), ptr(chunk))
+    def seq_desc(self, n_ar, n_clean, n_noisy, batch, rope_cs, chunk=None, mask_mode=L.COSMOT_MASK_FULL,
+                 n_cached=0) -> L.SeqDesc:
+        return L.SeqDesc(n_ar, n_clean, n_noisy, batch, mask_mode, n_cached, ptr(rope_cs), ptr(chunk))
 
     def workspace_bytes(self, seq: L.SeqDesc) -> int:
         return L.cosmot_layer_workspace_size(self.dims, seq)
@@ -101,6 +102,13 @@ class MoTLayer:
         if self._ws is None or self._ws.numel() < n:
             self._ws = torch.empty((n,), dtype=torch.uint8, device=device)
         return self._ws
+
+    def commit_kv(self, h: torch.Tensor, seq: L.SeqDesc, dst_row: int, workspace: Optional[torch.Tensor] = None,
+                  stream=None):
+        """K/V of rows [seq.n_cached, N) of h into cache rows [dst_row, ...) of the workspace."""
+        _need_cuda(h)
+        ws = workspace if workspace is not None else self.workspace(seq, h.device)
+        L.cosmot_layer_commit_kv(self.dims, self.cw, seq, ptr(h), dst_row, ptr(ws), ws.numel(), stream_handle(stream))
 
     def forward(self, h: torch.Tensor, h_out: torch.Tensor, sigma: float, sigma_next: float, seq: L.SeqDesc,
                 workspace: Optional[torch.Tensor] = None, stream=None):

@@ -281,7 +281,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     for (int32_t t = blockIdx.x; t < p.num_tiles; t += gridDim.x, ++local) {
       const uint32_t buf = local & 1;
       const uint32_t use = local >> 1;
-      if (!mbar_wait(bar_tfull + 8 * buf, use & 1, p.status, kWhereGemmEpilogue)) break;
+      // Warp-uniform: the tcgen05.ld below is .sync.aligned.
+      if (!__all_sync(0xffffffffu, mbar_wait(bar_tfull + 8 * buf, use & 1, p.status, kWhereGemmEpilogue))) break;
       tc_fence_after();
       const Tile tl = decode_tile(p, t);
       const bool valid = r < tl.rows;
@@ -311,7 +312,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       } else if (EPI == COSMOT_EPI_MROPE) {
         const int hd = p.head_dim;
         const int half = hd >> 1;
-        const int64_t trow = p.rope_period > 0 ? orow % p.rope_period : orow;
+        const int64_t arow = tl.a_row0 + r;  // positions follow the input row
+        const int64_t trow = p.rope_period > 0 ? arow % p.rope_period : arow;
         const float2* cs_row = p.rope_cs + trow * half;
 #pragma unroll 1
         for (int hb = 0; hb < BN / hd; ++hb) {

@@ -13,6 +13,14 @@
 //   7 routed down + residual     u, h1 -> h_out
 //   8 RMSNorm (noisy rows)       h_out -> a (packed)         (g_fin)
 //   9 velocity GEMM + Euler      a -> h[noisy rows] in place
+//
+// Cached prefix (seq.n_cached > 0): the first n_cached rows of every sequence
+// keep the K and V that an earlier call left in the workspace's qkv region and
+// are not recomputed; only rows [n_cached, N) go through the layer.  AR rows
+// never read DM rows ("Cosmos 3 方法原理全解" §3), so a sampler reuses the AR
+// K/V of its first step (§7.2: the Reasoner prompt is encoded once); a
+// streaming rollout keeps AR + history-block K/V there ("流式生成如何工作":
+// the key/value cache keeps attention information for the next prediction).
 #include "cosmot_internal.h"
 
 namespace cosmot {
@@ -46,7 +54,22 @@ cosmot_status check_seq(const cosmot_seq_desc* s) {
   if (s->mask_mode != COSMOT_MASK_FULL && s->mask_mode != COSMOT_MASK_BLOCK_CAUSAL) return COSMOT_ERR_INVALID_ARG;
   if (s->mask_mode == COSMOT_MASK_BLOCK_CAUSAL && !s->chunk) return COSMOT_ERR_INVALID_ARG;
   if (!s->rope_cs) return COSMOT_ERR_INVALID_ARG;
+  if (s->n_cached < 0 || s->n_cached > s->n_ar + s->n_clean) return COSMOT_ERR_INVALID_ARG;
   return COSMOT_OK;
+}
+
+// Routed row segments over rows [lo, N) of each sequence: AR rows through set 0,
+// DM rows through set 1; output row = input row + out_shift.
+int make_segments(const cosmot_seq_desc& S, int64_t lo, int64_t out_shift, cosmot_segment* segs) {
+  const int64_t N = (int64_t)S.n_ar + S.n_clean + S.n_noisy;
+  int ns = 0;
+  for (int b = 0; b < S.batch; ++b) {
+    const int64_t r0 = b * N;
+    if (lo < S.n_ar) segs[ns++] = cosmot_segment{r0 + lo, r0 + S.n_ar, r0 + lo + out_shift, 0, 0};
+    const int64_t dm0 = lo > S.n_ar ? lo : S.n_ar;
+    if (N > dm0) segs[ns++] = cosmot_segment{r0 + dm0, r0 + N, r0 + dm0 + out_shift, 1, 0};
+  }
+  return ns;
 }
 
 WsLayout ws_layout(const cosmot_dims& d, const cosmot_seq_desc& s) {
@@ -55,8 +78,9 @@ WsLayout ws_layout(const cosmot_dims& d, const cosmot_seq_desc& s) {
   const size_t q_cols = (size_t)d.n_heads * d.head_dim;
   WsLayout w;
   size_t off = 0;
-  w.a = off;   off += align256(rows * d.d_model * 2);
+  // qkv first: cached K/V rows keep their addresses whatever the other sizes.
   w.qkv = off; off += align256(rows * qkv_cols * 2);
+  w.a = off;   off += align256(rows * d.d_model * 2);
   w.o = off;   off += align256(rows * q_cols * 2);
   w.h1 = off;  off += align256(rows * d.d_model * 2);
   w.u = off;   off += align256(rows * d.ffn * 2);
@@ -122,14 +146,11 @@ cosmot_status layer_forward_impl(const cosmot_dims* dims, const cosmot_layer_wei
   void* u = ws + L.u;
   uint16_t* hb = static_cast<uint16_t*>(h);
 
-  // Row segments: AR rows of every sequence go through set 0, DM rows set 1.
+  // Row segments over the rows this call computes: AR rows through set 0, DM
+  // rows through set 1; rows before n_cached keep their cached K/V.
+  const int64_t c0 = S.n_cached;
   cosmot_segment segs[2 * kMaxBatch];
-  int ns = 0;
-  for (int b = 0; b < B; ++b) {
-    const int64_t r0 = b * N;
-    if (S.n_ar > 0) segs[ns++] = cosmot_segment{r0, r0 + S.n_ar, r0, 0, 0};
-    if (N > S.n_ar) segs[ns++] = cosmot_segment{r0 + S.n_ar, r0 + N, r0 + S.n_ar, 1, 0};
-  }
+  const int ns = make_segments(S, c0, 0, segs);
   const cosmot_set_weights& R = w->set[0];
   const cosmot_set_weights& G = w->set[1];
 
@@ -150,8 +171,8 @@ cosmot_status layer_forward_impl(const cosmot_dims* dims, const cosmot_layer_wei
   if ((st = M.mark(2)) != COSMOT_OK) return st;
   // 3. attention
   cosmot_attn_desc ad{};
-  ad.n_q = N;
-  ad.q_key_offset = 0;
+  ad.n_q = N - c0;
+  ad.q_key_offset = c0;
   ad.n_keys = N;
   ad.n_ar = S.n_ar;
   ad.n_heads = D.n_heads;
@@ -162,7 +183,8 @@ cosmot_status layer_forward_impl(const cosmot_dims* dims, const cosmot_layer_wei
   ad.batch = B;
   ad.q_batch_stride = ad.kv_batch_stride = ad.o_batch_stride = N;
   uint16_t* qkvp = static_cast<uint16_t*>(qkv);
-  st = cosmot_mot_attention(&ad, qkvp, qkvc, qkvp + qc, qkvp + qc + kvc, qkvc, o, qc, stream);
+  st = cosmot_mot_attention(&ad, qkvp + c0 * qkvc, qkvc, qkvp + qc, qkvp + qc + kvc, qkvc,
+                            static_cast<uint16_t*>(o) + c0 * qc, qc, stream);
   if (st != COSMOT_OK) return st;
   if ((st = M.mark(3)) != COSMOT_OK) return st;
   // 4. output projection + residual
@@ -227,6 +249,43 @@ cosmot_status cosmot_layer_forward(const cosmot_dims* dims, const cosmot_layer_w
                                    cosmot_stream_t stream) {
   return cosmot::layer_forward_impl(dims, w, seq, h, h_out, sigma, sigma_next, workspace, workspace_bytes, stream,
                                     nullptr);
+}
+
+cosmot_status cosmot_layer_commit_kv(const cosmot_dims* dims, const cosmot_layer_weights* w,
+                                     const cosmot_seq_desc* seq, const void* h, int64_t dst_row, void* workspace,
+                                     size_t workspace_bytes, cosmot_stream_t stream) {
+  using namespace cosmot;
+  cosmot_status st = check_dims(dims);
+  if (st != COSMOT_OK) return st;
+  st = check_seq(seq);
+  if (st != COSMOT_OK) return st;
+  if (!w || !h || !workspace) return COSMOT_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return COSMOT_ERR_INVALID_ARG;
+  const WsLayout L = ws_layout(*dims, *seq);
+  if (workspace_bytes < L.total) return COSMOT_ERR_WORKSPACE;
+  const cosmot_dims& D = *dims;
+  const cosmot_seq_desc& S = *seq;
+  const int64_t N = (int64_t)S.n_ar + S.n_clean + S.n_noisy;
+  const int64_t c0 = S.n_cached;
+  if (dst_row < 0 || dst_row + (N - c0) > N) return COSMOT_ERR_INVALID_ARG;
+  const int64_t d = D.d_model, hd = D.head_dim;
+  const int64_t qc = (int64_t)D.n_heads * hd, kvc = (int64_t)D.n_kv_heads * hd, qkvc = qc + 2 * kvc;
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  cosmot_segment segs[2 * kMaxBatch], dst[2 * kMaxBatch];
+  const int ns = make_segments(S, c0, 0, segs);
+  make_segments(S, c0, dst_row - c0, dst);
+  const cosmot_set_weights& R = w->set[0];
+  const cosmot_set_weights& G = w->set[1];
+  st = cosmot_rmsnorm_routed(h, d, segs, ns, R.g1, G.g1, d, D.eps, ws + L.a, d, stream);
+  if (st != COSMOT_OK) return st;
+  cosmot_epilogue e{};
+  e.kind = COSMOT_EPI_MROPE;
+  e.head_dim = D.head_dim;
+  e.rope_cols = qc + kvc;
+  e.rope_cs = S.rope_cs;
+  e.rope_period = N;
+  return cosmot_routed_linear(ws + L.a, d, d, dst, ns, R.wqkv, G.wqkv, nullptr, nullptr, qkvc, ws + L.qkv, qkvc, &e,
+                              stream);
 }
 
 cosmot_status cosmot_layer_forward_timed(const cosmot_dims* dims, const cosmot_layer_weights* w,

@@ -158,7 +158,7 @@ typedef struct {
   int32_t kind;
   int32_t head_dim;        /* MROPE: head width (64 or 128) */
   int64_t rope_cols;       /* MROPE: number of leading output columns rotated (Q and K heads) */
-  const float* rope_cs;    /* MROPE: table of cosmot_mrope_table, row = output row mod rope_period */
+  const float* rope_cs;    /* MROPE: table of cosmot_mrope_table, row = input row mod rope_period */
   int64_t rope_period;     /* MROPE: rows per sequence in the table (0 = no wrap) */
   const void* res;         /* RESIDUAL: [rows, n_out] bf16, indexed by output row */
   int64_t ld_res;
@@ -267,10 +267,22 @@ typedef struct {
   int32_t n_ar, n_clean, n_noisy; /* per sequence; N = n_ar + n_clean + n_noisy */
   int32_t batch;                  /* sequences laid out back to back: [batch][N][d] */
   int32_t mask_mode;              /* COSMOT_MASK_* among DM rows */
-  int32_t reserved;
+  int32_t n_cached;               /* leading rows of each sequence whose K/V are already in the
+                                     workspace (0 <= n_cached <= n_ar + n_clean); see below */
   const float* rope_cs;           /* device table of cosmot_mrope_table for one sequence [N] */
   const int32_t* chunk;           /* device [N] (BLOCK_CAUSAL only; may be NULL for FULL) */
 } cosmot_seq_desc;
+
+/*
+ * Key/value cache in the workspace.  The workspace starts with the layer's QKV
+ * rows [batch][N][(n_heads + 2 n_kv_heads) head_dim] (K rotated by mRoPE).  With
+ * seq.n_cached = c > 0, rows [0, c) of every sequence keep the K and V left there
+ * by earlier calls on the same workspace with the same batch and N; they are not
+ * recomputed, their h_out rows are not written, and only rows [c, N) are queries.
+ * Because AR rows never read DM rows ("Cosmos 3 方法原理全解" §3), a sampler loop
+ * reuses the AR K/V of its first step (c = n_ar, §7.2); a streaming rollout keeps
+ * AR + history-block K/V there (c = n_ar + history rows, "流式生成如何工作").
+ */
 
 /* Bytes of scratch cosmot_layer_forward needs for these sizes (host only). */
 COSMOT_API cosmot_status cosmot_layer_workspace_size(const cosmot_dims* dims, const cosmot_seq_desc* seq, size_t* bytes);
@@ -291,6 +303,19 @@ COSMOT_API cosmot_status cosmot_layer_forward(const cosmot_dims* dims, const cos
                                    const cosmot_seq_desc* seq, void* h, void* h_out, double sigma,
                                    double sigma_next, void* workspace, size_t workspace_bytes,
                                    cosmot_stream_t stream);
+
+/*
+ * Commit K/V into the workspace's cache: rows [seq.n_cached, N) of every sequence
+ * of h go through the pre-attention RMSNorm and the QKV projection with mRoPE
+ * (positions of those rows from seq.rope_cs), and the resulting QKV rows are
+ * written to rows [dst_row, dst_row + N - n_cached) of the cache.  Streaming: after
+ * a block's last denoising step, its final x is committed over the ring slot of
+ * the oldest history block; with n_cached = 0 and dst_row = 0 it fills the cache
+ * (AR rows and a prefilled history) in place.  Requires dst_row + N - n_cached <= N.
+ */
+COSMOT_API cosmot_status cosmot_layer_commit_kv(const cosmot_dims* dims, const cosmot_layer_weights* w,
+                                                const cosmot_seq_desc* seq, const void* h, int64_t dst_row,
+                                                void* workspace, size_t workspace_bytes, cosmot_stream_t stream);
 
 /* Stages of cosmot_layer_forward, in launch order. */
 enum {

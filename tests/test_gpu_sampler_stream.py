@@ -1,0 +1,132 @@
+"""Sampler loop with cached AR K/V and the streaming rollout with a key/value
+ring, against the fp64 oracle (needs a B200)."""
+
+import numpy as np
+import pytest
+
+import synth
+from oracle import layer as olayer
+from oracle import layout as olayout
+from synth import LayoutSpec, ModelDims, VideoSpec
+from tolerance import assert_close
+
+pytestmark = pytest.mark.gpu
+
+torch = pytest.importorskip("torch")
+if not torch.cuda.is_available():  # pragma: no cover
+    pytest.skip("no CUDA device", allow_module_level=True)
+
+from flow_matching_dit_cosmot_b200 import api as A  # noqa: E402
+from flow_matching_dit_cosmot_b200 import _lib as L  # noqa: E402
+from gpu_helpers import assert_device_ok, bits, device_weights, dims as cdims, layout_spec, to_dev, to_f64  # noqa
+
+MEDIUM = ModelDims(d_model=512, n_heads=4, n_kv_heads=4, head_dim=128, ffn=1536, rope_sections=(16, 24, 24))
+
+
+def _run_sampler(layer, dlay, cs, h0_bits, sigmas, batch, cached: bool):
+    h = to_dev(h0_bits)
+    h_out = torch.empty_like(h)
+    ws = None
+    states = []
+    for k, (s0, s1) in enumerate(zip(sigmas[:-1], sigmas[1:])):
+        seq = layer.seq_desc(dlay.n_ar, dlay.n_clean, dlay.n_noisy, batch, cs, dlay.chunk,
+                             n_cached=dlay.n_ar if (cached and k > 0) else 0)
+        if ws is None:
+            ws = torch.empty(layer.workspace_bytes(seq), dtype=torch.uint8, device="cuda")
+        layer.forward(h, h_out, s0, s1, seq, workspace=ws)
+        states.append(h.clone())
+    torch.cuda.synchronize()
+    assert_device_ok()
+    return h, h_out, states
+
+
+def test_sampler_loop_with_cached_ar_kv():
+    """DROID-style 10-step Euler sampler: step 1 computes every row, steps 2-10
+    reuse the AR K/V left in the workspace and compute DM rows only."""
+    wl = synth.preset("droid")
+    spec, sig, batch = wl.layout, wl.sigmas, 2
+    w = synth.make_weights(MEDIUM, 1003)
+    lay = olayout.build_layout(spec)
+    n = lay.n_tokens
+    h0 = np.stack([synth.make_activations(n, MEDIUM.d_model, 2003 + 100 * b) for b in range(batch)])
+    dlay = A.build_layout(layout_spec(A, spec))
+    cs = A.mrope_table(dlay.pos, MEDIUM.head_dim, MEDIUM.rope_sections)
+    layer = A.MoTLayer(cdims(A, MEDIUM), device_weights(w))
+    h_c, out_c, states = _run_sampler(layer, dlay, cs, h0, sig, batch, cached=True)
+    h_f, out_f, _ = _run_sampler(layer, dlay, cs, h0, sig, batch, cached=False)
+    # Caching the AR K/V is exact on the GPU too: same bits as recomputing them.
+    np.testing.assert_array_equal(bits(h_c), bits(h_f))
+    np.testing.assert_array_equal(bits(out_c), bits(out_f))
+    W = olayer.weights_from_bits(MEDIUM, w)
+    noisy = lay.region == olayout.REGION_NOISY
+    for b in range(batch):
+        hf, outs = olayer.sample(MEDIUM, W, synth.bf16_to_f64(h0[b]), lay, sig)
+        vel_rms = float(np.sqrt(np.mean(np.concatenate([o["vel"][noisy] for o in outs]) ** 2)))
+        # The bf16 state goes back through the layer at every step: after step k
+        # the per-step bounds apply accumulated over k steps (tests/tolerance.py).
+        for k, o in enumerate(outs):
+            assert_close(to_f64(states[k][b])[noisy], o["x_new"][noisy], f"x after step {k + 1} [{b}]",
+                         rounded_inputs=2, branch_rms=vel_rms, n_steps=k + 1)
+        np.testing.assert_array_equal(bits(h_c[b])[~noisy], h0[b][~noisy])
+        # h_out of the last step (AR rows kept from step 1)
+        assert_close(to_f64(out_c[b]), outs[-1]["h2"], f"h_out last step [{b}]", rounded_inputs=2,
+                     n_steps=len(sig) - 1)
+
+
+def _virtual_spec(n_text, video, hist, tau_offset):
+    """[AR; history blocks as clean steps; the current block as the noisy step]."""
+    v = video
+    return A.layout_spec(n_text, (v.views, v.grid_h, v.grid_w, v.fps, hist, 1), tau_offset=tau_offset)
+
+
+@pytest.mark.parametrize("mode", [L.COSMOT_MASK_BLOCK_CAUSAL, L.COSMOT_MASK_FULL])
+def test_streaming_rollout_with_kv_ring(mode):
+    dims = ModelDims(d_model=256, n_heads=4, n_kv_heads=2, head_dim=64, ffn=512, rope_sections=(8, 12, 12))
+    video = VideoSpec(2, 3, 5, 24, 0, 1)  # 30 tokens per block
+    n_text, hist, blocks, sig = 6, 3, 5, (1.0, 0.75, 0.5, 0.25, 0.0)
+    T = video.tokens_per_step
+    n_ar = n_text + 2
+    w = synth.make_weights(dims, 1004)
+    layer = A.MoTLayer(cdims(A, dims), device_weights(w))
+    # seeded inputs: AR rows, the prefilled history blocks, the noise of each new block
+    h_ar = synth.make_activations(n_ar, dims.d_model, 2004)
+    hist_x = [synth.make_activations(T, dims.d_model, 2104 + i) for i in range(hist)]
+    noise = [synth.make_activations(T, dims.d_model, 2204 + b) for b in range(blocks)]
+    N = n_ar + hist * T + T
+
+    def seq_for(b, n_cached):
+        dl = A.build_layout(_virtual_spec(n_text, video, hist, b))
+        cs = A.mrope_table(dl.pos, dims.head_dim, dims.rope_sections)
+        s = layer.seq_desc(dl.n_ar, dl.n_clean, dl.n_noisy, 1, cs, dl.chunk, mask_mode=mode, n_cached=n_cached)
+        return s, (dl, cs)
+
+    # prefill: AR + history K/V computed in place
+    h = to_dev(np.concatenate([h_ar] + hist_x + [noise[0]]))
+    seq0, keep0 = seq_for(0, 0)
+    ws = torch.empty(layer.workspace_bytes(seq0), dtype=torch.uint8, device="cuda")
+    layer.commit_kv(h, seq0, 0, workspace=ws)
+    h_out = torch.empty_like(h)
+    outs = []
+    for b in range(blocks):
+        h[n_ar + hist * T:] = to_dev(noise[b])
+        seq, keep = seq_for(b, n_ar + hist * T)
+        for s0, s1 in zip(sig[:-1], sig[1:]):
+            layer.forward(h, h_out, s0, s1, seq, workspace=ws)
+        outs.append(h[n_ar + hist * T:].clone())
+        layer.commit_kv(h, seq, n_ar + (b % hist) * T, workspace=ws)
+    torch.cuda.synchronize()
+    assert_device_ok()
+
+    # oracle: the same rollout with its own cache
+    W = olayer.weights_from_bits(dims, w)
+    spec_blk = LayoutSpec(n_text=n_text, video=video)
+    st = olayer.StreamState(slots=hist)
+    for i in range(hist):
+        olayer.stream_commit(dims, W, st, synth.bf16_to_f64(hist_x[i]), olayout.build_layout(spec_blk, tau_offset=i))
+    for b in range(blocks):
+        lb = olayout.build_layout(spec_blk, tau_offset=hist + b)
+        x, _ = olayer.stream_block(dims, W, st, synth.bf16_to_f64(h_ar), synth.bf16_to_f64(noise[b]), lb, sig)
+        got = to_f64(outs[b])
+        assert_close(got, x, f"block {b}", rounded_inputs=2, n_steps=len(sig) - 1)
+        # the committed K/V come from the GPU's own final x, as the oracle commits its own
+        olayer.stream_commit(dims, W, st, x, lb)
