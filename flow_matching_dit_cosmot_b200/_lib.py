@@ -101,11 +101,14 @@ SIGNATURES = {
                                      ctypes.c_size_t, c_vp]),
     "cosmot_layer_commit_kv": (c_i32, [_P(Dims), _P(LayerWeights), _P(SeqDesc), c_vp, c_i64, c_vp, ctypes.c_size_t,
                                        c_vp]),
+    "cosmot_layer_forward_noalloc": (c_i32, [_P(Dims), _P(LayerWeights), _P(SeqDesc), c_vp, c_vp, c_f64, c_f64,
+                                             c_vp]),
     "cosmot_layer_forward_timed": (c_i32, [_P(Dims), _P(LayerWeights), _P(SeqDesc), c_vp, c_vp, c_f64, c_f64, c_vp,
                                            ctypes.c_size_t, c_vp, _P(c_vp), c_i32]),
 }
 
 COSMOT_LAYER_STAGES = 9
+COSMOT_NOALLOC_SCRATCH_BYTES = 64 << 20
 STAGE_NAMES = ("norm1", "qkv_mrope", "attention", "oproj_residual", "norm2", "gateup_silu", "down_residual",
                "norm_final", "velocity_euler")
 
@@ -233,6 +236,13 @@ def cosmot_layer_commit_kv(dims: Dims, w: LayerWeights, seq: SeqDesc, h: int, ds
                            workspace_bytes: int, stream: int = 0, check=True):
     return _call("cosmot_layer_commit_kv", ctypes.byref(dims), ctypes.byref(w), ctypes.byref(seq), c_vp(h), dst_row,
                  c_vp(workspace), workspace_bytes, c_vp(stream), check=check)
+
+
+def cosmot_layer_forward_noalloc(dims: Dims, w: LayerWeights, seq: SeqDesc, h: int, h_out: int, sigma: float,
+                                 sigma_next: float, stream: int = 0, check=True):
+    """Layer forward with the library's fixed scratch array instead of a caller workspace."""
+    return _call("cosmot_layer_forward_noalloc", ctypes.byref(dims), ctypes.byref(w), ctypes.byref(seq), c_vp(h),
+                 c_vp(h_out), sigma, sigma_next, c_vp(stream), check=check)
 
 
 def cosmot_layer_forward_timed(dims: Dims, w: LayerWeights, seq: SeqDesc, h: int, h_out: int, sigma: float,

@@ -317,6 +317,36 @@ COSMOT_API cosmot_status cosmot_layer_commit_kv(const cosmot_dims* dims, const c
                                                 const cosmot_seq_desc* seq, const void* h, int64_t dst_row,
                                                 void* workspace, size_t workspace_bytes, cosmot_stream_t stream);
 
+/*
+ * cosmot_layer_forward without a caller workspace, for callers that may not
+ * allocate device memory while they run: a control loop with a hard per-step
+ * deadline (cudaMalloc can synchronise the device and stall for an unbounded
+ * time) or a host framework whose own pool owns all device memory.  The pages
+ * have no counterpart; this is a deployment convenience of this library.
+ *
+ * The workspace is a fixed array of COSMOT_NOALLOC_SCRATCH_BYTES compiled into
+ * the library; every GPU that loads the library keeps it until the process
+ * exits.  Inputs, outputs and semantics are those of cosmot_layer_forward.
+ *   - Sizes whose cosmot_layer_workspace_size exceeds the limit return
+ *     COSMOT_ERR_WORKSPACE before any launch (64 MiB covers a full-width DROID
+ *     policy step, 703 tokens at d_model 4096, batch 1).
+ *   - seq->n_cached must be 0 (COSMOT_ERR_UNSUPPORTED otherwise): nothing may
+ *     depend on the array's previous contents.  Every scratch byte a call reads
+ *     is written earlier in the same call, so nothing needs clearing.
+ *   - All calls on a device share its one array: calls that can run at the same
+ *     time on that GPU (issued on different streams, or from several host
+ *     threads) race on it and corrupt each other's results.  Issue them in order
+ *     on one stream.
+ *   - The first call on each device looks up the array's device address
+ *     (cudaGetSymbolAddress, with that device current); make that first call
+ *     before any stream capture.
+ * No device memory is allocated or freed on any path.
+ */
+#define COSMOT_NOALLOC_SCRATCH_BYTES ((size_t)64 << 20)
+COSMOT_API cosmot_status cosmot_layer_forward_noalloc(const cosmot_dims* dims, const cosmot_layer_weights* w,
+                                                      const cosmot_seq_desc* seq, void* h, void* h_out,
+                                                      double sigma, double sigma_next, cosmot_stream_t stream);
+
 /* Stages of cosmot_layer_forward, in launch order. */
 enum {
   COSMOT_STAGE_NORM1 = 0,    /* routed RMSNorm before attention */
