@@ -86,19 +86,16 @@ def attention_pairs(lay, mode: str) -> int:
     return int(pairs)
 
 
-def stage_work(wl, lay):
-    """(flops, bytes) per stage per step, algorithmic (no re-reads counted)."""
-    d, B = wl.dims, wl.batch
-    R = B * lay.n_tokens
-    dd, F, hd = d.d_model, d.ffn, d.head_dim
-    qc, qkvc = d.q_cols, d.qkv_cols
-    nz = B * lay.n_noisy
-    pairs = B * attention_pairs(lay, wl.mask_mode)
+def stage_work(dims, R, nz, pairs):
+    """(flops, bytes) per stage of one layer call, algorithmic (operands counted
+    once, only visible attention pairs): R rows computed, nz noisy rows."""
+    dd, F, hd = dims.d_model, dims.ffn, dims.head_dim
+    qc, qkvc = dims.q_cols, dims.qkv_cols
     w_set = 2  # bytes per bf16
     return {
         "norm1": (0, R * dd * 4),
         "qkv_mrope": (2 * R * dd * qkvc, (R * dd + 2 * qkvc * dd + R * qkvc) * w_set),
-        "attention": (4 * pairs * d.n_heads * hd, (R * qkvc + R * qc) * w_set),
+        "attention": (4 * pairs * dims.n_heads * hd, (R * qkvc + R * qc) * w_set),
         "oproj_residual": (2 * R * qc * dd, (R * qc + 2 * dd * qc + 2 * R * dd) * w_set),
         "norm2": (0, R * dd * 4),
         "gateup_silu": (2 * R * dd * 2 * F, (R * dd + 4 * F * dd + R * F) * w_set),
@@ -106,6 +103,20 @@ def stage_work(wl, lay):
         "norm_final": (0, nz * dd * 4),
         "velocity_euler": (2 * nz * dd * dd, (nz * dd * 3 + dd * dd) * w_set),
     }
+
+
+def workload_kind(wl) -> str:
+    if wl.stream is not None:
+        return "stream"
+    return "sampler" if len(wl.sigmas) > 2 else "layer"
+
+
+def stream_layout_spec(wl, block: int):
+    """One streaming step as a packed sequence: AR rows, the cached history
+    blocks as clean latent steps, the block being generated as the noisy step."""
+    v = wl.layout.video
+    return dict(n_text=wl.layout.n_text, video=(v.views, v.grid_h, v.grid_w, v.fps, wl.stream.cached_blocks, 1),
+                tau_offset=block)
 
 
 def load_peaks():
@@ -184,23 +195,95 @@ class ClockSampler:
 
 # ---------------------------------------------------------------- reference arm (fp64 CPU oracle)
 
-def oracle_sample(wl, lay, W, h64, rows_lo=16, rows_hi=48):
-    """Times the oracle on two row samples of the first sequence and extrapolates
-    linearly in query rows to the whole layer (K and V are always formed for
-    every row, so the fixed part is measured, not estimated)."""
+_ORACLE = {}
+
+
+def oracle_setup(wl):
+    """Oracle inputs of the workload (same seeded generators as the GPU arm)."""
+    if wl.name not in _ORACLE:
+        from oracle import layer as olayer
+        from oracle import layout as olayout
+        W = olayer.weights_from_bits(wl.dims, synth.make_weights(wl.dims, wl.weight_seed))
+        if workload_kind(wl) == "stream":
+            lay = olayout.build_layout(synth.LayoutSpec(n_text=wl.layout.n_text, video=wl.layout.video))
+            h_ar = synth.bf16_to_f64(synth.make_activations(lay.n_ar, wl.dims.d_model, wl.act_seed(0)))
+            hist = [synth.bf16_to_f64(synth.make_activations(lay.n_noisy, wl.dims.d_model, 4000 + k))
+                    for k in range(wl.stream.cached_blocks)]
+            st = olayer.StreamState(slots=wl.stream.cached_blocks)
+            spec_blk = synth.LayoutSpec(n_text=wl.layout.n_text, video=wl.layout.video)
+            for k, x in enumerate(hist):  # prefill, not timed
+                olayer.stream_commit(wl.dims, W, st, x, olayout.build_layout(spec_blk, tau_offset=k))
+            _ORACLE[wl.name] = (lay, W, (h_ar, hist, st))
+        else:
+            lay = olayout.build_layout(wl.layout)
+            h64 = synth.bf16_to_f64(synth.make_activations(lay.n_tokens, wl.dims.d_model, wl.act_seed(0)))
+            _ORACLE[wl.name] = (lay, W, h64)
+    return _ORACLE[wl.name]
+
+
+def oracle_sample(wl, quick: bool = False):
+    """Times the fp64 oracle on a bounded sample of one step of the workload.
+
+    Returns (seconds for one whole step, seconds spent, description).
+      layer:   two row samples (256 and 512 noisy query rows, fewer for small
+               layouts; K and V formed for every row each time), extrapolated
+               linearly to all rows and the batch;
+      sampler: the whole 10-step sampling of one sequence, times the batch;
+      stream:  one denoising step on 256 and 512 of the block's rows against
+               a cache of 8 prefilled history blocks (prefill not timed),
+               extrapolated to the block and its 4 steps, plus the K/V commit.
+    """
     from oracle import layer as olayer
-    dm0 = lay.n_ar + lay.n_clean
-    s0, s1 = wl.sigmas[0], wl.sigmas[1]
+    from oracle import layout as olayout
+    kind = workload_kind(wl)
+    lay, W, data = oracle_setup(wl)
+    # Row samples large enough that the per-row work (FFN, attention rows)
+    # is measured at full-size memory behaviour, not from cache.
+    big = 16 if quick else 256
+    rows_lo = min(big, max(lay.n_noisy // 4, 1))
+    rows_hi = min(2 * big, max(lay.n_noisy // 2, 2))
+    if kind == "layer":
+        dm0 = lay.n_ar + lay.n_clean
+        t = []
+        for r in (rows_lo, rows_hi):
+            rows = np.arange(dm0, min(lay.n_tokens, dm0 + r))
+            t0 = time.perf_counter()
+            olayer.layer_forward(wl.dims, W, data, lay.region, lay.pos, lay.chunk, wl.sigmas[0], wl.sigmas[1],
+                                 wl.mask_mode, rows=rows)
+            t.append(time.perf_counter() - t0)
+        per_row = max(t[1] - t[0], 0.0) / (rows_hi - rows_lo)
+        fixed = max(t[0] - rows_lo * per_row, 0.0)
+        return ((fixed + per_row * lay.n_tokens) * wl.batch, sum(t),
+                f"oracle layer forward on {rows_lo} and {rows_hi} noisy query rows (K/V of all {lay.n_tokens} "
+                f"rows each), extrapolated linearly to all rows and the batch")
+    if kind == "sampler":
+        # The oracle recomputes every row at every step, so its steps cost the
+        # same: time one and scale by the step count.
+        t0 = time.perf_counter()
+        olayer.layer_forward(wl.dims, W, data, lay.region, lay.pos, lay.chunk, wl.sigmas[0], wl.sigmas[1],
+                             wl.mask_mode)
+        t = time.perf_counter() - t0
+        n = len(wl.sigmas) - 1
+        return (t * n * wl.batch, t, f"one oracle layer forward of a {lay.n_tokens}-token sequence (all rows), "
+                                     f"times {n} sampler steps and the batch of {wl.batch}")
+    h_ar, hist, st = data
+    lb = olayout.build_layout(synth.LayoutSpec(n_text=wl.layout.n_text, video=wl.layout.video),
+                              tau_offset=len(hist))
+    x0 = synth.bf16_to_f64(synth.make_activations(lay.n_noisy, wl.dims.d_model, 5000))
     t = []
     for r in (rows_lo, rows_hi):
-        rows = np.arange(dm0, min(lay.n_tokens, dm0 + r))
         t0 = time.perf_counter()
-        olayer.layer_forward(wl.dims, W, h64, lay.region, lay.pos, lay.chunk, s0, s1, wl.mask_mode, rows=rows)
+        olayer.stream_block(wl.dims, W, st, h_ar, x0, lb, wl.sigmas, rows=np.arange(r))
         t.append(time.perf_counter() - t0)
     per_row = max(t[1] - t[0], 0.0) / (rows_hi - rows_lo)
     fixed = max(t[0] - rows_lo * per_row, 0.0)
-    t_full = (fixed + per_row * lay.n_tokens) * wl.batch
-    return t_full, sum(t)
+    t0 = time.perf_counter()
+    k, v = olayer.project_kv(wl.dims, W, x0, lb.region[lb.n_ar:], lb.pos[lb.n_ar:])  # the commit's work
+    t_commit = time.perf_counter() - t0
+    n = len(wl.sigmas) - 1
+    return (n * (fixed + per_row * lay.n_noisy) + t_commit, sum(t) + t_commit,
+            f"one oracle denoising step on {rows_lo} and {rows_hi} of the {lay.n_noisy} block rows against "
+            f"{len(hist)} cached blocks, extrapolated to the block, times {n} steps, plus the timed K/V commit")
 
 
 def cpu_threads():
@@ -214,38 +297,35 @@ def cpu_threads():
     return os.cpu_count()
 
 
-def oracle_setup(wl):
-    from oracle import layer as olayer
-    from oracle import layout as olayout
-    lay = olayout.build_layout(wl.layout)
-    W = olayer.weights_from_bits(wl.dims, synth.make_weights(wl.dims, wl.weight_seed))
-    h64 = synth.bf16_to_f64(synth.make_activations(lay.n_tokens, wl.dims.d_model, wl.act_seed(0)))
-    return lay, W, h64
-
-
 def run_reference(args, wl):
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return
-    lay, W, h64 = oracle_setup(wl)
+    kind = workload_kind(wl)
+    lay = oracle_setup(wl)[0]
+    if kind == "stream":
+        tokens = lay.n_noisy * (len(wl.sigmas) - 1)
+        seq_len = lay.n_ar + wl.stream.cached_blocks * lay.n_noisy + lay.n_noisy
+    else:
+        tokens = wl.batch * lay.n_tokens * (len(wl.sigmas) - 1 if kind == "sampler" else 1)
+        seq_len = lay.n_tokens
     for _ in range(args.warmup):
-        oracle_sample(wl, lay, W, h64)
-    t_full, t_spent = [], 0.0
+        oracle_sample(wl, quick=True)  # warm-up: the smallest sample
+    t_full, t_spent, sample = [], 0.0, ""
     for _ in range(args.steps):
-        tf, ts = oracle_sample(wl, lay, W, h64)
+        tf, ts, sample = oracle_sample(wl)
         t_full.append(tf)
         t_spent += ts
-    tokens = wl.batch * lay.n_tokens
     value = tokens * len(t_full) / sum(t_full)
     cores = cpu_threads()
-    sample = (f"per step: oracle layer forward on 16 and on 48 noisy query rows of sequence 0 (K/V of all "
-              f"{lay.n_tokens} rows each time), extrapolated linearly to all rows and the batch")
+    cfg = config_block(wl, lay, args.gpus)
+    cfg["seq_len"] = seq_len
     line = {
         "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * statistics.mean(t_full),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
         "data": "synthetic (seeded Philox: activations N(0,1), weights N(0,0.02), gains 1+N(0,0.02))",
-        "config": config_block(wl, lay, args.gpus),
+        "config": cfg,
         "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle", "sample": sample},
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
         "wall_s_sampled": t_spent,
@@ -284,14 +364,24 @@ def run_native(args, wl):
     from flow_matching_dit_cosmot_b200 import _lib as L
     from flow_matching_dit_cosmot_b200 import api as A
 
+    kind = workload_kind(wl)
     dims_s = wl.dims
     dev = torch.device("cuda", local)
-    v = wl.layout.video
-    spec = A.layout_spec(wl.layout.n_text,
-                         None if v is None else (v.views, v.grid_h, v.grid_w, v.fps, v.clean_steps, v.noisy_steps),
-                         wl.layout.audio_clean, wl.layout.audio_noisy, wl.layout.audio_rate, wl.layout.action_clean,
-                         wl.layout.action_noisy, wl.layout.action_hz, wl.layout.proprio)
-    dl = A.build_layout(spec, dev)
+    sh = torch.cuda.current_stream().cuda_stream
+    stream = torch.cuda.current_stream()
+    n_stage = L.COSMOT_LAYER_STAGES
+    mode = L.COSMOT_MASK_FULL if wl.mask_mode == "full" else L.COSMOT_MASK_BLOCK_CAUSAL
+
+    def spec_for(step_idx):
+        if kind == "stream":
+            return A.layout_spec(**stream_layout_spec(wl, step_idx % 16))
+        v = wl.layout.video
+        return A.layout_spec(wl.layout.n_text,
+                             None if v is None else (v.views, v.grid_h, v.grid_w, v.fps, v.clean_steps, v.noisy_steps),
+                             wl.layout.audio_clean, wl.layout.audio_noisy, wl.layout.audio_rate,
+                             wl.layout.action_clean, wl.layout.action_noisy, wl.layout.action_hz, wl.layout.proprio)
+
+    dl = A.build_layout(spec_for(0), dev)
     lay = Counts(dl.n_ar, dl.n_clean, dl.n_noisy, dl.chunk.cpu().numpy())
     B, N, d = wl.batch, lay.n_tokens, dims_s.d_model
 
@@ -300,8 +390,7 @@ def run_native(args, wl):
 
     w = {k: to_dev(v) for k, v in synth.make_weights(dims_s, wl.weight_seed).items()}
     h_host = np.stack([synth.make_activations(N, d, wl.act_seed(rank * B + b)) for b in range(B)])
-    h_src = to_dev(h_host)
-    h = h_src.clone()
+    h = to_dev(h_host)
     h_out = torch.empty_like(h)
     pos = torch.empty((N, 3), dtype=torch.float32, device=dev)
     chunk = torch.empty((N,), dtype=torch.int32, device=dev)
@@ -309,14 +398,77 @@ def run_native(args, wl):
     dims = A.make_dims(dims_s.d_model, dims_s.n_heads, dims_s.n_kv_heads, dims_s.head_dim, dims_s.ffn,
                        dims_s.rope_sections, dims_s.rope_base, dims_s.eps)
     layer = A.MoTLayer(dims, w)
-    mode = L.COSMOT_MASK_FULL if wl.mask_mode == "full" else L.COSMOT_MASK_BLOCK_CAUSAL
-    seq = layer.seq_desc(lay.n_ar, lay.n_clean, lay.n_noisy, B, cs, chunk, mode)
-    ws = layer.workspace(seq, dev)
+    z0 = lay.n_ar + lay.n_clean  # first noisy row of a sequence
+
+    def seq(n_cached):
+        return layer.seq_desc(lay.n_ar, lay.n_clean, lay.n_noisy, B, cs, chunk, mode, n_cached=n_cached)
+
+    ws = layer.workspace(seq(0), dev)
     flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
-    stream = torch.cuda.current_stream()
-    sh = stream.cuda_stream
-    s0, s1 = wl.sigmas[0], wl.sigmas[1]
-    n_stage = L.COSMOT_LAYER_STAGES
+
+    # ---- the plan of one step: (n_cached, sigma, sigma_next) per layer call
+    sig = wl.sigmas
+    if kind == "layer":
+        calls = [(0, sig[0], sig[1])]
+    elif kind == "sampler":
+        calls = [(0, sig[0], sig[1])] + [(lay.n_ar, a, b) for a, b in zip(sig[1:-1], sig[2:])]
+    else:
+        calls = [(z0, a, b) for a, b in zip(sig[:-1], sig[1:])]
+    seqs = {c: seq(c) for c in {c for c, _, _ in calls}}
+    if kind == "stream":
+        noise = [to_dev(synth.make_activations(lay.n_noisy, d, 5000 + k)) for k in range(4)]
+        # prefill the cache: AR rows and the 8 seeded history blocks, K/V in place
+        L.cosmot_build_layout(spec_for(0), pos.data_ptr(), chunk.data_ptr(), 0, sh)
+        L.cosmot_mrope_table(pos.data_ptr(), N, dims_s.head_dim, dims_s.rope_sections, dims_s.rope_base,
+                             cs.data_ptr(), sh)
+        L.cosmot_layer_commit_kv(dims, layer.cw, seq(0), h.data_ptr(), 0, ws.data_ptr(), ws.numel(), sh)
+        commit_seq = seq(z0)
+
+    def layer_pairs(n_cached):
+        """Visible attention pairs of one call (queries = rows >= n_cached)."""
+        if n_cached == 0:
+            return attention_pairs(lay, wl.mask_mode)
+        # DM queries only; every key is visible to them here (full mask, or a
+        # block-causal cache that holds only earlier chunks)
+        return (N - n_cached) * N
+
+    work = [stage_work(dims_s, B * (N - c), B * lay.n_noisy, B * layer_pairs(c)) for c, _, _ in calls]
+    commit_flops = 2 * lay.n_noisy * d * dims_s.qkv_cols if kind == "stream" else 0
+    tokens_per_step = {"layer": B * N, "sampler": B * N * len(calls), "stream": B * lay.n_noisy * len(calls)}[kind]
+
+    step_no = [0]
+
+    def step(stage_evs=None, commit_evs=None):
+        b = step_no[0]
+        step_no[0] += 1
+        L.cosmot_build_layout(spec_for(b), pos.data_ptr(), chunk.data_ptr(), 0, sh)
+        L.cosmot_mrope_table(pos.data_ptr(), N, dims_s.head_dim, dims_s.rope_sections, dims_s.rope_base,
+                             cs.data_ptr(), sh)
+        for i, (c, s0, s1) in enumerate(calls):
+            if stage_evs is None:
+                L.cosmot_layer_forward(dims, layer.cw, seqs[c], h.data_ptr(), h_out.data_ptr(), s0, s1,
+                                       ws.data_ptr(), ws.numel(), sh)
+            else:
+                L.cosmot_layer_forward_timed(dims, layer.cw, seqs[c], h.data_ptr(), h_out.data_ptr(), s0, s1,
+                                             ws.data_ptr(), ws.numel(), sh, [e.cuda_event for e in stage_evs[i]])
+        if kind == "stream":
+            if commit_evs is not None:
+                commit_evs[0].record(stream)
+            slot = b % wl.stream.cached_blocks
+            L.cosmot_layer_commit_kv(dims, layer.cw, commit_seq, h.data_ptr(),
+                                     lay.n_ar + slot * lay.n_noisy, ws.data_ptr(), ws.numel(), sh)
+            if commit_evs is not None:
+                commit_evs[1].record(stream)
+
+    def pre_step():
+        flush.zero_()
+        if kind == "stream":  # the new block starts from fresh noise
+            h[0, z0:].copy_(noise[step_no[0] % len(noise)])
+        elif kind == "sampler":  # a new sampling starts from the same seeded noise
+            h.copy_(h_src)
+
+    h_src = h.clone() if kind == "sampler" else None
+    launches_per_step = 2 + n_stage * len(calls) + (2 if kind == "stream" else 0)
 
     def new_events(n):
         evs = [torch.cuda.Event(enable_timing=True) for _ in range(n)]
@@ -324,21 +476,8 @@ def run_native(args, wl):
             e.record(stream)  # creates the underlying cudaEvent_t
         return evs
 
-    def step(stage_evs=None):
-        L.cosmot_build_layout(spec, pos.data_ptr(), chunk.data_ptr(), 0, sh)
-        L.cosmot_mrope_table(pos.data_ptr(), N, dims_s.head_dim, dims_s.rope_sections, dims_s.rope_base,
-                             cs.data_ptr(), sh)
-        if stage_evs is None:
-            L.cosmot_layer_forward(dims, layer.cw, seq, h.data_ptr(), h_out.data_ptr(), s0, s1, ws.data_ptr(),
-                                   ws.numel(), sh)
-        else:
-            L.cosmot_layer_forward_timed(dims, layer.cw, seq, h.data_ptr(), h_out.data_ptr(), s0, s1, ws.data_ptr(),
-                                         ws.numel(), sh, [e.cuda_event for e in stage_evs])
-
-    launches_per_step = 2 + (n_stage if lay.n_noisy > 0 else n_stage - 2)
-
     for _ in range(args.warmup):
-        flush.zero_()
+        pre_step()
         step()
     torch.cuda.synchronize()
     st, where = L.cosmot_get_device_status(sh)
@@ -346,7 +485,8 @@ def run_native(args, wl):
         raise RuntimeError(f"device status {L.status_string(st)} at {where}")
 
     starts, ends = new_events(args.steps), new_events(args.steps)
-    stage_evs = [new_events(n_stage + 1) for _ in range(args.steps)]
+    stage_evs = [[new_events(n_stage + 1) for _ in calls] for _ in range(args.steps)]
+    commit_evs = [new_events(2) for _ in range(args.steps)]
     torch.cuda.synchronize()
     if world > 1:
         dist.barrier()
@@ -355,9 +495,9 @@ def run_native(args, wl):
     clocks.start()
     time.sleep(0.3)
     for i in range(args.steps):
-        flush.zero_()
+        pre_step()
         starts[i].record(stream)
-        step(stage_evs[i])
+        step(stage_evs[i], commit_evs[i])
         ends[i].record(stream)
     torch.cuda.synchronize()
     clk = clocks.stop()
@@ -368,33 +508,39 @@ def run_native(args, wl):
     if st:
         raise RuntimeError(f"device status {L.status_string(st)} at {where}")
 
-    step_ms = [starts[i].elapsed_time(ends[i]) for i in range(args.steps)]
-    total_ms = sum(step_ms)
-    stage_ms = np.zeros(n_stage)
-    for evs in stage_evs:
-        for j in range(n_stage):
-            stage_ms[j] += evs[j].elapsed_time(evs[j + 1])
+    total_ms = sum(starts[i].elapsed_time(ends[i]) for i in range(args.steps))
+    stage_ms = np.zeros(n_stage)  # per step, summed over the step's layer calls
+    for per_call in stage_evs:
+        for evs in per_call:
+            for j in range(n_stage):
+                stage_ms[j] += evs[j].elapsed_time(evs[j + 1])
     stage_ms /= args.steps
+    commit_ms = (sum(e[0].elapsed_time(e[1]) for e in commit_evs) / args.steps) if kind == "stream" else 0.0
 
     # ---------------------------------------------------------------- end to end (host buffers)
     e2e = None
     if not args.no_e2e:
-        h_pin = torch.from_numpy(h_host.view(np.int16)).view(torch.bfloat16).pin_memory()
-        z0 = lay.n_ar + lay.n_clean
-        x_pin = torch.empty((B, lay.n_noisy, d), dtype=torch.bfloat16).pin_memory()
+        if kind == "stream":
+            in_pin = noise[0].cpu().pin_memory()
+            out_pin = torch.empty_like(in_pin).pin_memory()
+            dst_in, src_out = h[0, z0:], h[0, z0:]
+        else:
+            in_pin = torch.from_numpy(h_host.view(np.int16)).view(torch.bfloat16).pin_memory()
+            out_pin = torch.empty((B, lay.n_noisy, d), dtype=torch.bfloat16).pin_memory()
+            dst_in, src_out = h, h[:, z0:]
         for _ in range(max(1, args.warmup)):
-            h.copy_(h_pin, non_blocking=True)
+            dst_in.copy_(in_pin, non_blocking=True)
             step()
-            x_pin.copy_(h[:, z0:], non_blocking=True)
+            out_pin.copy_(src_out, non_blocking=True)
         torch.cuda.synchronize()
         e_s, e_e = new_events(args.steps), new_events(args.steps)
         torch.cuda.synchronize()
         for i in range(args.steps):
             flush.zero_()
             e_s[i].record(stream)
-            h.copy_(h_pin, non_blocking=True)
+            dst_in.copy_(in_pin, non_blocking=True)
             step()
-            x_pin.copy_(h[:, z0:], non_blocking=True)
+            out_pin.copy_(src_out, non_blocking=True)
             e_e[i].record(stream)
         torch.cuda.synchronize()
         e2e_ms = sum(e_s[i].elapsed_time(e_e[i]) for i in range(args.steps))
@@ -402,10 +548,12 @@ def run_native(args, wl):
             t = torch.tensor([e2e_ms], device=dev, dtype=torch.float64)
             dist.all_reduce(t, op=dist.ReduceOp.MAX)
             e2e_ms = float(t.item())
-        e2e = {"value": world * B * N * args.steps / (e2e_ms / 1e3), "unit": UNIT,
-               "h2d_bytes_per_step": int(h_pin.numel() * 2), "d2h_bytes_per_step": int(x_pin.numel() * 2),
-               "ms_per_step": e2e_ms / args.steps, "path": "cosmot_build_layout + cosmot_mrope_table + "
-               "cosmot_layer_forward, pinned host h in, x' (noisy rows) out"}
+        e2e = {"value": world * tokens_per_step * args.steps / (e2e_ms / 1e3), "unit": UNIT,
+               "h2d_bytes_per_step": int(in_pin.numel() * 2), "d2h_bytes_per_step": int(out_pin.numel() * 2),
+               "ms_per_step": e2e_ms / args.steps,
+               "path": "cosmot_build_layout + cosmot_mrope_table + cosmot_layer_forward"
+                       + (" + cosmot_layer_commit_kv" if kind == "stream" else "")
+                       + ", pinned host input in, x' (noisy rows) out"}
 
     if world > 1:
         t = torch.tensor([total_ms], device=dev, dtype=torch.float64)
@@ -413,9 +561,9 @@ def run_native(args, wl):
         total_ms = float(t.item())
 
     if rank == 0:
-        work = stage_work(wl, lay)
         names = L.STAGE_NAMES
-        flops_total = sum(f for f, _ in work.values())
+        wsum = {nm: (sum(wk[nm][0] for wk in work), sum(wk[nm][1] for wk in work)) for nm in names}
+        flops_total = sum(f for f, _ in wsum.values()) + commit_flops
         peaks, peak_src = load_peaks()
         peak_tf = float(peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"]))
         peak_tf_burst = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
@@ -423,9 +571,9 @@ def run_native(args, wl):
         ms_step = total_ms / args.steps
         stages = {}
         for j, nm in enumerate(names):
-            f, b = work[nm]
+            f, b = wsum[nm]
             t_s = stage_ms[j] / 1e3
-            ent = {"ms": round(float(stage_ms[j]), 4), "share": round(float(stage_ms[j] / stage_ms.sum()), 4)}
+            ent = {"ms": round(float(stage_ms[j]), 4), "share": round(float(stage_ms[j] / ms_step), 4)}
             if f:
                 ent["tflops"] = round(f / t_s / 1e12, 1) if t_s > 0 else None
                 ent["frac_of_peak"] = round(f / t_s / 1e12 / peak_tf, 3) if t_s > 0 else None
@@ -433,34 +581,46 @@ def run_native(args, wl):
                 ent["gbs"] = round(b / t_s / 1e9, 1) if t_s > 0 else None
                 ent["frac_of_hbm"] = round(b / t_s / 1e9 / peak_bw, 3) if t_s > 0 else None
             stages[nm] = ent
+        if kind == "stream":
+            stages["kv_commit"] = {"ms": round(commit_ms, 4), "share": round(commit_ms / ms_step, 4),
+                                   "tflops": round(commit_flops / (commit_ms / 1e3) / 1e12, 1) if commit_ms else None}
         dom = max(range(n_stage), key=lambda j: stage_ms[j])
         dname = names[dom]
-        f, b = work[dname]
-        t_dom = stage_ms[dom] / 1e3
+        f, b = wsum[dname]
+        t_dom = stage_ms[dom] / 1e3  # per step; one launch per layer call
+        per_launch = len(calls)
         src = "attention.cu" if dname == "attention" else ("gemm.cu" if f else "elementwise.cu")
         traffic = None
-        rec = NCU_TRAFFIC.get(dname)
+        rec = NCU_TRAFFIC.get(f"{wl.name}:{dname}")
         if rec and rec.get("src_sha") == src_sha(src):
             traffic = rec["bytes_per_launch"]
         if f:
             achieved = f / t_dom / 1e12
             roof = {"bound": "tensor", "kernel": dname, "achieved": round(achieved, 1), "peak": peak_tf,
                     "unit": "TFLOP/s", "frac": round(achieved / peak_tf, 3), "traffic": traffic,
-                    "algorithmic_flops_per_launch": f, "peak_source": f"{peak_src} bf16_tflops_sustained"}
+                    "algorithmic_flops_per_launch": f // per_launch, "launches_per_step": per_launch,
+                    "peak_source": f"{peak_src} bf16_tflops_sustained"}
         else:
             achieved = b / t_dom / 1e9
             roof = {"bound": "hbm", "kernel": dname, "achieved": round(achieved, 1), "peak": peak_bw,
                     "unit": "GB/s", "frac": round(achieved / peak_bw, 3), "traffic": traffic,
-                    "algorithmic_bytes_per_launch": b, "peak_source": f"{peak_src} hbm_gbs"}
-        tokens = world * B * N * args.steps
-        value = tokens / (total_ms / 1e3)
+                    "algorithmic_bytes_per_launch": b // per_launch, "launches_per_step": per_launch,
+                    "peak_source": f"{peak_src} hbm_gbs"}
+        value = world * tokens_per_step * args.steps / (total_ms / 1e3)
         layer_tflops = flops_total / (ms_step / 1e3) / 1e12
+        cfg = config_block(wl, lay, world)
+        cfg["step"] = {"layer": "one layer forward + Euler step",
+                       "sampler": f"one {len(calls)}-step Euler sampling (step 1 all rows, then DM rows with the "
+                                  f"AR K/V kept in the workspace)",
+                       "stream": f"one streaming block: {len(calls)} denoising steps of {lay.n_noisy} tokens "
+                                 f"against {N - lay.n_noisy} cached key rows, then the block's K/V commit"}[kind]
+        cfg["tokens_per_step"] = tokens_per_step
         line = {
             "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "bf16",
             "data": "synthetic (seeded Philox: activations N(0,1), weights N(0,0.02), gains 1+N(0,0.02))",
-            "config": config_block(wl, lay, world),
+            "config": cfg,
             "tflops": round(layer_tflops, 1),
             "tflops_frac_of_peak": round(layer_tflops / peak_tf, 3),
             "tflops_frac_of_burst_peak": round(layer_tflops / peak_tf_burst, 3),
@@ -469,12 +629,9 @@ def run_native(args, wl):
             "roofline": roof, "stages": stages,
         }
         if world == 1 and not args.no_cpu_baseline:
-            lay_o, W, h64 = oracle_setup(wl)
-            t_full, t_spent = oracle_sample(wl, lay_o, W, h64)
-            line["cpu_baseline"] = {
-                "value": B * N / t_full, "unit": UNIT, "cores": cpu_threads(), "kind": "oracle",
-                "sample": f"oracle layer forward on 16 and 48 noisy query rows (K/V of all {N} rows each), "
-                          f"extrapolated linearly to all rows and the batch; {t_spent:.1f} s of CPU wall time"}
+            t_full, t_spent, sample = oracle_sample(wl)
+            line["cpu_baseline"] = {"value": tokens_per_step / t_full, "unit": UNIT, "cores": cpu_threads(),
+                                    "kind": "oracle", "sample": f"{sample}; {t_spent:.1f} s of CPU wall time"}
         print(json.dumps(line), flush=True)
 
     if world > 1:

@@ -22,6 +22,13 @@
 //               rescaled in TMEM only when the running max grows by more than
 //               2^8 (the exponent headroom keeps P and O finite meanwhile).
 // TMEM columns: S0 [0,128), S1 [128,256), O0 and O1 after them.
+//
+// Measured on B200 (18,978 tokens, 32 heads of 128): the period of one key
+// block is set by the chain softmax(tile 0) -> PV0 -> next S0 -> softmax, not by
+// the SFU; variants that moved exponentials to the FMA pipe, used packed
+// f32x2 arithmetic, split the row between two warpgroups or served both tiles
+// from one warpgroup were all slower than this plain form.  Every tcgen05.ld/st
+// is reached through warp-uniform control flow (they are .sync.aligned).
 #include <cuda_bf16.h>
 
 #include <mutex>
@@ -39,64 +46,6 @@ constexpr int BOX_BYTES = 128 * 64 * 2;  // one 128-row x 64-column bf16 box
 constexpr int NUM_THREADS = 320;
 constexpr int TMEM_COLS = 512;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
-
-// 2^f ~ c0 + f (c1 + f (c2 + f c3)) on [-1/2, 1/2], relative error < 7.5e-5;
-// near-minimax coefficients from csrc/gen_exp2_poly.py (Lawson's algorithm).
-constexpr float kExp2C0 = 0.9999280571937561f;
-constexpr float kExp2C1 = 0.6932609677314758f;
-constexpr float kExp2C2 = 0.24261093139648438f;
-constexpr float kExp2C3 = 0.05517149344086647f;
-constexpr float kRoundMagic = 12582912.0f;  // 1.5 * 2^23: x + magic rounds x to an integer in the low bits
-
-// 2^x for a pair of x in [-125, 126] on the FMA/ALU pipes: x = j + f with j
-// the nearest integer (magic-number rounding) and f in [-1/2, 1/2]; 2^f by
-// the polynomial above; 2^j added to the exponent field in integer form.
-// Relieves the SFU, which would otherwise bound the softmax.
-__device__ __forceinline__ float2 exp2_poly_x2(float2 x) {
-  x.x = fmaxf(x.x, -125.0f);
-  x.y = fmaxf(x.y, -125.0f);
-  const uint64_t xx = f2_pack(x.x, x.y);
-  const uint64_t t = f2_add(xx, f2_pack(kRoundMagic, kRoundMagic));
-  const uint64_t j = f2_add(t, f2_pack(-kRoundMagic, -kRoundMagic));
-  const uint64_t f = f2_fma(j, f2_pack(-1.0f, -1.0f), xx);
-  uint64_t p = f2_fma(f, f2_pack(kExp2C3, kExp2C3), f2_pack(kExp2C2, kExp2C2));
-  p = f2_fma(p, f, f2_pack(kExp2C1, kExp2C1));
-  p = f2_fma(p, f, f2_pack(kExp2C0, kExp2C0));
-  const float2 tf = f2_unpack(t);
-  const float2 pf = f2_unpack(p);
-  // the integer j sits in the low mantissa bits of t; (t << 23) moves it into
-  // the exponent field (the magic constant's own bits shift out).
-  return make_float2(__uint_as_float(__float_as_uint(pf.x) + (__float_as_uint(tf.x) << 23)),
-                     __uint_as_float(__float_as_uint(pf.y) + (__float_as_uint(tf.y) << 23)));
-}
-
-// Pairs (of 16 in a 32-column chunk) whose exponentials go through
-// exp2_poly_x2 on the FMA pipe; the rest use the SFU.
-#ifndef COSMOT_ATTN_POLY_PAIRS
-#define COSMOT_ATTN_POLY_PAIRS 6
-#endif
-constexpr int kPolyPairs = COSMOT_ATTN_POLY_PAIRS;
-
-// One 32-column chunk of P: p = 2^(s * sl2 - mu).  With kPoly, kPolyPairs of
-// the 16 pairs go through exp2_poly_x2 and the rest through the SFU; masked
-// tiles use the SFU only, so masked entries (-inf) become exact zeros.
-template <bool kPoly>
-__device__ __forceinline__ void softmax_chunk(const uint32_t* s, uint64_t sl2x2, uint64_t nmux2, uint32_t* pk,
-                                              uint64_t& acc) {
-#pragma unroll
-  for (int e = 0; e < 16; ++e) {
-    const uint64_t x2 = f2_fma(f2_pack(__uint_as_float(s[2 * e]), __uint_as_float(s[2 * e + 1])), sl2x2, nmux2);
-    float2 pp;
-    if (kPoly && (e % 16) * kPolyPairs / 16 != ((e % 16) + 1) * kPolyPairs / 16) {
-      pp = exp2_poly_x2(f2_unpack(x2));
-    } else {
-      const float2 xf = f2_unpack(x2);
-      pp = make_float2(ex2_approx(xf.x), ex2_approx(xf.y));
-    }
-    acc = f2_add(acc, f2_pack(pp.x, pp.y));
-    pk[e] = pack_bf16x2(pp.x, pp.y);
-  }
-}
 
 template <int HD>
 struct Cfg {
@@ -164,8 +113,6 @@ __device__ __forceinline__ Work decode_work(const Params& p) {
   return w;
 }
 
-// 320 threads, one CTA per SM.  Registers are granted per group of four
-// warps, so ten warps are charged as twelve: 168 registers per thread.
 template <int HD>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
     mot_attention_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__ CUtensorMap tmap_k,
@@ -346,40 +293,25 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         break;
       }
       tc_fence_after();
+      uint32_t s[128];
+      tmem_ld32(s_addr + 0, *reinterpret_cast<uint32_t(*)[32]>(&s[0]));
+      tmem_ld32(s_addr + 32, *reinterpret_cast<uint32_t(*)[32]>(&s[32]));
+      tmem_ld32(s_addr + 64, *reinterpret_cast<uint32_t(*)[32]>(&s[64]));
+      tmem_ld32(s_addr + 96, *reinterpret_cast<uint32_t(*)[32]>(&s[96]));
+      tmem_ld_wait();
       const int64_t kbase = (int64_t)j * BKV;
-      const bool masked_row = kbase + BKV > klimit || (bc_dm && kbase + BKV > p.n_ar);
-      const bool masked = __any_sync(0xffffffffu, masked_row);  // selects a code path with collectives
-      // Reads 64 columns of S from TMEM; masked entries become -inf.
-      auto load_half = [&](int h0, uint32_t (&sv)[64]) {
-        tmem_ld32(s_addr + h0, *reinterpret_cast<uint32_t(*)[32]>(&sv[0]));
-        tmem_ld32(s_addr + h0 + 32, *reinterpret_cast<uint32_t(*)[32]>(&sv[32]));
-        tmem_ld_wait();
-        if (masked_row) {
+      if (kbase + BKV > klimit || (bc_dm && kbase + BKV > p.n_ar)) {
 #pragma unroll
-          for (int c = 0; c < 64; ++c) {
-            const int64_t key = kbase + h0 + c;
-            bool vis = key < klimit;
-            if (bc_dm && key >= p.n_ar && vis) vis = __ldg(p.chunk + key) <= my_chunk;
-            if (!vis) sv[c] = __float_as_uint(-INFINITY);
-          }
-        }
-      };
-      // pass 1: row max
-      float mx[4];
-#pragma unroll
-      for (int k = 0; k < 4; ++k) mx[k] = -INFINITY;
-#pragma unroll
-      for (int h0 = 0; h0 < 128; h0 += 64) {
-        uint32_t sv[64];
-        load_half(h0, sv);
-#pragma unroll
-        for (int c = 0; c < 64; c += 8) {
-#pragma unroll
-          for (int k = 0; k < 4; ++k)
-            mx[k] = fmax3(mx[k], __uint_as_float(sv[c + 2 * k]), __uint_as_float(sv[c + 2 * k + 1]));
+        for (int c = 0; c < 128; ++c) {
+          const int64_t key = kbase + c;
+          bool vis = key < klimit;
+          if (bc_dm && key >= p.n_ar && vis) vis = __ldg(p.chunk + key) <= my_chunk;
+          if (!vis) s[c] = __float_as_uint(-INFINITY);
         }
       }
-      const float mt = fmax3(fmaxf(mx[0], mx[1]), mx[2], mx[3]);
+      float mt = -INFINITY;
+#pragma unroll
+      for (int c = 0; c < 128; ++c) mt = fmaxf(mt, __uint_as_float(s[c]));
       const float m_new = fmaxf(m, mt * sl2);
       const bool first = (m == -INFINITY);
       const bool need = !first && (m_new > m + kRescaleThreshold);
@@ -404,28 +336,20 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         tmem_st_wait();
       }
       const float mu = (m == -INFINITY) ? 0.f : m;
-      const uint64_t sl2x2 = f2_pack(sl2, sl2), nmux2 = f2_pack(-mu, -mu);
-      uint64_t acc[4];
+      float rs = 0.f;
 #pragma unroll
-      for (int k = 0; k < 4; ++k) acc[k] = f2_pack(0.f, 0.f);
-      // pass 2: P = 2^(s*sl2 - mu) as packed bf16 over the first 64 columns of S
+      for (int c0 = 0; c0 < 128; c0 += 32) {
+        uint32_t pk[16];
 #pragma unroll
-      for (int h0 = 0; h0 < 128; h0 += 64) {
-        uint32_t sv[64];
-        load_half(h0, sv);
-#pragma unroll
-        for (int c0 = 0; c0 < 64; c0 += 32) {
-          uint32_t pk[16];
-          if (masked)
-            softmax_chunk<false>(sv + c0, sl2x2, nmux2, pk, acc[(h0 + c0) >> 5]);
-          else
-            softmax_chunk<true>(sv + c0, sl2x2, nmux2, pk, acc[(h0 + c0) >> 5]);
-          tmem_st16(s_addr + ((h0 + c0) >> 1), pk);
+        for (int e = 0; e < 16; ++e) {
+          const float p0 = ex2_approx(fmaf(__uint_as_float(s[c0 + 2 * e]), sl2, -mu));
+          const float p1 = ex2_approx(fmaf(__uint_as_float(s[c0 + 2 * e + 1]), sl2, -mu));
+          rs += p0 + p1;
+          pk[e] = pack_bf16x2(p0, p1);
         }
+        tmem_st16(s_addr + (c0 >> 1), pk);
       }
-      const float2 a01 = f2_unpack(f2_add(acc[0], acc[1]));
-      const float2 a23 = f2_unpack(f2_add(acc[2], acc[3]));
-      l += (a01.x + a01.y) + (a23.x + a23.y);
+      l += rs;
       tmem_st_wait();
       tc_fence_before();
       mbar_arrive(bar_p_full + 8 * t);
