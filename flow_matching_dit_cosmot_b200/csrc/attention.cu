@@ -280,13 +280,28 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     const bool bc_dm = !w.is_ar && p.mask_mode == COSMOT_MASK_BLOCK_CAUSAL;
     int64_t klimit = p.n_keys;
     if (w.is_ar) klimit = qk + 1 < p.n_ar ? qk + 1 : p.n_ar;
-    const int32_t my_chunk = (bc_dm && valid) ? __ldg(p.chunk + qk) : 0;
+    // Rows past the segment are padding (never stored): they see everything,
+    // so they never force the element-mask path on their warp.
+    const int32_t my_chunk = bc_dm ? (valid ? __ldg(p.chunk + qk) : INT32_MAX) : 0;
     const uint32_t s_addr = tmem_base + ((uint32_t)lane_base << 16) + C::s_col(t);
     const uint32_t o_addr = tmem_base + ((uint32_t)lane_base << 16) + C::o_col(t);
     const float sl2 = p.scale_log2;
     float m = -INFINITY, l = 0.f;
     bool ok = true;
     for (int j = 0; j < n_kt; ++j) {
+      const int64_t kbase = (int64_t)j * BKV;
+      // Block-causal rows need element masks only where the tile holds a DM
+      // key of a later chunk.  The warp reads the tile's 128 chunk ids (AR keys
+      // and keys past the end count as visible) before waiting for S, so the
+      // load latency hides behind the wait; the max is reduced after it.
+      int32_t ck[4] = {INT32_MIN, INT32_MIN, INT32_MIN, INT32_MIN};
+      if (bc_dm) {
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const int64_t key = kbase + lane + 32 * i;
+          if (key >= p.n_ar && key < p.n_keys) ck[i] = __ldg(p.chunk + key);
+        }
+      }
       // Warp-uniform decisions only: every tcgen05.ld/st below is .sync.aligned.
       if (!__all_sync(0xffffffffu, mbar_wait(bar_s_full + 8 * t, j & 1, p.status, kWhereAttnSoftmax))) {
         ok = false;
@@ -299,8 +314,14 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       tmem_ld32(s_addr + 64, *reinterpret_cast<uint32_t(*)[32]>(&s[64]));
       tmem_ld32(s_addr + 96, *reinterpret_cast<uint32_t(*)[32]>(&s[96]));
       tmem_ld_wait();
-      const int64_t kbase = (int64_t)j * BKV;
-      if (kbase + BKV > klimit || (bc_dm && kbase + BKV > p.n_ar)) {
+      bool chunk_mask = false;
+      if (bc_dm) {
+        int32_t tmax = max(max(ck[0], ck[1]), max(ck[2], ck[3]));
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) tmax = max(tmax, __shfl_xor_sync(0xffffffffu, tmax, off));
+        chunk_mask = tmax > my_chunk;
+      }
+      if (kbase + BKV > klimit || chunk_mask) {
 #pragma unroll
         for (int c = 0; c < 128; ++c) {
           const int64_t key = kbase + c;
