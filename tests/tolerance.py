@@ -7,12 +7,14 @@ the arithmetic; two terms come on top of it, both derived from bf16 storage:
 
   * the output's own rounding to bf16: half an ulp of the reference value
     (at |x| >= 8 that alone is 0.031, above 2e-2);
-  * for outputs downstream of reductions whose *inputs* were stored in bf16
-    (the normalised activations and the gated FFN hidden state of a layer),
+  * for outputs downstream of reductions whose *inputs* were stored in bf16,
     each such rounding point adds an error of standard deviation about
     2^-9/sqrt(3) * rms(branch) (first-order propagation of a uniform relative
     rounding error through a long dot product), whose maximum over ~1e8
-    elements is about 6 sigma.  `rounded_inputs` counts those points.
+    elements is about 6 sigma.  `rounded_inputs` counts those points.  A
+    layer's h_out crosses three on its FFN path: the normalised FFN input
+    feeds both factors of the gated product (two) and the gated hidden state
+    feeds the down projection (one).
 
 A sampler loop stores its running state in bf16 after every step and feeds
 it back through the layer.  The stated bounds hold per step (every layer test
