@@ -123,6 +123,23 @@ def stream_layout_spec(wl, block: int):
                 tau_offset=block)
 
 
+def reduce_max(value: float, device=None) -> float:
+    """Max of `value` over all ranks (the job's time is its slowest rank's);
+    the value itself on a single process."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return float(value)
+    t = torch.tensor([float(value)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_throughput(tokens_per_rank_step: int, steps: int, world: int, max_ms: float) -> float:
+    """Whole-job tokens/s: every rank's tokens over the slowest rank's time."""
+    return world * tokens_per_rank_step * steps / (max_ms / 1e3)
+
+
 def load_peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(path):
@@ -547,22 +564,15 @@ def run_native(args, wl):
             out_pin.copy_(src_out, non_blocking=True)
             e_e[i].record(stream)
         torch.cuda.synchronize()
-        e2e_ms = sum(e_s[i].elapsed_time(e_e[i]) for i in range(args.steps))
-        if world > 1:
-            t = torch.tensor([e2e_ms], device=dev, dtype=torch.float64)
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            e2e_ms = float(t.item())
-        e2e = {"value": world * tokens_per_step * args.steps / (e2e_ms / 1e3), "unit": UNIT,
+        e2e_ms = reduce_max(sum(e_s[i].elapsed_time(e_e[i]) for i in range(args.steps)), dev)
+        e2e = {"value": job_throughput(tokens_per_step, args.steps, world, e2e_ms), "unit": UNIT,
                "h2d_bytes_per_step": int(in_pin.numel() * 2), "d2h_bytes_per_step": int(out_pin.numel() * 2),
                "ms_per_step": e2e_ms / args.steps,
                "path": "cosmot_build_layout + cosmot_mrope_table + cosmot_layer_forward"
                        + (" + cosmot_layer_commit_kv" if kind == "stream" else "")
                        + ", pinned host input in, x' (noisy rows) out"}
 
-    if world > 1:
-        t = torch.tensor([total_ms], device=dev, dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        total_ms = float(t.item())
+    total_ms = reduce_max(total_ms, dev)
 
     if rank == 0:
         names = L.STAGE_NAMES
@@ -610,7 +620,7 @@ def run_native(args, wl):
                     "unit": "GB/s", "frac": round(achieved / peak_bw, 3), "traffic": traffic,
                     "algorithmic_bytes_per_launch": b // per_launch, "launches_per_step": per_launch,
                     "peak_source": f"{peak_src} hbm_gbs"}
-        value = world * tokens_per_step * args.steps / (total_ms / 1e3)
+        value = job_throughput(tokens_per_step, args.steps, world, total_ms)
         layer_tflops = flops_total / (ms_step / 1e3) / 1e12
         cfg = config_block(wl, lay, world)
         cfg["step"] = {"layer": "one layer forward + Euler step",
