@@ -231,6 +231,33 @@ def euler_step(x, v, sigma, sigma_next):
     return np.asarray(x, np.float64) + (float(sigma_next) - float(sigma)) * np.asarray(v, np.float64)
 
 
+def cfg_combine(v_cond, v_base, guidance):
+    """Classifier-free guidance ("Cosmos 3 方法原理全解" §7.2):
+    v = v_base + w * (v_cond - v_base)."""
+    v_cond = np.asarray(v_cond, np.float64)
+    v_base = np.asarray(v_base, np.float64)
+    return v_base + float(guidance) * (v_cond - v_base)
+
+
+def cfg_step(dims, W, h_cond, h_base, lay, sigma, sigma_next, guidance, mode="full"):
+    """One guided sampler step ("Cosmos 3 方法原理全解" §7.2-7.3): two Generator
+    forwards that share the DM rows (the state x) and differ in their AR rows
+    (the prompt and the baseline prompt), the guided velocity, one Euler step.
+
+    Reading: both AR sequences have the same length (the baseline prompt is
+    padded to the prompt's length), so the two passes share one layout.
+    Returns x' of the noisy rows and both passes' outputs.
+    """
+    noisy = lay.region == REGION_NOISY
+    if not np.array_equal(np.asarray(h_cond)[lay.n_ar:], np.asarray(h_base)[lay.n_ar:]):
+        raise ValueError("the two guidance passes must share their DM rows")
+    oc = layer_forward(dims, W, h_cond, lay.region, lay.pos, lay.chunk, sigma, sigma_next, mode)
+    ob = layer_forward(dims, W, h_base, lay.region, lay.pos, lay.chunk, sigma, sigma_next, mode)
+    v = cfg_combine(oc["vel"][noisy], ob["vel"][noisy], guidance)
+    x = np.asarray(h_cond, np.float64)[noisy]
+    return euler_step(x, v, sigma, sigma_next), oc, ob
+
+
 def sample(dims, W, h, lay, sigmas, mode="full"):
     """Sampler loop: one layer forward and one Euler step per (sigma, sigma_next).
 

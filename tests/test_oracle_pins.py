@@ -443,6 +443,43 @@ def test_sampler_loop_equals_repeated_steps():
     np.testing.assert_array_equal(hf[~noisy], h[~noisy])
 
 
+# ---------------------------------------------------------------- guidance
+
+def _cfg_case():
+    lay = _small_layout(video=VideoSpec(1, 2, 2, 24, 1, 2))
+    W = _weights(TINY)
+    hc = _h(lay.n_tokens, TINY.d_model, seed=21)
+    hb = hc.copy()
+    hb[:lay.n_ar] = _h(lay.n_ar, TINY.d_model, seed=22)  # a different prompt, same DM rows
+    return lay, W, hc, hb
+
+
+def test_cfg_limits_reduce_to_single_passes():
+    """w = 1 is the conditioned step, w = 0 the baseline step (§7.2)."""
+    lay, W, hc, hb = _cfg_case()
+    noisy = lay.region == layout.REGION_NOISY
+    x1, oc, ob = layer.cfg_step(TINY, W, hc, hb, lay, 0.8, 0.7, 1.0)
+    np.testing.assert_allclose(x1, oc["x_new"][noisy], rtol=0, atol=1e-13)
+    x0, _, _ = layer.cfg_step(TINY, W, hc, hb, lay, 0.8, 0.7, 0.0)
+    np.testing.assert_allclose(x0, ob["x_new"][noisy], rtol=0, atol=1e-13)
+    assert np.abs(x1 - x0).max() > 1e-4, "the prompt must matter"
+
+
+def test_cfg_is_affine_in_guidance_and_inert_for_equal_prompts():
+    lay, W, hc, hb = _cfg_case()
+    xs = [layer.cfg_step(TINY, W, hc, hb, lay, 0.8, 0.7, g)[0] for g in (0.0, 3.0, 6.0)]
+    np.testing.assert_allclose(xs[2] - xs[1], xs[1] - xs[0], rtol=0, atol=1e-12)
+    # guidance weight w extrapolates past the conditioned velocity: x(6) - x(0) = 6 (x(1) - x(0))
+    x1 = layer.cfg_step(TINY, W, hc, hb, lay, 0.8, 0.7, 1.0)[0]
+    np.testing.assert_allclose(xs[2] - xs[0], 6.0 * (x1 - xs[0]), rtol=0, atol=1e-12)
+    same = [layer.cfg_step(TINY, W, hc, hc, lay, 0.8, 0.7, g)[0] for g in (0.0, 7.5)]
+    np.testing.assert_allclose(same[0], same[1], rtol=0, atol=1e-13)
+    with pytest.raises(ValueError):
+        hb2 = hb.copy()
+        hb2[-1] += 1.0
+        layer.cfg_step(TINY, W, hc, hb2, lay, 0.8, 0.7, 2.0)
+
+
 # ---------------------------------------------------------------- streaming
 
 def test_stream_cache_equals_block_causal_sequence():
