@@ -276,7 +276,8 @@ def oracle_sample(wl, quick: bool = False):
         fixed = max(t[0] - rows_lo * per_row, 0.0)
         return ((fixed + per_row * lay.n_tokens) * wl.batch, sum(t),
                 f"oracle layer forward on {rows_lo} and {rows_hi} noisy query rows (K/V of all {lay.n_tokens} "
-                f"rows each), extrapolated linearly to all rows and the batch")
+                f"rows each), extrapolated linearly to all rows and the batch"
+                + (" (both passes of each guided pair; the guided combine is not timed)" if wl.guidance else ""))
     if kind == "sampler":
         # The oracle recomputes every row at every step, so its steps cost the
         # same: time one and scale by the step count.
@@ -360,6 +361,7 @@ def config_block(wl, lay, n_gpus):
             "d_model": wl.dims.d_model, "heads": wl.dims.n_heads, "head_dim": wl.dims.head_dim,
             "ffn": wl.dims.ffn, "n_ar": lay.n_ar, "n_clean": lay.n_clean, "n_noisy": lay.n_noisy,
             "mask": wl.mask_mode, "sigma": [wl.sigmas[0], wl.sigmas[1]],
+            **({"guidance": wl.guidance, "prompt_pairs": wl.batch // 2} if wl.guidance is not None else {}),
             "l2": "flushed between steps (256 MiB write, outside the timed events)"}
 
 
@@ -411,6 +413,9 @@ def run_native(args, wl):
 
     w = {k: to_dev(v) for k, v in synth.make_weights(dims_s, wl.weight_seed).items()}
     h_host = np.stack([synth.make_activations(N, d, wl.act_seed(rank * B + b)) for b in range(B)])
+    guided = wl.guidance is not None
+    if guided:  # each (cond, base) pair shares its DM rows; the prompts (AR rows) differ
+        h_host[1::2, lay.n_ar:] = h_host[0::2, lay.n_ar:]
     h = to_dev(h_host)
     h_out = torch.empty_like(h)
     pos = torch.empty((N, 3), dtype=torch.float32, device=dev)
@@ -466,12 +471,16 @@ def run_native(args, wl):
         L.cosmot_mrope_table(pos.data_ptr(), N, dims_s.head_dim, dims_s.rope_sections, dims_s.rope_base,
                              cs.data_ptr(), sh)
         for i, (c, s0, s1) in enumerate(calls):
-            if stage_evs is None:
+            if stage_evs is not None:
+                L.cosmot_layer_forward_timed(dims, layer.cw, seqs[c], h.data_ptr(), h_out.data_ptr(), s0, s1,
+                                             ws.data_ptr(), ws.numel(), sh, [e.cuda_event for e in stage_evs[i]],
+                                             wl.guidance)
+            elif guided:
+                L.cosmot_layer_forward_cfg(dims, layer.cw, seqs[c], h.data_ptr(), h_out.data_ptr(), s0, s1,
+                                           wl.guidance, ws.data_ptr(), ws.numel(), sh)
+            else:
                 L.cosmot_layer_forward(dims, layer.cw, seqs[c], h.data_ptr(), h_out.data_ptr(), s0, s1,
                                        ws.data_ptr(), ws.numel(), sh)
-            else:
-                L.cosmot_layer_forward_timed(dims, layer.cw, seqs[c], h.data_ptr(), h_out.data_ptr(), s0, s1,
-                                             ws.data_ptr(), ws.numel(), sh, [e.cuda_event for e in stage_evs[i]])
         if kind == "stream":
             if commit_evs is not None:
                 commit_evs[0].record(stream)
@@ -568,7 +577,8 @@ def run_native(args, wl):
         e2e = {"value": job_throughput(tokens_per_step, args.steps, world, e2e_ms), "unit": UNIT,
                "h2d_bytes_per_step": int(in_pin.numel() * 2), "d2h_bytes_per_step": int(out_pin.numel() * 2),
                "ms_per_step": e2e_ms / args.steps,
-               "path": "cosmot_build_layout + cosmot_mrope_table + cosmot_layer_forward"
+               "path": "cosmot_build_layout + cosmot_mrope_table + "
+                       + ("cosmot_layer_forward_cfg" if guided else "cosmot_layer_forward")
                        + (" + cosmot_layer_commit_kv" if kind == "stream" else "")
                        + ", pinned host input in, x' (noisy rows) out"}
 
@@ -623,7 +633,8 @@ def run_native(args, wl):
         value = job_throughput(tokens_per_step, args.steps, world, total_ms)
         layer_tflops = flops_total / (ms_step / 1e3) / 1e12
         cfg = config_block(wl, lay, world)
-        cfg["step"] = {"layer": "one layer forward + Euler step",
+        cfg["step"] = {"layer": ("one guided layer step: both passes of each prompt pair, the guided velocity "
+                                  "and one Euler step" if guided else "one layer forward + Euler step"),
                        "sampler": f"one {len(calls)}-step Euler sampling (step 1 all rows, then DM rows with the "
                                   f"AR K/V kept in the workspace)",
                        "stream": f"one streaming block: {len(calls)} denoising steps of {lay.n_noisy} tokens "

@@ -96,6 +96,10 @@ SIGNATURES = {
     "cosmot_mrope_apply": (c_i32, [c_vp, c_i64, c_i32, c_vp, c_i64, c_i32, c_i64, c_i32, c_vp, c_vp]),
     "cosmot_mot_attention": (c_i32, [_P(AttnDesc), c_vp, c_i64, c_vp, c_vp, c_i64, c_vp, c_i64, c_vp]),
     "cosmot_flow_euler_step": (c_i32, [c_vp, c_i64, c_vp, c_i64, c_i64, c_i64, c_i64, c_f64, c_f64, c_vp]),
+    "cosmot_flow_cfg_euler_step": (c_i32, [c_vp, c_vp, c_i64, c_vp, c_vp, c_i64, c_i64, c_i64, c_f64, c_f64, c_f64,
+                                           c_vp]),
+    "cosmot_layer_forward_cfg": (c_i32, [_P(Dims), _P(LayerWeights), _P(SeqDesc), c_vp, c_vp, c_f64, c_f64, c_f64,
+                                         c_vp, ctypes.c_size_t, c_vp]),
     "cosmot_layer_workspace_size": (c_i32, [_P(Dims), _P(SeqDesc), _P(ctypes.c_size_t)]),
     "cosmot_layer_forward": (c_i32, [_P(Dims), _P(LayerWeights), _P(SeqDesc), c_vp, c_vp, c_f64, c_f64, c_vp,
                                      ctypes.c_size_t, c_vp]),
@@ -104,7 +108,7 @@ SIGNATURES = {
     "cosmot_layer_forward_noalloc": (c_i32, [_P(Dims), _P(LayerWeights), _P(SeqDesc), c_vp, c_vp, c_f64, c_f64,
                                              c_vp]),
     "cosmot_layer_forward_timed": (c_i32, [_P(Dims), _P(LayerWeights), _P(SeqDesc), c_vp, c_vp, c_f64, c_f64, c_vp,
-                                           ctypes.c_size_t, c_vp, _P(c_vp), c_i32]),
+                                           ctypes.c_size_t, c_vp, _P(c_vp), c_i32, _P(c_f64)]),
 }
 
 COSMOT_LAYER_STAGES = 9
@@ -220,6 +224,20 @@ def cosmot_flow_euler_step(x: int, ld_x: int, v: int, ld_v: int, row_begin: int,
                  sigma_next, c_vp(stream), check=check)
 
 
+def cosmot_flow_cfg_euler_step(x_cond: int, x_base: int, ld_x: int, v_cond: int, v_base: int, ld_v: int, n_rows: int,
+                               n_cols: int, sigma: float, sigma_next: float, guidance: float, stream: int = 0,
+                               check=True):
+    return _call("cosmot_flow_cfg_euler_step", c_vp(x_cond), c_vp(x_base), ld_x, c_vp(v_cond), c_vp(v_base), ld_v,
+                 n_rows, n_cols, sigma, sigma_next, guidance, c_vp(stream), check=check)
+
+
+def cosmot_layer_forward_cfg(dims: Dims, w: LayerWeights, seq: SeqDesc, h: int, h_out: int, sigma: float,
+                             sigma_next: float, guidance: float, workspace: int, workspace_bytes: int, stream: int = 0,
+                             check=True):
+    return _call("cosmot_layer_forward_cfg", ctypes.byref(dims), ctypes.byref(w), ctypes.byref(seq), c_vp(h),
+                 c_vp(h_out), sigma, sigma_next, guidance, c_vp(workspace), workspace_bytes, c_vp(stream), check=check)
+
+
 def cosmot_layer_workspace_size(dims: Dims, seq: SeqDesc) -> int:
     n = ctypes.c_size_t(0)
     _call("cosmot_layer_workspace_size", ctypes.byref(dims), ctypes.byref(seq), ctypes.byref(n))
@@ -247,9 +265,11 @@ def cosmot_layer_forward_noalloc(dims: Dims, w: LayerWeights, seq: SeqDesc, h: i
 
 def cosmot_layer_forward_timed(dims: Dims, w: LayerWeights, seq: SeqDesc, h: int, h_out: int, sigma: float,
                                sigma_next: float, workspace: int, workspace_bytes: int, stream: int, events,
-                               check=True):
-    """`events`: COSMOT_LAYER_STAGES + 1 raw cudaEvent_t handles (ints)."""
+                               guidance: float | None = None, check=True):
+    """`events`: COSMOT_LAYER_STAGES + 1 raw cudaEvent_t handles (ints); `guidance`
+    selects the guided step of cosmot_layer_forward_cfg."""
     arr = (c_vp * len(events))(*[c_vp(e) for e in events])
+    g = ctypes.byref(c_f64(guidance)) if guidance is not None else None
     return _call("cosmot_layer_forward_timed", ctypes.byref(dims), ctypes.byref(w), ctypes.byref(seq), c_vp(h),
-                 c_vp(h_out), sigma, sigma_next, c_vp(workspace), workspace_bytes, c_vp(stream), arr, len(events),
+                 c_vp(h_out), sigma, sigma_next, c_vp(workspace), workspace_bytes, c_vp(stream), arr, len(events), g,
                  check=check)

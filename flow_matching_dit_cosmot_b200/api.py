@@ -110,6 +110,14 @@ class MoTLayer:
         ws = workspace if workspace is not None else self.workspace(seq, h.device)
         L.cosmot_layer_commit_kv(self.dims, self.cw, seq, ptr(h), dst_row, ptr(ws), ws.numel(), stream_handle(stream))
 
+    def forward_cfg(self, h: torch.Tensor, h_out: torch.Tensor, sigma: float, sigma_next: float, guidance: float,
+                    seq: L.SeqDesc, workspace: Optional[torch.Tensor] = None, stream=None):
+        """Guided step: h [2P, N, d] holds (conditioned, baseline) pairs sharing their DM rows."""
+        _need_cuda(h, h_out)
+        ws = workspace if workspace is not None else self.workspace(seq, h.device)
+        L.cosmot_layer_forward_cfg(self.dims, self.cw, seq, ptr(h), ptr(h_out), float(sigma), float(sigma_next),
+                                   float(guidance), ptr(ws), ws.numel(), stream_handle(stream))
+
     def forward(self, h: torch.Tensor, h_out: torch.Tensor, sigma: float, sigma_next: float, seq: L.SeqDesc,
                 workspace: Optional[torch.Tensor] = None, stream=None):
         """h [batch, N, d] bf16 (noisy DM rows updated in place to x'); h_out [batch, N, d] bf16."""

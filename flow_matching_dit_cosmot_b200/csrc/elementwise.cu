@@ -1,6 +1,7 @@
-// HBM-bound kernels: routed RMSNorm, standalone mRoPE, the Euler sampler step.
+// HBM-bound kernels: routed RMSNorm, standalone mRoPE, the Euler sampler step
+// and its guided form.
 //
-// All three stream 16-byte vectors (8 bf16) per thread with fully coalesced
+// All of them stream 16-byte vectors (8 bf16) per thread with fully coalesced
 // warps; grids are sized in multiples of the SM count.
 #include <cuda_bf16.h>
 
@@ -167,6 +168,39 @@ __global__ void __launch_bounds__(256) euler_kernel(__nv_bfloat16* __restrict__ 
   }
 }
 
+// ---------------------------------------------------------------- guided Euler
+// x' = x + dsigma * (v_base + w * (v_cond - v_base)), written to both states of
+// a (conditioned, baseline) pair so they stay identical for the next step.
+__global__ void __launch_bounds__(256) cfg_euler_kernel(__nv_bfloat16* x_cond, __nv_bfloat16* x_base,
+                                                        int64_t ld_x,
+                                                        const __nv_bfloat16* __restrict__ v_cond,
+                                                        const __nv_bfloat16* __restrict__ v_base, int64_t ld_v,
+                                                        int64_t n_rows, int64_t n_cols, float dsigma, float w) {
+  const int64_t vec_per_row = n_cols >> 3;
+  const int64_t total = n_rows * vec_per_row;
+  for (int64_t e = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; e < total; e += (int64_t)gridDim.x * blockDim.x) {
+    const int64_t r = e / vec_per_row;
+    const int64_t c = (e % vec_per_row) << 3;
+    uint4 xv = *reinterpret_cast<const uint4*>(x_cond + r * ld_x + c);
+    const uint4 vc = __ldg(reinterpret_cast<const uint4*>(v_cond + r * ld_v + c));
+    const uint4 vb = __ldg(reinterpret_cast<const uint4*>(v_base + r * ld_v + c));
+    uint32_t* xu = reinterpret_cast<uint32_t*>(&xv);
+    const uint32_t* cu = reinterpret_cast<const uint32_t*>(&vc);
+    const uint32_t* bu = reinterpret_cast<const uint32_t*>(&vb);
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const float2 a = unpack_bf16x2(xu[j]);
+      const float2 fc = unpack_bf16x2(cu[j]);
+      const float2 fb = unpack_bf16x2(bu[j]);
+      const float v0 = fmaf(w, fc.x - fb.x, fb.x);
+      const float v1 = fmaf(w, fc.y - fb.y, fb.y);
+      xu[j] = pack_bf16x2(fmaf(dsigma, v0, a.x), fmaf(dsigma, v1, a.y));
+    }
+    *reinterpret_cast<uint4*>(x_cond + r * ld_x + c) = xv;
+    *reinterpret_cast<uint4*>(x_base + r * ld_x + c) = xv;
+  }
+}
+
 unsigned grid_for(int64_t work_items, int threads) {
   const int64_t want = (work_items + threads - 1) / threads;
   const int64_t cap = (int64_t)num_sms() * 16;
@@ -244,6 +278,23 @@ cosmot_status cosmot_flow_euler_step(void* x, int64_t ld_x, const void* v, int64
   euler_kernel<<<grid_for(items, threads), threads, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
       static_cast<__nv_bfloat16*>(x), ld_x, static_cast<const __nv_bfloat16*>(v), ld_v, row_begin,
       row_end - row_begin, n_cols, dsigma);
+  return launch_status();
+}
+
+cosmot_status cosmot_flow_cfg_euler_step(void* x_cond, void* x_base, int64_t ld_x, const void* v_cond,
+                                         const void* v_base, int64_t ld_v, int64_t n_rows, int64_t n_cols,
+                                         double sigma, double sigma_next, double guidance, cosmot_stream_t stream) {
+  using namespace cosmot;
+  if (!x_cond || !x_base || !v_cond || !v_base || n_rows < 0 || n_cols <= 0) return COSMOT_ERR_INVALID_ARG;
+  if (n_cols % 8 || ld_x % 8 || ld_v % 8 || ld_x < n_cols || ld_v < n_cols) return COSMOT_ERR_INVALID_ARG;
+  if (!aligned16(x_cond) || !aligned16(x_base) || !aligned16(v_cond) || !aligned16(v_base)) return COSMOT_ERR_INVALID_ARG;
+  const int64_t items = n_rows * (n_cols / 8);
+  if (items == 0) return COSMOT_OK;
+  const int threads = 256;
+  cfg_euler_kernel<<<grid_for(items, threads), threads, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
+      static_cast<__nv_bfloat16*>(x_cond), static_cast<__nv_bfloat16*>(x_base), ld_x,
+      static_cast<const __nv_bfloat16*>(v_cond), static_cast<const __nv_bfloat16*>(v_base), ld_v, n_rows, n_cols,
+      (float)(sigma_next - sigma), (float)guidance);
   return launch_status();
 }
 

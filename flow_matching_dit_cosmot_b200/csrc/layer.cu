@@ -121,7 +121,8 @@ struct StageMarks {
 
 cosmot_status layer_forward_impl(const cosmot_dims* dims, const cosmot_layer_weights* w, const cosmot_seq_desc* seq,
                                  void* h, void* h_out, double sigma, double sigma_next, void* workspace,
-                                 size_t workspace_bytes, cosmot_stream_t stream, const cudaEvent_t* events) {
+                                 size_t workspace_bytes, cosmot_stream_t stream, const cudaEvent_t* events,
+                                 const double* guidance = nullptr) {
   const StageMarks M{events, reinterpret_cast<cudaStream_t>(stream)};
   cosmot_status st = check_dims(dims);
   if (st != COSMOT_OK) return st;
@@ -227,6 +228,27 @@ cosmot_status layer_forward_impl(const cosmot_dims* dims, const cosmot_layer_wei
   st = cosmot_rmsnorm_routed(h_out, d, ns_in, B, w->gfin, w->gfin, d, D.eps, a, d, stream);
   if (st != COSMOT_OK) return st;
   if ((st = M.mark(8)) != COSMOT_OK) return st;
+  if (guidance) {
+    // 9'. guided step: velocities of every sequence into the (now free) FFN
+    // hidden region, then v_base + w (v_cond - v_base) and the Euler step for
+    // each (conditioned, baseline) pair, written to both states of the pair.
+    uint16_t* vbuf = static_cast<uint16_t*>(u);
+    const int64_t nz = S.n_noisy;
+    const cosmot_segment all{0, (int64_t)B * nz, 0, 1, 0};
+    e = cosmot_epilogue{};
+    e.kind = COSMOT_EPI_NONE;
+    st = cosmot_routed_linear(a, d, d, &all, 1, w->wvel, w->wvel, nullptr, nullptr, d, vbuf, d, &e, stream);
+    if (st != COSMOT_OK) return st;
+    for (int pr = 0; pr < B / 2; ++pr) {
+      const int64_t zc = (int64_t)(2 * pr) * N + S.n_ar + S.n_clean;
+      const int64_t zb = (int64_t)(2 * pr + 1) * N + S.n_ar + S.n_clean;
+      st = cosmot_flow_cfg_euler_step(hb + zc * d, hb + zb * d, d, vbuf + (int64_t)(2 * pr) * nz * d,
+                                      vbuf + (int64_t)(2 * pr + 1) * nz * d, d, nz, d, sigma, sigma_next, *guidance,
+                                      stream);
+      if (st != COSMOT_OK) return st;
+    }
+    return M.mark(9);
+  }
   // 9. velocity head with the Euler step, in place on the noisy rows of h
   e = cosmot_epilogue{};
   e.kind = COSMOT_EPI_EULER;
@@ -249,6 +271,18 @@ cosmot_status cosmot_layer_forward(const cosmot_dims* dims, const cosmot_layer_w
                                    cosmot_stream_t stream) {
   return cosmot::layer_forward_impl(dims, w, seq, h, h_out, sigma, sigma_next, workspace, workspace_bytes, stream,
                                     nullptr);
+}
+
+cosmot_status cosmot_layer_forward_cfg(const cosmot_dims* dims, const cosmot_layer_weights* w,
+                                       const cosmot_seq_desc* seq, void* h, void* h_out, double sigma,
+                                       double sigma_next, double guidance, void* workspace, size_t workspace_bytes,
+                                       cosmot_stream_t stream) {
+  if (!seq || !dims || seq->batch < 2 || seq->batch % 2) return COSMOT_ERR_INVALID_ARG;
+  // the velocities of all sequences reuse the FFN hidden region of the workspace
+  if ((int64_t)dims->ffn * (seq->n_ar + seq->n_clean + seq->n_noisy) < (int64_t)dims->d_model * seq->n_noisy)
+    return COSMOT_ERR_UNSUPPORTED;
+  return cosmot::layer_forward_impl(dims, w, seq, h, h_out, sigma, sigma_next, workspace, workspace_bytes, stream,
+                                    nullptr, &guidance);
 }
 
 cosmot_status cosmot_layer_commit_kv(const cosmot_dims* dims, const cosmot_layer_weights* w,
@@ -291,12 +325,18 @@ cosmot_status cosmot_layer_commit_kv(const cosmot_dims* dims, const cosmot_layer
 cosmot_status cosmot_layer_forward_timed(const cosmot_dims* dims, const cosmot_layer_weights* w,
                                          const cosmot_seq_desc* seq, void* h, void* h_out, double sigma,
                                          double sigma_next, void* workspace, size_t workspace_bytes,
-                                         cosmot_stream_t stream, void* const* stage_events, int32_t n_events) {
+                                         cosmot_stream_t stream, void* const* stage_events, int32_t n_events,
+                                         const double* guidance) {
   if (!stage_events || n_events != COSMOT_LAYER_STAGES + 1) return COSMOT_ERR_INVALID_ARG;
   for (int i = 0; i < n_events; ++i)
     if (!stage_events[i]) return COSMOT_ERR_INVALID_ARG;
+  if (guidance) {
+    if (!seq || !dims || seq->batch < 2 || seq->batch % 2) return COSMOT_ERR_INVALID_ARG;
+    if ((int64_t)dims->ffn * (seq->n_ar + seq->n_clean + seq->n_noisy) < (int64_t)dims->d_model * seq->n_noisy)
+      return COSMOT_ERR_UNSUPPORTED;
+  }
   return cosmot::layer_forward_impl(dims, w, seq, h, h_out, sigma, sigma_next, workspace, workspace_bytes, stream,
-                                    reinterpret_cast<const cudaEvent_t*>(stage_events));
+                                    reinterpret_cast<const cudaEvent_t*>(stage_events), guidance);
 }
 
 }  // extern "C"

@@ -237,6 +237,20 @@ COSMOT_API cosmot_status cosmot_flow_euler_step(void* x, int64_t ld_x, const voi
                                      int64_t row_end, int64_t n_cols, double sigma, double sigma_next,
                                      cosmot_stream_t stream);
 
+/*
+ * Guided Euler step for a (conditioned, baseline) pair of states
+ * ("Cosmos 3 方法原理全解" §7.2 classifier-free guidance):
+ *     x' = bf16( x + (sigma_next - sigma) * (v_base + w * (v_cond - v_base)) )
+ * computed from x_cond and written to both x_cond and x_base (the two states
+ * are equal on entry and stay equal).  All [n_rows, n_cols] bf16 device arrays;
+ * x_cond/x_base share ld_x, v_cond/v_base share ld_v.  One fp32 FMA for the
+ * guided velocity, one for the step.
+ */
+COSMOT_API cosmot_status cosmot_flow_cfg_euler_step(void* x_cond, void* x_base, int64_t ld_x, const void* v_cond,
+                                                    const void* v_base, int64_t ld_v, int64_t n_rows, int64_t n_cols,
+                                                    double sigma, double sigma_next, double guidance,
+                                                    cosmot_stream_t stream);
+
 /* ===================================================================== layer */
 
 typedef struct {
@@ -305,6 +319,22 @@ COSMOT_API cosmot_status cosmot_layer_forward(const cosmot_dims* dims, const cos
                                    cosmot_stream_t stream);
 
 /*
+ * One guided sampler step ("Cosmos 3 方法原理全解" §7.2-7.3): seq->batch holds
+ * (conditioned, baseline) pairs, sequences 2p and 2p+1, with equal layouts and
+ * equal DM rows (the state x) but different AR rows (the prompt and the
+ * baseline prompt).  Both passes run as one batch of the layer; then the
+ * velocities give v = v_base + guidance * (v_cond - v_base) and x' is written
+ * to the noisy rows of both sequences of every pair.  h_out holds each pass's
+ * h2.  Requires an even batch and ffn * N >= d_model * n_noisy (the velocities
+ * reuse the FFN hidden region of the workspace); otherwise as
+ * cosmot_layer_forward, including n_cached.
+ */
+COSMOT_API cosmot_status cosmot_layer_forward_cfg(const cosmot_dims* dims, const cosmot_layer_weights* w,
+                                                  const cosmot_seq_desc* seq, void* h, void* h_out, double sigma,
+                                                  double sigma_next, double guidance, void* workspace,
+                                                  size_t workspace_bytes, cosmot_stream_t stream);
+
+/*
  * Commit K/V into the workspace's cache: rows [seq.n_cached, N) of every sequence
  * of h go through the pre-attention RMSNorm and the QKV projection with mRoPE
  * (positions of those rows from seq.rope_cs), and the resulting QKV rows are
@@ -366,14 +396,16 @@ enum {
  * is recorded on `stream` just before stage i and stage_events[COSMOT_LAYER_STAGES]
  * after the last one, so cudaEventElapsedTime between consecutive events is the
  * device time of one stage.  The events are cudaEvent_t handles created by the
- * caller on the current device; n_events must be COSMOT_LAYER_STAGES + 1.  The
- * computation is identical to cosmot_layer_forward.
+ * caller on the current device; n_events must be COSMOT_LAYER_STAGES + 1.  With
+ * guidance == NULL the computation is identical to cosmot_layer_forward; with
+ * a guidance weight it is that of cosmot_layer_forward_cfg (the last stage then
+ * covers the velocity GEMM and the guided Euler step).
  */
 COSMOT_API cosmot_status cosmot_layer_forward_timed(const cosmot_dims* dims, const cosmot_layer_weights* w,
                                                     const cosmot_seq_desc* seq, void* h, void* h_out, double sigma,
                                                     double sigma_next, void* workspace, size_t workspace_bytes,
                                                     cosmot_stream_t stream, void* const* stage_events,
-                                                    int32_t n_events);
+                                                    int32_t n_events, const double* guidance);
 
 #ifdef __cplusplus
 }

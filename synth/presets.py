@@ -124,6 +124,7 @@ class Workload:
     batch: int = 1
     mask_mode: str = "full"  # "full" | "block_causal"
     stream: Optional[StreamSpec] = None
+    guidance: Optional[float] = None  # classifier-free guidance weight; batch = (cond, base) pairs
     description: str = ""
     extra: dict = field(default_factory=dict)
 
@@ -158,6 +159,12 @@ PRESETS = {
         layout=LayoutSpec(n_text=256, video=VideoSpec(1, 15, 26, 24, 0, 48)),
         sigmas=(1.0, 0.97),
         description="480p text-to-video layer: d 4096, 32x128 heads, FFN 14336; 258 AR + 18720 noisy"),
+    "t2v480_cfg": Workload(
+        name="t2v480_cfg", config_id=2, dims=_NANO_LIKE,
+        layout=LayoutSpec(n_text=256, video=VideoSpec(1, 15, 26, 24, 0, 48)),
+        sigmas=(1.0, 0.97), batch=2, guidance=6.0,
+        description="480p text-to-video guided step: one (cond, base) prompt pair sharing the 18720 noisy "
+                    "rows, guidance 6"),
     "droid": Workload(
         name="droid", config_id=3, dims=_NANO_LIKE,
         layout=LayoutSpec(n_text=128, video=VideoSpec(3, 6, 10, 15, 1, 2),
