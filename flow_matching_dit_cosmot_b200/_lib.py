@@ -95,6 +95,7 @@ SIGNATURES = {
                                      c_i64, _P(Epilogue), c_vp]),
     "cosmot_mrope_apply": (c_i32, [c_vp, c_i64, c_i32, c_vp, c_i64, c_i32, c_i64, c_i32, c_vp, c_vp]),
     "cosmot_mot_attention": (c_i32, [_P(AttnDesc), c_vp, c_i64, c_vp, c_vp, c_i64, c_vp, c_i64, c_vp]),
+    "cosmot_mot_mask_export": (c_i32, [_P(AttnDesc), c_vp, c_vp, c_vp]),
     "cosmot_flow_euler_step": (c_i32, [c_vp, c_i64, c_vp, c_i64, c_i64, c_i64, c_i64, c_f64, c_f64, c_vp]),
     "cosmot_flow_cfg_euler_step": (c_i32, [c_vp, c_vp, c_i64, c_vp, c_vp, c_i64, c_i64, c_i64, c_f64, c_f64, c_f64,
                                            c_vp]),
@@ -215,6 +216,13 @@ def cosmot_mrope_apply(q: int, ld_q: int, n_q_heads: int, k: int, ld_k: int, n_k
 def cosmot_mot_attention(desc: AttnDesc, q: int, ld_q: int, k: int, v: int, ld_kv: int, o: int, ld_o: int,
                          stream: int = 0, check=True):
     return _call("cosmot_mot_attention", ctypes.byref(desc), c_vp(q), ld_q, c_vp(k), c_vp(v), ld_kv, c_vp(o), ld_o,
+                 c_vp(stream), check=check)
+
+
+def cosmot_mot_mask_export(desc: AttnDesc, tile_codes: int, visible: int = 0, stream: int = 0, check=True):
+    """Tile codes [n_q][ceil(n_keys/128)] and element visibility [n_q][n_keys]
+    (uint8 device buffers) of the attention kernel's masking."""
+    return _call("cosmot_mot_mask_export", ctypes.byref(desc), c_vp(tile_codes), c_vp(visible or None),
                  c_vp(stream), check=check)
 
 

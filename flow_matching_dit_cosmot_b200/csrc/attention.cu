@@ -113,6 +113,46 @@ __device__ __forceinline__ Work decode_work(const Params& p) {
   return w;
 }
 
+// Masking decisions of one query row, shared by the attention kernel and the
+// debug export (cosmot_mot_mask_export), so that the export shows exactly what
+// the kernel does.
+struct RowMask {
+  int64_t klimit;    // keys >= klimit are hidden (causal AR limit, or n_keys)
+  int32_t my_chunk;  // block-causal DM rows: DM keys of later chunks are hidden
+  bool bc_dm;
+};
+
+__device__ __forceinline__ RowMask row_mask(const Params& p, const Work& w, int64_t qi, bool valid) {
+  RowMask m;
+  const int64_t qk = p.q_key_offset + qi;  // key index of this query row
+  m.bc_dm = !w.is_ar && p.mask_mode == COSMOT_MASK_BLOCK_CAUSAL;
+  m.klimit = p.n_keys;
+  if (w.is_ar) m.klimit = qk + 1 < p.n_ar ? qk + 1 : p.n_ar;
+  // Rows past the segment are padding (never stored): they see everything,
+  // so they never force the element-mask path on their warp.
+  m.my_chunk = m.bc_dm ? (valid ? __ldg(p.chunk + qk) : INT32_MAX) : 0;
+  return m;
+}
+
+// Chunk id of a key as the tile test sees it: AR keys and keys past the end
+// never hide a tile (INT32_MIN).
+__device__ __forceinline__ int32_t key_chunk_for_tile(const Params& p, int64_t key) {
+  return (key >= p.n_ar && key < p.n_keys) ? __ldg(p.chunk + key) : INT32_MIN;
+}
+
+// A key tile needs per-element masks when it reaches past the row's key limit
+// or (block-causal) holds a DM key of a later chunk; tile_chunk_max is the
+// largest key_chunk_for_tile over its 128 keys.
+__device__ __forceinline__ bool tile_needs_mask(const RowMask& m, int64_t kbase, int32_t tile_chunk_max) {
+  return kbase + BKV > m.klimit || (m.bc_dm && tile_chunk_max > m.my_chunk);
+}
+
+__device__ __forceinline__ bool key_visible(const Params& p, const RowMask& m, int64_t key) {
+  bool vis = key < m.klimit;
+  if (m.bc_dm && key >= p.n_ar && vis) vis = __ldg(p.chunk + key) <= m.my_chunk;
+  return vis;
+}
+
 template <int HD>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
     mot_attention_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__ CUtensorMap tmap_k,
@@ -276,13 +316,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     const int r = lane_base + lane;
     const int64_t qi = w.row0 + (int64_t)t * BQ + r;
     const bool valid = qi < w.seg_end;
-    const int64_t qk = p.q_key_offset + qi;  // key index of this query row
-    const bool bc_dm = !w.is_ar && p.mask_mode == COSMOT_MASK_BLOCK_CAUSAL;
-    int64_t klimit = p.n_keys;
-    if (w.is_ar) klimit = qk + 1 < p.n_ar ? qk + 1 : p.n_ar;
-    // Rows past the segment are padding (never stored): they see everything,
-    // so they never force the element-mask path on their warp.
-    const int32_t my_chunk = bc_dm ? (valid ? __ldg(p.chunk + qk) : INT32_MAX) : 0;
+    const RowMask rm = row_mask(p, w, qi, valid);
     const uint32_t s_addr = tmem_base + ((uint32_t)lane_base << 16) + C::s_col(t);
     const uint32_t o_addr = tmem_base + ((uint32_t)lane_base << 16) + C::o_col(t);
     const float sl2 = p.scale_log2;
@@ -295,12 +329,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       // and keys past the end count as visible) before waiting for S, so the
       // load latency hides behind the wait; the max is reduced after it.
       int32_t ck[4] = {INT32_MIN, INT32_MIN, INT32_MIN, INT32_MIN};
-      if (bc_dm) {
+      if (rm.bc_dm) {
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          const int64_t key = kbase + lane + 32 * i;
-          if (key >= p.n_ar && key < p.n_keys) ck[i] = __ldg(p.chunk + key);
-        }
+        for (int i = 0; i < 4; ++i) ck[i] = key_chunk_for_tile(p, kbase + lane + 32 * i);
       }
       // Warp-uniform decisions only: every tcgen05.ld/st below is .sync.aligned.
       if (!__all_sync(0xffffffffu, mbar_wait(bar_s_full + 8 * t, j & 1, p.status, kWhereAttnSoftmax))) {
@@ -314,21 +345,16 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       tmem_ld32(s_addr + 64, *reinterpret_cast<uint32_t(*)[32]>(&s[64]));
       tmem_ld32(s_addr + 96, *reinterpret_cast<uint32_t(*)[32]>(&s[96]));
       tmem_ld_wait();
-      bool chunk_mask = false;
-      if (bc_dm) {
-        int32_t tmax = max(max(ck[0], ck[1]), max(ck[2], ck[3]));
+      int32_t tmax = INT32_MIN;
+      if (rm.bc_dm) {
+        tmax = max(max(ck[0], ck[1]), max(ck[2], ck[3]));
 #pragma unroll
         for (int off = 16; off > 0; off >>= 1) tmax = max(tmax, __shfl_xor_sync(0xffffffffu, tmax, off));
-        chunk_mask = tmax > my_chunk;
       }
-      if (kbase + BKV > klimit || chunk_mask) {
+      if (tile_needs_mask(rm, kbase, tmax)) {
 #pragma unroll
-        for (int c = 0; c < 128; ++c) {
-          const int64_t key = kbase + c;
-          bool vis = key < klimit;
-          if (bc_dm && key >= p.n_ar && vis) vis = __ldg(p.chunk + key) <= my_chunk;
-          if (!vis) s[c] = __float_as_uint(-INFINITY);
-        }
+        for (int c = 0; c < 128; ++c)
+          if (!key_visible(p, rm, kbase + c)) s[c] = __float_as_uint(-INFINITY);
       }
       float mt = -INFINITY;
 #pragma unroll
@@ -428,12 +454,13 @@ cosmot_status launch(const CUtensorMap& tq, const CUtensorMap& tk, const CUtenso
 }  // namespace attn
 }  // namespace cosmot
 
-extern "C" cosmot_status cosmot_mot_attention(const cosmot_attn_desc* d, const void* q, int64_t ld_q, const void* k,
-                                              const void* v, int64_t ld_kv, void* o, int64_t ld_o,
-                                              cosmot_stream_t stream) {
-  using namespace cosmot;
-  using namespace cosmot::attn;
-  if (!d || !q || !k || !v || !o) return COSMOT_ERR_INVALID_ARG;
+namespace cosmot {
+namespace attn {
+
+// Descriptor checks and kernel parameters shared by the attention entry point
+// and the mask export.
+cosmot_status make_params(const cosmot_attn_desc* d, Params& p, int64_t& grid) {
+  if (!d) return COSMOT_ERR_INVALID_ARG;
   const int hd = d->head_dim;
   if (hd != 64 && hd != 128) return COSMOT_ERR_UNSUPPORTED;
   if (d->n_heads < 1 || d->n_kv_heads < 1 || d->n_heads % d->n_kv_heads) return COSMOT_ERR_INVALID_ARG;
@@ -442,14 +469,9 @@ extern "C" cosmot_status cosmot_mot_attention(const cosmot_attn_desc* d, const v
     return COSMOT_ERR_INVALID_ARG;
   if (d->mask_mode != COSMOT_MASK_FULL && d->mask_mode != COSMOT_MASK_BLOCK_CAUSAL) return COSMOT_ERR_INVALID_ARG;
   if (d->mask_mode == COSMOT_MASK_BLOCK_CAUSAL && !d->chunk) return COSMOT_ERR_INVALID_ARG;
-  const int64_t qcols = (int64_t)d->n_heads * hd, kvcols = (int64_t)d->n_kv_heads * hd;
-  if (ld_q < qcols || ld_kv < kvcols || ld_o < qcols || ld_q % 8 || ld_kv % 8 || ld_o % 8) return COSMOT_ERR_INVALID_ARG;
-  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o)) return COSMOT_ERR_INVALID_ARG;
   if (d->batch > 1 && (d->q_batch_stride < d->n_q || d->kv_batch_stride < d->n_keys || d->o_batch_stride < d->n_q))
     return COSMOT_ERR_INVALID_ARG;
-  if (d->n_q == 0) return COSMOT_OK;
-
-  Params p{};
+  p = Params{};
   p.n_q = d->n_q;
   p.q_key_offset = d->q_key_offset;
   p.n_keys = d->n_keys;
@@ -470,18 +492,67 @@ extern "C" cosmot_status cosmot_mot_attention(const cosmot_attn_desc* d, const v
   const float scale = d->softmax_scale > 0.f ? d->softmax_scale : 1.0f / sqrtf((float)hd);
   p.scale_log2 = scale * 1.4426950408889634f;
   p.chunk = d->chunk;
-  p.o = static_cast<__nv_bfloat16*>(o);
-  p.ld_o = ld_o;
   p.status = device_status_ptr();
   if (!p.status) return COSMOT_ERR_CUDA;
+  grid = (int64_t)d->batch * d->n_heads * (p.ar_pairs + p.dm_pairs);
+  if (grid > INT32_MAX) return COSMOT_ERR_UNSUPPORTED;
+  return COSMOT_OK;
+}
 
-  const int64_t grid = (int64_t)d->batch * d->n_heads * (p.ar_pairs + p.dm_pairs);
+// One CTA per work item of the attention grid; only sequence 0, head 0 writes
+// (the decisions depend on neither).  Thread i handles query row row0 + i.
+__global__ void __launch_bounds__(2 * BQ) mask_export_kernel(const __grid_constant__ Params p, uint8_t* tile_codes,
+                                                             int64_t n_kt_all, uint8_t* visible) {
+  const Work w = decode_work(p);
+  if (w.b != 0 || w.h != 0) return;
+  const int64_t qi = w.row0 + threadIdx.x;
+  if (qi >= w.seg_end) return;
+  const RowMask rm = row_mask(p, w, qi, true);
+  for (int64_t j = 0; j < n_kt_all; ++j) {
+    const int64_t kbase = j * BKV;
+    uint8_t code = 0;
+    bool masked = false;
+    if (j < w.n_kt) {
+      int32_t tmax = INT32_MIN;
+      if (rm.bc_dm)
+        for (int c = 0; c < BKV; ++c) tmax = max(tmax, key_chunk_for_tile(p, kbase + c));
+      masked = tile_needs_mask(rm, kbase, tmax);
+      code = masked ? 2 : 1;
+    }
+    tile_codes[qi * n_kt_all + j] = code;
+    if (visible)
+      for (int c = 0; c < BKV && kbase + c < p.n_keys; ++c)
+        visible[qi * p.n_keys + kbase + c] = (uint8_t)(code && (!masked || key_visible(p, rm, kbase + c)));
+  }
+}
+
+}  // namespace attn
+}  // namespace cosmot
+
+extern "C" cosmot_status cosmot_mot_attention(const cosmot_attn_desc* d, const void* q, int64_t ld_q, const void* k,
+                                              const void* v, int64_t ld_kv, void* o, int64_t ld_o,
+                                              cosmot_stream_t stream) {
+  using namespace cosmot;
+  using namespace cosmot::attn;
+  if (!d || !q || !k || !v || !o) return COSMOT_ERR_INVALID_ARG;
+  Params p;
+  int64_t grid = 0;
+  cosmot_status st = make_params(d, p, grid);
+  if (st != COSMOT_OK) return st;
+  const int hd = d->head_dim;
+  const int64_t qcols = (int64_t)d->n_heads * hd, kvcols = (int64_t)d->n_kv_heads * hd;
+  if (ld_q < qcols || ld_kv < kvcols || ld_o < qcols || ld_q % 8 || ld_kv % 8 || ld_o % 8) return COSMOT_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o)) return COSMOT_ERR_INVALID_ARG;
+  if (d->n_q == 0) return COSMOT_OK;
+  p.o = static_cast<__nv_bfloat16*>(o);
+  p.ld_o = ld_o;
+
   const int64_t q_rows = (d->batch - 1) * p.q_bstride + d->n_q;
   const int64_t kv_rows = (d->batch - 1) * p.kv_bstride + d->n_keys;
-  if (grid > INT32_MAX || q_rows + 2 * BQ > INT32_MAX || kv_rows + BKV > INT32_MAX) return COSMOT_ERR_UNSUPPORTED;
+  if (q_rows + 2 * BQ > INT32_MAX || kv_rows + BKV > INT32_MAX) return COSMOT_ERR_UNSUPPORTED;
 
   CUtensorMap tq, tk, tv;
-  cosmot_status st = make_tmap_bf16_2d(&tq, q, (uint64_t)q_rows, (uint64_t)qcols, (uint64_t)ld_q, BQ, 64);
+  st = make_tmap_bf16_2d(&tq, q, (uint64_t)q_rows, (uint64_t)qcols, (uint64_t)ld_q, BQ, 64);
   if (st != COSMOT_OK) return st;
   st = make_tmap_bf16_2d(&tk, k, (uint64_t)kv_rows, (uint64_t)kvcols, (uint64_t)ld_kv, BKV, 64);
   if (st != COSMOT_OK) return st;
@@ -489,4 +560,20 @@ extern "C" cosmot_status cosmot_mot_attention(const cosmot_attn_desc* d, const v
   if (st != COSMOT_OK) return st;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   return hd == 128 ? launch<128>(tq, tk, tv, p, (unsigned)grid, s) : launch<64>(tq, tk, tv, p, (unsigned)grid, s);
+}
+
+extern "C" cosmot_status cosmot_mot_mask_export(const cosmot_attn_desc* d, uint8_t* tile_codes, uint8_t* visible,
+                                                cosmot_stream_t stream) {
+  using namespace cosmot;
+  using namespace cosmot::attn;
+  if (!tile_codes) return COSMOT_ERR_INVALID_ARG;
+  Params p;
+  int64_t grid = 0;
+  cosmot_status st = make_params(d, p, grid);
+  if (st != COSMOT_OK) return st;
+  if (d->n_q == 0) return COSMOT_OK;
+  const int64_t n_kt_all = (d->n_keys + BKV - 1) / BKV;
+  mask_export_kernel<<<(unsigned)grid, 2 * BQ, 0, reinterpret_cast<cudaStream_t>(stream)>>>(p, tile_codes, n_kt_all,
+                                                                                             visible);
+  return launch_status();
 }

@@ -228,6 +228,23 @@ COSMOT_API cosmot_status cosmot_mot_attention(const cosmot_attn_desc* desc, cons
                                    const void* v, int64_t ld_kv, void* o, int64_t ld_o, cosmot_stream_t stream);
 
 /*
+ * Debug export of the masking decisions cosmot_mot_attention takes for the
+ * same descriptor (sequence 0; they depend on neither the sequence nor the
+ * head).  The pages define the mask only element by element (the §3 equations);
+ * this shows the kernel's tiling of it so that a test can hold both against
+ * the definition.  Key tiles are 128 keys wide; n_kt = ceil(n_keys / 128).
+ *   tile_codes  device uint8 [n_q][n_kt]: 0 = the query's CTA never visits the
+ *               key tile, 1 = visited with no element mask (every key visible),
+ *               2 = visited with per-element masks.  Required.
+ *   visible     device uint8 [n_q][n_keys] or NULL: 1 where the kernel lets the
+ *               query see the key, else 0.
+ * Caller-owned buffers; every element of both is written.  Argument errors as
+ * for cosmot_mot_attention (the q/k/v/o checks do not apply).
+ */
+COSMOT_API cosmot_status cosmot_mot_mask_export(const cosmot_attn_desc* desc, uint8_t* tile_codes, uint8_t* visible,
+                                                cosmot_stream_t stream);
+
+/*
  * Flow-matching Euler step ("Cosmos 3 方法原理全解" §7.2), in place:
  *     x[r, c] = bf16( x[r, c] + (sigma_next - sigma) * v[r, c] )  for r in [row_begin, row_end)
  * Rows outside the range are not touched (clean DM rows pass through bit-exact).

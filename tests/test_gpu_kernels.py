@@ -111,6 +111,23 @@ def test_routed_linear_plain(m_split, m_total, k, n_out):
     assert_device_ok()
 
 
+def test_routed_linear_equal_sets_equal_single_segment():
+    """With both weight sets holding the same matrix (in separate buffers) the
+    routed projection is bit-identical to one segment over all rows: routing
+    changes which weights a row meets, never how a row is computed."""
+    a, w0, _, segs, _ = _gemm_case(203, 700, 512, 264, seed=5)
+    ad, w0d, w1d = to_dev(a), to_dev(w0), to_dev(w0.copy())
+    routed = torch.empty((700, 264), dtype=torch.bfloat16, device="cuda")
+    single = torch.empty_like(routed)
+    L.cosmot_routed_linear(A.ptr(ad), 512, 512, segs, A.ptr(w0d), A.ptr(w1d), 264, A.ptr(routed), 264,
+                           stream=A.stream_handle())
+    L.cosmot_routed_linear(A.ptr(ad), 512, 512, [(0, 700, 0, 0)], A.ptr(w0d), A.ptr(w1d), 264, A.ptr(single), 264,
+                           stream=A.stream_handle())
+    torch.cuda.synchronize()
+    assert_device_ok()
+    np.testing.assert_array_equal(bits(routed), bits(single))
+
+
 def test_routed_linear_residual():
     m_split, m_total, k, n_out = 77, 400, 512, 264
     a, w0, w1, segs, acc = _gemm_case(m_split, m_total, k, n_out, seed=1)
@@ -261,6 +278,31 @@ def _attn_case(n_keys, n_ar, n_q, q_off, H, Hkv, hd, mode, chunk=None, batch=1, 
     got = to_f64(o)
     assert_device_ok()
     return got, np.concatenate(ref)
+
+
+def test_attention_of_constant_values_is_one():
+    """With V = 1 every visible set of softmax weights sums to one, so every
+    output is 1 ("Cosmos 3 方法原理全解" §3: attention is a convex combination of
+    values).  P is stored in bf16 for the PV product while the row sum is kept
+    in fp32, so the output may differ from 1 by the bf16 rounding of P: at most
+    2^-9 relative, plus the output's own rounding."""
+    n_keys, n_ar, H, hd = 700, 130, 2, 128
+    ch = np.full(n_keys, -1, np.int32)
+    ch[n_ar:] = np.arange(n_keys - n_ar) // 97
+    for mode in ("full", "block_causal"):
+        q = _bf16((n_keys, H * hd), 95)
+        k = _bf16((n_keys, H * hd), 96)
+        ones = torch.ones((n_keys, H * hd), dtype=torch.bfloat16, device="cuda")
+        o = torch.full((n_keys, H * hd), float("nan"), dtype=torch.bfloat16, device="cuda")
+        qd, kd, chd = to_dev(q), to_dev(k), torch.from_numpy(ch).cuda()
+        d = L.AttnDesc(n_q=n_keys, q_key_offset=0, n_keys=n_keys, n_ar=n_ar, n_heads=H, n_kv_heads=H, head_dim=hd,
+                       mask_mode=L.COSMOT_MASK_FULL if mode == "full" else L.COSMOT_MASK_BLOCK_CAUSAL,
+                       chunk=A.ptr(chd), batch=1)
+        L.cosmot_mot_attention(d, A.ptr(qd), H * hd, A.ptr(kd), A.ptr(ones), H * hd, A.ptr(o), H * hd,
+                               A.stream_handle())
+        torch.cuda.synchronize()
+        assert_device_ok()
+        assert np.abs(to_f64(o) - 1.0).max() <= 2.0 ** -8, mode
 
 
 @pytest.mark.parametrize("hd", [128, 64])

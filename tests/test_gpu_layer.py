@@ -110,6 +110,25 @@ def test_ar_rows_bit_identical_under_dm_perturbation():
     assert (bits(out_a[0])[n_ar:] != bits(out_b[0])[n_ar:]).any()
 
 
+def test_ar_rows_bit_identical_under_generator_weight_change():
+    """AR rows use only Reasoner weights: replacing every Generator weight
+    (norm gains, QKV, O, FFN) leaves the AR rows of h_out unchanged to the bit
+    and changes the DM rows."""
+    run = LayerRun(MEDIUM, synth.preset("droid").layout)
+    _, out_a = run.gpu()
+    other = synth.make_weights(MEDIUM, 1099)
+    w2 = {k: (other[k] if k.startswith("G.") else v) for k, v in run.w.items()}
+    layer2 = A.MoTLayer(cdims(A, MEDIUM), device_weights(w2))
+    h = to_dev(run.h)
+    out_b = torch.empty_like(h)
+    layer2.forward(h, out_b, 0.8, 0.7, run.seq)
+    torch.cuda.synchronize()
+    assert_device_ok()
+    n_ar = run.lay.n_ar
+    np.testing.assert_array_equal(bits(out_a[0])[:n_ar], bits(out_b[0])[:n_ar])
+    assert (bits(out_a[0])[n_ar:] != bits(out_b[0])[n_ar:]).any()
+
+
 def test_layer_is_deterministic():
     run = LayerRun(MEDIUM, synth.preset("droid").layout)
     a = run.gpu()
