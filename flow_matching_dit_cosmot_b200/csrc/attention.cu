@@ -23,12 +23,20 @@
 //               2^8 (the exponent headroom keeps P and O finite meanwhile).
 // TMEM columns: S0 [0,128), S1 [128,256), O0 and O1 after them.
 //
+// P is released in two halves (keys 0-63, then 64-127) so that the first half
+// of PV overlaps the exponentials of the second.
+//
 // Measured on B200 (18,978 tokens, 32 heads of 128): the period of one key
-// block is set by the chain softmax(tile 0) -> PV0 -> next S0 -> softmax, not by
-// the SFU; variants that moved exponentials to the FMA pipe, used packed
-// f32x2 arithmetic, split the row between two warpgroups or served both tiles
-// from one warpgroup were all slower than this plain form.  Every tcgen05.ld/st
-// is reached through warp-uniform control flow (they are .sync.aligned).
+// block (~3,600 cycles) is the chain softmax(tile 0) ~1,900 -> hand-off ~450 ->
+// PV0 rest and next S0 ~1,000 -> S-ready ~250; the tensor pipe is busy ~60 % and
+// the SFU ~55 %.  The softmax is bound by its own issue latency (one warp per
+// sub-partition per tile), not by the SFU: exponentials on the FMA pipe (25 %
+// or 37.5 % of them), packed f32x2 arithmetic, a row split between two
+// warpgroups and one warpgroup serving both tiles were all slower.  Smaller MMAs
+// do not help either: a tcgen05.mma with N = 64 costs 44-48 cycles instead of
+// 32 (fixed per-instruction cost), so 64-key blocks with double-buffered S, or
+// S issued as two N = 64 halves, were 23-58 % slower.  Every tcgen05.ld/st is
+// reached through warp-uniform control flow (they are .sync.aligned).
 #include <cuda_bf16.h>
 
 #include <mutex>
@@ -167,10 +175,11 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   const uint32_t bar_kv_full = bar_q + 8;                // [SLOTS]
   const uint32_t bar_kv_empty = bar_kv_full + 8 * SLOTS; // [SLOTS]
   const uint32_t bar_s_full = bar_kv_empty + 8 * SLOTS;  // [2]
-  const uint32_t bar_p_full = bar_s_full + 16;           // [2]
+  const uint32_t bar_p_half = bar_s_full + 16;           // [2] P of keys 0-63 written
+  const uint32_t bar_p_full = bar_p_half + 16;           // [2] P of keys 64-127 written
   const uint32_t bar_o_done = bar_p_full + 16;           // [2]
   const uint32_t bar_drain = bar_o_done + 16;            // [1]
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 1 + 2 * SLOTS + 7);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 1 + 2 * SLOTS + 9);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -185,6 +194,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     }
     for (int t = 0; t < 2; ++t) {
       mbar_init(bar_s_full + 8 * t, 1);
+      mbar_init(bar_p_half + 8 * t, 128);
       mbar_init(bar_p_full + 8 * t, 128);
       mbar_init(bar_o_done + 8 * t, 1);
     }
@@ -253,10 +263,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                   C::IDESC_S, k > 0 ? 1u : 0u);
         }
       };
-      auto issue_pv = [&](int t, int slot, bool acc) {
+      auto issue_pv = [&](int t, int slot, bool acc, int half) {  // keys 64*half .. 64*half+63
         const uint32_t va = sKV + slot * C::TILE_BYTES;
 #pragma unroll
-        for (int k = 0; k < BKV / 16; ++k) {
+        for (int k = 4 * half; k < 4 * half + 4; ++k) {
           // V rows k*16 .. k*16+15: two 8-row swizzle atoms = 2048 bytes.
           umma_ts(tmem_base + C::o_col(t), tmem_base + C::s_col(t) + 8 * k, sw128_desc(va + 2048 * k, BOX_BYTES, 1024),
                   C::IDESC_O, (acc || k > 0) ? 1u : 0u);
@@ -278,18 +288,26 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         const int LV = 2 * j + 1, LK = 2 * j + 2;
         const bool has_next = j + 1 < n_kt;
         const uint32_t par = j & 1;
-        if (!kv_wait(LV) || !mbar_wait(bar_p_full, par, p.status, kWhereAttnMma)) break;
+        // Order of the softmax events in steady state: tile 0 half, tile 0
+        // full, tile 1 half, tile 1 full (tile 1 runs about half a block later).
+        if (!kv_wait(LV) || !mbar_wait(bar_p_half, par, p.status, kWhereAttnMma)) break;
         tc_fence_after();
-        issue_pv(0, LV % SLOTS, j > 0);
+        issue_pv(0, LV % SLOTS, j > 0, 0);
+        if (!mbar_wait(bar_p_full, par, p.status, kWhereAttnMma)) break;
+        tc_fence_after();
+        issue_pv(0, LV % SLOTS, true, 1);
         if (has_next) {
           if (!kv_wait(LK)) break;
           tc_fence_after();
           issue_s(0, LK % SLOTS);
           umma_commit(bar_s_full);
         }
+        if (!mbar_wait(bar_p_half + 8, par, p.status, kWhereAttnMma)) break;
+        tc_fence_after();
+        issue_pv(1, LV % SLOTS, j > 0, 0);
         if (!mbar_wait(bar_p_full + 8, par, p.status, kWhereAttnMma)) break;
         tc_fence_after();
-        issue_pv(1, LV % SLOTS, j > 0);
+        issue_pv(1, LV % SLOTS, true, 1);
         umma_commit(bar_kv_empty + 8 * (LV % SLOTS));
         if (has_next) {
           issue_s(1, LK % SLOTS);
@@ -356,9 +374,16 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         for (int c = 0; c < 128; ++c)
           if (!key_visible(p, rm, kbase + c)) s[c] = __float_as_uint(-INFINITY);
       }
-      float mt = -INFINITY;
+      // Row max with four independent three-input chains (16 deep, not 128).
+      float mx0 = -INFINITY, mx1 = -INFINITY, mx2 = -INFINITY, mx3 = -INFINITY;
 #pragma unroll
-      for (int c = 0; c < 128; ++c) mt = fmaxf(mt, __uint_as_float(s[c]));
+      for (int c = 0; c < 128; c += 8) {
+        mx0 = fmax3(mx0, __uint_as_float(s[c + 0]), __uint_as_float(s[c + 1]));
+        mx1 = fmax3(mx1, __uint_as_float(s[c + 2]), __uint_as_float(s[c + 3]));
+        mx2 = fmax3(mx2, __uint_as_float(s[c + 4]), __uint_as_float(s[c + 5]));
+        mx3 = fmax3(mx3, __uint_as_float(s[c + 6]), __uint_as_float(s[c + 7]));
+      }
+      const float mt = fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3));
       const float m_new = fmaxf(m, mt * sl2);
       const bool first = (m == -INFINITY);
       const bool need = !first && (m_new > m + kRescaleThreshold);
@@ -383,7 +408,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         tmem_st_wait();
       }
       const float mu = (m == -INFINITY) ? 0.f : m;
-      float rs = 0.f;
+      float rs0 = 0.f, rs1 = 0.f;  // two running sums: half the dependent-add chain
 #pragma unroll
       for (int c0 = 0; c0 < 128; c0 += 32) {
         uint32_t pk[16];
@@ -391,12 +416,18 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         for (int e = 0; e < 16; ++e) {
           const float p0 = ex2_approx(fmaf(__uint_as_float(s[c0 + 2 * e]), sl2, -mu));
           const float p1 = ex2_approx(fmaf(__uint_as_float(s[c0 + 2 * e + 1]), sl2, -mu));
-          rs += p0 + p1;
+          rs0 += p0;
+          rs1 += p1;
           pk[e] = pack_bf16x2(p0, p1);
         }
         tmem_st16(s_addr + (c0 >> 1), pk);
+        if (c0 == 32) {  // P of keys 0-63 is in TMEM: PV over them may start
+          tmem_st_wait();
+          tc_fence_before();
+          mbar_arrive(bar_p_half + 8 * t);
+        }
       }
-      l += rs;
+      l += rs0 + rs1;
       tmem_st_wait();
       tc_fence_before();
       mbar_arrive(bar_p_full + 8 * t);
