@@ -152,7 +152,7 @@ def project_kv(dims, W: LayerWeights, h, region, pos):
 
 
 def layer_forward(dims, W: LayerWeights, h, region, pos, chunk, sigma, sigma_next,
-                  mode="full", rows=None, cache=None):
+                  mode="full", rows=None, cache=None, head=True):
     """One MoT layer forward over one packed sequence, plus the Euler step.
 
     h [N, d] float64 (DM rows are the sampler state x), region/pos/chunk from
@@ -163,6 +163,8 @@ def layer_forward(dims, W: LayerWeights, h, region, pos, chunk, sigma, sigma_nex
 
     Returns a dict with h2 [len(rows), d], x_new [len(rows), d] (NaN on AR
     rows), vel [len(rows), d] (NaN except on noisy rows) and the row indices.
+    With head=False the velocity head and the Euler step are left out (x_new
+    and vel all NaN): a layer inside a stack.
     """
     h = np.asarray(h, dtype=np.float64)
     region = np.asarray(region)
@@ -216,6 +218,8 @@ def layer_forward(dims, W: LayerWeights, h, region, pos, chunk, sigma, sigma_nex
 
     x_new = np.full_like(h2, np.nan)
     vel = np.full_like(h2, np.nan)
+    if not head:
+        return {"rows": rows, "h2": h2, "x_new": x_new, "vel": vel}
     reg_r = region[rows]
     clean = reg_r == REGION_CLEAN
     noisy = reg_r == REGION_NOISY
@@ -256,6 +260,49 @@ def cfg_step(dims, W, h_cond, h_base, lay, sigma, sigma_next, guidance, mode="fu
     v = cfg_combine(oc["vel"][noisy], ob["vel"][noisy], guidance)
     x = np.asarray(h_cond, np.float64)[noisy]
     return euler_step(x, v, sigma, sigma_next), oc, ob
+
+
+def stack_forward(dims, layers, h, region, pos, chunk, sigma, sigma_next, mode="full"):
+    """A stack of MoT layers, then the flow-matching step ("Cosmos 3 方法原理全解"
+    §3 for the layer, §12.4 for the stacked models, §7.2 for the step).
+
+    h^0 = h; h^l = layer_l(h^{l-1}) for each entry of `layers` (LayerWeights,
+    applied in order); on the noisy rows v = RMSNorm(h^L; g_fin) W_vel^T with
+    the final norm and velocity head of the last entry, and x' = x + (sigma_next
+    - sigma) v where x is the noisy rows of h (the state is the stack's input).
+    Returns h_out = h^L, the hidden states after every layer, vel and x_new as
+    layer_forward does.
+    """
+    h = np.asarray(h, dtype=np.float64)
+    region = np.asarray(region)
+    x = h
+    hidden = []
+    for W in layers:
+        x = layer_forward(dims, W, x, region, pos, chunk, sigma, sigma_next, mode, head=False)["h2"]
+        hidden.append(x)
+    vel = np.full_like(x, np.nan)
+    x_new = np.full_like(x, np.nan)
+    clean = region == REGION_CLEAN
+    noisy = region == REGION_NOISY
+    x_new[clean] = h[clean]
+    if noisy.any():
+        last = layers[-1]
+        vel[noisy] = rms_norm(x[noisy], last.gfin, dims.eps) @ last.wvel.T
+        x_new[noisy] = euler_step(h[noisy], vel[noisy], sigma, sigma_next)
+    return {"h_out": x, "hidden": hidden, "vel": vel, "x_new": x_new}
+
+
+def stack_sample(dims, layers, h, lay, sigmas, mode="full"):
+    """Sampler loop over a layer stack: one stack forward and one Euler step per
+    (sigma, sigma_next); the noisy rows of h carry the state."""
+    h = np.array(h, dtype=np.float64)
+    noisy = lay.region == REGION_NOISY
+    outs = []
+    for s0, s1 in zip(sigmas[:-1], sigmas[1:]):
+        out = stack_forward(dims, layers, h, lay.region, lay.pos, lay.chunk, s0, s1, mode)
+        h[noisy] = out["x_new"][noisy]
+        outs.append(out)
+    return h, outs
 
 
 def sample(dims, W, h, lay, sigmas, mode="full"):

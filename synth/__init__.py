@@ -22,6 +22,8 @@ from .rng import (  # noqa: F401
     bf16_to_f64,
     normal_bf16,
     make_weights,
+    make_stack_weights,
+    stack_layer_seed,
     make_activations,
     WEIGHT_NAMES,
 )

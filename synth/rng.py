@@ -87,6 +87,23 @@ def make_weights(dims: ModelDims, seed: int, names=None) -> dict:
     return out
 
 
+def stack_layer_seed(seed: int, layer: int) -> int:
+    """Seed of layer `layer` of a stack whose first layer has `seed`."""
+    return seed + 7919 * layer
+
+
+def make_stack_weights(dims: ModelDims, seed: int, n_layers: int, distinct: int = 0) -> list:
+    """Weights of an n_layers stack, one make_weights draw per layer.
+
+    With distinct > 0 only that many layers are drawn and layer l uses draw
+    l % distinct (large stacks whose weights take long to generate on the host;
+    every layer's weights still stream from HBM, as each is far larger than L2).
+    """
+    n_draw = n_layers if distinct <= 0 else min(distinct, n_layers)
+    draws = [make_weights(dims, stack_layer_seed(seed, l)) for l in range(n_draw)]
+    return [draws[l % n_draw] for l in range(n_layers)]
+
+
 def make_activations(n_tokens: int, d_model: int, seed: int, tensor_id: int = 0) -> np.ndarray:
     """Layer input h [n_tokens, d_model] ~ N(0, 1) bf16 bits."""
     return normal_bf16((n_tokens, d_model), seed, 10_000 + tensor_id)

@@ -293,6 +293,82 @@ def test_dm_outputs_use_reasoner_kv_but_not_reasoner_o_or_mlp():
     assert np.abs(p3["h2"][lay.n_ar:] - base["h2"][lay.n_ar:]).max() > 1e-6
 
 
+# ---------------------------------------------------------------- layer stacks
+
+def _stack(dims, n, seed=21):
+    return [layer.weights_from_bits(dims, w) for w in synth.make_stack_weights(dims, seed, n)]
+
+
+def test_stack_of_one_layer_is_the_layer():
+    lay = _small_layout()
+    Ws = _stack(TINY, 1)
+    h = _h(lay.n_tokens, TINY.d_model)
+    one = _run(TINY, Ws[0], h, lay)
+    st = layer.stack_forward(TINY, Ws, h, lay.region, lay.pos, lay.chunk, 0.8, 0.7)
+    np.testing.assert_array_equal(st["h_out"], one["h2"])
+    np.testing.assert_array_equal(st["x_new"], one["x_new"])
+    np.testing.assert_array_equal(st["vel"], one["vel"])
+
+
+def test_stack_of_residual_only_layers_is_the_identity():
+    """With W_o = W_down = 0 in every layer each layer returns its input, so the
+    stack output is h and the step is the velocity head applied to h itself
+    (closed form)."""
+    lay = _small_layout()
+    Ws = _stack(TINY, 3)
+    for W in Ws:
+        for s_ in (W.R, W.G):
+            s_.wo = np.zeros_like(s_.wo)
+            s_.wd = np.zeros_like(s_.wd)
+    h = _h(lay.n_tokens, TINY.d_model)
+    st = layer.stack_forward(TINY, Ws, h, lay.region, lay.pos, lay.chunk, 0.8, 0.7)
+    np.testing.assert_array_equal(st["h_out"], h)
+    noisy = lay.region == layout.REGION_NOISY
+    g, wv = Ws[-1].gfin, Ws[-1].wvel
+    x = h[noisy]
+    v = (x / np.sqrt(np.mean(x * x, axis=1, keepdims=True) + TINY.eps) * g) @ wv.T
+    np.testing.assert_allclose(st["x_new"][noisy], x - 0.1 * v, rtol=0, atol=1e-12)
+
+
+@pytest.mark.parametrize("mode", ["full", "block_causal"])
+def test_stack_ar_rows_independent_of_dm_rows_and_generator_weights(mode):
+    """AR rows stay Reasoner-only through any depth: their outputs after every
+    layer ignore DM inputs and every Generator weight (so AR K/V can be cached
+    across sampler steps for a whole stack)."""
+    lay = _small_layout()
+    Ws = _stack(TINY, 3)
+    h = _h(lay.n_tokens, TINY.d_model)
+    base = layer.stack_forward(TINY, Ws, h, lay.region, lay.pos, lay.chunk, 0.8, 0.7, mode)
+    h2 = h.copy()
+    h2[lay.n_ar:] += 0.5
+    Ws2 = _stack(TINY, 3)
+    for W in Ws2:
+        W.G.wv = W.G.wv * -1.0
+        W.G.wd = W.G.wd * 2.0
+    pert = layer.stack_forward(TINY, Ws2, h2, lay.region, lay.pos, lay.chunk, 0.8, 0.7, mode)
+    for a, b in zip(base["hidden"], pert["hidden"]):
+        np.testing.assert_array_equal(a[:lay.n_ar], b[:lay.n_ar])
+    assert np.abs(pert["h_out"][lay.n_ar:] - base["h_out"][lay.n_ar:]).max() > 1e-3
+
+
+def test_stack_clean_rows_read_noisy_rows_from_the_second_layer():
+    """Full mask: clean DM rows attend to noisy rows, so after the first layer
+    their hidden state (and the next layer's clean K/V) changes with the noisy
+    state; block-causal: clean chunks before every noisy chunk do not."""
+    lay = _small_layout(video=VideoSpec(1, 2, 3, 24, 1, 2))
+    Ws = _stack(TINY, 2)
+    h = _h(lay.n_tokens, TINY.d_model)
+    clean = lay.region == layout.REGION_CLEAN
+    noisy = lay.region == layout.REGION_NOISY
+    h2 = h.copy()
+    h2[noisy] += 0.5
+    for mode, changes in (("full", True), ("block_causal", False)):
+        a = layer.stack_forward(TINY, Ws, h, lay.region, lay.pos, lay.chunk, 0.8, 0.7, mode)
+        b = layer.stack_forward(TINY, Ws, h2, lay.region, lay.pos, lay.chunk, 0.8, 0.7, mode)
+        d = np.abs(a["hidden"][0][clean] - b["hidden"][0][clean]).max()
+        assert (d > 1e-6) == changes, (mode, d)
+
+
 def test_clean_rows_pass_through_unchanged():
     lay = _small_layout(video=VideoSpec(1, 2, 2, 24, 2, 2), proprio=1)
     W = _weights(TINY)
