@@ -286,8 +286,9 @@ def oracle_sample(wl, quick: bool = False):
                              wl.mask_mode)
         t = time.perf_counter() - t0
         n = len(wl.sigmas) - 1
-        return (t * n * wl.batch, t, f"one oracle layer forward of a {lay.n_tokens}-token sequence (all rows), "
-                                     f"times {n} sampler steps and the batch of {wl.batch}")
+        return (t * n * wl.batch * wl.n_layers, t,
+                f"one oracle layer forward of a {lay.n_tokens}-token sequence (all rows), times {n} sampler steps, "
+                f"the batch of {wl.batch}" + (f" and the {wl.n_layers} layers" if wl.n_layers > 1 else ""))
     h_ar, hist, st = data
     lb = olayout.build_layout(synth.LayoutSpec(n_text=wl.layout.n_text, video=wl.layout.video),
                               tau_offset=len(hist))
@@ -362,6 +363,8 @@ def config_block(wl, lay, n_gpus):
             "ffn": wl.dims.ffn, "n_ar": lay.n_ar, "n_clean": lay.n_clean, "n_noisy": lay.n_noisy,
             "mask": wl.mask_mode, "sigma": [wl.sigmas[0], wl.sigmas[1]],
             **({"guidance": wl.guidance, "prompt_pairs": wl.batch // 2} if wl.guidance is not None else {}),
+            **({"layers": wl.n_layers, "distinct_layer_weight_draws": wl.weight_draws or wl.n_layers}
+               if wl.n_layers > 1 else {}),
             "l2": "flushed between steps (256 MiB write, outside the timed events)"}
 
 
@@ -411,7 +414,17 @@ def run_native(args, wl):
     def to_dev(u16):
         return torch.from_numpy(np.ascontiguousarray(u16).view(np.int16)).view(torch.bfloat16).to(dev)
 
-    w = {k: to_dev(v) for k, v in synth.make_weights(dims_s, wl.weight_seed).items()}
+    n_layers = wl.n_layers
+    if n_layers > 1:  # a stack: distinct draws go to the device once, layers share them
+        draws = synth.make_stack_weights(dims_s, wl.weight_seed, n_layers, distinct=wl.weight_draws)
+        dev_draws = {}
+        for dw in draws:
+            if id(dw) not in dev_draws:
+                dev_draws[id(dw)] = {k: to_dev(v) for k, v in dw.items()}
+        stack_w = [dev_draws[id(dw)] for dw in draws]
+        w = stack_w[-1]
+    else:
+        w = {k: to_dev(v) for k, v in synth.make_weights(dims_s, wl.weight_seed).items()}
     h_host = np.stack([synth.make_activations(N, d, wl.act_seed(rank * B + b)) for b in range(B)])
     guided = wl.guidance is not None
     if guided:  # each (cond, base) pair shares its DM rows; the prompts (AR rows) differ
@@ -424,12 +437,13 @@ def run_native(args, wl):
     dims = A.make_dims(dims_s.d_model, dims_s.n_heads, dims_s.n_kv_heads, dims_s.head_dim, dims_s.ffn,
                        dims_s.rope_sections, dims_s.rope_base, dims_s.eps)
     layer = A.MoTLayer(dims, w)
+    stack = A.MoTStack(dims, stack_w) if n_layers > 1 else None
     z0 = lay.n_ar + lay.n_clean  # first noisy row of a sequence
 
     def seq(n_cached):
         return layer.seq_desc(lay.n_ar, lay.n_clean, lay.n_noisy, B, cs, chunk, mode, n_cached=n_cached)
 
-    ws = layer.workspace(seq(0), dev)
+    ws = stack.workspace(seq(0), dev) if stack is not None else layer.workspace(seq(0), dev)
     flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
 
     # ---- the plan of one step: (n_cached, sigma, sigma_next) per layer call
@@ -459,6 +473,9 @@ def run_native(args, wl):
         return (N - n_cached) * N
 
     work = [stage_work(dims_s, B * (N - c), B * lay.n_noisy, B * layer_pairs(c)) for c, _, _ in calls]
+    if n_layers > 1:  # every layer runs the body stages; the head runs once
+        work = [{nm: ((f * n_layers, b * n_layers) if i < 7 else (f, b)) for i, (nm, (f, b)) in enumerate(wk.items())}
+                for wk in work]
     commit_flops = 2 * lay.n_noisy * d * dims_s.qkv_cols if kind == "stream" else 0
     tokens_per_step = {"layer": B * N, "sampler": B * N * len(calls), "stream": B * lay.n_noisy * len(calls)}[kind]
 
@@ -471,7 +488,14 @@ def run_native(args, wl):
         L.cosmot_mrope_table(pos.data_ptr(), N, dims_s.head_dim, dims_s.rope_sections, dims_s.rope_base,
                              cs.data_ptr(), sh)
         for i, (c, s0, s1) in enumerate(calls):
-            if stage_evs is not None:
+            if stack is not None:
+                if stage_evs is not None:
+                    L.cosmot_stack_forward_timed(dims, stack.cw, seqs[c], h.data_ptr(), h_out.data_ptr(), s0, s1,
+                                                 ws.data_ptr(), ws.numel(), sh, [e.cuda_event for e in stage_evs[i]])
+                else:
+                    L.cosmot_stack_forward(dims, stack.cw, seqs[c], h.data_ptr(), h_out.data_ptr(), s0, s1,
+                                           ws.data_ptr(), ws.numel(), sh)
+            elif stage_evs is not None:
                 L.cosmot_layer_forward_timed(dims, layer.cw, seqs[c], h.data_ptr(), h_out.data_ptr(), s0, s1,
                                              ws.data_ptr(), ws.numel(), sh, [e.cuda_event for e in stage_evs[i]],
                                              wl.guidance)
@@ -499,6 +523,9 @@ def run_native(args, wl):
 
     h_src = h.clone() if kind == "sampler" else None
     launches_per_step = 2 + n_stage * len(calls) + (2 if kind == "stream" else 0)
+    if n_layers > 1:  # 7 kernels per layer body, 2 for the head (the AR K/V copies are memcpys)
+        launches_per_step = 2 + (7 * n_layers + 2) * len(calls)
+    n_ev = 8 * n_layers + 2 if n_layers > 1 else n_stage + 1
 
     def new_events(n):
         evs = [torch.cuda.Event(enable_timing=True) for _ in range(n)]
@@ -515,7 +542,7 @@ def run_native(args, wl):
         raise RuntimeError(f"device status {L.status_string(st)} at {where}")
 
     starts, ends = new_events(args.steps), new_events(args.steps)
-    stage_evs = [[new_events(n_stage + 1) for _ in calls] for _ in range(args.steps)]
+    stage_evs = [[new_events(n_ev) for _ in calls] for _ in range(args.steps)]
     commit_evs = [new_events(2) for _ in range(args.steps)]
     torch.cuda.synchronize()
     if world > 1:
@@ -542,6 +569,13 @@ def run_native(args, wl):
     stage_ms = np.zeros(n_stage)  # per step, summed over the step's layer calls
     for per_call in stage_evs:
         for evs in per_call:
+            if n_layers > 1:
+                for lyr in range(n_layers):
+                    for j in range(7):
+                        stage_ms[j] += evs[8 * lyr + j].elapsed_time(evs[8 * lyr + j + 1])
+                stage_ms[7] += evs[8 * n_layers - 1].elapsed_time(evs[8 * n_layers])
+                stage_ms[8] += evs[8 * n_layers].elapsed_time(evs[8 * n_layers + 1])
+                continue
             for j in range(n_stage):
                 stage_ms[j] += evs[j].elapsed_time(evs[j + 1])
     stage_ms /= args.steps
@@ -578,7 +612,8 @@ def run_native(args, wl):
                "h2d_bytes_per_step": int(in_pin.numel() * 2), "d2h_bytes_per_step": int(out_pin.numel() * 2),
                "ms_per_step": e2e_ms / args.steps,
                "path": "cosmot_build_layout + cosmot_mrope_table + "
-                       + ("cosmot_layer_forward_cfg" if guided else "cosmot_layer_forward")
+                       + ("cosmot_stack_forward" if n_layers > 1 else
+                          "cosmot_layer_forward_cfg" if guided else "cosmot_layer_forward")
                        + (" + cosmot_layer_commit_kv" if kind == "stream" else "")
                        + ", pinned host input in, x' (noisy rows) out"}
 
@@ -612,7 +647,7 @@ def run_native(args, wl):
         dname = names[dom]
         f, b = wsum[dname]
         t_dom = stage_ms[dom] / 1e3  # per step; one launch per layer call
-        per_launch = len(calls)
+        per_launch = len(calls) * (n_layers if dom < 7 else 1)  # launches of the dominant kernel per step
         src = "attention.cu" if dname == "attention" else ("gemm.cu" if f else "elementwise.cu")
         traffic = None
         rec = NCU_TRAFFIC.get(f"{wl.name}:{dname}")
@@ -635,7 +670,8 @@ def run_native(args, wl):
         cfg = config_block(wl, lay, world)
         cfg["step"] = {"layer": ("one guided layer step: both passes of each prompt pair, the guided velocity "
                                   "and one Euler step" if guided else "one layer forward + Euler step"),
-                       "sampler": f"one {len(calls)}-step Euler sampling (step 1 all rows, then DM rows with the "
+                       "sampler": (f"{n_layers}-layer stack, " if n_layers > 1 else "")
+                                  + f"one {len(calls)}-step Euler sampling (step 1 all rows, then DM rows with the "
                                   f"AR K/V kept in the workspace)",
                        "stream": f"one streaming block: {len(calls)} denoising steps of {lay.n_noisy} tokens "
                                  f"against {N - lay.n_noisy} cached key rows, then the block's K/V commit"}[kind]

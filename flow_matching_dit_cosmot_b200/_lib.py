@@ -104,6 +104,11 @@ SIGNATURES = {
     "cosmot_layer_workspace_size": (c_i32, [_P(Dims), _P(SeqDesc), _P(ctypes.c_size_t)]),
     "cosmot_layer_forward": (c_i32, [_P(Dims), _P(LayerWeights), _P(SeqDesc), c_vp, c_vp, c_f64, c_f64, c_vp,
                                      ctypes.c_size_t, c_vp]),
+    "cosmot_stack_workspace_size": (c_i32, [_P(Dims), c_i32, _P(SeqDesc), _P(ctypes.c_size_t)]),
+    "cosmot_stack_forward": (c_i32, [_P(Dims), _P(LayerWeights), c_i32, _P(SeqDesc), c_vp, c_vp, c_f64, c_f64, c_vp,
+                                     ctypes.c_size_t, c_vp]),
+    "cosmot_stack_forward_timed": (c_i32, [_P(Dims), _P(LayerWeights), c_i32, _P(SeqDesc), c_vp, c_vp, c_f64, c_f64,
+                                           c_vp, ctypes.c_size_t, c_vp, _P(c_vp), c_i32]),
     "cosmot_layer_commit_kv": (c_i32, [_P(Dims), _P(LayerWeights), _P(SeqDesc), c_vp, c_i64, c_vp, ctypes.c_size_t,
                                        c_vp]),
     "cosmot_layer_forward_noalloc": (c_i32, [_P(Dims), _P(LayerWeights), _P(SeqDesc), c_vp, c_vp, c_f64, c_f64,
@@ -262,6 +267,33 @@ def cosmot_layer_commit_kv(dims: Dims, w: LayerWeights, seq: SeqDesc, h: int, ds
                            workspace_bytes: int, stream: int = 0, check=True):
     return _call("cosmot_layer_commit_kv", ctypes.byref(dims), ctypes.byref(w), ctypes.byref(seq), c_vp(h), dst_row,
                  c_vp(workspace), workspace_bytes, c_vp(stream), check=check)
+
+
+def cosmot_stack_workspace_size(dims: Dims, n_layers: int, seq: SeqDesc) -> int:
+    n = ctypes.c_size_t(0)
+    _call("cosmot_stack_workspace_size", ctypes.byref(dims), n_layers, ctypes.byref(seq), ctypes.byref(n))
+    return n.value
+
+
+def cosmot_stack_forward(dims: Dims, layers, seq: SeqDesc, h: int, h_out: int, sigma: float, sigma_next: float,
+                         workspace: int, workspace_bytes: int, stream: int = 0, check=True):
+    """`layers`: a ctypes array of LayerWeights (or a sequence of them)."""
+    if not isinstance(layers, ctypes.Array):
+        layers = (LayerWeights * len(layers))(*layers)
+    return _call("cosmot_stack_forward", ctypes.byref(dims), layers, len(layers), ctypes.byref(seq), c_vp(h),
+                 c_vp(h_out), sigma, sigma_next, c_vp(workspace), workspace_bytes, c_vp(stream), check=check)
+
+
+def cosmot_stack_forward_timed(dims: Dims, layers, seq: SeqDesc, h: int, h_out: int, sigma: float,
+                               sigma_next: float, workspace: int, workspace_bytes: int, stream: int, events,
+                               check=True):
+    """`events`: 8 * len(layers) + 2 raw cudaEvent_t handles (ints)."""
+    if not isinstance(layers, ctypes.Array):
+        layers = (LayerWeights * len(layers))(*layers)
+    arr = (c_vp * len(events))(*[c_vp(e) for e in events])
+    return _call("cosmot_stack_forward_timed", ctypes.byref(dims), layers, len(layers), ctypes.byref(seq), c_vp(h),
+                 c_vp(h_out), sigma, sigma_next, c_vp(workspace), workspace_bytes, c_vp(stream), arr, len(events),
+                 check=check)
 
 
 def cosmot_layer_forward_noalloc(dims: Dims, w: LayerWeights, seq: SeqDesc, h: int, h_out: int, sigma: float,

@@ -125,3 +125,37 @@ class MoTLayer:
         ws = workspace if workspace is not None else self.workspace(seq, h.device)
         L.cosmot_layer_forward(self.dims, self.cw, seq, ptr(h), ptr(h_out), float(sigma), float(sigma_next),
                                ptr(ws), ws.numel(), stream_handle(stream))
+
+
+class MoTStack:
+    """A stack of MoT layers with one velocity head (that of the last layer).
+
+    `layers` is a list of weight dicts as MoTLayer takes (bf16 CUDA tensors);
+    the same dict may appear more than once.
+    """
+
+    def __init__(self, dims: L.Dims, layers: list):
+        self.dims = dims
+        self.layers = [MoTLayer(dims, w) for w in layers]
+        self.cw = (L.LayerWeights * len(self.layers))(*[m.cw for m in self.layers])
+        self._ws = None
+
+    def seq_desc(self, *args, **kw) -> L.SeqDesc:
+        return self.layers[0].seq_desc(*args, **kw)
+
+    def workspace_bytes(self, seq: L.SeqDesc) -> int:
+        return L.cosmot_stack_workspace_size(self.dims, len(self.layers), seq)
+
+    def workspace(self, seq: L.SeqDesc, device="cuda") -> torch.Tensor:
+        n = self.workspace_bytes(seq)
+        if self._ws is None or self._ws.numel() < n:
+            self._ws = torch.empty((n,), dtype=torch.uint8, device=device)
+        return self._ws
+
+    def forward(self, h: torch.Tensor, h_out: torch.Tensor, sigma: float, sigma_next: float, seq: L.SeqDesc,
+                workspace: Optional[torch.Tensor] = None, stream=None):
+        """h^L into h_out; x' into the noisy rows of h (see cosmot_stack_forward)."""
+        _need_cuda(h, h_out)
+        ws = workspace if workspace is not None else self.workspace(seq, h.device)
+        L.cosmot_stack_forward(self.dims, self.cw, seq, ptr(h), ptr(h_out), sigma, sigma_next, ptr(ws), ws.numel(),
+                               stream_handle(stream))

@@ -119,33 +119,23 @@ struct StageMarks {
   }
 };
 
-cosmot_status layer_forward_impl(const cosmot_dims* dims, const cosmot_layer_weights* w, const cosmot_seq_desc* seq,
-                                 void* h, void* h_out, double sigma, double sigma_next, void* workspace,
-                                 size_t workspace_bytes, cosmot_stream_t stream, const cudaEvent_t* events,
-                                 const double* guidance = nullptr) {
-  const StageMarks M{events, reinterpret_cast<cudaStream_t>(stream)};
-  cosmot_status st = check_dims(dims);
-  if (st != COSMOT_OK) return st;
-  st = check_seq(seq);
-  if (st != COSMOT_OK) return st;
-  if (!w || !h || !h_out || !workspace) return COSMOT_ERR_INVALID_ARG;
-  if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return COSMOT_ERR_INVALID_ARG;
-  const WsLayout L = ws_layout(*dims, *seq);
-  if (workspace_bytes < L.total) return COSMOT_ERR_WORKSPACE;
-
-  const cosmot_dims& D = *dims;
-  const cosmot_seq_desc& S = *seq;
+// Steps 1-7 for the rows [n_cached, N) of every sequence: x_in -> x_out.
+// kv_cache (a stack's per-layer AR K/V store, or null): with n_cached == 0 the
+// AR rows' q/k/v rows are copied there after the QKV projection; with
+// n_cached > 0 they are copied back before the attention.
+cosmot_status layer_body(const cosmot_dims& D, const cosmot_layer_weights* w, const cosmot_seq_desc& S,
+                         const WsLayout& L, uint8_t* ws, const void* x_in, void* x_out, void* kv_cache,
+                         cosmot_stream_t stream, const StageMarks& M) {
+  cosmot_status st;
   const int64_t N = (int64_t)S.n_ar + S.n_clean + S.n_noisy;
   const int64_t d = D.d_model, F = D.ffn, hd = D.head_dim;
   const int64_t qc = (int64_t)D.n_heads * hd, kvc = (int64_t)D.n_kv_heads * hd, qkvc = qc + 2 * kvc;
   const int B = S.batch;
-  uint8_t* ws = static_cast<uint8_t*>(workspace);
   void* a = ws + L.a;
   void* qkv = ws + L.qkv;
   void* o = ws + L.o;
   void* h1 = ws + L.h1;
   void* u = ws + L.u;
-  uint16_t* hb = static_cast<uint16_t*>(h);
 
   // Row segments over the rows this call computes: AR rows through set 0, DM
   // rows through set 1; rows before n_cached keep their cached K/V.
@@ -157,7 +147,7 @@ cosmot_status layer_forward_impl(const cosmot_dims* dims, const cosmot_layer_wei
 
   if ((st = M.mark(0)) != COSMOT_OK) return st;
   // 1. pre-attention norm
-  st = cosmot_rmsnorm_routed(h, d, segs, ns, R.g1, G.g1, d, D.eps, a, d, stream);
+  st = cosmot_rmsnorm_routed(x_in, d, segs, ns, R.g1, G.g1, d, D.eps, a, d, stream);
   if (st != COSMOT_OK) return st;
   if ((st = M.mark(1)) != COSMOT_OK) return st;
   // 2. QKV projection with mRoPE on the Q and K heads
@@ -169,6 +159,15 @@ cosmot_status layer_forward_impl(const cosmot_dims* dims, const cosmot_layer_wei
   e.rope_period = N;
   st = cosmot_routed_linear(a, d, d, segs, ns, R.wqkv, G.wqkv, nullptr, nullptr, qkvc, qkv, qkvc, &e, stream);
   if (st != COSMOT_OK) return st;
+  if (kv_cache && S.n_ar > 0) {
+    // One strided copy per direction: the n_ar leading rows of every sequence.
+    const size_t width = (size_t)S.n_ar * qkvc * 2, seq_pitch = (size_t)N * qkvc * 2;
+    cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
+    const cudaError_t ce = c0 == 0
+        ? cudaMemcpy2DAsync(kv_cache, width, qkv, seq_pitch, width, B, cudaMemcpyDeviceToDevice, cs)
+        : cudaMemcpy2DAsync(qkv, seq_pitch, kv_cache, width, width, B, cudaMemcpyDeviceToDevice, cs);
+    if (ce != cudaSuccess) return COSMOT_ERR_CUDA;
+  }
   if ((st = M.mark(2)) != COSMOT_OK) return st;
   // 3. attention
   cosmot_attn_desc ad{};
@@ -191,7 +190,7 @@ cosmot_status layer_forward_impl(const cosmot_dims* dims, const cosmot_layer_wei
   // 4. output projection + residual
   e = cosmot_epilogue{};
   e.kind = COSMOT_EPI_RESIDUAL;
-  e.res = h;
+  e.res = x_in;
   e.ld_res = d;
   st = cosmot_routed_linear(o, qc, qc, segs, ns, R.wo, G.wo, nullptr, nullptr, d, h1, d, &e, stream);
   if (st != COSMOT_OK) return st;
@@ -211,13 +210,27 @@ cosmot_status layer_forward_impl(const cosmot_dims* dims, const cosmot_layer_wei
   e.kind = COSMOT_EPI_RESIDUAL;
   e.res = h1;
   e.ld_res = d;
-  st = cosmot_routed_linear(u, F, F, segs, ns, R.wd, G.wd, nullptr, nullptr, d, h_out, d, &e, stream);
+  st = cosmot_routed_linear(u, F, F, segs, ns, R.wd, G.wd, nullptr, nullptr, d, x_out, d, &e, stream);
   if (st != COSMOT_OK) return st;
+  return M.mark(7);
+}
+
+// Steps 8-9: final norm of the noisy rows of h_last, velocity head, Euler step
+// (or the guided step) into the noisy rows of `state`.
+cosmot_status layer_head(const cosmot_dims& D, const cosmot_layer_weights* w, const cosmot_seq_desc& S,
+                         const WsLayout& L, uint8_t* ws, const void* h_last, void* state, double sigma,
+                         double sigma_next, cosmot_stream_t stream, const StageMarks& M, const double* guidance) {
+  cosmot_status st;
+  const int64_t N = (int64_t)S.n_ar + S.n_clean + S.n_noisy;
+  const int64_t d = D.d_model;
+  const int B = S.batch;
+  void* a = ws + L.a;
+  void* u = ws + L.u;
+  uint16_t* hb = static_cast<uint16_t*>(state);
   if (S.n_noisy == 0) {
-    if ((st = M.mark(7)) != COSMOT_OK || (st = M.mark(8)) != COSMOT_OK) return st;
+    if ((st = M.mark(8)) != COSMOT_OK) return st;
     return M.mark(9);
   }
-  if ((st = M.mark(7)) != COSMOT_OK) return st;
   // 8. final norm of the noisy rows, packed into a
   cosmot_segment vs[kMaxBatch], ns_in[kMaxBatch];
   for (int b = 0; b < B; ++b) {
@@ -225,9 +238,10 @@ cosmot_status layer_forward_impl(const cosmot_dims* dims, const cosmot_layer_wei
     ns_in[b] = cosmot_segment{z0, z0 + S.n_noisy, (int64_t)b * S.n_noisy, 1, 0};
     vs[b] = cosmot_segment{(int64_t)b * S.n_noisy, (int64_t)(b + 1) * S.n_noisy, z0, 1, 0};
   }
-  st = cosmot_rmsnorm_routed(h_out, d, ns_in, B, w->gfin, w->gfin, d, D.eps, a, d, stream);
+  st = cosmot_rmsnorm_routed(h_last, d, ns_in, B, w->gfin, w->gfin, d, D.eps, a, d, stream);
   if (st != COSMOT_OK) return st;
   if ((st = M.mark(8)) != COSMOT_OK) return st;
+  cosmot_epilogue e{};
   if (guidance) {
     // 9'. guided step: velocities of every sequence into the (now free) FFN
     // hidden region, then v_base + w (v_cond - v_base) and the Euler step for
@@ -235,7 +249,6 @@ cosmot_status layer_forward_impl(const cosmot_dims* dims, const cosmot_layer_wei
     uint16_t* vbuf = static_cast<uint16_t*>(u);
     const int64_t nz = S.n_noisy;
     const cosmot_segment all{0, (int64_t)B * nz, 0, 1, 0};
-    e = cosmot_epilogue{};
     e.kind = COSMOT_EPI_NONE;
     st = cosmot_routed_linear(a, d, d, &all, 1, w->wvel, w->wvel, nullptr, nullptr, d, vbuf, d, &e, stream);
     if (st != COSMOT_OK) return st;
@@ -249,15 +262,94 @@ cosmot_status layer_forward_impl(const cosmot_dims* dims, const cosmot_layer_wei
     }
     return M.mark(9);
   }
-  // 9. velocity head with the Euler step, in place on the noisy rows of h
-  e = cosmot_epilogue{};
+  // 9. velocity head with the Euler step, in place on the noisy rows of the state
   e.kind = COSMOT_EPI_EULER;
-  e.x = h;
+  e.x = state;
   e.ld_x = d;
   e.dsigma = (float)(sigma_next - sigma);
   st = cosmot_routed_linear(a, d, d, vs, B, w->wvel, w->wvel, nullptr, nullptr, d, hb, d, &e, stream);
   if (st != COSMOT_OK) return st;
   return M.mark(9);
+}
+
+cosmot_status layer_forward_impl(const cosmot_dims* dims, const cosmot_layer_weights* w, const cosmot_seq_desc* seq,
+                                 void* h, void* h_out, double sigma, double sigma_next, void* workspace,
+                                 size_t workspace_bytes, cosmot_stream_t stream, const cudaEvent_t* events,
+                                 const double* guidance = nullptr) {
+  const StageMarks M{events, reinterpret_cast<cudaStream_t>(stream)};
+  cosmot_status st = check_dims(dims);
+  if (st != COSMOT_OK) return st;
+  st = check_seq(seq);
+  if (st != COSMOT_OK) return st;
+  if (!w || !h || !h_out || !workspace) return COSMOT_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return COSMOT_ERR_INVALID_ARG;
+  const WsLayout L = ws_layout(*dims, *seq);
+  if (workspace_bytes < L.total) return COSMOT_ERR_WORKSPACE;
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  st = layer_body(*dims, w, *seq, L, ws, h, h_out, nullptr, stream, M);
+  if (st != COSMOT_OK) return st;
+  return layer_head(*dims, w, *seq, L, ws, h_out, h, sigma, sigma_next, stream, M, guidance);
+}
+
+// Stack workspace: one layer's working set, a second hidden-state buffer for
+// the layer outputs, and the AR rows' q/k/v of every layer.
+struct StackWs {
+  WsLayout layer;
+  size_t tmp, cache, cache_per_layer, total;
+};
+
+StackWs stack_ws_layout(const cosmot_dims& d, int32_t n_layers, const cosmot_seq_desc& s) {
+  StackWs w;
+  w.layer = ws_layout(d, s);
+  size_t off = w.layer.total;
+  const size_t rows = (size_t)s.batch * (size_t)(s.n_ar + s.n_clean + s.n_noisy);
+  const size_t qkv_cols = (size_t)(d.n_heads + 2 * d.n_kv_heads) * d.head_dim;
+  w.tmp = off;
+  off += align256(rows * d.d_model * 2);
+  w.cache_per_layer = align256((size_t)s.batch * (size_t)s.n_ar * qkv_cols * 2);
+  w.cache = off;
+  off += (size_t)n_layers * w.cache_per_layer;
+  w.total = off;
+  return w;
+}
+
+constexpr int32_t kMaxLayers = 1024;
+
+// events (or null): 8 per layer (layer l records events[8l + i] before its
+// stage i, i < 7, and events[8l + 7] after its last stage), then 2 for the head
+// (before the velocity stage and after it).
+cosmot_status stack_forward_impl(const cosmot_dims* dims, const cosmot_layer_weights* layers, int32_t n_layers,
+                                 const cosmot_seq_desc* seq, void* h, void* h_out, double sigma, double sigma_next,
+                                 void* workspace, size_t workspace_bytes, cosmot_stream_t stream,
+                                 const cudaEvent_t* events) {
+  const cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
+  cosmot_status st = check_dims(dims);
+  if (st != COSMOT_OK) return st;
+  st = check_seq(seq);
+  if (st != COSMOT_OK) return st;
+  if (!layers || n_layers < 1 || n_layers > kMaxLayers || !h || !h_out || !workspace || h == h_out)
+    return COSMOT_ERR_INVALID_ARG;
+  // Clean DM rows read the noisy rows from the second layer on, so only the AR
+  // prefix has step-invariant K/V in a stack.
+  if (seq->n_cached != 0 && seq->n_cached != seq->n_ar) return COSMOT_ERR_UNSUPPORTED;
+  if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return COSMOT_ERR_INVALID_ARG;
+  const StackWs W = stack_ws_layout(*dims, n_layers, *seq);
+  if (workspace_bytes < W.total) return COSMOT_ERR_WORKSPACE;
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  // Layer outputs alternate between h_out and the workspace buffer so that the
+  // last one lands in h_out; the state h is only read until the final step.
+  for (int32_t l = 0; l < n_layers; ++l) {
+    void* out = ((n_layers - 1 - l) % 2 == 0) ? h_out : static_cast<void*>(ws + W.tmp);
+    const void* in = l == 0 ? h : (((n_layers - l) % 2 == 0) ? h_out : static_cast<void*>(ws + W.tmp));
+    const StageMarks M{events ? events + 8 * l : nullptr, cs};
+    st = layer_body(*dims, &layers[l], *seq, W.layer, ws, in, out, ws + W.cache + (size_t)l * W.cache_per_layer,
+                    stream, M);
+    if (st != COSMOT_OK) return st;
+  }
+  // the head's marks 8 and 9 land at events[8 n_layers] and [8 n_layers + 1]
+  const StageMarks MH{events ? events + 8 * (n_layers - 1) : nullptr, cs};
+  return layer_head(*dims, &layers[n_layers - 1], *seq, W.layer, ws, h_out, h, sigma, sigma_next, stream, MH,
+                    nullptr);
 }
 
 }  // namespace
@@ -320,6 +412,38 @@ cosmot_status cosmot_layer_commit_kv(const cosmot_dims* dims, const cosmot_layer
   e.rope_period = N;
   return cosmot_routed_linear(ws + L.a, d, d, dst, ns, R.wqkv, G.wqkv, nullptr, nullptr, qkvc, ws + L.qkv, qkvc, &e,
                               stream);
+}
+
+cosmot_status cosmot_stack_workspace_size(const cosmot_dims* dims, int32_t n_layers, const cosmot_seq_desc* seq,
+                                          size_t* bytes) {
+  using namespace cosmot;
+  if (!bytes) return COSMOT_ERR_INVALID_ARG;
+  cosmot_status st = check_dims(dims);
+  if (st != COSMOT_OK) return st;
+  if (!seq || seq->batch < 1 || seq->batch > kMaxBatch || seq->n_ar < 0 || seq->n_clean < 0 || seq->n_noisy < 0 ||
+      n_layers < 1 || n_layers > kMaxLayers)
+    return COSMOT_ERR_INVALID_ARG;
+  *bytes = stack_ws_layout(*dims, n_layers, *seq).total;
+  return COSMOT_OK;
+}
+
+cosmot_status cosmot_stack_forward(const cosmot_dims* dims, const cosmot_layer_weights* layers, int32_t n_layers,
+                                   const cosmot_seq_desc* seq, void* h, void* h_out, double sigma, double sigma_next,
+                                   void* workspace, size_t workspace_bytes, cosmot_stream_t stream) {
+  return cosmot::stack_forward_impl(dims, layers, n_layers, seq, h, h_out, sigma, sigma_next, workspace,
+                                    workspace_bytes, stream, nullptr);
+}
+
+cosmot_status cosmot_stack_forward_timed(const cosmot_dims* dims, const cosmot_layer_weights* layers,
+                                         int32_t n_layers, const cosmot_seq_desc* seq, void* h, void* h_out,
+                                         double sigma, double sigma_next, void* workspace, size_t workspace_bytes,
+                                         cosmot_stream_t stream, void* const* stage_events, int32_t n_events) {
+  if (!stage_events || n_layers < 1 || n_layers > cosmot::kMaxLayers || n_events != 8 * n_layers + 2)
+    return COSMOT_ERR_INVALID_ARG;
+  for (int i = 0; i < n_events; ++i)
+    if (!stage_events[i]) return COSMOT_ERR_INVALID_ARG;
+  return cosmot::stack_forward_impl(dims, layers, n_layers, seq, h, h_out, sigma, sigma_next, workspace,
+                                    workspace_bytes, stream, reinterpret_cast<const cudaEvent_t*>(stage_events));
 }
 
 cosmot_status cosmot_layer_forward_timed(const cosmot_dims* dims, const cosmot_layer_weights* w,

@@ -365,6 +365,52 @@ COSMOT_API cosmot_status cosmot_layer_commit_kv(const cosmot_dims* dims, const c
                                                 void* workspace, size_t workspace_bytes, cosmot_stream_t stream);
 
 /*
+ * A stack of MoT layers and one sampler step ("Cosmos 3 方法原理全解" §3 for the
+ * layer, §12.4 for the released models, which stack 28, 36 or 64 of them; §7.2
+ * for the step):
+ *     h^0 = h;  h^l = layer_l(h^{l-1})  for l = 1 .. n_layers
+ *     noisy rows:  v = RMSNorm(h^L; gfin) W_vel^T,  h <- h + (sigma_next - sigma) v
+ * layers: host array of n_layers weight descriptors (device pointers inside),
+ *         applied in order; the final norm and velocity head are the gfin and
+ *         wvel of the last entry (the others' are not read).
+ * h:      [batch, N, d] bf16 device, the stack input; its noisy rows are the
+ *         state and receive x'.  Its other rows are not written.
+ * h_out:  [batch, N, d] bf16 device, receives h^L (must not alias h).
+ * seq:    as for cosmot_layer_forward, with n_cached 0 or n_ar only.  With 0
+ *         every row is computed and the q/k/v rows of the AR prefix of every
+ *         layer are kept in the workspace; with n_ar those are reused (a
+ *         sampler's later steps: AR rows never read DM rows at any depth) and
+ *         rows < n_ar of h_out are not written.  Clean DM rows read the noisy
+ *         rows from the second layer on, so no longer prefix is step-invariant:
+ *         other values return COSMOT_ERR_UNSUPPORTED.
+ * workspace: cosmot_stack_workspace_size bytes, 256-byte aligned, owned by the
+ *         caller and kept between the steps of one sampling.
+ * Errors: INVALID_ARG for null pointers, h == h_out, n_layers outside
+ * [1, 1024] or bad dims/seq; WORKSPACE if the workspace is too small.
+ */
+COSMOT_API cosmot_status cosmot_stack_workspace_size(const cosmot_dims* dims, int32_t n_layers,
+                                                     const cosmot_seq_desc* seq, size_t* bytes);
+COSMOT_API cosmot_status cosmot_stack_forward(const cosmot_dims* dims, const cosmot_layer_weights* layers,
+                                              int32_t n_layers, const cosmot_seq_desc* seq, void* h, void* h_out,
+                                              double sigma, double sigma_next, void* workspace,
+                                              size_t workspace_bytes, cosmot_stream_t stream);
+
+/*
+ * cosmot_stack_forward with CUDA events (cudaEvent_t, created by the caller on
+ * the current device) recorded on the stream around every stage:
+ * n_events = 8 * n_layers + 2.  Layer l records events[8l + i] before its stage
+ * i (COSMOT_STAGE_NORM1 .. COSMOT_STAGE_DOWN_RESIDUAL) and events[8l + 7]
+ * after its last one (where the final-norm stage starts); events[8 n_layers]
+ * is recorded before the velocity stage and events[8 n_layers + 1] after it.
+ * The computation is identical to cosmot_stack_forward.
+ */
+COSMOT_API cosmot_status cosmot_stack_forward_timed(const cosmot_dims* dims, const cosmot_layer_weights* layers,
+                                                    int32_t n_layers, const cosmot_seq_desc* seq, void* h,
+                                                    void* h_out, double sigma, double sigma_next, void* workspace,
+                                                    size_t workspace_bytes, cosmot_stream_t stream,
+                                                    void* const* stage_events, int32_t n_events);
+
+/*
  * cosmot_layer_forward without a caller workspace, for callers that may not
  * allocate device memory while they run: a control loop with a hard per-step
  * deadline (cudaMalloc can synchronise the device and stall for an unbounded

@@ -125,6 +125,8 @@ class Workload:
     mask_mode: str = "full"  # "full" | "block_causal"
     stream: Optional[StreamSpec] = None
     guidance: Optional[float] = None  # classifier-free guidance weight; batch = (cond, base) pairs
+    n_layers: int = 1  # > 1: a layer stack with one velocity head
+    weight_draws: int = 0  # > 0: that many distinct layer weight draws, cycled over the stack
     description: str = ""
     extra: dict = field(default_factory=dict)
 
@@ -140,6 +142,12 @@ _NANO_LIKE = ModelDims(d_model=4096, n_heads=32, n_kv_heads=32, head_dim=128,
                        ffn=14336, rope_sections=(16, 24, 24))
 _SUPER_LIKE = ModelDims(d_model=5120, n_heads=40, n_kv_heads=40, head_dim=128,
                         ffn=20480, rope_sections=(16, 24, 24))
+# Page-exact widths ("Cosmos 3 方法原理全解" §12.4 model table): Nano 36 layers,
+# hidden 4096, 32 query / 8 key-value heads, FFN 12288; Super 64 layers, hidden
+# 5120, 64 / 8 heads, FFN 25600.  Head size 128 in both (not printed; the
+# Qwen3-VL-initialised Reasoner uses 128, so Super's query width is 8192).
+NANO = ModelDims(d_model=4096, n_heads=32, n_kv_heads=8, head_dim=128, ffn=12288, rope_sections=(16, 24, 24))
+SUPER = ModelDims(d_model=5120, n_heads=64, n_kv_heads=8, head_dim=128, ffn=25600, rope_sections=(16, 24, 24))
 _TINY = ModelDims(d_model=256, n_heads=4, n_kv_heads=4, head_dim=64, ffn=1024,
                   rope_sections=(8, 12, 12))
 
@@ -183,6 +191,25 @@ PRESETS = {
         sigmas=(1.0, 0.75, 0.5, 0.25, 0.0), mask_mode="block_causal",
         stream=StreamSpec(cached_blocks=8, blocks=16, steps_per_block=4),
         description="streaming block-causal rollout: 1560-token blocks, 8 cached blocks, 66 AR"),
+    "t2v480_nano": Workload(
+        name="t2v480_nano", config_id=2, dims=NANO,
+        layout=LayoutSpec(n_text=256, video=VideoSpec(1, 15, 26, 24, 0, 48)),
+        sigmas=(1.0, 0.97),
+        description="480p text-to-video layer at Nano's widths: d 4096, 32 query / 8 key-value heads of 128, "
+                    "FFN 12288; 258 AR + 18720 noisy"),
+    "i2v720_super": Workload(
+        name="i2v720_super", config_id=5, dims=SUPER,
+        layout=LayoutSpec(n_text=512, video=VideoSpec(1, 22, 40, 24, 1, 47)),
+        sigmas=(1.0, 0.97),
+        description="720p image-to-video layer at Super's widths: d 5120, 64 query / 8 key-value heads of 128, "
+                    "FFN 25600; 514 AR + 880 clean + 41360 noisy"),
+    "droid_nano36": Workload(
+        name="droid_nano36", config_id=3, dims=NANO,
+        layout=LayoutSpec(n_text=128, video=VideoSpec(3, 6, 10, 15, 1, 2),
+                          action_noisy=32, action_hz=15, proprio=1),
+        sigmas=_linear_sigmas(10), n_layers=36, weight_draws=4,
+        description="DROID policy step through Nano's 36-layer stack (page widths), 10 Euler steps; 4 distinct "
+                    "layer weight draws of 0.77 GB cycled over the 36 layers"),
     "i2v720": Workload(
         name="i2v720", config_id=5, dims=_SUPER_LIKE,
         layout=LayoutSpec(n_text=512, video=VideoSpec(1, 22, 40, 24, 1, 47)),

@@ -110,3 +110,30 @@ def test_layer_workspace_and_validation():
     bad = A.make_dims(4096, 32, 5, 128, 14336, (16, 24, 24))
     assert lib.cosmot_layer_forward(ctypes.byref(bad), ctypes.byref(A.L.LayerWeights()), ctypes.byref(seq), 256, 256,
                                     1.0, 0.97, 256, n, None) == A.L.COSMOT_ERR_INVALID_ARG
+
+
+def test_stack_workspace_and_validation():
+    """Stack workspace = one layer's working set + a hidden buffer + the AR
+    q/k/v rows of every layer; argument errors return before any launch."""
+    from flow_matching_dit_cosmot_b200 import api as A
+    dm = synth.preset("droid_nano36").dims
+    dims = A.make_dims(dm.d_model, dm.n_heads, dm.n_kv_heads, dm.head_dim, dm.ffn, dm.rope_sections)
+    seq = A.L.SeqDesc(130, 181, 392, 1, 0, 0, 16, 0)
+    one = A.L.cosmot_layer_workspace_size(dims, seq)
+    n36 = A.L.cosmot_stack_workspace_size(dims, 36, seq)
+    qkv_cols = (32 + 2 * 8) * 128
+    per_layer_cache = 130 * qkv_cols * 2
+    hidden = 703 * 4096 * 2
+    assert one + hidden + 36 * per_layer_cache <= n36 <= one + hidden + 36 * (per_layer_cache + 256) + 256
+    lib = A.L.lib()
+    arr = (A.L.LayerWeights * 2)()
+    args = lambda layers, n, s, h, ho, ws, wsb: (ctypes.byref(dims), layers, n, ctypes.byref(s), h, ho, 1.0, 0.9, ws,
+                                                 wsb, None)
+    n2 = A.L.cosmot_stack_workspace_size(dims, 2, seq)
+    assert lib.cosmot_stack_forward(*args(arr, 2, seq, 256, 256, 256, n2)) == A.L.COSMOT_ERR_INVALID_ARG  # h == h_out
+    assert lib.cosmot_stack_forward(*args(arr, 0, seq, 256, 512, 256, n2)) == A.L.COSMOT_ERR_INVALID_ARG
+    assert lib.cosmot_stack_forward(*args(arr, 2, seq, 256, 512, 256, n2 - 256)) == A.L.COSMOT_ERR_WORKSPACE
+    cached = A.L.SeqDesc(130, 181, 392, 1, 0, 311, 16, 0)  # clean prefix: not step-invariant in a stack
+    assert lib.cosmot_stack_forward(*args(arr, 2, cached, 256, 512, 256, n2)) == A.L.COSMOT_ERR_UNSUPPORTED
+    with pytest.raises(Exception):
+        A.L.cosmot_stack_workspace_size(dims, 0, seq)

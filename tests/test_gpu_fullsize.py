@@ -35,7 +35,7 @@ def _weights(wl):
     return _W[wl.name]
 
 
-@pytest.mark.parametrize("name", ["t2v480", "i2v720"])
+@pytest.mark.parametrize("name", ["t2v480", "i2v720", "t2v480_nano", "i2v720_super"])
 def test_full_size_layer_on_sampled_rows(name):
     wl = synth.preset(name)
     w, dw, W = _weights(wl)
