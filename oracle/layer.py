@@ -37,7 +37,7 @@ from dataclasses import dataclass
 import numpy as np
 
 from . import rope as _rope
-from .layout import REGION_AR, REGION_CLEAN, REGION_NOISY
+from .layout import MOD_ACTION, REGION_AR, REGION_CLEAN, REGION_NOISY
 from .mask import allow_matrix
 
 
@@ -303,6 +303,80 @@ def stack_sample(dims, layers, h, lay, sigmas, mode="full"):
         h[noisy] = out["x_new"][noisy]
         outs.append(out)
     return h, outs
+
+
+def shift_sigmas(n_steps: int, shift: float) -> np.ndarray:
+    """Sampler noise levels with the flow shift ("Cosmos 3 方法原理全解" §6.3:
+    t_bar = 1 - t, sigma = s t_bar / (1 + (s - 1) t_bar)), evaluated on the
+    uniform grid t_k = k / n_steps, k = 0 .. n_steps: sigma_0 = 1, sigma_n = 0.
+
+    Reading: the pages define the shift for the training-time noise draw and
+    quote an inference "shift" beside the step count; applying the same map to
+    the uniform inference grid is the plainest reading.
+    """
+    if n_steps < 1 or not shift > 0:
+        raise ValueError("n_steps >= 1 and shift > 0 required")
+    t_bar = 1.0 - np.arange(n_steps + 1, dtype=np.float64) / n_steps
+    return shift * t_bar / (1.0 + (shift - 1.0) * t_bar)
+
+
+def action_embed(x_a, w_in):
+    """Domain-specific action input projection ("Cosmos 3 方法原理全解" §4.2:
+    normalised actions, clean or noisy, enter the Generator through W_in):
+    rows x_a [n, C_a] -> x_a W_in^T [n, d]."""
+    return np.asarray(x_a, np.float64) @ np.asarray(w_in, np.float64).T
+
+
+def action_velocity(dims, h_last, g_fin, w_out):
+    """Action velocity from the last hidden states of the noisy action rows
+    (§4.2: W_out returns the velocity at the current sigma, in the normalised
+    action space): RMSNorm with the final DM gain, then W_out [C_a, d]."""
+    return rms_norm(np.asarray(h_last, np.float64), g_fin, dims.eps) @ np.asarray(w_out, np.float64).T
+
+
+def policy_step(dims, layers, h, x_a, w_in, w_out, lay, sigma, sigma_next, sigma_a, sigma_a_next, mode="full",
+                guidance=None, h_base=None, x_a_base=None):
+    """One sampler step of a policy with an action head (§4.2, §7.2, §7.3).
+
+    The action rows of the layer input (clean and noisy, in packed order) are
+    x_a W_in^T; the stack runs; the other noisy rows take the hidden-space
+    velocity head and the Euler step with (sigma, sigma_next); the noisy action
+    rows take v_a = RMSNorm(h^L; g_fin) W_out^T and x_a' = x_a + (sigma_a_next
+    - sigma_a) v_a (each modality has its own noise level, §6.3).  With a
+    guidance weight the baseline pass (h_base, x_a_base: same DM rows, other
+    AR rows) runs too and both velocities are combined before the steps.
+
+    Returns (h_new, x_a_new): h_new is the stack input (action rows = x_a
+    W_in^T) with its noisy non-action rows stepped; x_a_new has its noisy rows
+    stepped.
+    """
+    act = lay.modality == MOD_ACTION
+    noisy = lay.region == REGION_NOISY
+    act_noisy = act & noisy
+    vid_noisy = noisy & ~act
+
+    def forward(h_in, xa):
+        hh = np.array(h_in, dtype=np.float64)
+        hh[act] = action_embed(xa, w_in)
+        x = hh
+        for W in layers:
+            x = layer_forward(dims, W, x, lay.region, lay.pos, lay.chunk, sigma, sigma_next, mode, head=False)["h2"]
+        last = layers[-1]
+        v = rms_norm(x[vid_noisy], last.gfin, dims.eps) @ last.wvel.T
+        va = action_velocity(dims, x[act_noisy], last.gfin, w_out)
+        return hh, v, va
+
+    hh, v, va = forward(h, x_a)
+    if guidance is not None:
+        _, vb, vab = forward(h_base, x_a_base)
+        v = cfg_combine(v, vb, guidance)
+        va = cfg_combine(va, vab, guidance)
+    h_new = hh  # the action rows hold the embedding of x_a (the state is x_a)
+    h_new[vid_noisy] = euler_step(h_new[vid_noisy], v, sigma, sigma_next)
+    x_new = np.array(x_a, dtype=np.float64)
+    n_act_clean = int((act & (lay.region == REGION_CLEAN)).sum())
+    x_new[n_act_clean:] = euler_step(x_new[n_act_clean:], va, sigma_a, sigma_a_next)
+    return h_new, x_new
 
 
 def sample(dims, W, h, lay, sigmas, mode="full"):

@@ -369,6 +369,89 @@ def test_stack_clean_rows_read_noisy_rows_from_the_second_layer():
         assert (d > 1e-6) == changes, (mode, d)
 
 
+# ---------------------------------------------------------------- schedules and action heads
+
+def test_shift_schedule_properties():
+    """sigma = s t_bar / (1 + (s - 1) t_bar): identity at s = 1, endpoints 1
+    and 0, strictly decreasing, and t_bar = sigma / (s - (s - 1) sigma) maps it
+    back onto the uniform grid (the closed-form inverse)."""
+    np.testing.assert_array_equal(layer.shift_sigmas(10, 1.0), 1.0 - np.arange(11) / 10)
+    for s_ in (0.5, 3.0, 5.0, 10.0):
+        sig = layer.shift_sigmas(7, s_)
+        assert sig[0] == 1.0 and sig[-1] == 0.0
+        assert np.all(np.diff(sig) < 0)
+        t_bar = sig / (s_ - (s_ - 1.0) * sig)
+        np.testing.assert_allclose(t_bar, 1.0 - np.arange(8) / 7, rtol=0, atol=1e-15)
+    # a shift above 1 spends more of the steps at high noise
+    assert np.all(layer.shift_sigmas(4, 5.0)[1:-1] > layer.shift_sigmas(4, 1.0)[1:-1])
+    from fractions import Fraction as Fr
+    want = [Fr(1), Fr(15, 16), Fr(5, 6), Fr(5, 8), Fr(0)]  # 4 steps, shift 5, by hand
+    np.testing.assert_allclose(layer.shift_sigmas(4, 5.0), [float(v) for v in want], rtol=0, atol=1e-15)
+
+
+def _policy_case(n_layers=2, residual_only=False):
+    spec = LayoutSpec(n_text=5, video=VideoSpec(1, 2, 3, 24, 1, 1), action_clean=3, action_noisy=4, action_hz=15)
+    lay = layout.build_layout(spec)
+    Ws = _stack(TINY, n_layers)
+    if residual_only:
+        for W in Ws:
+            for s_ in (W.R, W.G):
+                s_.wo = np.zeros_like(s_.wo)
+                s_.wd = np.zeros_like(s_.wd)
+    ca = 6
+    w_in = synth.bf16_to_f64(synth.normal_bf16((TINY.d_model, ca), 40, 1, std=0.3))
+    w_out = synth.bf16_to_f64(synth.normal_bf16((ca, TINY.d_model), 41, 1, std=0.1))
+    x_a = synth.bf16_to_f64(synth.normal_bf16((7, ca), 42, 1))
+    h = _h(lay.n_tokens, TINY.d_model)
+    return lay, Ws, w_in, w_out, x_a, h
+
+
+def test_policy_step_with_residual_only_layers_is_the_closed_form():
+    """Residual-only layers pass the embedded actions through, so the action
+    velocity is RMSNorm(x_a W_in^T; g_fin) W_out^T exactly (closed form); clean
+    actions stay put; the action rows of h carry the embedding."""
+    lay, Ws, w_in, w_out, x_a, h = _policy_case(residual_only=True)
+    h_new, xa_new = layer.policy_step(TINY, Ws, h, x_a, w_in, w_out, lay, 0.9, 0.7, 0.6, 0.5)
+    e = x_a[3:] @ w_in.T
+    v = (e / np.sqrt(np.mean(e * e, axis=1, keepdims=True) + TINY.eps) * Ws[-1].gfin) @ w_out.T
+    np.testing.assert_allclose(xa_new[3:], x_a[3:] - 0.1 * v, rtol=0, atol=1e-12)
+    np.testing.assert_array_equal(xa_new[:3], x_a[:3])
+    act = lay.modality == layout.MOD_ACTION
+    np.testing.assert_allclose(h_new[act], x_a @ w_in.T, rtol=0, atol=1e-12)
+
+
+def test_policy_step_modalities_have_their_own_noise_levels():
+    lay, Ws, w_in, w_out, x_a, h = _policy_case()
+    vid = (lay.region == layout.REGION_NOISY) & (lay.modality != layout.MOD_ACTION)
+    h1, xa1 = layer.policy_step(TINY, Ws, h, x_a, w_in, w_out, lay, 0.9, 0.7, 0.6, 0.6)
+    np.testing.assert_array_equal(xa1, x_a)  # action noise level held: actions do not move
+    assert np.abs(h1[vid] - h[vid]).max() > 1e-4
+    h2, xa2 = layer.policy_step(TINY, Ws, h, x_a, w_in, w_out, lay, 0.9, 0.9, 0.6, 0.4)
+    np.testing.assert_array_equal(h2[vid], h[vid])  # video held
+    assert np.abs(xa2[3:] - x_a[3:]).max() > 1e-4
+    # the same forward pass: the action step is linear in its sigma step
+    _, xa3 = layer.policy_step(TINY, Ws, h, x_a, w_in, w_out, lay, 0.9, 0.9, 0.6, 0.2)
+    np.testing.assert_allclose(xa3[3:] - x_a[3:], 2.0 * (xa2[3:] - x_a[3:]), rtol=1e-12, atol=1e-15)
+
+
+def test_policy_step_guidance_limits():
+    """Guidance 1 is the conditioned pass alone; guidance 0 the baseline alone."""
+    lay, Ws, w_in, w_out, x_a, h = _policy_case()
+    hb = h.copy()
+    hb[:lay.n_ar] = _h(lay.n_ar, TINY.d_model, seed=99)
+    c = layer.policy_step(TINY, Ws, h, x_a, w_in, w_out, lay, 0.9, 0.7, 0.6, 0.5)
+    b = layer.policy_step(TINY, Ws, hb, x_a, w_in, w_out, lay, 0.9, 0.7, 0.6, 0.5)
+    g1 = layer.policy_step(TINY, Ws, h, x_a, w_in, w_out, lay, 0.9, 0.7, 0.6, 0.5, guidance=1.0, h_base=hb,
+                           x_a_base=x_a)
+    g0 = layer.policy_step(TINY, Ws, h, x_a, w_in, w_out, lay, 0.9, 0.7, 0.6, 0.5, guidance=0.0, h_base=hb,
+                           x_a_base=x_a)
+    noisy = lay.region == layout.REGION_NOISY
+    np.testing.assert_allclose(g1[1], c[1], rtol=0, atol=1e-13)
+    np.testing.assert_allclose(g0[1], b[1], rtol=0, atol=1e-13)
+    np.testing.assert_allclose(g1[0][noisy], c[0][noisy], rtol=0, atol=1e-13)
+    np.testing.assert_allclose(g0[0][noisy], b[0][noisy], rtol=0, atol=1e-13)
+
+
 def test_clean_rows_pass_through_unchanged():
     lay = _small_layout(video=VideoSpec(1, 2, 2, 24, 2, 2), proprio=1)
     W = _weights(TINY)
