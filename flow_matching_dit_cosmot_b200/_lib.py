@@ -75,6 +75,12 @@ class LayerWeights(ctypes.Structure):
     _fields_ = [("set", SetWeights * 2), ("gfin", c_vp), ("wvel", c_vp)]
 
 
+class ActionDesc(ctypes.Structure):
+    _fields_ = [("action_dim", c_i32), ("n_clean", c_i32), ("n_noisy", c_i32), ("clean_row", c_i32),
+                ("w_in", c_vp), ("w_out", c_vp), ("x", c_vp), ("ld_x", c_i64), ("sigma", c_f64),
+                ("sigma_next", c_f64)]
+
+
 class SeqDesc(ctypes.Structure):
     _fields_ = [("n_ar", c_i32), ("n_clean", c_i32), ("n_noisy", c_i32), ("batch", c_i32),
                 ("mask_mode", c_i32), ("n_cached", c_i32), ("rope_cs", c_vp), ("chunk", c_vp)]
@@ -104,6 +110,12 @@ SIGNATURES = {
     "cosmot_layer_workspace_size": (c_i32, [_P(Dims), _P(SeqDesc), _P(ctypes.c_size_t)]),
     "cosmot_layer_forward": (c_i32, [_P(Dims), _P(LayerWeights), _P(SeqDesc), c_vp, c_vp, c_f64, c_f64, c_vp,
                                      ctypes.c_size_t, c_vp]),
+    "cosmot_flow_shift_sigmas": (c_i32, [c_i32, c_f64, _P(c_f64)]),
+    "cosmot_action_embed": (c_i32, [c_vp, c_i64, _P(Segment), c_i32, c_vp, c_i32, c_i32, c_vp, c_i64, c_vp]),
+    "cosmot_action_head": (c_i32, [c_vp, c_i64, _P(Segment), c_i32, c_vp, c_f32, c_vp, c_i32, c_i32, c_vp, c_i64, c_f64,
+                                   c_f64, _P(c_f64), c_vp]),
+    "cosmot_policy_step": (c_i32, [_P(Dims), _P(LayerWeights), c_i32, _P(SeqDesc), _P(ActionDesc), c_vp, c_vp, c_f64,
+                                   c_f64, _P(c_f64), c_vp, ctypes.c_size_t, c_vp, _P(c_vp), c_i32]),
     "cosmot_stack_workspace_size": (c_i32, [_P(Dims), c_i32, _P(SeqDesc), _P(ctypes.c_size_t)]),
     "cosmot_stack_forward": (c_i32, [_P(Dims), _P(LayerWeights), c_i32, _P(SeqDesc), c_vp, c_vp, c_f64, c_f64, c_vp,
                                      ctypes.c_size_t, c_vp]),
@@ -267,6 +279,47 @@ def cosmot_layer_commit_kv(dims: Dims, w: LayerWeights, seq: SeqDesc, h: int, ds
                            workspace_bytes: int, stream: int = 0, check=True):
     return _call("cosmot_layer_commit_kv", ctypes.byref(dims), ctypes.byref(w), ctypes.byref(seq), c_vp(h), dst_row,
                  c_vp(workspace), workspace_bytes, c_vp(stream), check=check)
+
+
+def cosmot_flow_shift_sigmas(n_steps: int, shift: float) -> list:
+    out = (c_f64 * (n_steps + 1))()
+    _call("cosmot_flow_shift_sigmas", n_steps, shift, out)
+    return list(out)
+
+
+def _segs(segs):
+    arr = (Segment * len(segs))(*[Segment(*s) for s in segs])
+    return arr, len(segs)
+
+
+def cosmot_action_embed(x: int, ld_x: int, segs, w_in: int, action_dim: int, d_model: int, h: int, ld_h: int,
+                        stream: int = 0, check=True):
+    """`segs`: (row_begin, row_end, out_row, weight_set, reserved) tuples."""
+    arr, n = _segs(segs)
+    return _call("cosmot_action_embed", c_vp(x), ld_x, arr, n, c_vp(w_in), action_dim, d_model, c_vp(h), ld_h,
+                 c_vp(stream), check=check)
+
+
+def cosmot_action_head(h_last: int, ld_h: int, segs, g_fin: int, eps: float, w_out: int, action_dim: int,
+                       d_model: int, x: int, ld_x: int, sigma: float, sigma_next: float, guidance=None,
+                       stream: int = 0, check=True):
+    arr, n = _segs(segs)
+    g = ctypes.byref(c_f64(guidance)) if guidance is not None else None
+    return _call("cosmot_action_head", c_vp(h_last), ld_h, arr, n, c_vp(g_fin), eps, c_vp(w_out), action_dim,
+                 d_model, c_vp(x), ld_x, sigma, sigma_next, g, c_vp(stream), check=check)
+
+
+def cosmot_policy_step(dims: Dims, layers, seq: SeqDesc, act: ActionDesc, h: int, h_out: int, sigma: float,
+                       sigma_next: float, guidance, workspace: int, workspace_bytes: int, stream: int = 0,
+                       events=None, check=True):
+    """`events`: None, or 8 * len(layers) + 2 raw cudaEvent_t handles (ints)."""
+    if not isinstance(layers, ctypes.Array):
+        layers = (LayerWeights * len(layers))(*layers)
+    g = ctypes.byref(c_f64(guidance)) if guidance is not None else None
+    arr = (c_vp * len(events))(*[c_vp(e) for e in events]) if events else None
+    return _call("cosmot_policy_step", ctypes.byref(dims), layers, len(layers), ctypes.byref(seq), ctypes.byref(act),
+                 c_vp(h), c_vp(h_out), sigma, sigma_next, g, c_vp(workspace), workspace_bytes, c_vp(stream), arr,
+                 len(events) if events else 0, check=check)
 
 
 def cosmot_stack_workspace_size(dims: Dims, n_layers: int, seq: SeqDesc) -> int:

@@ -215,11 +215,12 @@ cosmot_status layer_body(const cosmot_dims& D, const cosmot_layer_weights* w, co
   return M.mark(7);
 }
 
-// Steps 8-9: final norm of the noisy rows of h_last, velocity head, Euler step
-// (or the guided step) into the noisy rows of `state`.
+// Steps 8-9: final norm of the first nz noisy rows of h_last, velocity head,
+// Euler step (or the guided step) into the same rows of `state`.
 cosmot_status layer_head(const cosmot_dims& D, const cosmot_layer_weights* w, const cosmot_seq_desc& S,
                          const WsLayout& L, uint8_t* ws, const void* h_last, void* state, double sigma,
-                         double sigma_next, cosmot_stream_t stream, const StageMarks& M, const double* guidance) {
+                         double sigma_next, cosmot_stream_t stream, const StageMarks& M, const double* guidance,
+                         int64_t nz) {
   cosmot_status st;
   const int64_t N = (int64_t)S.n_ar + S.n_clean + S.n_noisy;
   const int64_t d = D.d_model;
@@ -227,7 +228,7 @@ cosmot_status layer_head(const cosmot_dims& D, const cosmot_layer_weights* w, co
   void* a = ws + L.a;
   void* u = ws + L.u;
   uint16_t* hb = static_cast<uint16_t*>(state);
-  if (S.n_noisy == 0) {
+  if (nz == 0) {
     if ((st = M.mark(8)) != COSMOT_OK) return st;
     return M.mark(9);
   }
@@ -235,8 +236,8 @@ cosmot_status layer_head(const cosmot_dims& D, const cosmot_layer_weights* w, co
   cosmot_segment vs[kMaxBatch], ns_in[kMaxBatch];
   for (int b = 0; b < B; ++b) {
     const int64_t z0 = b * N + S.n_ar + S.n_clean;
-    ns_in[b] = cosmot_segment{z0, z0 + S.n_noisy, (int64_t)b * S.n_noisy, 1, 0};
-    vs[b] = cosmot_segment{(int64_t)b * S.n_noisy, (int64_t)(b + 1) * S.n_noisy, z0, 1, 0};
+    ns_in[b] = cosmot_segment{z0, z0 + nz, (int64_t)b * nz, 1, 0};
+    vs[b] = cosmot_segment{(int64_t)b * nz, (int64_t)(b + 1) * nz, z0, 1, 0};
   }
   st = cosmot_rmsnorm_routed(h_last, d, ns_in, B, w->gfin, w->gfin, d, D.eps, a, d, stream);
   if (st != COSMOT_OK) return st;
@@ -247,7 +248,6 @@ cosmot_status layer_head(const cosmot_dims& D, const cosmot_layer_weights* w, co
     // hidden region, then v_base + w (v_cond - v_base) and the Euler step for
     // each (conditioned, baseline) pair, written to both states of the pair.
     uint16_t* vbuf = static_cast<uint16_t*>(u);
-    const int64_t nz = S.n_noisy;
     const cosmot_segment all{0, (int64_t)B * nz, 0, 1, 0};
     e.kind = COSMOT_EPI_NONE;
     st = cosmot_routed_linear(a, d, d, &all, 1, w->wvel, w->wvel, nullptr, nullptr, d, vbuf, d, &e, stream);
@@ -288,7 +288,7 @@ cosmot_status layer_forward_impl(const cosmot_dims* dims, const cosmot_layer_wei
   uint8_t* ws = static_cast<uint8_t*>(workspace);
   st = layer_body(*dims, w, *seq, L, ws, h, h_out, nullptr, stream, M);
   if (st != COSMOT_OK) return st;
-  return layer_head(*dims, w, *seq, L, ws, h_out, h, sigma, sigma_next, stream, M, guidance);
+  return layer_head(*dims, w, *seq, L, ws, h_out, h, sigma, sigma_next, stream, M, guidance, seq->n_noisy);
 }
 
 // Stack workspace: one layer's working set, a second hidden-state buffer for
@@ -315,14 +315,10 @@ StackWs stack_ws_layout(const cosmot_dims& d, int32_t n_layers, const cosmot_seq
 
 constexpr int32_t kMaxLayers = 1024;
 
-// events (or null): 8 per layer (layer l records events[8l + i] before its
-// stage i, i < 7, and events[8l + 7] after its last stage), then 2 for the head
-// (before the velocity stage and after it).
-cosmot_status stack_forward_impl(const cosmot_dims* dims, const cosmot_layer_weights* layers, int32_t n_layers,
-                                 const cosmot_seq_desc* seq, void* h, void* h_out, double sigma, double sigma_next,
-                                 void* workspace, size_t workspace_bytes, cosmot_stream_t stream,
-                                 const cudaEvent_t* events) {
-  const cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
+// Checks shared by the stack entries; fills W.
+cosmot_status stack_check(const cosmot_dims* dims, const cosmot_layer_weights* layers, int32_t n_layers,
+                          const cosmot_seq_desc* seq, const void* h, const void* h_out, const void* workspace,
+                          size_t workspace_bytes, StackWs* W) {
   cosmot_status st = check_dims(dims);
   if (st != COSMOT_OK) return st;
   st = check_seq(seq);
@@ -333,23 +329,100 @@ cosmot_status stack_forward_impl(const cosmot_dims* dims, const cosmot_layer_wei
   // prefix has step-invariant K/V in a stack.
   if (seq->n_cached != 0 && seq->n_cached != seq->n_ar) return COSMOT_ERR_UNSUPPORTED;
   if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return COSMOT_ERR_INVALID_ARG;
-  const StackWs W = stack_ws_layout(*dims, n_layers, *seq);
-  if (workspace_bytes < W.total) return COSMOT_ERR_WORKSPACE;
-  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  *W = stack_ws_layout(*dims, n_layers, *seq);
+  if (workspace_bytes < W->total) return COSMOT_ERR_WORKSPACE;
+  return COSMOT_OK;
+}
+
+// The layer bodies of a stack: h -> h_out.  events (or null): 8 per layer
+// (layer l records events[8l + i] before its stage i, i < 7, and
+// events[8l + 7] after its last stage).
+cosmot_status stack_bodies(const cosmot_dims* dims, const cosmot_layer_weights* layers, int32_t n_layers,
+                           const cosmot_seq_desc* seq, const StackWs& W, uint8_t* ws, const void* h, void* h_out,
+                           cosmot_stream_t stream, const cudaEvent_t* events) {
+  const cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
   // Layer outputs alternate between h_out and the workspace buffer so that the
   // last one lands in h_out; the state h is only read until the final step.
   for (int32_t l = 0; l < n_layers; ++l) {
     void* out = ((n_layers - 1 - l) % 2 == 0) ? h_out : static_cast<void*>(ws + W.tmp);
-    const void* in = l == 0 ? h : (((n_layers - l) % 2 == 0) ? h_out : static_cast<void*>(ws + W.tmp));
+    const void* in = l == 0 ? h : (((n_layers - l) % 2 == 0) ? h_out : static_cast<const void*>(ws + W.tmp));
     const StageMarks M{events ? events + 8 * l : nullptr, cs};
-    st = layer_body(*dims, &layers[l], *seq, W.layer, ws, in, out, ws + W.cache + (size_t)l * W.cache_per_layer,
-                    stream, M);
+    cosmot_status st = layer_body(*dims, &layers[l], *seq, W.layer, ws, in, out,
+                                  ws + W.cache + (size_t)l * W.cache_per_layer, stream, M);
     if (st != COSMOT_OK) return st;
   }
+  return COSMOT_OK;
+}
+
+// events: as stack_bodies, then 2 for the head (before the velocity stage and
+// after it).
+cosmot_status stack_forward_impl(const cosmot_dims* dims, const cosmot_layer_weights* layers, int32_t n_layers,
+                                 const cosmot_seq_desc* seq, void* h, void* h_out, double sigma, double sigma_next,
+                                 void* workspace, size_t workspace_bytes, cosmot_stream_t stream,
+                                 const cudaEvent_t* events) {
+  StackWs W;
+  cosmot_status st = stack_check(dims, layers, n_layers, seq, h, h_out, workspace, workspace_bytes, &W);
+  if (st != COSMOT_OK) return st;
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  st = stack_bodies(dims, layers, n_layers, seq, W, ws, h, h_out, stream, events);
+  if (st != COSMOT_OK) return st;
   // the head's marks 8 and 9 land at events[8 n_layers] and [8 n_layers + 1]
-  const StageMarks MH{events ? events + 8 * (n_layers - 1) : nullptr, cs};
+  const StageMarks MH{events ? events + 8 * (n_layers - 1) : nullptr, reinterpret_cast<cudaStream_t>(stream)};
   return layer_head(*dims, &layers[n_layers - 1], *seq, W.layer, ws, h_out, h, sigma, sigma_next, stream, MH,
-                    nullptr);
+                    nullptr, seq->n_noisy);
+}
+
+cosmot_status policy_step_impl(const cosmot_dims* dims, const cosmot_layer_weights* layers, int32_t n_layers,
+                               const cosmot_seq_desc* seq, const cosmot_action_desc* act, void* h, void* h_out,
+                               double sigma, double sigma_next, const double* guidance, void* workspace,
+                               size_t workspace_bytes, cosmot_stream_t stream, const cudaEvent_t* events) {
+  StackWs W;
+  cosmot_status st = stack_check(dims, layers, n_layers, seq, h, h_out, workspace, workspace_bytes, &W);
+  if (st != COSMOT_OK) return st;
+  const cosmot_seq_desc& S = *seq;
+  if (!act || !act->w_in || !act->w_out || !act->x || act->n_clean < 0 || act->n_noisy < 0 ||
+      act->n_noisy > S.n_noisy || act->ld_x < act->action_dim)
+    return COSMOT_ERR_INVALID_ARG;
+  if (act->n_clean > 0 && (act->clean_row < S.n_ar || act->clean_row + act->n_clean > S.n_ar + S.n_clean))
+    return COSMOT_ERR_INVALID_ARG;
+  if (guidance) {
+    if (S.batch < 2 || S.batch % 2) return COSMOT_ERR_INVALID_ARG;
+    if ((int64_t)dims->ffn * (S.n_ar + S.n_clean + S.n_noisy) < (int64_t)dims->d_model * S.n_noisy)
+      return COSMOT_ERR_UNSUPPORTED;
+  }
+  const int64_t N = (int64_t)S.n_ar + S.n_clean + S.n_noisy;
+  const int64_t na = act->n_clean + act->n_noisy;
+  const int32_t d = dims->d_model;
+  // 0. action rows of the layer input: x W_in^T (clean conditions and the noisy
+  // variable alike); the noisy action rows close the noisy group.
+  cosmot_segment es[2 * kMaxBatch], hs[kMaxBatch];
+  int ne = 0;
+  for (int b = 0; b < S.batch; ++b) {
+    if (act->n_clean > 0)
+      es[ne++] = cosmot_segment{b * na, b * na + act->n_clean, b * N + act->clean_row, 0, 0};
+    if (act->n_noisy > 0)
+      es[ne++] = cosmot_segment{b * na + act->n_clean, (b + 1) * na, b * N + N - act->n_noisy, 0, 0};
+    hs[b] = cosmot_segment{b * N + N - act->n_noisy, (b + 1) * N, b * na + act->n_clean, 0, 0};
+  }
+  if (ne > 0) {
+    st = cosmot_action_embed(act->x, act->ld_x, es, ne, act->w_in, act->action_dim, d, h, d, stream);
+    if (st != COSMOT_OK) return st;
+  }
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  st = stack_bodies(dims, layers, n_layers, seq, W, ws, h, h_out, stream, events);
+  if (st != COSMOT_OK) return st;
+  const cosmot_layer_weights* last = &layers[n_layers - 1];
+  // the noisy action rows: W_out velocity and the action's own Euler step (it
+  // reads h^L and writes the action state only; timed with the final norm)
+  if (act->n_noisy > 0) {
+    st = cosmot_action_head(h_out, d, hs, S.batch, last->gfin, dims->eps, act->w_out, act->action_dim, d, act->x,
+                            act->ld_x, act->sigma, act->sigma_next, guidance, stream);
+    if (st != COSMOT_OK) return st;
+  }
+  // the other noisy rows: hidden-space velocity head and their Euler step
+  const StageMarks MH{events ? events + 8 * (n_layers - 1) : nullptr, reinterpret_cast<cudaStream_t>(stream)};
+  return layer_head(*dims, last, S, W.layer, ws, h_out, h, sigma, sigma_next, stream, MH, guidance,
+                    S.n_noisy - act->n_noisy);
 }
 
 }  // namespace
@@ -432,6 +505,20 @@ cosmot_status cosmot_stack_forward(const cosmot_dims* dims, const cosmot_layer_w
                                    void* workspace, size_t workspace_bytes, cosmot_stream_t stream) {
   return cosmot::stack_forward_impl(dims, layers, n_layers, seq, h, h_out, sigma, sigma_next, workspace,
                                     workspace_bytes, stream, nullptr);
+}
+
+cosmot_status cosmot_policy_step(const cosmot_dims* dims, const cosmot_layer_weights* layers, int32_t n_layers,
+                                 const cosmot_seq_desc* seq, const cosmot_action_desc* act, void* h, void* h_out,
+                                 double sigma, double sigma_next, const double* guidance, void* workspace,
+                                 size_t workspace_bytes, cosmot_stream_t stream, void* const* stage_events,
+                                 int32_t n_events) {
+  if (stage_events) {
+    if (n_layers < 1 || n_layers > cosmot::kMaxLayers || n_events != 8 * n_layers + 2) return COSMOT_ERR_INVALID_ARG;
+    for (int i = 0; i < n_events; ++i)
+      if (!stage_events[i]) return COSMOT_ERR_INVALID_ARG;
+  }
+  return cosmot::policy_step_impl(dims, layers, n_layers, seq, act, h, h_out, sigma, sigma_next, guidance, workspace,
+                                  workspace_bytes, stream, reinterpret_cast<const cudaEvent_t*>(stage_events));
 }
 
 cosmot_status cosmot_stack_forward_timed(const cosmot_dims* dims, const cosmot_layer_weights* layers,

@@ -396,6 +396,81 @@ COSMOT_API cosmot_status cosmot_stack_forward(const cosmot_dims* dims, const cos
                                               size_t workspace_bytes, cosmot_stream_t stream);
 
 /*
+ * Sampler noise levels with the flow shift ("Cosmos 3 方法原理全解" §6.3:
+ * t_bar = 1 - t, sigma = s t_bar / (1 + (s - 1) t_bar)) on the uniform grid
+ * t_k = k / n_steps: sigmas[k] for k = 0 .. n_steps (n_steps + 1 host doubles,
+ * sigmas[0] = 1, sigmas[n_steps] = 0).  Host arithmetic, no stream.  INVALID_ARG
+ * for n_steps < 1, a shift that is not a positive finite number, or NULL.
+ */
+COSMOT_API cosmot_status cosmot_flow_shift_sigmas(int32_t n_steps, double shift, double* sigmas);
+
+/*
+ * Domain-specific action input projection ("Cosmos 3 方法原理全解" §4.2:
+ * normalised actions, clean conditions and the noisy variable alike, enter the
+ * Generator through W_in):  for every segment, rows [row_begin, row_end) of x
+ * ([*, ld_x] bf16, action_dim <= 32 columns used) give rows out_row.. of h
+ * ([*, ld_h] bf16, 16-byte aligned, ld_h % 8 == 0):
+ *     h[out, n] = bf16( sum_c x[row, c] * w_in[n, c] ),  w_in [d_model, action_dim] bf16.
+ * weight_set of the segments is ignored; at most 64 segments.
+ */
+COSMOT_API cosmot_status cosmot_action_embed(const void* x, int64_t ld_x, const cosmot_segment* segs, int32_t n_segs,
+                                             const void* w_in, int32_t action_dim, int32_t d_model, void* h,
+                                             int64_t ld_h, cosmot_stream_t stream);
+
+/*
+ * Action velocity head and the action's own Euler step (§4.2: W_out returns the
+ * velocity at the current sigma in the normalised action space; §6.3: each
+ * modality has its own noise level).  For every segment, row r of h_last
+ * ([*, ld_h] bf16) and row o = out_row + (r - row_begin) of x ([*, ld_x] bf16):
+ *     v = RMSNorm(h_last[r]; g_fin, eps) . w_out^T      (fp32; w_out [action_dim, d_model])
+ *     x[o] = bf16( x[o] + (sigma_next - sigma) v )
+ * With guidance != NULL the segments come in (conditioned, baseline) pairs of
+ * equal length (segment 2p and 2p + 1): v = v_base + w (v_cond - v_base) and
+ * both x rows receive the same result (they are equal on entry).
+ */
+COSMOT_API cosmot_status cosmot_action_head(const void* h_last, int64_t ld_h, const cosmot_segment* segs,
+                                            int32_t n_segs, const void* g_fin, float eps, const void* w_out,
+                                            int32_t action_dim, int32_t d_model, void* x, int64_t ld_x, double sigma,
+                                            double sigma_next, const double* guidance, cosmot_stream_t stream);
+
+/* Actions of a policy step (see cosmot_policy_step). */
+typedef struct {
+  int32_t action_dim; /* C_a, 1..32 (8 for DROID joint positions, 10 for a generic arm) */
+  int32_t n_clean;    /* clean (conditioning) action rows per sequence */
+  int32_t n_noisy;    /* noisy action rows per sequence: the last rows of each sequence */
+  int32_t clean_row;  /* first clean action row within a sequence (inside the clean group) */
+  const void* w_in;   /* [d_model, C_a] bf16 device */
+  const void* w_out;  /* [C_a, d_model] bf16 device */
+  void* x;            /* [batch * (n_clean + n_noisy), ld_x] bf16 device: per sequence its clean rows,
+                         then its noisy rows (the action state, updated in place) */
+  int64_t ld_x;
+  double sigma, sigma_next; /* the action modality's noise levels for this step */
+} cosmot_action_desc;
+
+/*
+ * One sampler step of a policy with an action head (§4.2, §6.3, §7.2-7.3):
+ *   1. the action rows of h (clean and noisy) receive x W_in^T;
+ *   2. the layer stack runs as in cosmot_stack_forward (h^L into h_out);
+ *   3. the other noisy rows take the hidden-space head and the Euler step with
+ *      (sigma, sigma_next) into h;
+ *   4. the noisy action rows take v_a = RMSNorm(h^L; gfin) W_out^T and the Euler
+ *      step with (act->sigma, act->sigma_next) into act->x.
+ * guidance (NULL or a weight): sequences 2p and 2p + 1 are a (conditioned,
+ * baseline) pair sharing their DM rows and action state; both steps use the
+ * guided velocity and write both states.  Workspace, n_cached and errors as for
+ * cosmot_stack_forward; INVALID_ARG also for a bad action descriptor.
+ * stage_events: NULL, or n_events = 8 * n_layers + 2 CUDA events recorded as
+ * for cosmot_stack_forward_timed (the action head falls in the final-norm
+ * stage); the computation is the same either way.
+ */
+COSMOT_API cosmot_status cosmot_policy_step(const cosmot_dims* dims, const cosmot_layer_weights* layers,
+                                            int32_t n_layers, const cosmot_seq_desc* seq,
+                                            const cosmot_action_desc* act, void* h, void* h_out, double sigma,
+                                            double sigma_next, const double* guidance, void* workspace,
+                                            size_t workspace_bytes, cosmot_stream_t stream,
+                                            void* const* stage_events, int32_t n_events);
+
+/*
  * cosmot_stack_forward with CUDA events (cudaEvent_t, created by the caller on
  * the current device) recorded on the stream around every stage:
  * n_events = 8 * n_layers + 2.  Layer l records events[8l + i] before its stage

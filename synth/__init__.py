@@ -25,5 +25,7 @@ from .rng import (  # noqa: F401
     make_stack_weights,
     stack_layer_seed,
     make_activations,
+    make_action_weights,
+    make_actions,
     WEIGHT_NAMES,
 )

@@ -104,6 +104,18 @@ def make_stack_weights(dims: ModelDims, seed: int, n_layers: int, distinct: int 
     return [draws[l % n_draw] for l in range(n_layers)]
 
 
+def make_action_weights(d_model: int, action_dim: int, seed: int) -> tuple:
+    """Domain action projections: W_in [d_model, action_dim] and W_out
+    [action_dim, d_model], both ~ N(0, 0.02) bf16 bits."""
+    return (normal_bf16((d_model, action_dim), seed, 20_000, std=WEIGHT_STD),
+            normal_bf16((action_dim, d_model), seed, 20_001, std=WEIGHT_STD))
+
+
+def make_actions(n_rows: int, action_dim: int, seed: int, tensor_id: int = 0) -> np.ndarray:
+    """Normalised action state [n_rows, action_dim] ~ N(0, 1) bf16 bits."""
+    return normal_bf16((n_rows, action_dim), seed, 30_000 + tensor_id)
+
+
 def make_activations(n_tokens: int, d_model: int, seed: int, tensor_id: int = 0) -> np.ndarray:
     """Layer input h [n_tokens, d_model] ~ N(0, 1) bf16 bits."""
     return normal_bf16((n_tokens, d_model), seed, 10_000 + tensor_id)

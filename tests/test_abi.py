@@ -137,3 +137,19 @@ def test_stack_workspace_and_validation():
     assert lib.cosmot_stack_forward(*args(arr, 2, cached, 256, 512, 256, n2)) == A.L.COSMOT_ERR_UNSUPPORTED
     with pytest.raises(Exception):
         A.L.cosmot_stack_workspace_size(dims, 0, seq)
+
+
+def test_shift_schedule_host_function_matches_oracle():
+    """cosmot_flow_shift_sigmas is host arithmetic: bit-identical to the
+    oracle's schedule; bad arguments rejected."""
+    from flow_matching_dit_cosmot_b200 import api as A
+    from oracle import layer as olayer
+    for n, s in ((1, 1.0), (4, 5.0), (10, 1.0), (30, 5.0), (35, 10.0), (7, 0.5)):
+        got = np.array(A.L.cosmot_flow_shift_sigmas(n, s))
+        np.testing.assert_array_equal(got, olayer.shift_sigmas(n, s))
+    lib = A.L.lib()
+    buf = (ctypes.c_double * 8)()
+    assert lib.cosmot_flow_shift_sigmas(0, 5.0, buf) == A.L.COSMOT_ERR_INVALID_ARG
+    assert lib.cosmot_flow_shift_sigmas(4, 0.0, buf) == A.L.COSMOT_ERR_INVALID_ARG
+    assert lib.cosmot_flow_shift_sigmas(4, float("inf"), buf) == A.L.COSMOT_ERR_INVALID_ARG
+    assert lib.cosmot_flow_shift_sigmas(4, 5.0, None) == A.L.COSMOT_ERR_INVALID_ARG
