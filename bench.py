@@ -109,6 +109,22 @@ def stage_work(dims, R, nz, pairs):
     }
 
 
+def resolve_schedule(wl, use_oracle: bool):
+    """A workload with its sampler noise levels filled in: the flow-shift
+    schedule comes from the library's host function (native arm) or the
+    oracle (reference arm); tests check that the two agree bit for bit."""
+    if wl.sigmas or wl.shift <= 0:
+        return wl
+    import dataclasses
+    if use_oracle:
+        from oracle import layer as olayer
+        sig = olayer.shift_sigmas(wl.n_sampler_steps, wl.shift)
+    else:
+        from flow_matching_dit_cosmot_b200 import _lib as L
+        sig = L.cosmot_flow_shift_sigmas(wl.n_sampler_steps, wl.shift)
+    return dataclasses.replace(wl, sigmas=tuple(float(x) for x in sig))
+
+
 def workload_kind(wl) -> str:
     if wl.stream is not None:
         return "stream"
@@ -365,6 +381,9 @@ def config_block(wl, lay, n_gpus):
             **({"guidance": wl.guidance, "prompt_pairs": wl.batch // 2} if wl.guidance is not None else {}),
             **({"layers": wl.n_layers, "distinct_layer_weight_draws": wl.weight_draws or wl.n_layers}
                if wl.n_layers > 1 else {}),
+            **({"shift": wl.shift, "sigmas": list(wl.sigmas)} if wl.shift > 0 else {}),
+            **({"action_dim": wl.action_dim, "action_rows": wl.layout.action_clean + wl.layout.action_noisy}
+               if wl.action_dim else {}),
             "l2": "flushed between steps (256 MiB write, outside the timed events)"}
 
 
@@ -438,6 +457,24 @@ def run_native(args, wl):
                        dims_s.rope_sections, dims_s.rope_base, dims_s.eps)
     layer = A.MoTLayer(dims, w)
     stack = A.MoTStack(dims, stack_w) if n_layers > 1 else None
+    ca = wl.action_dim
+    if ca:  # domain action heads; the action state of each (cond, base) pair is shared
+        a_clean, a_noisy = wl.layout.action_clean, wl.layout.action_noisy
+        na = a_clean + a_noisy
+        v = wl.layout.video
+        clean_row = lay.n_ar + (v.views * v.grid_h * v.grid_w * v.clean_steps if v else 0) + wl.layout.audio_clean
+        wi_h, wo_h = synth.make_action_weights(d, ca, wl.weight_seed + 500)
+        w_in, w_out = to_dev(wi_h), to_dev(wo_h)
+        xa_host = np.concatenate([synth.make_actions(na, ca, wl.act_seed(rank * B + b)) for b in range(B)])
+        if guided:
+            for pr in range(B // 2):
+                xa_host[(2 * pr + 1) * na:(2 * pr + 2) * na] = xa_host[2 * pr * na:(2 * pr + 1) * na]
+        xa = to_dev(xa_host)
+        xa_src = xa.clone()
+
+        def act_desc(s0, s1):  # the actions follow the same schedule as the video
+            return L.ActionDesc(ca, a_clean, a_noisy, clean_row, w_in.data_ptr(), w_out.data_ptr(), xa.data_ptr(),
+                                ca, s0, s1)
     z0 = lay.n_ar + lay.n_clean  # first noisy row of a sequence
 
     def seq(n_cached):
@@ -488,7 +525,11 @@ def run_native(args, wl):
         L.cosmot_mrope_table(pos.data_ptr(), N, dims_s.head_dim, dims_s.rope_sections, dims_s.rope_base,
                              cs.data_ptr(), sh)
         for i, (c, s0, s1) in enumerate(calls):
-            if stack is not None:
+            if ca:
+                L.cosmot_policy_step(dims, stack.cw, seqs[c], act_desc(s0, s1), h.data_ptr(), h_out.data_ptr(), s0,
+                                     s1, wl.guidance, ws.data_ptr(), ws.numel(), sh,
+                                     [e.cuda_event for e in stage_evs[i]] if stage_evs is not None else None)
+            elif stack is not None:
                 if stage_evs is not None:
                     L.cosmot_stack_forward_timed(dims, stack.cw, seqs[c], h.data_ptr(), h_out.data_ptr(), s0, s1,
                                                  ws.data_ptr(), ws.numel(), sh, [e.cuda_event for e in stage_evs[i]])
@@ -520,11 +561,15 @@ def run_native(args, wl):
             h[0, z0:].copy_(noise[step_no[0] % len(noise)])
         elif kind == "sampler":  # a new sampling starts from the same seeded noise
             h.copy_(h_src)
+            if ca:
+                xa.copy_(xa_src)
 
     h_src = h.clone() if kind == "sampler" else None
     launches_per_step = 2 + n_stage * len(calls) + (2 if kind == "stream" else 0)
     if n_layers > 1:  # 7 kernels per layer body, 2 for the head (the AR K/V copies are memcpys)
         launches_per_step = 2 + (7 * n_layers + 2) * len(calls)
+        if ca:  # the action embedding and the action head; the guided head adds one kernel per pair
+            launches_per_step += (2 + (B // 2 if guided else 0)) * len(calls)
     n_ev = 8 * n_layers + 2 if n_layers > 1 else n_stage + 1
 
     def new_events(n):
@@ -586,36 +631,44 @@ def run_native(args, wl):
     if not args.no_e2e:
         if kind == "stream":
             in_pin = noise[0].cpu().pin_memory()
-            out_pin = torch.empty_like(in_pin).pin_memory()
-            dst_in, src_out = h[0, z0:], h[0, z0:]
+            ins = [(h[0, z0:], in_pin)]
+            outs = [(torch.empty_like(in_pin).pin_memory(), h[0, z0:])]
         else:
-            in_pin = torch.from_numpy(h_host.view(np.int16)).view(torch.bfloat16).pin_memory()
-            out_pin = torch.empty((B, lay.n_noisy, d), dtype=torch.bfloat16).pin_memory()
-            dst_in, src_out = h, h[:, z0:]
-        for _ in range(max(1, args.warmup)):
-            dst_in.copy_(in_pin, non_blocking=True)
+            ins = [(h, torch.from_numpy(h_host.view(np.int16)).view(torch.bfloat16).pin_memory())]
+            outs = [(torch.empty((B, lay.n_noisy, d), dtype=torch.bfloat16).pin_memory(), h[:, z0:])]
+        if ca:  # a policy reads the action state in and the actions out
+            ins.append((xa, torch.from_numpy(xa_host.view(np.int16)).view(torch.bfloat16).pin_memory()))
+            outs = [(torch.empty_like(xa, device="cpu").pin_memory(), xa)]
+
+        def e2e_step():
+            for dst, src in ins:
+                dst.copy_(src, non_blocking=True)
             step()
-            out_pin.copy_(src_out, non_blocking=True)
+            for dst, src in outs:
+                dst.copy_(src, non_blocking=True)
+
+        for _ in range(max(1, args.warmup)):
+            e2e_step()
         torch.cuda.synchronize()
         e_s, e_e = new_events(args.steps), new_events(args.steps)
         torch.cuda.synchronize()
         for i in range(args.steps):
             flush.zero_()
             e_s[i].record(stream)
-            dst_in.copy_(in_pin, non_blocking=True)
-            step()
-            out_pin.copy_(src_out, non_blocking=True)
+            e2e_step()
             e_e[i].record(stream)
         torch.cuda.synchronize()
         e2e_ms = reduce_max(sum(e_s[i].elapsed_time(e_e[i]) for i in range(args.steps)), dev)
         e2e = {"value": job_throughput(tokens_per_step, args.steps, world, e2e_ms), "unit": UNIT,
-               "h2d_bytes_per_step": int(in_pin.numel() * 2), "d2h_bytes_per_step": int(out_pin.numel() * 2),
+               "h2d_bytes_per_step": int(sum(src.numel() * 2 for _, src in ins)),
+               "d2h_bytes_per_step": int(sum(dst.numel() * 2 for dst, _ in outs)),
                "ms_per_step": e2e_ms / args.steps,
                "path": "cosmot_build_layout + cosmot_mrope_table + "
-                       + ("cosmot_stack_forward" if n_layers > 1 else
+                       + ("cosmot_policy_step" if ca else "cosmot_stack_forward" if n_layers > 1 else
                           "cosmot_layer_forward_cfg" if guided else "cosmot_layer_forward")
                        + (" + cosmot_layer_commit_kv" if kind == "stream" else "")
-                       + ", pinned host input in, x' (noisy rows) out"}
+                       + (", pinned host inputs (h, action state) in, actions out" if ca else
+                          ", pinned host input in, x' (noisy rows) out")}
 
     total_ms = reduce_max(total_ms, dev)
 
@@ -670,7 +723,9 @@ def run_native(args, wl):
         cfg = config_block(wl, lay, world)
         cfg["step"] = {"layer": ("one guided layer step: both passes of each prompt pair, the guided velocity "
                                   "and one Euler step" if guided else "one layer forward + Euler step"),
-                       "sampler": (f"{n_layers}-layer stack, " if n_layers > 1 else "")
+                       "sampler": ("policy inference with W_in / W_out action heads, " if ca else "")
+                                  + (f"guided (cond, base) pairs, w {wl.guidance}, " if guided else "")
+                                  + (f"{n_layers}-layer stack, " if n_layers > 1 else "")
                                   + f"one {len(calls)}-step Euler sampling (step 1 all rows, then DM rows with the "
                                   f"AR K/V kept in the workspace)",
                        "stream": f"one streaming block: {len(calls)} denoising steps of {lay.n_noisy} tokens "
@@ -803,9 +858,9 @@ def main():
         run_micro(args, wl)
         return
     if args.impl == "reference":
-        run_reference(args, wl)
+        run_reference(args, resolve_schedule(wl, use_oracle=True))
     else:
-        run_native(args, wl)
+        run_native(args, resolve_schedule(wl, use_oracle=False))
 
 
 if __name__ == "__main__":

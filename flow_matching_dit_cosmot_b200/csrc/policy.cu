@@ -11,7 +11,7 @@
 // contraction (C_a = 8 for DROID joint positions, 10 for a generic arm) done on
 // the CUDA cores, one thread per 8 output columns; the head is one warp per
 // action row (or per conditioned/baseline row pair under guidance) that forms
-// the RMS of the row, then each of the C_a dot products with W_out, in fp32.
+// the RMS of the row and the C_a dot products with W_out in one pass, in fp32.
 #include <cuda_bf16.h>
 
 #include <cmath>
@@ -81,29 +81,56 @@ __global__ void __launch_bounds__(256) action_embed_kernel(const __nv_bfloat16* 
   }
 }
 
-// Velocity of one action row: lane c (< ca) returns v_c = sum_j hn_j w_out[c, j]
-// with hn = h * rstd * g (fp32 throughout).
+// Velocity of one action row in one pass: lane c (< ca) returns
+// v_c = rstd * sum_j h_j g_j w_out[c, j] (the RMS scale factored out of the
+// sums), fp32 throughout; 16-byte loads of h, g and each W_out row.
 __device__ __forceinline__ float action_velocity_row(const __nv_bfloat16* __restrict__ hr,
                                                      const __nv_bfloat16* __restrict__ g,
                                                      const __nv_bfloat16* __restrict__ w_out, int32_t ca, int32_t d,
                                                      float eps, int lane) {
+  float acc[kMaxActionDim];
+#pragma unroll
+  for (int c = 0; c < kMaxActionDim; ++c) acc[c] = 0.f;
   float ss = 0.f;
-  for (int j = lane; j < d; j += 32) {
-    const float v = __bfloat162float(hr[j]);
-    ss = fmaf(v, v, ss);
+  for (int j8 = lane * 8; j8 < d; j8 += 256) {
+    const uint4 hv = __ldg(reinterpret_cast<const uint4*>(hr + j8));
+    const uint4 gv = __ldg(reinterpret_cast<const uint4*>(g + j8));
+    const uint32_t* hu = reinterpret_cast<const uint32_t*>(&hv);
+    const uint32_t* gu = reinterpret_cast<const uint32_t*>(&gv);
+    float hg[8];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const float2 hh = unpack_bf16x2(hu[e]);
+      const float2 gg = unpack_bf16x2(gu[e]);
+      ss = fmaf(hh.x, hh.x, fmaf(hh.y, hh.y, ss));
+      hg[2 * e] = hh.x * gg.x;
+      hg[2 * e + 1] = hh.y * gg.y;
+    }
+#pragma unroll
+    for (int c = 0; c < kMaxActionDim; ++c) {
+      if (c < ca) {
+        const uint4 wv = __ldg(reinterpret_cast<const uint4*>(w_out + (int64_t)c * d + j8));
+        const uint32_t* wu = reinterpret_cast<const uint32_t*>(&wv);
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const float2 ww = unpack_bf16x2(wu[e]);
+          acc[c] = fmaf(hg[2 * e], ww.x, fmaf(hg[2 * e + 1], ww.y, acc[c]));
+        }
+      }
+    }
   }
 #pragma unroll
   for (int off = 16; off > 0; off >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, off);
   const float rstd = rsqrtf(ss / (float)d + eps);
   float mine = 0.f;
-  for (int c = 0; c < ca; ++c) {
-    const __nv_bfloat16* wr = w_out + (int64_t)c * d;
-    float acc = 0.f;
-    for (int j = lane; j < d; j += 32)
-      acc = fmaf(__bfloat162float(hr[j]) * rstd * __bfloat162float(g[j]), __bfloat162float(wr[j]), acc);
 #pragma unroll
-    for (int off = 16; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
-    if (lane == c) mine = acc;
+  for (int c = 0; c < kMaxActionDim; ++c) {
+    if (c < ca) {
+      float v = acc[c];
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1) v += __shfl_xor_sync(0xffffffffu, v, off);
+      if (lane == c) mine = v * rstd;
+    }
   }
   return mine;
 }
@@ -195,8 +222,9 @@ cosmot_status cosmot_action_head(const void* h_last, int64_t ld_h, const cosmot_
                                  void* x, int64_t ld_x, double sigma, double sigma_next, const double* guidance,
                                  cosmot_stream_t stream) {
   using namespace cosmot;
-  if (!h_last || !g_fin || !w_out || !x || action_dim < 1 || action_dim > kMaxActionDim || d_model < 1 ||
-      ld_h < d_model || ld_x < action_dim || !(eps >= 0.f))
+  if (!h_last || !g_fin || !w_out || !x || action_dim < 1 || action_dim > kMaxActionDim || d_model < 8 ||
+      d_model % 8 || ld_h < d_model || ld_h % 8 || ld_x < action_dim || !(eps >= 0.f) || !aligned16(h_last) ||
+      !aligned16(g_fin) || !aligned16(w_out))
     return COSMOT_ERR_INVALID_ARG;
   ActSegs t;
   if (!fill_act_segs(segs, n_segs, &t)) return COSMOT_ERR_INVALID_ARG;

@@ -426,7 +426,8 @@ COSMOT_API cosmot_status cosmot_action_embed(const void* x, int64_t ld_x, const 
  *     x[o] = bf16( x[o] + (sigma_next - sigma) v )
  * With guidance != NULL the segments come in (conditioned, baseline) pairs of
  * equal length (segment 2p and 2p + 1): v = v_base + w (v_cond - v_base) and
- * both x rows receive the same result (they are equal on entry).
+ * both x rows receive the same result (they are equal on entry).  h_last, g_fin
+ * and w_out 16-byte aligned, d_model and ld_h multiples of 8.
  */
 COSMOT_API cosmot_status cosmot_action_head(const void* h_last, int64_t ld_h, const cosmot_segment* segs,
                                             int32_t n_segs, const void* g_fin, float eps, const void* w_out,

@@ -127,6 +127,9 @@ class Workload:
     guidance: Optional[float] = None  # classifier-free guidance weight; batch = (cond, base) pairs
     n_layers: int = 1  # > 1: a layer stack with one velocity head
     weight_draws: int = 0  # > 0: that many distinct layer weight draws, cycled over the stack
+    shift: float = 0.0  # > 0: sigmas come from the flow-shift schedule over n_sampler_steps (sigmas left empty)
+    n_sampler_steps: int = 0
+    action_dim: int = 0  # > 0: the action rows go through W_in / W_out heads of this width
     description: str = ""
     extra: dict = field(default_factory=dict)
 
@@ -210,6 +213,15 @@ PRESETS = {
         sigmas=_linear_sigmas(10), n_layers=36, weight_draws=4,
         description="DROID policy step through Nano's 36-layer stack (page widths), 10 Euler steps; 4 distinct "
                     "layer weight draws of 0.77 GB cycled over the 36 layers"),
+    "droid_policy": Workload(
+        name="droid_policy", config_id=3, dims=NANO,
+        layout=LayoutSpec(n_text=128, video=VideoSpec(3, 6, 10, 15, 1, 2),
+                          action_noisy=32, action_hz=15, proprio=1),
+        sigmas=(), n_layers=36, weight_draws=4, shift=5.0, n_sampler_steps=4, guidance=3.0, batch=2,
+        action_dim=8,
+        description="DROID policy inference: Nano's 36-layer stack, a (cond, base) prompt pair with guidance 3, "
+                    "4 steps of the shift-5 schedule, 32 x 8-D joint-position actions through W_in / W_out; 4 "
+                    "distinct layer weight draws cycled over the 36 layers"),
     "i2v720": Workload(
         name="i2v720", config_id=5, dims=_SUPER_LIKE,
         layout=LayoutSpec(n_text=512, video=VideoSpec(1, 22, 40, 24, 1, 47)),
