@@ -52,6 +52,30 @@ def test_latent_sizes_golden(golden_dir):
     assert (lay3.n_ar, lay3.n_clean, lay3.n_noisy) == (130, 181, 392)
 
 
+def test_resolution_table_golden(golden_dir):
+    """The published resolutions against the stride-32 latent grid read from
+    §4.1 (832x480 -> 26x15).  In the 480p and 720p classes the five aspect
+    buckets have the same pixel area to within 3 %, and so the same number of
+    tokens per latent step (the 256p class on the page is not equal-area);
+    transposed aspects swap the grid; every 256p and 480p side divides by 32;
+    1280x720 floors to 40x22 (the 720p workload's grid)."""
+    g = json.load(open(os.path.join(golden_dir, "resolutions.json")))
+    for cls in ("256p", "480p", "720p"):
+        grids = [(w // 32, h // 32) for w, h in g[cls]]
+        assert grids[0] == grids[4][::-1] and grids[1] == grids[3][::-1], cls
+        if cls in ("256p", "480p"):
+            assert all(w % 32 == 0 and h % 32 == 0 for w, h in g[cls]), cls
+        if cls in ("480p", "720p"):
+            areas = [w * h for w, h in g[cls]]
+            tokens = [gw * gh for gw, gh in grids]
+            assert max(areas) <= 1.03 * min(areas), (cls, areas)
+            assert max(tokens) <= 1.03 * min(tokens), (cls, tokens)
+    v = synth.preset("t2v480").layout.video
+    assert (g["480p"][0][0] // 32, g["480p"][0][1] // 32) == (v.grid_w, v.grid_h) == (26, 15)
+    v = synth.preset("i2v720").layout.video
+    assert (g["720p"][0][0] // 32, g["720p"][0][1] // 32) == (v.grid_w, v.grid_h) == (40, 22)
+
+
 def test_time_steps_golden(golden_dir):
     g = json.load(open(os.path.join(golden_dir, "time_steps.json")))
     assert layout.video_time_step(g["video_fps"]) == g["video_dt"]
