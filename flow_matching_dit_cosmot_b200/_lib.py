@@ -29,6 +29,7 @@ COSMOT_EPI_EULER = 4
 
 COSMOT_MASK_FULL = 0
 COSMOT_MASK_BLOCK_CAUSAL = 1
+COSMOT_ATTN_NO_TILE_SKIP = 1
 
 c_i32, c_i64, c_f32, c_f64, c_vp = ctypes.c_int32, ctypes.c_int64, ctypes.c_float, ctypes.c_double, ctypes.c_void_p
 
@@ -56,7 +57,7 @@ class Epilogue(ctypes.Structure):
 class AttnDesc(ctypes.Structure):
     _fields_ = [("n_q", c_i64), ("q_key_offset", c_i64), ("n_keys", c_i64), ("n_ar", c_i64),
                 ("n_heads", c_i32), ("n_kv_heads", c_i32), ("head_dim", c_i32), ("mask_mode", c_i32),
-                ("chunk", c_vp), ("batch", c_i32), ("reserved", c_i32),
+                ("chunk", c_vp), ("batch", c_i32), ("flags", c_i32),
                 ("q_batch_stride", c_i64), ("kv_batch_stride", c_i64), ("o_batch_stride", c_i64),
                 ("softmax_scale", c_f32), ("reserved2", c_f32)]
 

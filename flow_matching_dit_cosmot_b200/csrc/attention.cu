@@ -54,12 +54,16 @@ constexpr int BOX_BYTES = 128 * 64 * 2;  // one 128-row x 64-column bf16 box
 constexpr int NUM_THREADS = 320;
 constexpr int TMEM_COLS = 512;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
+// Block-causal DM work items skip key tiles that none of their rows sees; the
+// visit list is a bitmask in shared memory (one bit per 128-key tile).
+constexpr int kMaxVisitWords = 2048;
+constexpr int64_t kMaxVisitTiles = (int64_t)kMaxVisitWords * 32;
 
 template <int HD>
 struct Cfg {
   static constexpr int NBOX = HD / 64;
   static constexpr int TILE_BYTES = 128 * HD * 2;
-  static constexpr int SMEM_BYTES = (2 + SLOTS) * TILE_BYTES + 256 + 1024;
+  static constexpr int SMEM_BYTES = (2 + SLOTS) * TILE_BYTES + 256 + 4 * kMaxVisitWords + 1024;
   static constexpr uint32_t IDESC_S = idesc_bf16_f32(BQ, BKV, false, false);
   static constexpr uint32_t IDESC_O = idesc_bf16_f32(BQ, HD, false, true);
   __device__ static constexpr uint32_t s_col(int t) { return (uint32_t)t * 128u; }
@@ -74,6 +78,7 @@ struct Params {
   int32_t mask_mode;
   int32_t batch;
   int32_t dm_pairs, ar_pairs;
+  int32_t skip;  // block-causal DM items skip key tiles none of their rows sees
   float scale_log2;
   const int32_t* chunk;
   __nv_bfloat16* o;
@@ -161,7 +166,47 @@ __device__ __forceinline__ bool key_visible(const Params& p, const RowMask& m, i
   return vis;
 }
 
-template <int HD>
+// Key-tile skipping for block-causal DM work items.  A tile is visited iff
+// its smallest key chunk is at most the largest chunk among the item's query
+// rows (AR keys count as the smallest chunk, keys past the end are ignored):
+// exactly the tiles that one of the item's rows sees.  FULL mode and AR items
+// visit every tile of [0, n_kt).
+__device__ __forceinline__ bool skips_tiles(const Params& p, const Work& w) { return p.skip && !w.is_ar; }
+
+__device__ __forceinline__ int32_t key_chunk_for_visit(const Params& p, int64_t key) {
+  if (key < p.n_ar) return INT32_MIN;
+  return key < p.n_keys ? __ldg(p.chunk + key) : INT32_MAX;
+}
+
+// Largest chunk among the item's valid query rows (warp-cooperative).
+__device__ __forceinline__ int32_t item_max_chunk(const Params& p, const Work& w, int lane) {
+  int32_t m = INT32_MIN;
+  for (int i = lane; i < 2 * BQ; i += 32) {
+    const int64_t qi = w.row0 + i;
+    if (qi < w.seg_end) m = max(m, __ldg(p.chunk + p.q_key_offset + qi));
+  }
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) m = max(m, __shfl_xor_sync(0xffffffffu, m, off));
+  return m;
+}
+
+// Smallest visited tile >= kt, or n_kt.
+__device__ __forceinline__ int32_t next_visit(const uint32_t* visit, bool use, int32_t kt, int32_t n_kt) {
+  if (!use) return kt < n_kt ? kt : n_kt;
+  while (kt < n_kt) {
+    const uint32_t word = visit[kt >> 5] >> (kt & 31);
+    if (word) {
+      kt += __ffs(word) - 1;
+      return kt < n_kt ? kt : n_kt;
+    }
+    kt = (kt | 31) + 1;
+  }
+  return n_kt;
+}
+
+// kSkip: the instance that may skip block-causal DM tiles (p.skip set); the
+// other one carries none of that machinery.
+template <int HD, bool kSkip>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
     mot_attention_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__ CUtensorMap tmap_k,
                          const __grid_constant__ CUtensorMap tmap_v, const __grid_constant__ Params p) {
@@ -180,6 +225,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   const uint32_t bar_o_done = bar_p_full + 16;           // [2]
   const uint32_t bar_drain = bar_o_done + 16;            // [1]
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 1 + 2 * SLOTS + 9);
+  uint32_t* visit = reinterpret_cast<uint32_t*>(smem + (2 + SLOTS) * C::TILE_BYTES + 256);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -205,11 +251,44 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     tmem_alloc(smem_u32(tmem_slot), TMEM_COLS);
     tmem_relinquish();
   }
+  bool use_visit = kSkip && skips_tiles(p, w);  // CTA-uniform
+  if (use_visit) {
+    // A tile is visited iff one of its keys is visible to the item's latest
+    // chunk; each warp tests 32 consecutive keys (inside one tile) at a time
+    // with coalesced loads and sets the tile's bit once if any passes.
+    const int32_t n_words = (w.n_kt + 31) >> 5;
+    for (int32_t i = threadIdx.x; i < n_words; i += NUM_THREADS) visit[i] = 0;
+    const int32_t qmax = item_max_chunk(p, w, lane);
+    __syncthreads();
+    const int64_t span = (int64_t)w.n_kt * BKV;
+    constexpr int U = 8;  // independent loads in flight per thread before any vote
+    for (int64_t base = (int64_t)warp * 32; base < span; base += (int64_t)NUM_THREADS * U) {
+      int32_t c[U];
+#pragma unroll
+      for (int u = 0; u < U; ++u) c[u] = key_chunk_for_visit(p, base + (int64_t)u * NUM_THREADS + lane);
+#pragma unroll
+      for (int u = 0; u < U; ++u) {
+        const int64_t k0 = base + (int64_t)u * NUM_THREADS;  // 32 keys inside one tile
+        if (__any_sync(0xffffffffu, c[u] <= qmax) && lane == 0 && k0 < span) {
+          const int64_t kt = k0 / BKV;
+          atomicOr(&visit[kt >> 5], 1u << (kt & 31));
+        }
+      }
+    }
+  }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *reinterpret_cast<volatile uint32_t*>(tmem_slot);
   const int32_t n_kt = w.n_kt;
+  if (use_visit) {
+    // Nothing to skip (a streaming block sees every cached key): walk the
+    // tiles plainly.  Every thread reads the same words, so this stays uniform.
+    bool all = true;
+    for (int32_t wd = 0; wd < (n_kt >> 5); ++wd) all = all && visit[wd] == 0xffffffffu;
+    if (n_kt & 31) all = all && (visit[n_kt >> 5] | (0xffffffffu << (n_kt & 31))) == 0xffffffffu;
+    use_visit = !all;
+  }
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer
@@ -224,18 +303,26 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           tma_load_2d(sQ + t * C::TILE_BYTES + bx * BOX_BYTES, &tmap_q, bar_q, w.h * HD + bx * 64, qrow + t * BQ);
       uint32_t armed_mask = 0, armed_parity = 0;
       const int kvrow = (int)(w.b * p.kv_bstride);
-      for (int L = 0; L < 2 * n_kt; ++L) {
-        const int slot = L % SLOTS;
-        const uint32_t par = (L / SLOTS) & 1;
-        if (!mbar_wait(bar_kv_empty + 8 * slot, par ^ 1, p.status, kWhereAttnProducer)) break;
-        const uint32_t fb = bar_kv_full + 8 * slot;
-        mbar_arrive_expect_tx(fb, C::TILE_BYTES);
-        const CUtensorMap* m = (L & 1) ? &tmap_v : &tmap_k;
-        const int krow = kvrow + (L >> 1) * BKV;
-        for (int bx = 0; bx < C::NBOX; ++bx)
-          tma_load_2d(sKV + slot * C::TILE_BYTES + bx * BOX_BYTES, m, fb, g * HD + bx * 64, krow);
-        armed_mask |= 1u << slot;
-        armed_parity = (armed_parity & ~(1u << slot)) | (par << slot);
+      // Load L = 2j (K) and 2j + 1 (V) of the j-th visited key tile.
+      bool ok = true;
+      for (int32_t kt = next_visit(visit, use_visit, 0, n_kt), L = 0; kt < n_kt && ok;
+           kt = next_visit(visit, use_visit, kt + 1, n_kt)) {
+        for (int kv = 0; kv < 2; ++kv, ++L) {
+          const int slot = L % SLOTS;
+          const uint32_t par = (L / SLOTS) & 1;
+          if (!mbar_wait(bar_kv_empty + 8 * slot, par ^ 1, p.status, kWhereAttnProducer)) {
+            ok = false;
+            break;
+          }
+          const uint32_t fb = bar_kv_full + 8 * slot;
+          mbar_arrive_expect_tx(fb, C::TILE_BYTES);
+          const CUtensorMap* m = kv ? &tmap_v : &tmap_k;
+          const int krow = kvrow + kt * BKV;
+          for (int bx = 0; bx < C::NBOX; ++bx)
+            tma_load_2d(sKV + slot * C::TILE_BYTES + bx * BOX_BYTES, m, fb, g * HD + bx * 64, krow);
+          armed_mask |= 1u << slot;
+          armed_parity = (armed_parity & ~(1u << slot)) | (par << slot);
+        }
       }
       // Let every bulk copy land before the CTA may exit.
       const uint64_t t0 = globaltimer_ns();
@@ -284,9 +371,12 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         umma_commit(bar_s_full + 8);
         umma_commit(bar_kv_empty + 8 * 0);
       }
-      for (int j = 0; j < n_kt && ok; ++j) {
+      // j counts visited key tiles; kt is the j-th one.
+      int32_t kt = next_visit(visit, use_visit, 0, n_kt);
+      for (int j = 0; kt < n_kt && ok; ++j) {
+        const int32_t kt_next = next_visit(visit, use_visit, kt + 1, n_kt);
         const int LV = 2 * j + 1, LK = 2 * j + 2;
-        const bool has_next = j + 1 < n_kt;
+        const bool has_next = kt_next < n_kt;
         const uint32_t par = j & 1;
         // Order of the softmax events in steady state: tile 0 half, tile 0
         // full, tile 1 half, tile 1 full (tile 1 runs about half a block later).
@@ -314,6 +404,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           umma_commit(bar_s_full + 8);
           umma_commit(bar_kv_empty + 8 * (LK % SLOTS));
         }
+        kt = kt_next;
       }
       umma_commit(bar_o_done);
       umma_commit(bar_o_done + 8);
@@ -340,8 +431,11 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     const float sl2 = p.scale_log2;
     float m = -INFINITY, l = 0.f;
     bool ok = true;
-    for (int j = 0; j < n_kt; ++j) {
-      const int64_t kbase = (int64_t)j * BKV;
+    // j counts visited key tiles (it sets the barrier phases); kt is the j-th.
+    int j = 0;
+    for (int32_t kt = next_visit(visit, use_visit, 0, n_kt); kt < n_kt;
+         kt = next_visit(visit, use_visit, kt + 1, n_kt), ++j) {
+      const int64_t kbase = (int64_t)kt * BKV;
       // Block-causal rows need element masks only where the tile holds a DM
       // key of a later chunk.  The warp reads the tile's 128 chunk ids (AR keys
       // and keys past the end count as visible) before waiting for S, so the
@@ -462,7 +556,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   if (warp == 1) tmem_dealloc(tmem_base, TMEM_COLS);
 }
 
-template <int HD>
+template <int HD, bool kSkip>
 cosmot_status launch(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, const Params& p,
                      unsigned grid, cudaStream_t s) {
   static std::mutex mu;
@@ -472,13 +566,13 @@ cosmot_status launch(const CUtensorMap& tq, const CUtensorMap& tk, const CUtenso
   {
     std::lock_guard<std::mutex> lk(mu);
     if (dev >= 64 || !(done_mask & (1ull << dev))) {
-      if (cudaFuncSetAttribute(mot_attention_kernel<HD>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+      if (cudaFuncSetAttribute(mot_attention_kernel<HD, kSkip>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                Cfg<HD>::SMEM_BYTES) != cudaSuccess)
         return COSMOT_ERR_CUDA;
       if (dev < 64) done_mask |= 1ull << dev;
     }
   }
-  mot_attention_kernel<HD><<<grid, NUM_THREADS, Cfg<HD>::SMEM_BYTES, s>>>(tq, tk, tv, p);
+  mot_attention_kernel<HD, kSkip><<<grid, NUM_THREADS, Cfg<HD>::SMEM_BYTES, s>>>(tq, tk, tv, p);
   return launch_status();
 }
 
@@ -500,6 +594,9 @@ cosmot_status make_params(const cosmot_attn_desc* d, Params& p, int64_t& grid) {
     return COSMOT_ERR_INVALID_ARG;
   if (d->mask_mode != COSMOT_MASK_FULL && d->mask_mode != COSMOT_MASK_BLOCK_CAUSAL) return COSMOT_ERR_INVALID_ARG;
   if (d->mask_mode == COSMOT_MASK_BLOCK_CAUSAL && !d->chunk) return COSMOT_ERR_INVALID_ARG;
+  // the shared-memory visit mask of block-causal DM items holds kMaxVisitTiles key tiles
+  if (d->mask_mode == COSMOT_MASK_BLOCK_CAUSAL && (d->n_keys + BKV - 1) / BKV > kMaxVisitTiles)
+    return COSMOT_ERR_UNSUPPORTED;
   if (d->batch > 1 && (d->q_batch_stride < d->n_q || d->kv_batch_stride < d->n_keys || d->o_batch_stride < d->n_q))
     return COSMOT_ERR_INVALID_ARG;
   p = Params{};
@@ -523,6 +620,7 @@ cosmot_status make_params(const cosmot_attn_desc* d, Params& p, int64_t& grid) {
   const float scale = d->softmax_scale > 0.f ? d->softmax_scale : 1.0f / sqrtf((float)hd);
   p.scale_log2 = scale * 1.4426950408889634f;
   p.chunk = d->chunk;
+  p.skip = d->mask_mode == COSMOT_MASK_BLOCK_CAUSAL && !(d->flags & COSMOT_ATTN_NO_TILE_SKIP);
   p.status = device_status_ptr();
   if (!p.status) return COSMOT_ERR_CUDA;
   grid = (int64_t)d->batch * d->n_heads * (p.ar_pairs + p.dm_pairs);
@@ -539,11 +637,22 @@ __global__ void __launch_bounds__(2 * BQ) mask_export_kernel(const __grid_consta
   const int64_t qi = w.row0 + threadIdx.x;
   if (qi >= w.seg_end) return;
   const RowMask rm = row_mask(p, w, qi, true);
+  const bool skip = skips_tiles(p, w);
+  int32_t qmax = INT32_MIN;  // the item's largest query chunk, as the kernel forms it
+  if (skip)
+    for (int i = 0; i < 2 * BQ; ++i)
+      if (w.row0 + i < w.seg_end) qmax = max(qmax, __ldg(p.chunk + p.q_key_offset + w.row0 + i));
   for (int64_t j = 0; j < n_kt_all; ++j) {
     const int64_t kbase = j * BKV;
     uint8_t code = 0;
     bool masked = false;
-    if (j < w.n_kt) {
+    bool visited = j < w.n_kt;
+    if (visited && skip) {
+      int32_t mn = INT32_MAX;
+      for (int c = 0; c < BKV; ++c) mn = min(mn, key_chunk_for_visit(p, kbase + c));
+      visited = mn <= qmax;
+    }
+    if (visited) {
       int32_t tmax = INT32_MIN;
       if (rm.bc_dm)
         for (int c = 0; c < BKV; ++c) tmax = max(tmax, key_chunk_for_tile(p, kbase + c));
@@ -590,7 +699,11 @@ extern "C" cosmot_status cosmot_mot_attention(const cosmot_attn_desc* d, const v
   st = make_tmap_bf16_2d(&tv, v, (uint64_t)kv_rows, (uint64_t)kvcols, (uint64_t)ld_kv, BKV, 64);
   if (st != COSMOT_OK) return st;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  return hd == 128 ? launch<128>(tq, tk, tv, p, (unsigned)grid, s) : launch<64>(tq, tk, tv, p, (unsigned)grid, s);
+  if (p.skip)
+    return hd == 128 ? launch<128, true>(tq, tk, tv, p, (unsigned)grid, s)
+                     : launch<64, true>(tq, tk, tv, p, (unsigned)grid, s);
+  return hd == 128 ? launch<128, false>(tq, tk, tv, p, (unsigned)grid, s)
+                   : launch<64, false>(tq, tk, tv, p, (unsigned)grid, s);
 }
 
 extern "C" cosmot_status cosmot_mot_mask_export(const cosmot_attn_desc* d, uint8_t* tile_codes, uint8_t* visible,

@@ -181,6 +181,9 @@ cosmot_status layer_body(const cosmot_dims& D, const cosmot_layer_weights* w, co
   ad.mask_mode = S.mask_mode;
   ad.chunk = S.chunk;
   ad.batch = B;
+  // A streaming step's queries are its newest block; its cache holds earlier
+  // chunks only, so no key tile is hidden from every query.
+  if (c0 >= (int64_t)S.n_ar + S.n_clean && S.n_noisy > 0) ad.flags = COSMOT_ATTN_NO_TILE_SKIP;
   ad.q_batch_stride = ad.kv_batch_stride = ad.o_batch_stride = N;
   uint16_t* qkvp = static_cast<uint16_t*>(qkv);
   st = cosmot_mot_attention(&ad, qkvp + c0 * qkvc, qkvc, qkvp + qc, qkvp + qc + kvc, qkvc,

@@ -209,11 +209,17 @@ typedef struct {
   int32_t mask_mode;    /* COSMOT_MASK_* */
   const int32_t* chunk; /* BLOCK_CAUSAL: device int32 [n_keys] latent step of each key row */
   int32_t batch;        /* independent sequences */
-  int32_t reserved;
+  int32_t flags;        /* COSMOT_ATTN_* hints, 0 = none */
   int64_t q_batch_stride, kv_batch_stride, o_batch_stride; /* rows between sequences */
   float softmax_scale;  /* 0 = 1/sqrt(head_dim) */
   float reserved2;
 } cosmot_attn_desc;
+
+/* BLOCK_CAUSAL hint: no DM query row can have a fully hidden key tile (a
+ * streaming step, whose cache holds only earlier chunks), so the kernel need
+ * not look for tiles to skip.  Results are the same either way: element masks
+ * still apply; a wrong hint only costs the skipped work. */
+#define COSMOT_ATTN_NO_TILE_SKIP 1
 
 /*
  * MoT attention ("Cosmos 3 方法原理全解" §3 equations; block-causal variant from
@@ -223,6 +229,9 @@ typedef struct {
  * FULL mode, every DM key; in BLOCK_CAUSAL mode the DM keys with
  * chunk[j] <= chunk[query].  q: [n_q, ld_q] (heads of head_dim from column 0),
  * k, v: [n_keys, ld_kv], o: [n_q, ld_o], all bf16 device.  head_dim 128 or 64.
+ * Key tiles that none of a CTA's query rows sees are skipped: causally hidden
+ * AR tiles always, and in BLOCK_CAUSAL mode DM tiles of later chunks (unless
+ * COSMOT_ATTN_NO_TILE_SKIP); block-causal calls need ceil(n_keys / 128) <= 65536.
  */
 COSMOT_API cosmot_status cosmot_mot_attention(const cosmot_attn_desc* desc, const void* q, int64_t ld_q, const void* k,
                                    const void* v, int64_t ld_kv, void* o, int64_t ld_o, cosmot_stream_t stream);

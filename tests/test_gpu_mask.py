@@ -5,9 +5,9 @@ block-causal variant of "流式生成如何工作").  Needs a B200.
 The element visibility must equal the oracle's bit for bit.  The tile codes
 are the kernel's own choice; the test checks what the definition fixes about
 them: a skipped tile holds no key the row sees, an unmasked tile holds only
-keys the row sees, a masked tile holds at least one it does not, DM query
-tiles visit every key tile, and an AR CTA visits no tile that none of its
-rows needs.
+keys the row sees, a masked tile holds at least one it does not, and every
+CTA (AR or DM, full or block-causal mask) visits exactly the key tiles that
+one of its rows needs: fully masked tiles are skipped.
 """
 
 import numpy as np
@@ -15,6 +15,7 @@ import pytest
 
 from oracle import layout as olayout
 from oracle import mask as omask
+import synth
 from synth import LayoutSpec, VideoSpec
 
 pytestmark = pytest.mark.gpu
@@ -28,7 +29,7 @@ from flow_matching_dit_cosmot_b200 import _lib as L  # noqa: E402
 from gpu_helpers import assert_device_ok  # noqa: E402
 
 BKV = 128
-AR_CTA_ROWS = 256  # two 128-row query tiles per CTA
+CTA_ROWS = 256  # two 128-row query tiles per CTA
 
 
 def _export(region, chunk, mode, q_off, n_q):
@@ -67,15 +68,15 @@ def _check(region, chunk, mode, q_off=0, n_q=None):
     assert not (all_vis[codes == 2]).any(), "a fully visible tile was masked"
 
     is_ar_q = region[rows] == olayout.REGION_AR
-    assert (codes[~is_ar_q] != 0).all(), "a DM query tile skipped a key tile"
-    # AR rows are grouped into CTAs of 256 consecutive query rows from the first
-    # query row; a CTA visits only key tiles that one of its rows needs.
-    ar_idx = np.nonzero(is_ar_q)[0]
-    for g0 in range(0, len(ar_idx), AR_CTA_ROWS):
-        grp = ar_idx[g0:g0 + AR_CTA_ROWS]
-        needed = any_vis[grp].any(axis=0)
-        visited = (codes[grp] != 0)
-        assert (visited == needed[None, :]).all(), "an AR CTA's visited tiles differ from what its rows need"
+    # AR query rows and DM query rows are each grouped into CTAs of 256
+    # consecutive rows from their first row; a CTA visits exactly the key tiles
+    # that one of its rows needs.
+    for idx in (np.nonzero(is_ar_q)[0], np.nonzero(~is_ar_q)[0]):
+        for g0 in range(0, len(idx), CTA_ROWS):
+            grp = idx[g0:g0 + CTA_ROWS]
+            needed = any_vis[grp].any(axis=0)
+            visited = (codes[grp] != 0)
+            assert (visited == needed[None, :]).all(), "a CTA's visited tiles differ from what its rows need"
     return codes
 
 
@@ -85,7 +86,7 @@ def _layout(spec):
 
 
 @pytest.mark.parametrize("mode", [omask.FULL, omask.BLOCK_CAUSAL])
-@pytest.mark.parametrize("name", ["tiny", "droid", "unaligned_chunks", "long_ar"])
+@pytest.mark.parametrize("name", ["tiny", "droid", "unaligned_chunks", "long_ar", "long_block_causal"])
 def test_mask_export_matches_oracle(name, mode):
     spec = {
         "tiny": LayoutSpec(n_text=32, video=VideoSpec(1, 4, 4, 24, 2, 4)),
@@ -93,11 +94,15 @@ def test_mask_export_matches_oracle(name, mode):
                             proprio=1),
         "unaligned_chunks": LayoutSpec(n_text=20, video=VideoSpec(2, 5, 13, 24, 2, 3)),
         "long_ar": LayoutSpec(n_text=600, video=VideoSpec(1, 4, 4, 24, 0, 2)),
+        "long_block_causal": LayoutSpec(n_text=30, video=VideoSpec(1, 8, 16, 24, 2, 6)),
     }[name]
     _, region, chunk = _layout(spec)
     codes = _check(region, chunk, mode)
     if mode == omask.BLOCK_CAUSAL and name != "tiny":
         assert (codes == 2).any()
+    if mode == omask.BLOCK_CAUSAL and name == "long_block_causal":
+        dm = region != olayout.REGION_AR
+        assert (codes[dm] == 0).any()  # early DM rows skip the tiles of later chunks
 
 
 def test_mask_export_query_suffixes():
@@ -117,3 +122,38 @@ def test_mask_export_rejects_bad_descriptor():
     d = L.AttnDesc(n_q=10, q_key_offset=0, n_keys=10, n_ar=2, n_heads=2, n_kv_heads=2, head_dim=128, batch=1,
                    mask_mode=L.COSMOT_MASK_BLOCK_CAUSAL)
     assert L.cosmot_mot_mask_export(d, 256, 0, A.stream_handle(), check=False) == L.COSMOT_ERR_INVALID_ARG
+
+
+def test_no_tile_skip_hint_changes_visits_not_results():
+    """COSMOT_ATTN_NO_TILE_SKIP only stops the search for skippable tiles:
+    every DM tile is visited, the element visibility is unchanged, and the
+    attention output is bit-identical (a visited fully hidden tile adds exact
+    zeros)."""
+    from gpu_helpers import to_dev
+    _, region, chunk = _layout(LayoutSpec(n_text=30, video=VideoSpec(1, 8, 16, 24, 2, 6)))
+    n = len(region)
+    n_ar = int((region == olayout.REGION_AR).sum())
+    chd = torch.from_numpy(np.ascontiguousarray(chunk, dtype=np.int32)).cuda()
+    n_kt = (n + BKV - 1) // BKV
+    H, hd = 4, 128
+    q = to_dev(synth.normal_bf16((n, H * hd), 61, 1))
+    k = to_dev(synth.normal_bf16((n, H * hd), 62, 1))
+    v = to_dev(synth.normal_bf16((n, H * hd), 63, 1))
+    outs, codes, viss = [], [], []
+    for flags in (0, L.COSMOT_ATTN_NO_TILE_SKIP):
+        d = L.AttnDesc(n_q=n, q_key_offset=0, n_keys=n, n_ar=n_ar, n_heads=H, n_kv_heads=H, head_dim=hd,
+                       mask_mode=L.COSMOT_MASK_BLOCK_CAUSAL, chunk=A.ptr(chd), batch=1, flags=flags)
+        tiles = torch.full((n, n_kt), 255, dtype=torch.uint8, device="cuda")
+        vis = torch.full((n, n), 255, dtype=torch.uint8, device="cuda")
+        L.cosmot_mot_mask_export(d, A.ptr(tiles), A.ptr(vis), A.stream_handle())
+        o = torch.empty((n, H * hd), dtype=torch.bfloat16, device="cuda")
+        L.cosmot_mot_attention(d, A.ptr(q), H * hd, A.ptr(k), A.ptr(v), H * hd, A.ptr(o), H * hd, A.stream_handle())
+        torch.cuda.synchronize()
+        assert_device_ok()
+        outs.append(o.cpu().view(torch.int16).numpy())
+        codes.append(tiles.cpu().numpy())
+        viss.append(vis.cpu().numpy())
+    dm = region != olayout.REGION_AR
+    assert (codes[0][dm] == 0).any() and not (codes[1][dm] == 0).any()
+    np.testing.assert_array_equal(viss[0], viss[1])
+    np.testing.assert_array_equal(outs[0], outs[1])
