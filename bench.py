@@ -44,8 +44,8 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # is unchanged.  Summaries live under profiles/.
 NCU_TRAFFIC = {
     # profiles/attention_t2v480_dram.md: one launch at the 480p shape (18,978 rows x 32 heads),
-    # dram__bytes_read.sum 476,272,128 + dram__bytes_write.sum 135,506,432
-    "t2v480:attention": {"bytes_per_launch": 611778560, "src_sha": "2d4e4f243ccfec14"},
+    # dram__bytes_read.sum 474,001,152 + dram__bytes_write.sum 134,097,408
+    "t2v480:attention": {"bytes_per_launch": 608098560, "src_sha": "e7f276c09bdeb691"},
 }
 
 
