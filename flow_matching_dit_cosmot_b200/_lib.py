@@ -205,7 +205,8 @@ def cosmot_mrope_table(pos: int, n_rows: int, head_dim: int, sections, rope_base
 
 
 def _segs(segs):
-    arr = (Segment * len(segs))(*[Segment(int(b), int(e), int(o), int(s), 0) for (b, e, o, s) in segs])
+    """(row_begin, row_end, out_row, weight_set[, reserved]) tuples -> Segment array."""
+    arr = (Segment * len(segs))(*[Segment(int(t[0]), int(t[1]), int(t[2]), int(t[3]), 0) for t in segs])
     return arr, len(segs)
 
 
@@ -286,11 +287,6 @@ def cosmot_flow_shift_sigmas(n_steps: int, shift: float) -> list:
     out = (c_f64 * (n_steps + 1))()
     _call("cosmot_flow_shift_sigmas", n_steps, shift, out)
     return list(out)
-
-
-def _segs(segs):
-    arr = (Segment * len(segs))(*[Segment(*s) for s in segs])
-    return arr, len(segs)
 
 
 def cosmot_action_embed(x: int, ld_x: int, segs, w_in: int, action_dim: int, d_model: int, h: int, ld_h: int,
