@@ -117,6 +117,12 @@ SIGNATURES = {
                                    c_f64, _P(c_f64), c_vp]),
     "cosmot_policy_step": (c_i32, [_P(Dims), _P(LayerWeights), c_i32, _P(SeqDesc), _P(ActionDesc), c_vp, c_vp, c_f64,
                                    c_f64, _P(c_f64), c_vp, ctypes.c_size_t, c_vp, _P(c_vp), c_i32]),
+    "cosmot_shard_workspace_size": (c_i32, [_P(Dims), c_i64, _P(ctypes.c_size_t)]),
+    "cosmot_layer_shard_pre": (c_i32, [_P(Dims), _P(LayerWeights), _P(SeqDesc), c_i64, c_i64, c_vp, c_vp, c_vp,
+                                       ctypes.c_size_t, c_vp]),
+    "cosmot_layer_shard_post": (c_i32, [_P(Dims), _P(LayerWeights), _P(SeqDesc), c_i64, c_i64, c_vp, c_vp, c_vp,
+                                        c_f64, c_f64, c_vp, ctypes.c_size_t, c_vp]),
+    "cosmot_copy_columns": (c_i32, [c_vp, c_i64, c_vp, c_i64, c_i64, c_i64, c_vp]),
     "cosmot_stack_workspace_size": (c_i32, [_P(Dims), c_i32, _P(SeqDesc), _P(ctypes.c_size_t)]),
     "cosmot_stack_forward": (c_i32, [_P(Dims), _P(LayerWeights), c_i32, _P(SeqDesc), c_vp, c_vp, c_f64, c_f64, c_vp,
                                      ctypes.c_size_t, c_vp]),
@@ -317,6 +323,32 @@ def cosmot_policy_step(dims: Dims, layers, seq: SeqDesc, act: ActionDesc, h: int
     return _call("cosmot_policy_step", ctypes.byref(dims), layers, len(layers), ctypes.byref(seq), ctypes.byref(act),
                  c_vp(h), c_vp(h_out), sigma, sigma_next, g, c_vp(workspace), workspace_bytes, c_vp(stream), arr,
                  len(events) if events else 0, check=check)
+
+
+def cosmot_shard_workspace_size(dims: Dims, rows: int) -> int:
+    n = ctypes.c_size_t(0)
+    _call("cosmot_shard_workspace_size", ctypes.byref(dims), rows, ctypes.byref(n))
+    return n.value
+
+
+def cosmot_layer_shard_pre(dims: Dims, w: LayerWeights, seq: SeqDesc, row0: int, row1: int, h_local: int,
+                           qkv_local: int, workspace: int, workspace_bytes: int, stream: int = 0, check=True):
+    return _call("cosmot_layer_shard_pre", ctypes.byref(dims), ctypes.byref(w), ctypes.byref(seq), row0, row1,
+                 c_vp(h_local), c_vp(qkv_local), c_vp(workspace), workspace_bytes, c_vp(stream), check=check)
+
+
+def cosmot_layer_shard_post(dims: Dims, w: LayerWeights, seq: SeqDesc, row0: int, row1: int, h_local: int,
+                            o_local: int, h_out_local: int, sigma: float, sigma_next: float, workspace: int,
+                            workspace_bytes: int, stream: int = 0, check=True):
+    return _call("cosmot_layer_shard_post", ctypes.byref(dims), ctypes.byref(w), ctypes.byref(seq), row0, row1,
+                 c_vp(h_local), c_vp(o_local), c_vp(h_out_local), sigma, sigma_next, c_vp(workspace),
+                 workspace_bytes, c_vp(stream), check=check)
+
+
+def cosmot_copy_columns(src: int, ld_src: int, dst: int, ld_dst: int, rows: int, n_cols: int, stream: int = 0,
+                        check=True):
+    return _call("cosmot_copy_columns", c_vp(src), ld_src, c_vp(dst), ld_dst, rows, n_cols, c_vp(stream),
+                 check=check)
 
 
 def cosmot_stack_workspace_size(dims: Dims, n_layers: int, seq: SeqDesc) -> int:

@@ -375,6 +375,115 @@ cosmot_status stack_forward_impl(const cosmot_dims* dims, const cosmot_layer_wei
                     nullptr, seq->n_noisy);
 }
 
+// ---------------------------------------------------------------- row shards
+// Rows [row0, row1) of one sequence held by one rank of a sequence-parallel
+// layer, in local buffers indexed from row0 (global row row0 + i is local
+// row i).  Routing follows the global index: AR rows through set 0.
+int make_shard_segments(const cosmot_seq_desc& S, int64_t row0, int64_t row1, cosmot_segment* segs) {
+  int ns = 0;
+  const int64_t ar_end = row1 < S.n_ar ? row1 : S.n_ar;
+  if (row0 < ar_end) segs[ns++] = cosmot_segment{0, ar_end - row0, 0, 0, 0};
+  const int64_t dm0 = row0 > S.n_ar ? row0 : S.n_ar;
+  if (row1 > dm0) segs[ns++] = cosmot_segment{dm0 - row0, row1 - row0, dm0 - row0, 1, 0};
+  return ns;
+}
+
+cosmot_status check_shard(const cosmot_dims* dims, const cosmot_seq_desc* seq, int64_t row0, int64_t row1,
+                          const void* workspace, size_t workspace_bytes, WsLayout* L) {
+  cosmot_status st = check_dims(dims);
+  if (st != COSMOT_OK) return st;
+  st = check_seq(seq);
+  if (st != COSMOT_OK) return st;
+  const int64_t N = (int64_t)seq->n_ar + seq->n_clean + seq->n_noisy;
+  if (seq->batch != 1 || seq->n_cached != 0) return COSMOT_ERR_UNSUPPORTED;
+  if (row0 < 0 || row1 <= row0 || row1 > N || !workspace) return COSMOT_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return COSMOT_ERR_INVALID_ARG;
+  cosmot_seq_desc local = *seq;  // a shard's working set is that of a row1 - row0 row sequence
+  local.n_ar = (int32_t)(row1 - row0);
+  local.n_clean = local.n_noisy = 0;
+  *L = ws_layout(*dims, local);
+  if (workspace_bytes < L->total) return COSMOT_ERR_WORKSPACE;
+  return COSMOT_OK;
+}
+
+cosmot_status shard_pre(const cosmot_dims* dims, const cosmot_layer_weights* w, const cosmot_seq_desc* seq,
+                        int64_t row0, int64_t row1, const void* h_local, void* qkv_local, void* workspace,
+                        size_t workspace_bytes, cosmot_stream_t stream) {
+  WsLayout L;
+  cosmot_status st = check_shard(dims, seq, row0, row1, workspace, workspace_bytes, &L);
+  if (st != COSMOT_OK) return st;
+  if (!w || !h_local || !qkv_local) return COSMOT_ERR_INVALID_ARG;
+  const cosmot_dims& D = *dims;
+  const int64_t d = D.d_model, hd = D.head_dim;
+  const int64_t qc = (int64_t)D.n_heads * hd, kvc = (int64_t)D.n_kv_heads * hd, qkvc = qc + 2 * kvc;
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  cosmot_segment segs[2];
+  const int ns = make_shard_segments(*seq, row0, row1, segs);
+  const cosmot_set_weights& R = w->set[0];
+  const cosmot_set_weights& G = w->set[1];
+  st = cosmot_rmsnorm_routed(h_local, d, segs, ns, R.g1, G.g1, d, D.eps, ws + L.a, d, stream);
+  if (st != COSMOT_OK) return st;
+  cosmot_epilogue e{};
+  e.kind = COSMOT_EPI_MROPE;
+  e.head_dim = D.head_dim;
+  e.rope_cols = qc + kvc;
+  e.rope_cs = seq->rope_cs + row0 * hd;  // (cos, sin) pairs of the shard's global rows
+  e.rope_period = 0;
+  return cosmot_routed_linear(ws + L.a, d, d, segs, ns, R.wqkv, G.wqkv, nullptr, nullptr, qkvc, qkv_local, qkvc, &e,
+                              stream);
+}
+
+cosmot_status shard_post(const cosmot_dims* dims, const cosmot_layer_weights* w, const cosmot_seq_desc* seq,
+                         int64_t row0, int64_t row1, void* h_local, const void* o_local, void* h_out_local,
+                         double sigma, double sigma_next, void* workspace, size_t workspace_bytes,
+                         cosmot_stream_t stream) {
+  WsLayout L;
+  cosmot_status st = check_shard(dims, seq, row0, row1, workspace, workspace_bytes, &L);
+  if (st != COSMOT_OK) return st;
+  if (!w || !h_local || !o_local || !h_out_local || h_local == h_out_local) return COSMOT_ERR_INVALID_ARG;
+  const cosmot_dims& D = *dims;
+  const cosmot_seq_desc& S = *seq;
+  const int64_t d = D.d_model, F = D.ffn, qc = (int64_t)D.n_heads * D.head_dim;
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  cosmot_segment segs[2];
+  const int ns = make_shard_segments(S, row0, row1, segs);
+  const cosmot_set_weights& R = w->set[0];
+  const cosmot_set_weights& G = w->set[1];
+  cosmot_epilogue e{};
+  e.kind = COSMOT_EPI_RESIDUAL;
+  e.res = h_local;
+  e.ld_res = d;
+  st = cosmot_routed_linear(o_local, qc, qc, segs, ns, R.wo, G.wo, nullptr, nullptr, d, ws + L.h1, d, &e, stream);
+  if (st != COSMOT_OK) return st;
+  st = cosmot_rmsnorm_routed(ws + L.h1, d, segs, ns, R.g2, G.g2, d, D.eps, ws + L.a, d, stream);
+  if (st != COSMOT_OK) return st;
+  e = cosmot_epilogue{};
+  e.kind = COSMOT_EPI_SILU_MUL;
+  st = cosmot_routed_linear(ws + L.a, d, d, segs, ns, R.wg, G.wg, R.wu, G.wu, F, ws + L.u, F, &e, stream);
+  if (st != COSMOT_OK) return st;
+  e = cosmot_epilogue{};
+  e.kind = COSMOT_EPI_RESIDUAL;
+  e.res = ws + L.h1;
+  e.ld_res = d;
+  st = cosmot_routed_linear(ws + L.u, F, F, segs, ns, R.wd, G.wd, nullptr, nullptr, d, h_out_local, d, &e, stream);
+  if (st != COSMOT_OK) return st;
+  // the noisy rows of the shard: final norm, velocity head and the Euler step
+  const int64_t z0 = (int64_t)S.n_ar + S.n_clean;
+  const int64_t nz0 = row0 > z0 ? row0 : z0;
+  if (row1 <= nz0) return COSMOT_OK;
+  const int64_t nz = row1 - nz0;
+  const cosmot_segment ns_in{nz0 - row0, row1 - row0, 0, 1, 0};
+  st = cosmot_rmsnorm_routed(h_out_local, d, &ns_in, 1, w->gfin, w->gfin, d, D.eps, ws + L.a, d, stream);
+  if (st != COSMOT_OK) return st;
+  const cosmot_segment vs{0, nz, nz0 - row0, 1, 0};
+  e = cosmot_epilogue{};
+  e.kind = COSMOT_EPI_EULER;
+  e.x = h_local;
+  e.ld_x = d;
+  e.dsigma = (float)(sigma_next - sigma);
+  return cosmot_routed_linear(ws + L.a, d, d, &vs, 1, w->wvel, w->wvel, nullptr, nullptr, d, h_local, d, &e, stream);
+}
+
 cosmot_status policy_step_impl(const cosmot_dims* dims, const cosmot_layer_weights* layers, int32_t n_layers,
                                const cosmot_seq_desc* seq, const cosmot_action_desc* act, void* h, void* h_out,
                                double sigma, double sigma_next, const double* guidance, void* workspace,
@@ -522,6 +631,43 @@ cosmot_status cosmot_policy_step(const cosmot_dims* dims, const cosmot_layer_wei
   }
   return cosmot::policy_step_impl(dims, layers, n_layers, seq, act, h, h_out, sigma, sigma_next, guidance, workspace,
                                   workspace_bytes, stream, reinterpret_cast<const cudaEvent_t*>(stage_events));
+}
+
+cosmot_status cosmot_shard_workspace_size(const cosmot_dims* dims, int64_t rows, size_t* bytes) {
+  using namespace cosmot;
+  if (!bytes || rows < 1 || rows > INT32_MAX) return COSMOT_ERR_INVALID_ARG;
+  cosmot_status st = check_dims(dims);
+  if (st != COSMOT_OK) return st;
+  cosmot_seq_desc local{};
+  local.n_ar = (int32_t)rows;
+  local.batch = 1;
+  *bytes = ws_layout(*dims, local).total;
+  return COSMOT_OK;
+}
+
+cosmot_status cosmot_layer_shard_pre(const cosmot_dims* dims, const cosmot_layer_weights* w,
+                                     const cosmot_seq_desc* seq, int64_t row0, int64_t row1, const void* h_local,
+                                     void* qkv_local, void* workspace, size_t workspace_bytes,
+                                     cosmot_stream_t stream) {
+  return cosmot::shard_pre(dims, w, seq, row0, row1, h_local, qkv_local, workspace, workspace_bytes, stream);
+}
+
+cosmot_status cosmot_layer_shard_post(const cosmot_dims* dims, const cosmot_layer_weights* w,
+                                      const cosmot_seq_desc* seq, int64_t row0, int64_t row1, void* h_local,
+                                      const void* o_local, void* h_out_local, double sigma, double sigma_next,
+                                      void* workspace, size_t workspace_bytes, cosmot_stream_t stream) {
+  return cosmot::shard_post(dims, w, seq, row0, row1, h_local, o_local, h_out_local, sigma, sigma_next, workspace,
+                            workspace_bytes, stream);
+}
+
+cosmot_status cosmot_copy_columns(const void* src, int64_t ld_src, void* dst, int64_t ld_dst, int64_t rows,
+                                  int64_t n_cols, cosmot_stream_t stream) {
+  if (!src || !dst || rows < 0 || n_cols < 0 || ld_src < n_cols || ld_dst < n_cols) return COSMOT_ERR_INVALID_ARG;
+  if (rows == 0 || n_cols == 0) return COSMOT_OK;
+  const cudaError_t e = cudaMemcpy2DAsync(dst, (size_t)ld_dst * 2, src, (size_t)ld_src * 2, (size_t)n_cols * 2,
+                                          (size_t)rows, cudaMemcpyDeviceToDevice,
+                                          reinterpret_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? COSMOT_OK : COSMOT_ERR_CUDA;
 }
 
 cosmot_status cosmot_stack_forward_timed(const cosmot_dims* dims, const cosmot_layer_weights* layers,

@@ -481,6 +481,42 @@ COSMOT_API cosmot_status cosmot_policy_step(const cosmot_dims* dims, const cosmo
                                             void* const* stage_events, int32_t n_events);
 
 /*
+ * A layer split around its attention for sequence parallelism over P ranks
+ * (one sequence, batch 1, no cached prefix).  A rank holds rows [row0, row1)
+ * of the packed sequence in local buffers (global row row0 + i is local row i);
+ * routing, positions and the noisy rows follow the global index.
+ *   cosmot_layer_shard_pre:  qkv_local [row1 - row0, (H + 2 Hkv) hd] bf16 =
+ *       routed RMSNorm and QKV projection with mRoPE of h_local's rows.
+ *   (the caller trades rows for heads, runs cosmot_mot_attention on its heads
+ *    over all rows, and trades back)
+ *   cosmot_layer_shard_post: o_local [row1 - row0, H hd] (heads in order) ->
+ *       O projection + residual, routed norm, gate/up, down + residual into
+ *       h_out_local, and for the shard's noisy rows the velocity head and the
+ *       Euler step into h_local.
+ * Every output element is computed with the same arithmetic as in
+ * cosmot_layer_forward.  Workspace: cosmot_shard_workspace_size(row1 - row0),
+ * 256-byte aligned.  UNSUPPORTED for batch != 1 or n_cached != 0.
+ */
+COSMOT_API cosmot_status cosmot_shard_workspace_size(const cosmot_dims* dims, int64_t rows, size_t* bytes);
+COSMOT_API cosmot_status cosmot_layer_shard_pre(const cosmot_dims* dims, const cosmot_layer_weights* w,
+                                                const cosmot_seq_desc* seq, int64_t row0, int64_t row1,
+                                                const void* h_local, void* qkv_local, void* workspace,
+                                                size_t workspace_bytes, cosmot_stream_t stream);
+COSMOT_API cosmot_status cosmot_layer_shard_post(const cosmot_dims* dims, const cosmot_layer_weights* w,
+                                                 const cosmot_seq_desc* seq, int64_t row0, int64_t row1,
+                                                 void* h_local, const void* o_local, void* h_out_local, double sigma,
+                                                 double sigma_next, void* workspace, size_t workspace_bytes,
+                                                 cosmot_stream_t stream);
+
+/*
+ * dst[r, 0:n_cols] = src[r, 0:n_cols] for r < rows (bf16, row pitches ld_src
+ * and ld_dst in elements): packs and unpacks column blocks for the exchanges
+ * of a sequence-parallel layer.  One strided device-to-device copy.
+ */
+COSMOT_API cosmot_status cosmot_copy_columns(const void* src, int64_t ld_src, void* dst, int64_t ld_dst, int64_t rows,
+                                             int64_t n_cols, cosmot_stream_t stream);
+
+/*
  * cosmot_stack_forward with CUDA events (cudaEvent_t, created by the caller on
  * the current device) recorded on the stream around every stage:
  * n_events = 8 * n_layers + 2.  Layer l records events[8l + i] before its stage
