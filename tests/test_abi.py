@@ -153,3 +153,32 @@ def test_shift_schedule_host_function_matches_oracle():
     assert lib.cosmot_flow_shift_sigmas(4, 0.0, buf) == A.L.COSMOT_ERR_INVALID_ARG
     assert lib.cosmot_flow_shift_sigmas(4, float("inf"), buf) == A.L.COSMOT_ERR_INVALID_ARG
     assert lib.cosmot_flow_shift_sigmas(4, 5.0, None) == A.L.COSMOT_ERR_INVALID_ARG
+
+
+def _random_specs():
+    from hypothesis import strategies as st
+    video = st.one_of(st.none(), st.tuples(st.integers(1, 4), st.integers(1, 8), st.integers(1, 8),
+                                            st.sampled_from([10, 15, 24, 30]), st.integers(0, 3), st.integers(0, 3)))
+    return st.builds(lambda nt, v, ac, an, rate, xc, xn, hz, pr: synth.LayoutSpec(
+        n_text=nt, video=None if v is None else synth.VideoSpec(*v), audio_clean=ac, audio_noisy=an, audio_rate=rate,
+        action_clean=xc, action_noisy=xn, action_hz=hz, proprio=pr),
+        st.integers(0, 40), video, st.integers(0, 9), st.integers(0, 9), st.sampled_from([25, 50]),
+        st.integers(0, 9), st.integers(0, 9), st.sampled_from([10, 15, 20]), st.integers(0, 2))
+
+
+def test_layout_counts_match_oracle_on_random_layouts():
+    """cosmot_layout_counts (host arithmetic) agrees with the oracle's layout
+    builder on random layouts: any mix of text, views, clean/noisy steps,
+    audio, actions and proprioception."""
+    from hypothesis import given, settings
+    from flow_matching_dit_cosmot_b200 import api as A
+    from gpu_helpers import layout_spec
+
+    @settings(max_examples=150, deadline=None)
+    @given(_random_specs())
+    def check(spec):
+        lay = olayout.build_layout(spec)
+        n, a, c, z = A.L.cosmot_layout_counts(layout_spec(A, spec))
+        assert (n, a, c, z) == (lay.n_tokens, lay.n_ar, lay.n_clean, lay.n_noisy)
+
+    check()

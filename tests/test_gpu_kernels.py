@@ -56,6 +56,29 @@ def test_build_layout_bit_exact(case, tau_offset):
     assert_device_ok()
 
 
+def test_build_layout_bit_exact_on_random_layouts():
+    """Positions, chunk ids and regions from the GPU equal the oracle's bit for
+    bit on random layouts (text, views, clean/noisy steps, audio, actions,
+    proprioception, time offsets)."""
+    from hypothesis import given, settings
+    from hypothesis import strategies as st
+    from test_abi import _random_specs
+
+    @settings(max_examples=60, deadline=None)
+    @given(_random_specs(), st.integers(0, 12))
+    def check(spec, tau):
+        ref = olayout.build_layout(spec, tau_offset=tau)
+        dev = A.build_layout(layout_spec(A, spec, tau))
+        torch.cuda.synchronize()
+        assert (dev.n_ar, dev.n_clean, dev.n_noisy) == (ref.n_ar, ref.n_clean, ref.n_noisy)
+        np.testing.assert_array_equal(dev.pos.cpu().numpy().view(np.uint32), ref.pos.view(np.uint32))
+        np.testing.assert_array_equal(dev.chunk.cpu().numpy(), ref.chunk)
+        np.testing.assert_array_equal(dev.region.cpu().numpy(), ref.region)
+
+    check()
+    assert_device_ok()
+
+
 @pytest.mark.parametrize("hd,sections", [(128, (16, 24, 24)), (64, (8, 12, 12))])
 def test_mrope_table(hd, sections):
     ref = olayout.build_layout(synth.preset("i2v720").layout)
