@@ -12,16 +12,22 @@ the definitions state.  Each function names the passage it follows:
 
   * "Cosmos 3 方法原理全解" (cnblogs): §2 packed sequence S=[S_AR, S_DM] and
     its internal order; §2.2 clean/noisy condition mask; §3 MoT: two weight
-    sets, causal AR attention and full DM attention over [K_AR; K_DM]; §5
-    unified 3D mRoPE, real-time step sizes and the 15000 offset; §6.3 the
-    linear flow path; §7.2 the Euler sampler step.
+    sets, causal AR attention and full DM attention over [K_AR; K_DM]; §4.2
+    domain action projections W_in / W_out; §5 unified 3D mRoPE, real-time
+    step sizes and the 15000 offset; §6.3 the linear flow path, per-modality
+    noise levels and the flow shift; §7.2-7.3 the Euler sampler step and
+    classifier-free guidance; §12.4 the stacked model sizes.
   * "NVIDIA 发布 Cosmos 3 系列四个开放权重世界模型", "流式生成如何工作":
     time-causal block attention with a key/value cache.
 
-Where the pages are silent the oracle takes the readings listed in the design doc
-(norm type, RoPE base and pairing, t/h/w split, EOS/BOG region, position
-formulas, streaming commit).  Every function is pinned by tests under
-``tests/test_oracle_*.py`` except where a docstring says "parity unpinned".
+Where the pages are silent the oracle takes a stated reading, given in the
+docstring of the function concerned (norm type, RoPE base and pairing, t/h/w
+split, EOS/BOG region, position formulas, streaming commit, the head of a
+stack, the inference grid of the shift).  Every function is pinned by tests
+under ``tests/test_oracle_pins.py`` (closed forms, invariants, brute force and
+the values the pages print) except where a docstring says "parity unpinned";
+none does.  No page prints a layer output, so a layer's numerical value is
+pinned only through those tests.
 """
 
 from . import layout, rope, mask, layer  # noqa: F401

@@ -10,7 +10,7 @@ velocity v and the sampler moves x_next = x + (sigma_next - sigma) * v, with
 sigma_next < sigma; §2.2 / §4.2: clean tokens are fixed conditions and are not
 updated.
 
-Readings where the pages are silent (listed in the design doc):
+Readings where the pages are silent:
   * norms are pre-norm RMSNorm with a gain and eps = 1e-6, no biases anywhere;
   * the FFN is SiLU-gated: (silu(b Wg^T) * (b Wu^T)) Wd^T, silu(z) = z/(1+e^-z);
   * the DM state x lives in the hidden space: the DM rows of the layer input

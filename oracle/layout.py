@@ -16,7 +16,7 @@ Follows "Cosmos 3 方法原理全解":
   §8.2 several camera views are tiled into one canvas; here views sit side by
        side along w.
 
-Readings where the pages leave the formula open (also listed in the design doc):
+Readings where the pages leave the formula open:
   * EOS and BOG are AR tokens (Reasoner weights, causal, visible to DM).
   * AR token k has (k, k, k); the DM time origin is T0 = n_ar + 15000.
   * video token (step tau, view v, row y, col x) -> (T0 + tau*dt_v, y, x + v*W).

@@ -10,7 +10,7 @@ streaming models ("NVIDIA 发布 Cosmos 3 系列四个开放权重世界模型",
 "流式生成如何工作") use time-causal attention: a block reads the history and
 the controls but not future targets.
 
-Reading: key j is visible to query i iff
+Reading taken where the pages leave details open: key j is visible to query i iff
   * i is AR:  j is AR and j <= i;
   * i is DM, FULL mode:          every AR key and every DM key;
   * i is DM, BLOCK_CAUSAL mode:  every AR key, and DM keys with

@@ -6,7 +6,7 @@ TEST INFRASTRUCTURE (see the package docstring).
 say every token carries a (t, h, w) coordinate and that text, with
 t = h = w, reduces to ordinary 1D RoPE.  The pages give neither the base, the
 pairing, nor how the frequency pairs are split between the three axes.
-Readings (the design doc lists them):
+Readings where the pages are silent:
   * base 10000, inv_freq_i = base^(-2i/head_dim) for pair i in [0, head_dim/2);
   * rotate-half pairing: element i is paired with element i + head_dim/2;
   * the pairs are cut into three contiguous sections (n_t, n_h, n_w) with
