@@ -24,7 +24,7 @@
  *   - Alignment: every bf16 matrix base pointer must be 16-byte aligned and every
  *     leading dimension a multiple of 8 elements (the 16-byte TMA stride rule).
  *   - Argument errors are reported synchronously as COSMOT_ERR_INVALID_ARG (or
- *     COSMOT_ERR_UNSUPPORTED for shapes this build does not handle) and nothing is
+ *     COSMOT_ERR_UNSUPPORTED for shapes the library does not handle) and nothing is
  *     launched.  Launch failures return COSMOT_ERR_CUDA.
  *   - Device-side failures (a bounded wait that ran out, recorded instead of
  *     hanging) are latched into a device status word; read and clear it with
