@@ -349,6 +349,16 @@ def test_attention_block_causal_and_batch():
     assert_close(got, ref, "block causal", rounded_inputs=1)
 
 
+def test_attention_block_causal_hd64_gqa():
+    """The tile-skipping instance at head_dim 64 with grouped key/value heads:
+    chunks of 200 keys, so early DM query tiles skip the later key tiles."""
+    n_keys, n_ar = 1100, 50
+    ch = np.full(n_keys, -1, np.int32)
+    ch[n_ar:] = np.arange(n_keys - n_ar) // 200
+    got, ref = _attn_case(n_keys, n_ar, n_keys, 0, H=4, Hkv=2, hd=64, mode="block_causal", chunk=ch, batch=2, seed=5)
+    assert_close(got, ref, "block causal hd64", rounded_inputs=1)
+
+
 def test_attention_query_suffix_streaming():
     """Queries are the last block of the key sequence (a streaming step)."""
     n_keys, n_ar = 66 + 3 * 250 + 250, 66
