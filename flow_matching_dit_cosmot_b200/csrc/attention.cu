@@ -8,7 +8,7 @@
 // formulation, exact up to rounding.
 //
 // One CTA per (sequence, head, pair of 128-row query tiles); a pair never
-// mixes AR and DM rows.  320 threads:
+// mixes AR and DM rows.  384 threads in three warpgroups:
 //   warp 0      TMA: both Q tiles once, then K_j and V_j tiles (128 keys x
 //               head_dim, 128-byte swizzle) through a 4-slot ring.
 //   warp 1      owns TMEM and issues the MMAs from one thread:
@@ -16,7 +16,10 @@
 //                 O_t += P_t V_j           (M=128, N=head_dim, K=128;  A = P in TMEM)
 //               in the order S0 S1 | PV0 S0' PV1 S1' | ..., so the tensor core
 //               works on one tile while the other tile's softmax runs.
-//   warps 2-5   softmax of query tile 0, warps 6-9 of tile 1 (one row per
+//   warps 2-3   idle: they complete warpgroup 0, which hands registers to
+//               the softmax (setmaxnreg: 88 a thread for warpgroup 0, 200 for
+//               warpgroups 1 and 2, out of the 168 a thread at launch).
+//   warps 4-7   softmax of query tile 0, warps 8-11 of tile 1 (one row per
 //               thread): read S from TMEM, mask, running max, P = 2^(s*c - m)
 //               written back over S as packed bf16, running sum; O is
 //               rescaled in TMEM only when the running max grows by more than
@@ -24,15 +27,20 @@
 // TMEM columns: S0 [0,128), S1 [128,256), O0 and O1 after them.
 //
 // P is released in two halves (keys 0-63, then 64-127) so that the first half
-// of PV overlaps the exponentials of the second.
+// of PV overlaps the exponentials of the second; each softmax warp signals a
+// half with one arrive after its lanes' tensor-memory stores have completed.
 //
 // Measured on B200 (18,978 tokens, 32 heads of 128): the period of one key
-// block (~3,600 cycles) is the chain softmax(tile 0) ~1,900 -> hand-off ~450 ->
-// PV0 rest and next S0 ~1,000 -> S-ready ~250; the tensor pipe is busy ~60 % and
-// the SFU ~55 %.  The softmax is bound by its own issue latency (one warp per
-// sub-partition per tile), not by the SFU: exponentials on the FMA pipe (25 %
-// or 37.5 % of them), packed f32x2 arithmetic, a row split between two
-// warpgroups and one warpgroup serving both tiles were all slower.  Smaller MMAs
+// block (~3,600 cycles before the register hand-over) is the chain
+// softmax(tile 0) ~1,900 -> hand-off ~450 -> PV0 rest and next S0 ~1,000 ->
+// S-ready ~250.  The softmax was held back by the 168-register ceiling of a
+// CTA this size: giving it 200 registers a thread took the kernel from 5.6 to
+// 5.1 ms on one box (tensor pipe 54 -> 59 %, SFU 54 -> 60 %).  It is bound by
+// its own issue latency (one warp per sub-partition per tile), not by the SFU:
+// exponentials on the FMA pipe (25 % or 37.5 % of them), packed f32x2
+// arithmetic, a row split between two warpgroups, one warpgroup serving both
+// tiles, and starting the exponentials of keys 0-63 from the previous running
+// max while the tile max is reduced were all slower.  Smaller MMAs
 // do not help either: a tcgen05.mma with N = 64 costs 44-48 cycles instead of
 // 32 (fixed per-instruction cost), so 64-key blocks with double-buffered S, or
 // S issued as two N = 64 halves, were 23-58 % slower.  Every tcgen05.ld/st is
@@ -51,7 +59,12 @@ constexpr int BQ = 128;
 constexpr int BKV = 128;
 constexpr int SLOTS = 4;
 constexpr int BOX_BYTES = 128 * 64 * 2;  // one 128-row x 64-column bf16 box
-constexpr int NUM_THREADS = 320;
+constexpr int NUM_THREADS = 384;
+// Registers a thread after the hand-over; 128 x kRegsIo + 256 x kRegsSoftmax
+// must not exceed the launch's pool (384 x registers at launch), or the
+// increase would wait forever: the launch checks it.
+constexpr int kRegsIo = 88;
+constexpr int kRegsSoftmax = 200;
 constexpr int TMEM_COLS = 512;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
 // Block-causal DM work items skip key tiles that none of their rows sees; the
@@ -240,8 +253,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     }
     for (int t = 0; t < 2; ++t) {
       mbar_init(bar_s_full + 8 * t, 1);
-      mbar_init(bar_p_half + 8 * t, 128);
-      mbar_init(bar_p_full + 8 * t, 128);
+      mbar_init(bar_p_half + 8 * t, 4);  // one arrive per softmax warp
+      mbar_init(bar_p_full + 8 * t, 4);
       mbar_init(bar_o_done + 8 * t, 1);
     }
     mbar_init(bar_drain, 1);
@@ -290,6 +303,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     use_visit = !all;
   }
 
+  if (warp < 4) {
+  setmaxnreg_dec<kRegsIo>();
   if (warp == 0) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
@@ -418,9 +433,11 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       }
     }
     __syncwarp();
+  }
   } else {
+    setmaxnreg_inc<kRegsSoftmax>();
     // ------------------------------------------------------------ softmax
-    const int t = (warp - 2) >> 2;           // query tile of this warpgroup
+    const int t = (warp - 4) >> 2;           // query tile of this warpgroup
     const int lane_base = (warp & 3) * 32;   // TMEM lanes this warp may access
     const int r = lane_base + lane;
     const int64_t qi = w.row0 + (int64_t)t * BQ + r;
@@ -518,13 +535,15 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         if (c0 == 32) {  // P of keys 0-63 is in TMEM: PV over them may start
           tmem_st_wait();
           tc_fence_before();
-          mbar_arrive(bar_p_half + 8 * t);
+          __syncwarp();
+          if (lane == 0) mbar_arrive(bar_p_half + 8 * t);
         }
       }
       l += rs0 + rs1;
       tmem_st_wait();
       tc_fence_before();
-      mbar_arrive(bar_p_full + 8 * t);
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar_p_full + 8 * t);
     }
     if (ok && __all_sync(0xffffffffu, mbar_wait(bar_o_done + 8 * t, 0, p.status, kWhereAttnSoftmax))) {
       tc_fence_after();
@@ -569,6 +588,10 @@ cosmot_status launch(const CUtensorMap& tq, const CUtensorMap& tk, const CUtenso
       if (cudaFuncSetAttribute(mot_attention_kernel<HD, kSkip>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                Cfg<HD>::SMEM_BYTES) != cudaSuccess)
         return COSMOT_ERR_CUDA;
+      cudaFuncAttributes fa{};
+      if (cudaFuncGetAttributes(&fa, mot_attention_kernel<HD, kSkip>) != cudaSuccess) return COSMOT_ERR_CUDA;
+      // a build whose register count cannot fund the hand-over is not launched
+      if (128 * kRegsIo + 256 * kRegsSoftmax > NUM_THREADS * fa.numRegs) return COSMOT_ERR_CUDA;
       if (dev < 64) done_mask |= 1ull << dev;
     }
   }
