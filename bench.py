@@ -389,19 +389,21 @@ def config_block(wl, lay, n_gpus):
 
 # ---------------------------------------------------------------- native arm
 
-def src_sha(name):
-    """sha256 of a kernel source with its // comments and blank lines removed, so
+def code_sha(text):
+    """sha256 of source text with its // comments and blank lines removed, so
     that a comment edit keeps the counters taken on the same code."""
-    p = os.path.join(ROOT, "flow_matching_dit_cosmot_b200", "csrc", name)
-    if not os.path.exists(p):
-        return None
     code = []
-    for line in open(p, encoding="utf-8").read().splitlines():
+    for line in text.splitlines():
         cut = line.find("//")
         line = (line if cut < 0 else line[:cut]).rstrip()
         if line:
             code.append(line)
     return hashlib.sha256("\n".join(code).encode()).hexdigest()[:16]
+
+
+def src_sha(name):
+    p = os.path.join(ROOT, "flow_matching_dit_cosmot_b200", "csrc", name)
+    return code_sha(open(p, encoding="utf-8").read()) if os.path.exists(p) else None
 
 
 def run_native(args, wl):

@@ -50,3 +50,14 @@ def test_stage_flops_follow_the_layer_shapes():
     assert w["down_residual"][0] == 2 * R * d.ffn * d.d_model
     assert w["velocity_euler"][0] == 2 * nz * d.d_model * d.d_model
     assert all(w[k][0] == 0 for k in ("norm1", "norm2", "norm_final"))
+
+
+def test_traffic_counters_follow_the_kernel_code_not_its_comments():
+    """The ncu traffic a bench line reports is keyed on the kernel's code: a
+    comment edit keeps it, any code edit drops it."""
+    import bench
+    code = "int f(int a) {  // add one\n  return a + 1;\n}\n"
+    assert bench.code_sha(code) == bench.code_sha("// header\nint f(int a) {\n\n  return a + 1;  // note\n}\n")
+    assert bench.code_sha(code) != bench.code_sha(code.replace("a + 1", "a + 2"))
+    for rec in bench.NCU_TRAFFIC.values():
+        assert len(rec["src_sha"]) == 16 and rec["bytes_per_launch"] > 0
