@@ -64,8 +64,7 @@ def build(verbose: bool = False, force: bool = False, ptxas_verbose: bool = Fals
                 print(err)
     objs = [os.path.join(BUILD, os.path.basename(s) + ".o") for s in srcs]
     if force or todo or not os.path.exists(LIB) or any(os.path.getmtime(o) > os.path.getmtime(LIB) for o in objs):
-        cmd = [NVCC, *ARCH, "-shared", "-o", LIB, *objs, "-lcudart", "-lcuda"] if False else \
-            [NVCC, *ARCH, "-shared", "-o", LIB, *objs]
+        cmd = [NVCC, *ARCH, "-shared", "-o", LIB, *objs]
         if verbose:
             print(" ".join(cmd), flush=True)
         r = subprocess.run(cmd, capture_output=True, text=True)
