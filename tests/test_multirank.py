@@ -68,3 +68,31 @@ def test_reference_arm_skips_non_zero_ranks(monkeypatch, capsys):
 
     bench.run_reference(Args(), synth.preset("tiny"))
     assert capsys.readouterr().out == ""
+
+
+def test_reference_arm_line_carries_the_contract_keys(monkeypatch, capsys):
+    """Rank 0 prints one JSON line: the metric keys, the oracle as its own CPU
+    baseline, and an e2e block with no host copies."""
+    import json
+    sys.path.insert(0, ROOT)
+    import bench
+    import synth
+    monkeypatch.setenv("RANK", "0")
+
+    class Args:
+        steps, warmup, gpus = 2, 1, 1
+
+    bench.run_reference(Args(), bench.resolve_schedule(synth.preset("tiny"), use_oracle=True))
+    lines = [ln for ln in capsys.readouterr().out.splitlines() if ln.strip()]
+    assert len(lines) == 1
+    rec = json.loads(lines[0])
+    for key in ("metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step", "higher_is_better",
+                "scaling", "vs_baseline", "dtype", "data", "config", "impl", "cpu_baseline", "e2e"):
+        assert key in rec, key
+    assert rec["impl"] == "reference" and rec["steps"] == 2 and rec["warmup"] == 1 and rec["value"] > 0
+    assert rec["unit"] == bench.UNIT and rec["metric"] == bench.METRIC and rec["higher_is_better"] is True
+    assert "workload" in rec["config"]
+    cb = rec["cpu_baseline"]
+    assert cb["kind"] == "oracle" and cb["value"] == rec["value"] and cb["cores"] >= 1 and cb["sample"]
+    assert rec["e2e"] == {"value": rec["value"], "unit": rec["unit"], "h2d_bytes_per_step": 0,
+                          "d2h_bytes_per_step": 0}
