@@ -31,6 +31,49 @@ def _need_cuda(*ts):
             raise ValueError("libcosmot takes CUDA tensors only (no CPU fallback)")
 
 
+WEIGHT_TENSORS = ("g1", "wqkv", "wo", "g2", "wg", "wu", "wd")
+
+
+def weight_shapes(dims: L.Dims) -> dict:
+    """Shape of every tensor of a layer's weight dict (row-major [out, in])."""
+    d, f, hd = dims.d_model, dims.ffn, dims.head_dim
+    per_set = {"g1": (d,), "wqkv": ((dims.n_heads + 2 * dims.n_kv_heads) * hd, d), "wo": (d, dims.n_heads * hd),
+               "g2": (d,), "wg": (f, d), "wu": (f, d), "wd": (d, f)}
+    shapes = {f"{s}.{t}": shp for s in ("R", "G") for t, shp in per_set.items()}
+    shapes["gfin"] = (d,)
+    shapes["wvel"] = (d, d)
+    return shapes
+
+
+def _check_bf16(t: torch.Tensor, name: str):
+    if t.dtype != torch.bfloat16 or not t.is_contiguous():
+        raise ValueError(f"{name}: libcosmot takes contiguous bf16 tensors (got {t.dtype}, "
+                         f"{'contiguous' if t.is_contiguous() else 'strided'})")
+
+
+def check_weights(dims: L.Dims, weights: dict):
+    """The kernels read every weight through a bare pointer, so a tensor of the
+    wrong shape, dtype or layout would be read out of bounds: refuse it here."""
+    for name, shp in weight_shapes(dims).items():
+        if name not in weights:
+            raise ValueError(f"weight {name!r} missing")
+        t = weights[name]
+        if tuple(t.shape) != shp:
+            raise ValueError(f"weight {name!r} has shape {tuple(t.shape)}, expected {shp}")
+        _check_bf16(t, f"weight {name!r}")
+    _need_cuda(*weights.values())
+
+
+def _check_state(seq: L.SeqDesc, d: int, **ts):
+    """h / h_out hold [batch][N][d] bf16 (N = n_ar + n_clean + n_noisy)."""
+    rows = seq.batch * (seq.n_ar + seq.n_clean + seq.n_noisy)
+    for name, t in ts.items():
+        _check_bf16(t, name)
+        if t.numel() < rows * d:
+            raise ValueError(f"{name} holds {t.numel()} elements, fewer than batch x N x d = {rows * d}")
+    _need_cuda(*ts.values())
+
+
 def layout_spec(n_text: int, video=None, audio_clean=0, audio_noisy=0, audio_rate=25, action_clean=0,
                 action_noisy=0, action_hz=15, proprio=0, tau_offset=0) -> L.LayoutSpec:
     """`video` = (views, grid_h, grid_w, fps, clean_steps, noisy_steps) or None."""
@@ -83,7 +126,7 @@ class MoTLayer:
     def __init__(self, dims: L.Dims, weights: dict):
         self.dims = dims
         self.weights = weights
-        _need_cuda(*weights.values())
+        check_weights(dims, weights)
         sets = []
         for s in ("R", "G"):
             sets.append(L.SetWeights(*[ptr(weights[f"{s}.{t}"]) for t in ("g1", "wqkv", "wo", "g2", "wg", "wu", "wd")]))
@@ -92,6 +135,7 @@ class MoTLayer:
 
     def seq_desc(self, n_ar, n_clean, n_noisy, batch, rope_cs, chunk=None, mask_mode=L.COSMOT_MASK_FULL,
                  n_cached=0) -> L.SeqDesc:
+        """The descriptor holds raw pointers: rope_cs and chunk must stay alive while it is used."""
         return L.SeqDesc(n_ar, n_clean, n_noisy, batch, mask_mode, n_cached, ptr(rope_cs), ptr(chunk))
 
     def workspace_bytes(self, seq: L.SeqDesc) -> int:
@@ -106,14 +150,14 @@ class MoTLayer:
     def commit_kv(self, h: torch.Tensor, seq: L.SeqDesc, dst_row: int, workspace: Optional[torch.Tensor] = None,
                   stream=None):
         """K/V of rows [seq.n_cached, N) of h into cache rows [dst_row, ...) of the workspace."""
-        _need_cuda(h)
+        _check_state(seq, self.dims.d_model, h=h)
         ws = workspace if workspace is not None else self.workspace(seq, h.device)
         L.cosmot_layer_commit_kv(self.dims, self.cw, seq, ptr(h), dst_row, ptr(ws), ws.numel(), stream_handle(stream))
 
     def forward_cfg(self, h: torch.Tensor, h_out: torch.Tensor, sigma: float, sigma_next: float, guidance: float,
                     seq: L.SeqDesc, workspace: Optional[torch.Tensor] = None, stream=None):
         """Guided step: h [2P, N, d] holds (conditioned, baseline) pairs sharing their DM rows."""
-        _need_cuda(h, h_out)
+        _check_state(seq, self.dims.d_model, h=h, h_out=h_out)
         ws = workspace if workspace is not None else self.workspace(seq, h.device)
         L.cosmot_layer_forward_cfg(self.dims, self.cw, seq, ptr(h), ptr(h_out), float(sigma), float(sigma_next),
                                    float(guidance), ptr(ws), ws.numel(), stream_handle(stream))
@@ -121,7 +165,7 @@ class MoTLayer:
     def forward(self, h: torch.Tensor, h_out: torch.Tensor, sigma: float, sigma_next: float, seq: L.SeqDesc,
                 workspace: Optional[torch.Tensor] = None, stream=None):
         """h [batch, N, d] bf16 (noisy DM rows updated in place to x'); h_out [batch, N, d] bf16."""
-        _need_cuda(h, h_out)
+        _check_state(seq, self.dims.d_model, h=h, h_out=h_out)
         ws = workspace if workspace is not None else self.workspace(seq, h.device)
         L.cosmot_layer_forward(self.dims, self.cw, seq, ptr(h), ptr(h_out), float(sigma), float(sigma_next),
                                ptr(ws), ws.numel(), stream_handle(stream))
@@ -155,7 +199,7 @@ class MoTStack:
     def forward(self, h: torch.Tensor, h_out: torch.Tensor, sigma: float, sigma_next: float, seq: L.SeqDesc,
                 workspace: Optional[torch.Tensor] = None, stream=None):
         """h^L into h_out; x' into the noisy rows of h (see cosmot_stack_forward)."""
-        _need_cuda(h, h_out)
+        _check_state(seq, self.dims.d_model, h=h, h_out=h_out)
         ws = workspace if workspace is not None else self.workspace(seq, h.device)
         L.cosmot_stack_forward(self.dims, self.cw, seq, ptr(h), ptr(h_out), sigma, sigma_next, ptr(ws), ws.numel(),
                                stream_handle(stream))

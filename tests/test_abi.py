@@ -182,3 +182,59 @@ def test_layout_counts_match_oracle_on_random_layouts():
         assert (n, a, c, z) == (lay.n_tokens, lay.n_ar, lay.n_clean, lay.n_noisy)
 
     check()
+
+
+def _all_model_widths():
+    from synth import ModelDims
+    from synth import presets
+    widths = {p.dims for p in (synth.preset(n) for n in presets.PRESETS)}
+    widths |= {presets.NANO, presets.SUPER,
+               ModelDims(d_model=512, n_heads=4, n_kv_heads=4, head_dim=128, ffn=1536, rope_sections=(16, 24, 24)),
+               ModelDims(d_model=512, n_heads=4, n_kv_heads=2, head_dim=128, ffn=1024, rope_sections=(16, 24, 24)),
+               ModelDims(d_model=256, n_heads=4, n_kv_heads=2, head_dim=64, ffn=512, rope_sections=(8, 12, 12)),
+               ModelDims(d_model=512, n_heads=8, n_kv_heads=4, head_dim=64, ffn=1024, rope_sections=(8, 12, 12))}
+    return widths
+
+
+def test_api_weight_shapes_match_the_weights_synth_draws():
+    """MoTLayer refuses weights whose shapes differ from api.weight_shapes;
+    every width the tests, the bench and smoke() use draws exactly those."""
+    from flow_matching_dit_cosmot_b200 import api as A
+    for d in _all_model_widths():
+        cd = A.make_dims(d.d_model, d.n_heads, d.n_kv_heads, d.head_dim, d.ffn, d.rope_sections, d.rope_base, d.eps)
+        assert A.weight_shapes(cd) == synth.rng.weight_shapes(d), d
+
+
+def test_api_refuses_weights_and_states_it_cannot_read_safely():
+    import torch
+    from flow_matching_dit_cosmot_b200 import api as A
+    d = synth.ModelDims(d_model=64, n_heads=4, n_kv_heads=2, head_dim=16, ffn=96, rope_sections=(2, 3, 3))
+    cd = A.make_dims(d.d_model, d.n_heads, d.n_kv_heads, d.head_dim, d.ffn, d.rope_sections)
+
+    def weights():
+        return {k: torch.from_numpy(v.view(np.int16)).view(torch.bfloat16) for k, v in synth.make_weights(d, 7).items()}
+
+    with pytest.raises(ValueError, match="CUDA tensors only"):  # shapes, dtype and layout pass; the device does not
+        A.check_weights(cd, weights())
+    w = weights()
+    w["G.wo"] = w["G.wo"][:, :-16].contiguous()
+    with pytest.raises(ValueError, match="'G.wo' has shape"):
+        A.check_weights(cd, w)
+    w = weights()
+    w["R.wqkv"] = w["R.wqkv"].float()
+    with pytest.raises(ValueError, match="contiguous bf16"):
+        A.check_weights(cd, w)
+    w = weights()
+    w["wvel"] = w["wvel"].t()
+    with pytest.raises(ValueError, match="strided"):
+        A.check_weights(cd, w)
+    w = weights()
+    del w["gfin"]
+    with pytest.raises(ValueError, match="'gfin' missing"):
+        A.check_weights(cd, w)
+    seq = A.L.SeqDesc(3, 4, 5, 2, 0, 0, 0, 0)  # batch 2 x N 12 rows
+    ok = torch.zeros((2, 12, 64), dtype=torch.bfloat16)
+    with pytest.raises(ValueError, match="CUDA tensors only"):
+        A._check_state(seq, 64, h=ok, h_out=ok.clone())
+    with pytest.raises(ValueError, match="fewer than"):
+        A._check_state(seq, 64, h=ok[:1].clone())
