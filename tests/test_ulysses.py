@@ -41,15 +41,20 @@ def test_row_shards_and_head_blocks_partition_the_work():
         shard_rows(3, 4)
     with pytest.raises(ValueError):
         head_split(32, 8, 128, 3)
-    hs = head_split(32, 8, 128, 4)
-    covered = np.zeros((32 + 16) * 128, int)
-    for s in range(4):
-        packed = np.zeros(hs.packed_cols, int)
-        for src, width, dst in hs.blocks(s):
-            covered[src:src + width] += 1
-            packed[dst:dst + width] += 1
-        assert (packed == 1).all()  # each rank's packed row is filled exactly once
-    assert (covered == 1).all()      # every column of a q/k/v row goes to exactly one rank
+    for H, Hkv, p in ((32, 8, 4), (32, 8, 8), (64, 8, 8), (40, 40, 8), (4, 2, 2)):
+        hs = head_split(H, Hkv, 128, p)
+        covered = np.zeros((H + 2 * Hkv) * 128, int)
+        for s in range(p):
+            packed = np.zeros(hs.packed_cols, int)
+            for src, width, dst in hs.blocks(s):
+                covered[src:src + width] += 1
+                packed[dst:dst + width] += 1
+            # a rank's query heads read its own key/value heads (GQA groups stay whole)
+            q0 = hs.blocks(s)[0][0] // 128
+            k0 = (hs.blocks(s)[1][0] - H * 128) // 128
+            assert q0 // (H // Hkv) == k0
+            assert (packed == 1).all()  # each rank's packed row is filled exactly once
+        assert (covered == 1).all()      # every column of a q/k/v row goes to exactly one rank
 
 
 def _worker(rank, world, port, q, mode):
