@@ -2,8 +2,8 @@
 // (TMEM allocation, UMMA issue/commit, TMEM loads and stores) and bounded
 // waits that latch a device status word instead of spinning forever.
 //
-// Written from the PTX ISA (8.7+) instruction descriptions.  Nothing here
-// uses cluster multicast: every CTA issues its own loads.
+// Written from the PTX ISA (8.7+) instruction descriptions.  Every CTA issues
+// its own tile loads; no load is shared across the CTAs of a cluster.
 #pragma once
 
 #include <cstdint>
