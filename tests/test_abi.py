@@ -238,3 +238,39 @@ def test_api_refuses_weights_and_states_it_cannot_read_safely():
         A._check_state(seq, 64, h=ok, h_out=ok.clone())
     with pytest.raises(ValueError, match="fewer than"):
         A._check_state(seq, 64, h=ok[:1].clone())
+
+
+def test_ctypes_structs_and_constants_match_the_header(tmp_path):
+    """gcc compiles the header and prints every struct's size and field
+    offsets and every constant; the ctypes binding must agree on all of them."""
+    import shutil
+    from flow_matching_dit_cosmot_b200 import _lib as L
+    cc = shutil.which("gcc") or shutil.which("cc")
+    if cc is None:
+        pytest.skip("no C compiler")
+    structs = {"cosmot_layout_spec": L.LayoutSpec, "cosmot_segment": L.Segment, "cosmot_epilogue": L.Epilogue,
+               "cosmot_attn_desc": L.AttnDesc, "cosmot_dims": L.Dims, "cosmot_set_weights": L.SetWeights,
+               "cosmot_layer_weights": L.LayerWeights, "cosmot_seq_desc": L.SeqDesc,
+               "cosmot_action_desc": L.ActionDesc}
+    consts = [n for n in dir(L) if re.fullmatch(r"COSMOT_[A-Z_]+", n)]
+    lines = ["#include <stdio.h>", "#include <stddef.h>", '#include "cosmot.h"', "int main(void) {"]
+    for cname, cls in structs.items():
+        lines.append(f'  printf("{cname} %zu\\n", sizeof({cname}));')
+        for f, _ in cls._fields_:
+            lines.append(f'  printf("{cname}.{f} %zu\\n", offsetof({cname}, {f}));')
+    for n in consts:
+        lines.append(f'  printf("{n} %lld\\n", (long long)({n}));')
+    lines += ["  return 0;", "}"]
+    src = tmp_path / "layout.c"
+    src.write_text("\n".join(lines) + "\n")
+    exe = tmp_path / "layout"
+    include = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))), "include")
+    subprocess.run([cc, "-std=c11", "-I", include, str(src), "-o", str(exe)], check=True, capture_output=True)
+    got = dict(line.rsplit(" ", 1) for line in subprocess.run([str(exe)], capture_output=True, text=True,
+                                                               check=True).stdout.splitlines())
+    for cname, cls in structs.items():
+        assert int(got[cname]) == ctypes.sizeof(cls), cname
+        for f, _ in cls._fields_:
+            assert int(got[f"{cname}.{f}"]) == getattr(cls, f).offset, f"{cname}.{f}"
+    for n in consts:
+        assert int(got[n]) == getattr(L, n), n
