@@ -274,3 +274,40 @@ def test_ctypes_structs_and_constants_match_the_header(tmp_path):
             assert int(got[f"{cname}.{f}"]) == getattr(cls, f).offset, f"{cname}.{f}"
     for n in consts:
         assert int(got[n]) == getattr(L, n), n
+
+
+def _c_kind(param: str) -> str:
+    """Kind of one C parameter declaration: ptr, i32, i64, size, f32 or f64."""
+    p = param.strip()
+    if "*" in p or "[" in p or p.startswith("cosmot_stream_t"):
+        return "ptr"
+    for ctype, kind in (("int32_t", "i32"), ("int64_t", "i64"), ("size_t", "size"), ("double", "f64"),
+                        ("float", "f32"), ("cosmot_status", "i32")):
+        if p.startswith(ctype) or p.startswith("const " + ctype):
+            return kind
+    raise AssertionError(f"unclassified parameter {p!r}")
+
+
+def _py_kind(t) -> str:
+    if t in (ctypes.c_void_p, ctypes.c_char_p) or (isinstance(t, type) and issubclass(t, ctypes._Pointer)):
+        return "ptr"
+    return {ctypes.c_int32: "i32", ctypes.c_int64: "i64", ctypes.c_size_t: "size", ctypes.c_double: "f64",
+            ctypes.c_float: "f32"}[t]
+
+
+def test_binding_signatures_match_the_header_prototypes():
+    """Every entry the binding declares has the header's argument count and,
+    argument by argument, the same kind (pointer, 32/64-bit integer, size_t,
+    float, double), so ctypes marshals each value the way the C side reads it."""
+    from flow_matching_dit_cosmot_b200 import _lib as L
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    header = open(os.path.join(root, "include", "cosmot.h")).read()
+    header = re.sub(r"/\*.*?\*/", "", header, flags=re.S)
+    protos = {m.group(2): m.group(3) for m in
+              re.finditer(r"COSMOT_API\s+([\w\s\*]+?)\s*\b(cosmot_\w+)\s*\(([^)]*)\)\s*;", header)}
+    assert set(L.SIGNATURES) <= set(protos), set(L.SIGNATURES) - set(protos)
+    for name, (_, argtypes) in L.SIGNATURES.items():
+        params = [x for x in protos[name].split(",") if x.strip() and x.strip() != "void"]
+        assert len(params) == len(argtypes), name
+        for i, (cp, pt) in enumerate(zip(params, argtypes)):
+            assert _c_kind(cp) == _py_kind(pt), f"{name} argument {i}: {cp.strip()!r} vs {pt}"
