@@ -305,7 +305,7 @@ def test_binding_signatures_match_the_header_prototypes():
     header = re.sub(r"/\*.*?\*/", "", header, flags=re.S)
     protos = {m.group(2): m.group(3) for m in
               re.finditer(r"COSMOT_API\s+([\w\s\*]+?)\s*\b(cosmot_\w+)\s*\(([^)]*)\)\s*;", header)}
-    assert set(L.SIGNATURES) <= set(protos), set(L.SIGNATURES) - set(protos)
+    assert set(L.SIGNATURES) == set(protos), set(L.SIGNATURES) ^ set(protos)  # one binding per entry
     for name, (_, argtypes) in L.SIGNATURES.items():
         params = [x for x in protos[name].split(",") if x.strip() and x.strip() != "void"]
         assert len(params) == len(argtypes), name
