@@ -5,6 +5,7 @@ import ctypes
 import os
 import re
 import subprocess
+import sys
 
 import numpy as np
 import pytest
@@ -311,3 +312,31 @@ def test_binding_signatures_match_the_header_prototypes():
         assert len(params) == len(argtypes), name
         for i, (cp, pt) in enumerate(zip(params, argtypes)):
             assert _c_kind(cp) == _py_kind(pt), f"{name} argument {i}: {cp.strip()!r} vs {pt}"
+
+
+def test_product_never_reaches_the_oracle_and_has_no_fallback():
+    """The package and the CUDA sources neither import nor name the oracle, and
+    the binding raises when libcosmot.so is absent instead of computing on the
+    CPU."""
+    import ast
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    pkg = os.path.join(root, "flow_matching_dit_cosmot_b200")
+    for dirpath, _, files in os.walk(pkg):
+        for f in files:
+            path = os.path.join(dirpath, f)
+            if f.endswith(".py"):
+                tree = ast.parse(open(path).read())
+                for node in ast.walk(tree):
+                    names = []
+                    if isinstance(node, ast.Import):
+                        names = [a.name for a in node.names]
+                    elif isinstance(node, ast.ImportFrom):
+                        names = [node.module or ""]
+                    assert not any(n == "oracle" or n.startswith("oracle.") for n in names), (path, names)
+            elif f.endswith((".cu", ".cuh", ".h")):
+                assert "oracle" not in open(path).read(), path
+    code = ("import sys; sys.path.insert(0, %r); from flow_matching_dit_cosmot_b200 import _lib as L; "
+            "L.LIB_PATH = L.LIB_PATH + '.absent'; L._lib = None\n"
+            "try:\n    L.lib()\nexcept ImportError:\n    print('refused')\n" % root)
+    out = subprocess.run([sys.executable, "-c", code], capture_output=True, text=True)
+    assert out.stdout.strip() == "refused", out.stdout + out.stderr
