@@ -119,6 +119,22 @@ def _routed_sets_swapped(orig):
     return routed
 
 
+def _video_group_views_stacked(video, taus, t0, dt_v):
+    """Views share the canvas columns instead of sitting side by side along w."""
+    tau, view, y, x = np.meshgrid(np.asarray(taus, dtype=np.int64), np.arange(video.views),
+                                  np.arange(video.grid_h), np.arange(video.grid_w), indexing="ij")
+    tau, view, y, x = (a.reshape(-1) for a in (tau, view, y, x))
+    pos = np.stack([t0 + tau.astype(np.float64) * dt_v, y.astype(np.float64), x.astype(np.float64)], axis=1)
+    return pos, tau.astype(np.int32)
+
+
+def _commit_over_newest(self, k, v, chunk):
+    """The ring keeps writing one slot after it is full (the newest is lost)."""
+    i = min(self.next, self.slots - 1)
+    self.k[i], self.v[i], self.chunk[i] = k, v, chunk
+    self.next += 1
+
+
 # ---------------------------------------------------------------- cases
 
 MUTATIONS = {
@@ -176,6 +192,16 @@ MUTATIONS = {
         lambda mp: mp.setattr(layer, "shift_sigmas", lambda n, s: (1.0 - np.arange(n + 1) / n) /
                               (s + (1.0 - s) * (1.0 - np.arange(n + 1) / n))),
         [P.test_shift_schedule_properties]),
+    "action velocity without the final norm": (
+        lambda mp: mp.setattr(layer, "action_velocity",
+                              lambda dims, h_last, g_fin, w_out: np.asarray(h_last) @ np.asarray(w_out).T),
+        [P.test_policy_step_with_residual_only_layers_is_the_closed_form]),
+    "camera views not tiled along w": (
+        lambda mp: mp.setattr(layout, "_video_group", _video_group_views_stacked),
+        [P.test_views_tile_along_w]),
+    "stream ring overwrites its newest block": (
+        lambda mp: mp.setattr(layer.StreamState, "commit", _commit_over_newest),
+        [P.test_stream_ring_evicts_oldest]),
     "guidance extrapolates from the conditioned velocity": (
         lambda mp: mp.setattr(layer, "cfg_combine", lambda vc, vb, w: np.asarray(vc) + float(w) * (np.asarray(vc) -
                                                                                                    np.asarray(vb))),
