@@ -30,6 +30,7 @@ COSMOT_EPI_EULER = 4
 COSMOT_MASK_FULL = 0
 COSMOT_MASK_BLOCK_CAUSAL = 1
 COSMOT_ATTN_NO_TILE_SKIP = 1
+COSMOT_SITE_SELFTEST = 900
 
 c_i32, c_i64, c_f32, c_f64, c_vp = ctypes.c_int32, ctypes.c_int64, ctypes.c_float, ctypes.c_double, ctypes.c_void_p
 
@@ -94,6 +95,7 @@ SIGNATURES = {
     "cosmot_status_string": (ctypes.c_char_p, [c_i32]),
     "cosmot_version": (c_i32, []),
     "cosmot_get_device_status": (c_i32, [c_vp, _P(c_i32), _P(c_i32)]),
+    "cosmot_selftest_wait_timeout": (c_i32, [c_vp]),
     "cosmot_layout_counts": (c_i32, [_P(LayoutSpec), _P(c_i32), _P(c_i32), _P(c_i32), _P(c_i32)]),
     "cosmot_build_layout": (c_i32, [_P(LayoutSpec), c_vp, c_vp, c_vp, c_vp]),
     "cosmot_mrope_table": (c_i32, [c_vp, c_i64, c_i32, _P(c_i32), c_f64, c_vp, c_vp]),
@@ -190,6 +192,11 @@ def cosmot_get_device_status(stream: int = 0):
     st, where = c_i32(0), c_i32(0)
     _call("cosmot_get_device_status", c_vp(stream), ctypes.byref(st), ctypes.byref(where))
     return st.value, where.value
+
+
+def cosmot_selftest_wait_timeout(stream: int = 0):
+    """Test-only: a bounded wait that never completes; latches COSMOT_ERR_TIMEOUT."""
+    _call("cosmot_selftest_wait_timeout", c_vp(stream))
 
 
 def cosmot_layout_counts(spec: LayoutSpec):

@@ -20,6 +20,7 @@ enum Where : int {
   kWhereAttnMma = 201,
   kWhereAttnSoftmax = 202,
   kWhereAttnDrain = 203,
+  kWhereSelftest = COSMOT_SITE_SELFTEST,
 };
 
 // Encodes a 2D bf16 tensor map: `rows` x `cols` elements with row pitch

@@ -5,6 +5,7 @@
 #include <mutex>
 
 #include "cosmot_internal.h"
+#include "ptx.cuh"
 
 namespace cosmot {
 
@@ -75,9 +76,30 @@ cosmot_status make_tmap_bf16_2d(CUtensorMap* map, const void* base, uint64_t row
   return r == CUDA_SUCCESS ? COSMOT_OK : COSMOT_ERR_INVALID_ARG;
 }
 
+// Test-only: warp 0 is a producer that never arrives on the barrier; thread 32
+// waits for it with the library's bounded wait, which gives up after
+// kWaitLimitNs and latches COSMOT_ERR_TIMEOUT at kWhereSelftest.
+__global__ void __launch_bounds__(64) selftest_timeout_kernel(int* status) {
+  __shared__ alignas(8) uint64_t bar;
+  if (threadIdx.x == 0) {
+    mbar_init(smem_u32(&bar), 1);
+    fence_barrier_init();
+  }
+  __syncthreads();
+  if (threadIdx.x == 32) mbar_wait(smem_u32(&bar), 0, status, kWhereSelftest);
+  __syncthreads();
+}
+
 }  // namespace cosmot
 
 extern "C" {
+
+cosmot_status cosmot_selftest_wait_timeout(cosmot_stream_t stream) {
+  int* st = cosmot::device_status_ptr();
+  if (!st) return COSMOT_ERR_CUDA;
+  cosmot::selftest_timeout_kernel<<<1, 64, 0, reinterpret_cast<cudaStream_t>(stream)>>>(st);
+  return cosmot::launch_status();
+}
 
 const char* cosmot_status_string(cosmot_status s) {
   switch (s) {

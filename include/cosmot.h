@@ -72,6 +72,21 @@ COSMOT_API int32_t cosmot_version(void);
  */
 COSMOT_API cosmot_status cosmot_get_device_status(cosmot_stream_t stream, cosmot_status* out, int32_t* where_out);
 
+/* Site code that cosmot_selftest_wait_timeout latches with its timeout. */
+#define COSMOT_SITE_SELFTEST 900
+
+/*
+ * Test-only check of the failure path.  One CTA whose consumer thread waits on
+ * an mbarrier that its producer warp never arrives on, through the same bounded
+ * wait every kernel of the library uses.  The wait gives up after its bound
+ * (one second), latches COSMOT_ERR_TIMEOUT with site COSMOT_SITE_SELFTEST into
+ * the device status word, and the kernel returns: nothing faults or traps, and
+ * the context stays usable.  Returns the launch status; read the outcome with
+ * cosmot_get_device_status.  If the status word already holds a failure, the
+ * wait gives up at once and leaves that failure in place.
+ */
+COSMOT_API cosmot_status cosmot_selftest_wait_timeout(cosmot_stream_t stream);
+
 /* ===================================================================== layout */
 
 /*
