@@ -340,3 +340,21 @@ def test_product_never_reaches_the_oracle_and_has_no_fallback():
             "try:\n    L.lib()\nexcept ImportError:\n    print('refused')\n" % root)
     out = subprocess.run([sys.executable, "-c", code], capture_output=True, text=True)
     assert out.stdout.strip() == "refused", out.stdout + out.stderr
+
+
+def test_readme_c_example_compiles_against_the_header(tmp_path):
+    """The C usage example in README.md stays in step with include/cosmot.h."""
+    import shutil
+    cc = shutil.which("gcc") or shutil.which("cc")
+    cuda_inc = "/usr/local/cuda/include"
+    if cc is None or not os.path.exists(os.path.join(cuda_inc, "cuda_runtime.h")):
+        pytest.skip("no C compiler or CUDA headers")
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    text = open(os.path.join(root, "README.md"), encoding="utf-8").read()
+    blocks = re.findall(r"```c\n(.*?)```", text, flags=re.S)
+    assert blocks, "README has no C example"
+    src = tmp_path / "example.c"
+    src.write_text(blocks[0])
+    r = subprocess.run([cc, "-std=c11", "-fsyntax-only", "-Wall", "-Werror", "-I", os.path.join(root, "include"),
+                        "-I", cuda_inc, str(src)], capture_output=True, text=True)
+    assert r.returncode == 0, r.stderr
