@@ -41,9 +41,9 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # DRAM traffic per launch of the dominant kernel from an ncu capture
 # (dram__bytes_read.sum + dram__bytes_write.sum), keyed by stage, with the
 # sha256 of the kernel source it was taken on (comments excluded); reported
-# only while that code is unchanged.  Summaries live under profiles/.
+# only while that code is unchanged.
 NCU_TRAFFIC = {
-    # profiles/attention_t2v480_dram.md: one launch at the 480p shape (18,978 rows x 32 heads),
+    # one attention launch at the 480p shape (18,978 rows x 32 heads):
     # dram__bytes_read.sum 474,648,832 + dram__bytes_write.sum 136,260,608
     "t2v480:attention": {"bytes_per_launch": 610909440, "src_sha": "abea48bb2bacaadf"},
 }
@@ -58,8 +58,10 @@ def parse_args():
     p.add_argument("--impl", default="native", choices=["native", "reference"])
     p.add_argument("--no-e2e", action="store_true")
     p.add_argument("--no-cpu-baseline", action="store_true")
-    p.add_argument("--micro", choices=["attention", "gemm", "mrope", "euler", "rmsnorm"],
-                   help="time one kernel alone on the workload's widths (prints its own JSON line)")
+    p.add_argument("--micro", choices=["attention", "gemm", "mrope", "euler", "rmsnorm", "epilogues"],
+                   help="time one kernel alone on the workload's widths (prints its own JSON line); "
+                        "'epilogues' times the QKV and velocity GEMMs with their fused mRoPE and Euler "
+                        "epilogues against the same GEMMs with a plain epilogue")
     p.add_argument("--tokens", type=int, default=0, help="rows for --micro (default: the workload's N)")
     return p.parse_args()
 
@@ -96,14 +98,16 @@ def stage_work(dims, R, nz, pairs):
     dd, F, hd = dims.d_model, dims.ffn, dims.head_dim
     qc, qkvc = dims.q_cols, dims.qkv_cols
     w_set = 2  # bytes per bf16
+    # h1 (the residual stream between the two halves) is float32: written by the
+    # O projection, read by the pre-FFN norm and by the down projection
     return {
         "norm1": (0, R * dd * 4),
         "qkv_mrope": (2 * R * dd * qkvc, (R * dd + 2 * qkvc * dd + R * qkvc) * w_set),
         "attention": (4 * pairs * dims.n_heads * hd, (R * qkvc + R * qc) * w_set),
-        "oproj_residual": (2 * R * qc * dd, (R * qc + 2 * dd * qc + 2 * R * dd) * w_set),
-        "norm2": (0, R * dd * 4),
+        "oproj_residual": (2 * R * qc * dd, (R * qc + 2 * dd * qc + R * dd) * w_set + R * dd * 4),
+        "norm2": (0, R * dd * 4 + R * dd * 2),
         "gateup_silu": (2 * R * dd * 2 * F, (R * dd + 4 * F * dd + R * F) * w_set),
-        "down_residual": (2 * R * F * dd, (R * F + 2 * dd * F + 2 * R * dd) * w_set),
+        "down_residual": (2 * R * F * dd, (R * F + 2 * dd * F + R * dd) * w_set + R * dd * 4),
         "norm_final": (0, nz * dd * 4),
         "velocity_euler": (2 * nz * dd * dd, (nz * dd * 3 + dd * dd) * w_set),
     }
@@ -504,6 +508,14 @@ def run_native(args, wl):
     else:
         calls = [(z0, a, b) for a, b in zip(sig[:-1], sig[1:])]
     seqs = {c: seq(c) for c in {c for c, _, _ in calls}}
+    # samplers keep the state of the noisy rows in float32 between steps
+    # (cosmot_layer_forward_io / cosmot_stack_forward_io); the first call of a
+    # sampling or of a streaming block takes it from the bf16 rows of h
+    x_state = None
+    step_ios = [None] * len(calls)
+    if kind in ("sampler", "stream") and not guided and not ca:
+        x_state = torch.empty((B, lay.n_noisy, d), dtype=torch.float32, device=dev)
+        step_ios = [L.step_io(x_state.data_ptr(), d, 0, 0, i == 0) for i in range(len(calls))]
     if kind == "stream":
         noise = [to_dev(synth.make_activations(lay.n_noisy, d, 5000 + k)) for k in range(4)]
         # prefill the cache: AR rows and the 8 seeded history blocks, K/V in place
@@ -544,20 +556,21 @@ def run_native(args, wl):
             elif stack is not None:
                 if stage_evs is not None:
                     L.cosmot_stack_forward_timed(dims, stack.cw, seqs[c], h.data_ptr(), h_out.data_ptr(), s0, s1,
-                                                 ws.data_ptr(), ws.numel(), sh, [e.cuda_event for e in stage_evs[i]])
+                                                 ws.data_ptr(), ws.numel(), sh, [e.cuda_event for e in stage_evs[i]],
+                                                 step_ios[i])
                 else:
-                    L.cosmot_stack_forward(dims, stack.cw, seqs[c], h.data_ptr(), h_out.data_ptr(), s0, s1,
-                                           ws.data_ptr(), ws.numel(), sh)
+                    L.cosmot_stack_forward_io(dims, stack.cw, seqs[c], h.data_ptr(), h_out.data_ptr(), s0, s1,
+                                              step_ios[i], ws.data_ptr(), ws.numel(), sh)
             elif stage_evs is not None:
                 L.cosmot_layer_forward_timed(dims, layer.cw, seqs[c], h.data_ptr(), h_out.data_ptr(), s0, s1,
                                              ws.data_ptr(), ws.numel(), sh, [e.cuda_event for e in stage_evs[i]],
-                                             wl.guidance)
+                                             wl.guidance, step_ios[i])
             elif guided:
                 L.cosmot_layer_forward_cfg(dims, layer.cw, seqs[c], h.data_ptr(), h_out.data_ptr(), s0, s1,
                                            wl.guidance, ws.data_ptr(), ws.numel(), sh)
             else:
-                L.cosmot_layer_forward(dims, layer.cw, seqs[c], h.data_ptr(), h_out.data_ptr(), s0, s1,
-                                       ws.data_ptr(), ws.numel(), sh)
+                L.cosmot_layer_forward_io(dims, layer.cw, seqs[c], h.data_ptr(), h_out.data_ptr(), s0, s1,
+                                          step_ios[i], ws.data_ptr(), ws.numel(), sh)
         if kind == "stream":
             if commit_evs is not None:
                 commit_evs[0].record(stream)
@@ -622,7 +635,11 @@ def run_native(args, wl):
     if st:
         raise RuntimeError(f"device status {L.status_string(st)} at {where}")
 
-    total_ms = sum(starts[i].elapsed_time(ends[i]) for i in range(args.steps))
+    # `value` is throughput over the K timed steps (their summed device time);
+    # the median step is reported beside it
+    step_ms = [starts[i].elapsed_time(ends[i]) for i in range(args.steps)]
+    total_ms = sum(step_ms)
+    median_ms = statistics.median(step_ms)
     stage_ms = np.zeros(n_stage)  # per step, summed over the step's layer calls
     for per_call in stage_evs:
         for evs in per_call:
@@ -729,8 +746,9 @@ def run_native(args, wl):
                "serial": {"value": job_throughput(tokens_per_step, args.steps, world, serial_ms),
                           "ms_per_step": serial_ms / args.steps},
                "path": "cosmot_build_layout + cosmot_mrope_table + "
-                       + ("cosmot_policy_step" if ca else "cosmot_stack_forward" if n_layers > 1 else
-                          "cosmot_layer_forward_cfg" if guided else "cosmot_layer_forward")
+                       + ("cosmot_policy_step" if ca else
+                          ("cosmot_stack_forward" if n_layers > 1 else "cosmot_layer_forward_cfg" if guided else
+                           "cosmot_layer_forward") + ("_io (float32 state)" if x_state is not None else ""))
                        + (" + cosmot_layer_commit_kv" if kind == "stream" else "")
                        + (", pinned host inputs (h, action state) in, actions out" if ca else
                           ", pinned host input in, x' (noisy rows) out")}
@@ -798,7 +816,8 @@ def run_native(args, wl):
         cfg["tokens_per_step"] = tokens_per_step
         line = {
             "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
-            "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
+            "warmup": args.warmup, "ms_per_step": ms_step, "median_ms_per_step": round(median_ms, 4),
+            "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "bf16",
             "data": "synthetic (seeded Philox: activations N(0,1), weights N(0,0.02), gains 1+N(0,0.02))",
             "config": cfg,
@@ -843,6 +862,75 @@ def run_micro(args, wl):
     sh = torch.cuda.current_stream().cuda_stream
     peaks, peak_src = load_peaks()
     qkvc = dm.qkv_cols
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+
+    def time_launch(launch):
+        for _ in range(args.warmup):
+            flush.zero_()
+            launch()
+        torch.cuda.synchronize()
+        st_ev = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+        en_ev = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+        for i in range(args.steps):
+            flush.zero_()
+            st_ev[i].record()
+            launch()
+            en_ev[i].record()
+        torch.cuda.synchronize()
+        st, where = L.cosmot_get_device_status(sh)
+        if st:
+            raise RuntimeError(f"device status {L.status_string(st)} at {where}")
+        t = [st_ev[i].elapsed_time(en_ev[i]) for i in range(args.steps)]
+        return statistics.mean(t), statistics.median(t)
+
+    if args.micro == "epilogues":
+        # the QKV projection (mRoPE on its Q and K heads) and the velocity head
+        # (Euler step into the state), each against the same GEMM with a plain
+        # epilogue: the fused epilogue's cost is the extra time
+        a = rnd(T, d)
+        w = rnd(qkvc, d, std=0.02)
+        out = torch.empty((T, qkvc), dtype=torch.bfloat16, device=dev)
+        segs = [(0, n_ar, 0, 0), (n_ar, T, n_ar, 1)]
+        pos = torch.empty((T, 3), dtype=torch.float32, device=dev)
+        pos[:, 0] = torch.arange(T, device=dev, dtype=torch.float32)
+        pos[:, 1:] = (torch.arange(T, device=dev, dtype=torch.float32) % 26)[:, None]
+        cs = A.mrope_table(pos, hd, dm.rope_sections, dm.rope_base)
+        e_rope = L.Epilogue(kind=L.COSMOT_EPI_MROPE, head_dim=hd, rope_cols=(H + Hkv) * hd, rope_cs=cs.data_ptr(),
+                            rope_period=0)
+        nz = T - n_ar
+        wv = rnd(d, d, std=0.02)
+        x = rnd(nz, d)
+        xo = torch.empty_like(x)
+        vsegs = [(0, nz, 0, 1)]
+        e_euler = L.Epilogue(kind=L.COSMOT_EPI_EULER, x=x.data_ptr(), ld_x=d, dsigma=-0.03)
+        cases = {
+            "qkv_plain": lambda: L.cosmot_routed_linear(a.data_ptr(), d, d, segs, w.data_ptr(), w.data_ptr(), qkvc,
+                                                        out.data_ptr(), qkvc, stream=sh),
+            "qkv_mrope": lambda: L.cosmot_routed_linear(a.data_ptr(), d, d, segs, w.data_ptr(), w.data_ptr(), qkvc,
+                                                        out.data_ptr(), qkvc, e_rope, stream=sh),
+            "velocity_plain": lambda: L.cosmot_routed_linear(a.data_ptr(), d, d, vsegs, wv.data_ptr(), wv.data_ptr(),
+                                                             d, xo.data_ptr(), d, stream=sh),
+            "velocity_euler": lambda: L.cosmot_routed_linear(a.data_ptr(), d, d, vsegs, wv.data_ptr(), wv.data_ptr(),
+                                                             d, xo.data_ptr(), d, e_euler, stream=sh),
+        }
+        res = {k: time_launch(f) for k, f in cases.items()}
+        f_qkv, f_vel = 2 * T * d * qkvc, 2 * nz * d * d
+        burst = float(peaks["bf16_tflops"])
+        line = {"micro": "epilogues", "workload": wl.name, "tokens": T, "steps": args.steps, "warmup": args.warmup,
+                "peak_tflops": burst, "peak_source": f"{peak_src} burst"}
+        for k, (mean_ms, med_ms) in res.items():
+            fl = f_qkv if k.startswith("qkv") else f_vel
+            line[k] = {"ms": round(mean_ms, 4), "median_ms": round(med_ms, 4),
+                       "tflops": round(fl / (mean_ms / 1e3) / 1e12, 1),
+                       "frac": round(fl / (mean_ms / 1e3) / 1e12 / burst, 3)}
+        line["mrope_extra_ms"] = round(res["qkv_mrope"][0] - res["qkv_plain"][0], 4)
+        line["euler_extra_ms"] = round(res["velocity_euler"][0] - res["velocity_plain"][0], 4)
+        # what the same work would cost as a standalone HBM pass at the measured bandwidth
+        hbm = float(peaks["hbm_gbs"]) * 1e9
+        line["mrope_standalone_floor_ms"] = round((4 * T * (H + Hkv) * hd + T * (hd // 2) * 8) / hbm * 1e3, 4)
+        line["euler_standalone_floor_ms"] = round(6 * nz * d / hbm * 1e3, 4)
+        print(json.dumps(line), flush=True)
+        return
     if args.micro == "attention":
         qkv = rnd(T, qkvc)
         o = torch.empty((T, H * hd), dtype=torch.bfloat16, device=dev)
@@ -891,26 +979,11 @@ def run_micro(args, wl):
                                     sh)
         work, unit, peak = 4 * T * d, "GB/s", float(peaks["hbm_gbs"])
 
-    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
-    for _ in range(args.warmup):
-        flush.zero_()
-        launch()
-    torch.cuda.synchronize()
-    st_ev = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
-    en_ev = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
-    for i in range(args.steps):
-        flush.zero_()
-        st_ev[i].record()
-        launch()
-        en_ev[i].record()
-    torch.cuda.synchronize()
-    st, where = L.cosmot_get_device_status(sh)
-    if st:
-        raise RuntimeError(f"device status {L.status_string(st)} at {where}")
-    ms = statistics.mean(st_ev[i].elapsed_time(en_ev[i]) for i in range(args.steps))
+    ms, med = time_launch(launch)
     scale = 1e12 if unit == "TFLOP/s" else 1e9
     achieved = work / (ms / 1e3) / scale
-    print(json.dumps({"micro": args.micro, "workload": wl.name, "tokens": T, "ms": ms, "achieved": round(achieved, 1),
+    print(json.dumps({"micro": args.micro, "workload": wl.name, "tokens": T, "ms": ms, "median_ms": med,
+                      "achieved": round(achieved, 1),
                       "unit": unit, "peak": peak, "frac": round(achieved / peak, 3),
                       "peak_source": f"{peak_src} burst", "algorithmic_per_launch": work,
                       "steps": args.steps, "warmup": args.warmup}), flush=True)

@@ -26,6 +26,8 @@ COSMOT_EPI_RESIDUAL = 1
 COSMOT_EPI_SILU_MUL = 2
 COSMOT_EPI_MROPE = 3
 COSMOT_EPI_EULER = 4
+COSMOT_EPI_OUT_F32 = 1
+COSMOT_EPI_RES_F32 = 2
 
 COSMOT_MASK_FULL = 0
 COSMOT_MASK_BLOCK_CAUSAL = 1
@@ -52,7 +54,8 @@ class Segment(ctypes.Structure):
 class Epilogue(ctypes.Structure):
     _fields_ = [("kind", c_i32), ("head_dim", c_i32), ("rope_cols", c_i64), ("rope_cs", c_vp),
                 ("rope_period", c_i64), ("res", c_vp), ("ld_res", c_i64), ("x", c_vp), ("ld_x", c_i64),
-                ("dsigma", c_f32), ("reserved", c_f32)]
+                ("dsigma", c_f32), ("reserved", c_f32), ("x_state", c_vp), ("ld_state", c_i64), ("vel", c_vp),
+                ("ld_vel", c_i64), ("state_from_x", c_i32), ("flags", c_i32)]
 
 
 class AttnDesc(ctypes.Structure):
@@ -81,6 +84,11 @@ class ActionDesc(ctypes.Structure):
     _fields_ = [("action_dim", c_i32), ("n_clean", c_i32), ("n_noisy", c_i32), ("clean_row", c_i32),
                 ("w_in", c_vp), ("w_out", c_vp), ("x", c_vp), ("ld_x", c_i64), ("sigma", c_f64),
                 ("sigma_next", c_f64)]
+
+
+class StepIO(ctypes.Structure):
+    _fields_ = [("x_state", c_vp), ("ld_state", c_i64), ("vel", c_vp), ("ld_vel", c_i64), ("state_from_h", c_i32),
+                ("reserved", c_i32)]
 
 
 class SeqDesc(ctypes.Structure):
@@ -113,6 +121,8 @@ SIGNATURES = {
     "cosmot_layer_workspace_size": (c_i32, [_P(Dims), _P(SeqDesc), _P(ctypes.c_size_t)]),
     "cosmot_layer_forward": (c_i32, [_P(Dims), _P(LayerWeights), _P(SeqDesc), c_vp, c_vp, c_f64, c_f64, c_vp,
                                      ctypes.c_size_t, c_vp]),
+    "cosmot_layer_forward_io": (c_i32, [_P(Dims), _P(LayerWeights), _P(SeqDesc), c_vp, c_vp, c_f64, c_f64,
+                                        _P(StepIO), c_vp, ctypes.c_size_t, c_vp]),
     "cosmot_flow_shift_sigmas": (c_i32, [c_i32, c_f64, _P(c_f64)]),
     "cosmot_action_embed": (c_i32, [c_vp, c_i64, _P(Segment), c_i32, c_vp, c_i32, c_i32, c_vp, c_i64, c_vp]),
     "cosmot_action_head": (c_i32, [c_vp, c_i64, _P(Segment), c_i32, c_vp, c_f32, c_vp, c_i32, c_i32, c_vp, c_i64, c_f64,
@@ -128,14 +138,16 @@ SIGNATURES = {
     "cosmot_stack_workspace_size": (c_i32, [_P(Dims), c_i32, _P(SeqDesc), _P(ctypes.c_size_t)]),
     "cosmot_stack_forward": (c_i32, [_P(Dims), _P(LayerWeights), c_i32, _P(SeqDesc), c_vp, c_vp, c_f64, c_f64, c_vp,
                                      ctypes.c_size_t, c_vp]),
+    "cosmot_stack_forward_io": (c_i32, [_P(Dims), _P(LayerWeights), c_i32, _P(SeqDesc), c_vp, c_vp, c_f64, c_f64,
+                                        _P(StepIO), c_vp, ctypes.c_size_t, c_vp]),
     "cosmot_stack_forward_timed": (c_i32, [_P(Dims), _P(LayerWeights), c_i32, _P(SeqDesc), c_vp, c_vp, c_f64, c_f64,
-                                           c_vp, ctypes.c_size_t, c_vp, _P(c_vp), c_i32]),
+                                           c_vp, ctypes.c_size_t, c_vp, _P(c_vp), c_i32, _P(StepIO)]),
     "cosmot_layer_commit_kv": (c_i32, [_P(Dims), _P(LayerWeights), _P(SeqDesc), c_vp, c_i64, c_vp, ctypes.c_size_t,
                                        c_vp]),
     "cosmot_layer_forward_noalloc": (c_i32, [_P(Dims), _P(LayerWeights), _P(SeqDesc), c_vp, c_vp, c_f64, c_f64,
                                              c_vp]),
     "cosmot_layer_forward_timed": (c_i32, [_P(Dims), _P(LayerWeights), _P(SeqDesc), c_vp, c_vp, c_f64, c_f64, c_vp,
-                                           ctypes.c_size_t, c_vp, _P(c_vp), c_i32, _P(c_f64)]),
+                                           ctypes.c_size_t, c_vp, _P(c_vp), c_i32, _P(c_f64), _P(StepIO)]),
 }
 
 COSMOT_LAYER_STAGES = 9
@@ -290,6 +302,19 @@ def cosmot_layer_forward(dims: Dims, w: LayerWeights, seq: SeqDesc, h: int, h_ou
                  c_vp(h_out), sigma, sigma_next, c_vp(workspace), workspace_bytes, c_vp(stream), check=check)
 
 
+def step_io(x_state: int = 0, ld_state: int = 0, vel: int = 0, ld_vel: int = 0, state_from_h: bool = False):
+    """StepIO for cosmot_layer_forward_io / _timed (pointers as integers, 0 = absent)."""
+    return StepIO(x_state or None, ld_state, vel or None, ld_vel, 1 if state_from_h else 0, 0)
+
+
+def cosmot_layer_forward_io(dims: Dims, w: LayerWeights, seq: SeqDesc, h: int, h_out: int, sigma: float,
+                            sigma_next: float, io: StepIO | None, workspace: int, workspace_bytes: int,
+                            stream: int = 0, check=True):
+    return _call("cosmot_layer_forward_io", ctypes.byref(dims), ctypes.byref(w), ctypes.byref(seq), c_vp(h),
+                 c_vp(h_out), sigma, sigma_next, ctypes.byref(io) if io is not None else None, c_vp(workspace),
+                 workspace_bytes, c_vp(stream), check=check)
+
+
 def cosmot_layer_commit_kv(dims: Dims, w: LayerWeights, seq: SeqDesc, h: int, dst_row: int, workspace: int,
                            workspace_bytes: int, stream: int = 0, check=True):
     return _call("cosmot_layer_commit_kv", ctypes.byref(dims), ctypes.byref(w), ctypes.byref(seq), c_vp(h), dst_row,
@@ -373,16 +398,25 @@ def cosmot_stack_forward(dims: Dims, layers, seq: SeqDesc, h: int, h_out: int, s
                  c_vp(h_out), sigma, sigma_next, c_vp(workspace), workspace_bytes, c_vp(stream), check=check)
 
 
+def cosmot_stack_forward_io(dims: Dims, layers, seq: SeqDesc, h: int, h_out: int, sigma: float, sigma_next: float,
+                            io: StepIO | None, workspace: int, workspace_bytes: int, stream: int = 0, check=True):
+    if not isinstance(layers, ctypes.Array):
+        layers = (LayerWeights * len(layers))(*layers)
+    return _call("cosmot_stack_forward_io", ctypes.byref(dims), layers, len(layers), ctypes.byref(seq), c_vp(h),
+                 c_vp(h_out), sigma, sigma_next, ctypes.byref(io) if io is not None else None, c_vp(workspace),
+                 workspace_bytes, c_vp(stream), check=check)
+
+
 def cosmot_stack_forward_timed(dims: Dims, layers, seq: SeqDesc, h: int, h_out: int, sigma: float,
                                sigma_next: float, workspace: int, workspace_bytes: int, stream: int, events,
-                               check=True):
+                               io: StepIO | None = None, check=True):
     """`events`: 8 * len(layers) + 2 raw cudaEvent_t handles (ints)."""
     if not isinstance(layers, ctypes.Array):
         layers = (LayerWeights * len(layers))(*layers)
     arr = (c_vp * len(events))(*[c_vp(e) for e in events])
     return _call("cosmot_stack_forward_timed", ctypes.byref(dims), layers, len(layers), ctypes.byref(seq), c_vp(h),
                  c_vp(h_out), sigma, sigma_next, c_vp(workspace), workspace_bytes, c_vp(stream), arr, len(events),
-                 check=check)
+                 ctypes.byref(io) if io is not None else None, check=check)
 
 
 def cosmot_layer_forward_noalloc(dims: Dims, w: LayerWeights, seq: SeqDesc, h: int, h_out: int, sigma: float,
@@ -394,11 +428,12 @@ def cosmot_layer_forward_noalloc(dims: Dims, w: LayerWeights, seq: SeqDesc, h: i
 
 def cosmot_layer_forward_timed(dims: Dims, w: LayerWeights, seq: SeqDesc, h: int, h_out: int, sigma: float,
                                sigma_next: float, workspace: int, workspace_bytes: int, stream: int, events,
-                               guidance: float | None = None, check=True):
+                               guidance: float | None = None, io: StepIO | None = None, check=True):
     """`events`: COSMOT_LAYER_STAGES + 1 raw cudaEvent_t handles (ints); `guidance`
-    selects the guided step of cosmot_layer_forward_cfg."""
+    selects the guided step of cosmot_layer_forward_cfg; `io` the float32 state
+    and velocity output of cosmot_layer_forward_io."""
     arr = (c_vp * len(events))(*[c_vp(e) for e in events])
     g = ctypes.byref(c_f64(guidance)) if guidance is not None else None
     return _call("cosmot_layer_forward_timed", ctypes.byref(dims), ctypes.byref(w), ctypes.byref(seq), c_vp(h),
                  c_vp(h_out), sigma, sigma_next, c_vp(workspace), workspace_bytes, c_vp(stream), arr, len(events), g,
-                 check=check)
+                 ctypes.byref(io) if io is not None else None, check=check)

@@ -163,12 +163,40 @@ class MoTLayer:
                                    float(guidance), ptr(ws), ws.numel(), stream_handle(stream))
 
     def forward(self, h: torch.Tensor, h_out: torch.Tensor, sigma: float, sigma_next: float, seq: L.SeqDesc,
-                workspace: Optional[torch.Tensor] = None, stream=None):
-        """h [batch, N, d] bf16 (noisy DM rows updated in place to x'); h_out [batch, N, d] bf16."""
+                workspace: Optional[torch.Tensor] = None, stream=None, x_state: Optional[torch.Tensor] = None,
+                state_from_h: bool = False, vel: Optional[torch.Tensor] = None):
+        """h [batch, N, d] bf16 (noisy DM rows updated in place to x'); h_out [batch, N, d] bf16.
+
+        x_state: optional float32 [batch, n_noisy, d] sampler state of the noisy
+        rows, read (unless state_from_h) and written in float32; h's noisy rows
+        then receive its bf16 copy.  vel: optional bf16 [batch, n_noisy, d]
+        receiving the velocity (see cosmot_layer_forward_io)."""
         _check_state(seq, self.dims.d_model, h=h, h_out=h_out)
         ws = workspace if workspace is not None else self.workspace(seq, h.device)
-        L.cosmot_layer_forward(self.dims, self.cw, seq, ptr(h), ptr(h_out), float(sigma), float(sigma_next),
-                               ptr(ws), ws.numel(), stream_handle(stream))
+        io = self.step_io(seq, x_state, state_from_h, vel)
+        if io is None:
+            L.cosmot_layer_forward(self.dims, self.cw, seq, ptr(h), ptr(h_out), float(sigma), float(sigma_next),
+                                   ptr(ws), ws.numel(), stream_handle(stream))
+        else:
+            L.cosmot_layer_forward_io(self.dims, self.cw, seq, ptr(h), ptr(h_out), float(sigma), float(sigma_next),
+                                      io, ptr(ws), ws.numel(), stream_handle(stream))
+
+    def step_io(self, seq: L.SeqDesc, x_state: Optional[torch.Tensor] = None, state_from_h: bool = False,
+                vel: Optional[torch.Tensor] = None) -> Optional[L.StepIO]:
+        """The StepIO struct for an optional float32 state and velocity output,
+        both [batch, n_noisy, d] contiguous (checked here: the kernels read and
+        write them through bare pointers)."""
+        if x_state is None and vel is None:
+            return None
+        d, rows = self.dims.d_model, seq.batch * seq.n_noisy
+        for name, t, dt in (("x_state", x_state, torch.float32), ("vel", vel, torch.bfloat16)):
+            if t is None:
+                continue
+            _need_cuda(t)
+            if t.dtype != dt or not t.is_contiguous() or t.numel() < rows * d:
+                raise ValueError(f"{name}: expected a contiguous {dt} tensor of batch x n_noisy x d = {rows * d} "
+                                 f"elements (got {t.dtype}, {t.numel()})")
+        return L.step_io(ptr(x_state), d, ptr(vel), d, state_from_h)
 
 
 class MoTStack:
@@ -197,9 +225,16 @@ class MoTStack:
         return self._ws
 
     def forward(self, h: torch.Tensor, h_out: torch.Tensor, sigma: float, sigma_next: float, seq: L.SeqDesc,
-                workspace: Optional[torch.Tensor] = None, stream=None):
-        """h^L into h_out; x' into the noisy rows of h (see cosmot_stack_forward)."""
+                workspace: Optional[torch.Tensor] = None, stream=None, x_state: Optional[torch.Tensor] = None,
+                state_from_h: bool = False, vel: Optional[torch.Tensor] = None):
+        """h^L into h_out; x' into the noisy rows of h (see cosmot_stack_forward);
+        x_state / vel as for MoTLayer.forward."""
         _check_state(seq, self.dims.d_model, h=h, h_out=h_out)
         ws = workspace if workspace is not None else self.workspace(seq, h.device)
-        L.cosmot_stack_forward(self.dims, self.cw, seq, ptr(h), ptr(h_out), sigma, sigma_next, ptr(ws), ws.numel(),
-                               stream_handle(stream))
+        io = self.layers[0].step_io(seq, x_state, state_from_h, vel)
+        if io is None:
+            L.cosmot_stack_forward(self.dims, self.cw, seq, ptr(h), ptr(h_out), sigma, sigma_next, ptr(ws),
+                                   ws.numel(), stream_handle(stream))
+        else:
+            L.cosmot_stack_forward_io(self.dims, self.cw, seq, ptr(h), ptr(h_out), sigma, sigma_next, io, ptr(ws),
+                                      ws.numel(), stream_handle(stream))

@@ -38,6 +38,12 @@ inline cosmot_status launch_status() {
 
 int num_sms();
 
+// cosmot_rmsnorm_routed with a float32 input when h_f32 (the layer's h1, the
+// residual stream between the attention and FFN halves, is kept in float32).
+cosmot_status rmsnorm_routed(const void* h, bool h_f32, int64_t ld_h, const cosmot_segment* segs, int32_t n_segs,
+                             const void* g0, const void* g1, int64_t d, float eps, void* out, int64_t ld_out,
+                             cosmot_stream_t stream);
+
 // Per-device address of the status word that kernels latch failures into.
 int* device_status_ptr();
 

@@ -39,7 +39,70 @@ bool fill_segs(const cosmot_segment* segs, int32_t n, SegTable* t) {
 }
 
 // ---------------------------------------------------------------- RMSNorm
-// One warp per row; the row stays in registers between the two passes.
+// One warp per row.  A bf16 row stays in registers between the two passes; a
+// float32 row (a residual stream kept in float32) is read again in the second
+// pass, from L1/L2, so that the registers hold no more than for bf16.
+__device__ __forceinline__ void load8_f32(const float* p, float* f) {
+  const float4 a = *reinterpret_cast<const float4*>(p);
+  const float4 b = *reinterpret_cast<const float4*>(p + 4);
+  f[0] = a.x; f[1] = a.y; f[2] = a.z; f[3] = a.w;
+  f[4] = b.x; f[5] = b.y; f[6] = b.z; f[7] = b.w;
+}
+
+template <int kVecPerLane>
+__global__ void __launch_bounds__(256) rmsnorm_f32in_kernel(const float* __restrict__ h, int64_t ld_h,
+                                                            const SegTable segs, const __nv_bfloat16* __restrict__ g0,
+                                                            const __nv_bfloat16* __restrict__ g1, int32_t d, float eps,
+                                                            __nv_bfloat16* __restrict__ out, int64_t ld_out) {
+  const int lane = threadIdx.x & 31;
+  const int64_t warps_total = (int64_t)gridDim.x * (blockDim.x >> 5);
+  const int nvec = d >> 3;
+  for (int64_t gr = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); gr < segs.prefix[segs.n];
+       gr += warps_total) {
+    int s = 0;
+    while (s + 1 < segs.n && gr >= segs.prefix[s + 1]) ++s;
+    const int64_t local = gr - segs.prefix[s];
+    const int64_t r = segs.row_begin[s] + local;
+    const int64_t o = segs.out_row[s] + local;
+    const __nv_bfloat16* g = segs.set[s] ? g1 : g0;
+    const float* src = h + r * ld_h;
+    float ss = 0.f;
+#pragma unroll
+    for (int j = 0; j < kVecPerLane; ++j) {
+      const int c = lane + 32 * j;
+      if (c < nvec) {
+        float f[8];
+        load8_f32(src + 8 * c, f);
+#pragma unroll
+        for (int q = 0; q < 8; ++q) ss = fmaf(f[q], f[q], ss);
+      }
+    }
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, off);
+    const float rstd = rsqrtf(ss / (float)d + eps);
+    uint4* dst = reinterpret_cast<uint4*>(out + o * ld_out);
+    const uint4* gv = reinterpret_cast<const uint4*>(g);
+#pragma unroll
+    for (int j = 0; j < kVecPerLane; ++j) {
+      const int c = lane + 32 * j;
+      if (c < nvec) {
+        float f[8];
+        load8_f32(src + 8 * c, f);
+        uint4 gg = __ldg(gv + c);
+        const uint32_t* gu = reinterpret_cast<const uint32_t*>(&gg);
+        uint4 res;
+        uint32_t* ru = reinterpret_cast<uint32_t*>(&res);
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          float2 w = unpack_bf16x2(gu[q]);
+          ru[q] = pack_bf16x2(f[2 * q] * rstd * w.x, f[2 * q + 1] * rstd * w.y);
+        }
+        dst[c] = res;
+      }
+    }
+  }
+}
+
 template <int kVecPerLane>
 __global__ void __launch_bounds__(256) rmsnorm_kernel(const __nv_bfloat16* __restrict__ h, int64_t ld_h,
                                                       const SegTable segs, const __nv_bfloat16* __restrict__ g0,
@@ -210,12 +273,11 @@ unsigned grid_for(int64_t work_items, int threads) {
 }  // namespace
 }  // namespace cosmot
 
-extern "C" {
+namespace cosmot {
 
-cosmot_status cosmot_rmsnorm_routed(const void* h, int64_t ld_h, const cosmot_segment* segs, int32_t n_segs,
-                                    const void* g0, const void* g1, int64_t d, float eps, void* out,
-                                    int64_t ld_out, cosmot_stream_t stream) {
-  using namespace cosmot;
+cosmot_status rmsnorm_routed(const void* h, bool h_f32, int64_t ld_h, const cosmot_segment* segs, int32_t n_segs,
+                             const void* g0, const void* g1, int64_t d, float eps, void* out, int64_t ld_out,
+                             cosmot_stream_t stream) {
   SegTable t;
   if (!h || !out || !fill_segs(segs, n_segs, &t)) return COSMOT_ERR_INVALID_ARG;
   if (d <= 0 || d % 8 || ld_h % 8 || ld_out % 8 || ld_h < d || ld_out < d || !aligned16(h) || !aligned16(out))
@@ -235,6 +297,16 @@ cosmot_status cosmot_rmsnorm_routed(const void* h, int64_t ld_h, const cosmot_se
   const auto* gp1 = static_cast<const __nv_bfloat16*>(g1);
   auto* op = static_cast<__nv_bfloat16*>(out);
   const int vpl = (int)((d / 8 + 31) / 32);
+  if (h_f32) {
+    const auto* hf = static_cast<const float*>(h);
+    if (vpl <= 4)
+      rmsnorm_f32in_kernel<4><<<grid, threads, 0, s>>>(hf, ld_h, t, gp0, gp1, (int32_t)d, eps, op, ld_out);
+    else if (vpl <= 16)
+      rmsnorm_f32in_kernel<16><<<grid, threads, 0, s>>>(hf, ld_h, t, gp0, gp1, (int32_t)d, eps, op, ld_out);
+    else
+      rmsnorm_f32in_kernel<24><<<grid, threads, 0, s>>>(hf, ld_h, t, gp0, gp1, (int32_t)d, eps, op, ld_out);
+    return launch_status();
+  }
   if (vpl <= 4)
     rmsnorm_kernel<4><<<grid, threads, 0, s>>>(hp, ld_h, t, gp0, gp1, (int32_t)d, eps, op, ld_out);
   else if (vpl <= 16)
@@ -242,6 +314,16 @@ cosmot_status cosmot_rmsnorm_routed(const void* h, int64_t ld_h, const cosmot_se
   else
     rmsnorm_kernel<24><<<grid, threads, 0, s>>>(hp, ld_h, t, gp0, gp1, (int32_t)d, eps, op, ld_out);
   return launch_status();
+}
+
+}  // namespace cosmot
+
+extern "C" {
+
+cosmot_status cosmot_rmsnorm_routed(const void* h, int64_t ld_h, const cosmot_segment* segs, int32_t n_segs,
+                                    const void* g0, const void* g1, int64_t d, float eps, void* out,
+                                    int64_t ld_out, cosmot_stream_t stream) {
+  return cosmot::rmsnorm_routed(h, false, ld_h, segs, n_segs, g0, g1, d, eps, out, ld_out, stream);
 }
 
 cosmot_status cosmot_mrope_apply(void* q, int64_t ld_q, int32_t n_q_heads, void* k, int64_t ld_k,

@@ -61,12 +61,17 @@ struct Params {
   int64_t rope_cols;
   const float2* rope_cs;
   int64_t rope_period;
-  const __nv_bfloat16* res;
+  const void* res;        // bf16, or float32 with COSMOT_EPI_RES_F32
   int64_t ld_res;
   const __nv_bfloat16* x;
   int64_t ld_x;
   float dsigma;
-  __nv_bfloat16* out;
+  int32_t xs_from_x;      // EULER with xs: read x from the bf16 `x` this call
+  float* xs;              // EULER: optional float32 state, indexed by input row
+  int64_t ld_xs;
+  __nv_bfloat16* vel;     // EULER: optional bf16 copy of the accumulator, by input row
+  int64_t ld_vel;
+  __nv_bfloat16* out;     // float32 storage with COSMOT_EPI_OUT_F32
   int64_t ld_out;
   int* status;
 };
@@ -114,6 +119,26 @@ __device__ __forceinline__ void store_row32(__nv_bfloat16* dst, int32_t col0, in
   }
 }
 
+// Stores / loads 32 consecutive fp32 values of one row, clipped to n_out.
+__device__ __forceinline__ void store_row32_f32(float* dst, int32_t col0, int32_t n_out, const float* v) {
+#pragma unroll
+  for (int q = 0; q < 8; ++q)
+    if (col0 + 4 * q + 4 <= n_out)
+      *reinterpret_cast<float4*>(dst + 4 * q) = make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
+}
+
+__device__ __forceinline__ void load_row32_f32(const float* src, int32_t col0, int32_t n_out, float* v) {
+#pragma unroll
+  for (int q = 0; q < 8; ++q) {
+    float4 w = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (col0 + 4 * q + 4 <= n_out) w = *reinterpret_cast<const float4*>(src + 4 * q);
+    v[4 * q] = w.x;
+    v[4 * q + 1] = w.y;
+    v[4 * q + 2] = w.z;
+    v[4 * q + 3] = w.w;
+  }
+}
+
 // Loads 32 consecutive bf16 of one row as fp32 (zeros past n_out).
 __device__ __forceinline__ void load_row32(const __nv_bfloat16* src, int32_t col0, int32_t n_out, float* v) {
 #pragma unroll
@@ -134,7 +159,8 @@ __device__ __forceinline__ void load_row32(const __nv_bfloat16* src, int32_t col
   }
 }
 
-template <int EPI>
+// FL: COSMOT_EPI_OUT_F32 / COSMOT_EPI_RES_F32 bits of the RESIDUAL epilogue.
+template <int EPI, int FL>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
     routed_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUtensorMap tmap_b0,
                        const __grid_constant__ CUtensorMap tmap_b1, const __grid_constant__ CUtensorMap tmap_u0,
@@ -360,19 +386,37 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           if (valid && col0 < p.n_out) {
             if (EPI == COSMOT_EPI_RESIDUAL) {
               float rs[32];
-              load_row32(p.res + orow * p.ld_res + col0, col0, p.n_out, rs);
+              if (FL & COSMOT_EPI_RES_F32)
+                load_row32_f32(static_cast<const float*>(p.res) + orow * p.ld_res + col0, col0, p.n_out, rs);
+              else
+                load_row32(static_cast<const __nv_bfloat16*>(p.res) + orow * p.ld_res + col0, col0, p.n_out, rs);
 #pragma unroll
               for (int j = 0; j < 32; ++j) f[j] = __uint_as_float(v[j]) + rs[j];
             } else if (EPI == COSMOT_EPI_EULER) {
+              // x' = x + dsigma * v in fp32; x from the fp32 state when there is one
+              const int64_t arow = tl.a_row0 + r;
               float xs[32];
-              load_row32(p.x + orow * p.ld_x + col0, col0, p.n_out, xs);
+              if (p.xs && !p.xs_from_x)
+                load_row32_f32(p.xs + arow * p.ld_xs + col0, col0, p.n_out, xs);
+              else
+                load_row32(p.x + orow * p.ld_x + col0, col0, p.n_out, xs);
 #pragma unroll
               for (int j = 0; j < 32; ++j) f[j] = fmaf(p.dsigma, __uint_as_float(v[j]), xs[j]);
+              if (p.xs) store_row32_f32(p.xs + arow * p.ld_xs + col0, col0, p.n_out, f);
+              if (p.vel) {
+                float vv[32];
+#pragma unroll
+                for (int j = 0; j < 32; ++j) vv[j] = __uint_as_float(v[j]);
+                store_row32(p.vel + arow * p.ld_vel + col0, col0, p.n_out, vv);
+              }
             } else {
 #pragma unroll
               for (int j = 0; j < 32; ++j) f[j] = __uint_as_float(v[j]);
             }
-            store_row32(p.out + orow * p.ld_out + col0, col0, p.n_out, f);
+            if (FL & COSMOT_EPI_OUT_F32)
+              store_row32_f32(reinterpret_cast<float*>(p.out) + orow * p.ld_out + col0, col0, p.n_out, f);
+            else
+              store_row32(p.out + orow * p.ld_out + col0, col0, p.n_out, f);
           }
         }
       }
@@ -387,7 +431,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   if (warp == 1) tmem_dealloc(tmem_base, TMEM_COLS);
 }
 
-template <int EPI>
+template <int EPI, int FL = 0>
 cosmot_status launch(const CUtensorMap& ta, const CUtensorMap& tb0, const CUtensorMap& tb1, const CUtensorMap& tu0,
                      const CUtensorMap& tu1, const Params& p, cudaStream_t s) {
   static std::mutex mu;
@@ -397,7 +441,7 @@ cosmot_status launch(const CUtensorMap& ta, const CUtensorMap& tb0, const CUtens
   {
     std::lock_guard<std::mutex> lk(mu);
     if (dev >= 64 || !(done_mask & (1ull << dev))) {
-      if (cudaFuncSetAttribute(routed_gemm_kernel<EPI>, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES) !=
+      if (cudaFuncSetAttribute(routed_gemm_kernel<EPI, FL>, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES) !=
           cudaSuccess)
         return COSMOT_ERR_CUDA;
       if (dev < 64) done_mask |= 1ull << dev;
@@ -405,7 +449,7 @@ cosmot_status launch(const CUtensorMap& ta, const CUtensorMap& tb0, const CUtens
   }
   int grid = num_sms();
   if (p.num_tiles < grid) grid = p.num_tiles;
-  routed_gemm_kernel<EPI><<<grid, NUM_THREADS, SMEM_BYTES, s>>>(ta, tb0, tb1, tu0, tu1, p);
+  routed_gemm_kernel<EPI, FL><<<grid, NUM_THREADS, SMEM_BYTES, s>>>(ta, tb0, tb1, tu0, tu1, p);
   return launch_status();
 }
 
@@ -425,6 +469,9 @@ extern "C" cosmot_status cosmot_routed_linear(const void* a, int64_t ld_a, int64
   if (!aligned16(a) || !aligned16(out)) return COSMOT_ERR_INVALID_ARG;
   if (k > INT32_MAX || n_out > INT32_MAX) return COSMOT_ERR_UNSUPPORTED;
   if (kind < COSMOT_EPI_NONE || kind > COSMOT_EPI_EULER) return COSMOT_ERR_INVALID_ARG;
+  const int flags = epi ? epi->flags : 0;
+  if (flags & ~(COSMOT_EPI_OUT_F32 | COSMOT_EPI_RES_F32)) return COSMOT_ERR_INVALID_ARG;
+  if (flags && kind != COSMOT_EPI_RESIDUAL) return COSMOT_ERR_INVALID_ARG;
 
   Params p{};
   p.n_segs = n_segs;
@@ -464,13 +511,24 @@ extern "C" cosmot_status cosmot_routed_linear(const void* a, int64_t ld_a, int64
 
   if (kind == COSMOT_EPI_RESIDUAL) {
     if (!epi->res || !aligned16(epi->res) || epi->ld_res % 8 || epi->ld_res < n_out) return COSMOT_ERR_INVALID_ARG;
-    p.res = static_cast<const __nv_bfloat16*>(epi->res);
+    p.res = epi->res;
     p.ld_res = epi->ld_res;
   } else if (kind == COSMOT_EPI_EULER) {
     if (!epi->x || !aligned16(epi->x) || epi->ld_x % 8 || epi->ld_x < n_out) return COSMOT_ERR_INVALID_ARG;
     p.x = static_cast<const __nv_bfloat16*>(epi->x);
     p.ld_x = epi->ld_x;
     p.dsigma = epi->dsigma;
+    if (epi->x_state) {
+      if (!aligned16(epi->x_state) || epi->ld_state % 8 || epi->ld_state < n_out) return COSMOT_ERR_INVALID_ARG;
+      p.xs = epi->x_state;
+      p.ld_xs = epi->ld_state;
+      p.xs_from_x = epi->state_from_x ? 1 : 0;
+    }
+    if (epi->vel) {
+      if (!aligned16(epi->vel) || epi->ld_vel % 8 || epi->ld_vel < n_out) return COSMOT_ERR_INVALID_ARG;
+      p.vel = static_cast<__nv_bfloat16*>(epi->vel);
+      p.ld_vel = epi->ld_vel;
+    }
   } else if (kind == COSMOT_EPI_MROPE) {
     if (epi->head_dim != 64 && epi->head_dim != 128) return COSMOT_ERR_UNSUPPORTED;
     if (!epi->rope_cs || !aligned16(epi->rope_cs) || epi->rope_cols < 0 || epi->rope_cols % epi->head_dim ||
@@ -505,7 +563,15 @@ extern "C" cosmot_status cosmot_routed_linear(const void* a, int64_t ld_a, int64
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   switch (kind) {
     case COSMOT_EPI_NONE: return launch<COSMOT_EPI_NONE>(ta, tb[0], tb[1], tu[0], tu[1], p, s);
-    case COSMOT_EPI_RESIDUAL: return launch<COSMOT_EPI_RESIDUAL>(ta, tb[0], tb[1], tu[0], tu[1], p, s);
+    case COSMOT_EPI_RESIDUAL:
+      switch (flags) {
+        case COSMOT_EPI_OUT_F32: return launch<COSMOT_EPI_RESIDUAL, COSMOT_EPI_OUT_F32>(ta, tb[0], tb[1], tu[0], tu[1], p, s);
+        case COSMOT_EPI_RES_F32: return launch<COSMOT_EPI_RESIDUAL, COSMOT_EPI_RES_F32>(ta, tb[0], tb[1], tu[0], tu[1], p, s);
+        case COSMOT_EPI_OUT_F32 | COSMOT_EPI_RES_F32:
+          return launch<COSMOT_EPI_RESIDUAL, COSMOT_EPI_OUT_F32 | COSMOT_EPI_RES_F32>(ta, tb[0], tb[1], tu[0], tu[1],
+                                                                                     p, s);
+        default: return launch<COSMOT_EPI_RESIDUAL>(ta, tb[0], tb[1], tu[0], tu[1], p, s);
+      }
     case COSMOT_EPI_SILU_MUL: return launch<COSMOT_EPI_SILU_MUL>(ta, tb[0], tb[1], tu[0], tu[1], p, s);
     case COSMOT_EPI_MROPE: return launch<COSMOT_EPI_MROPE>(ta, tb[0], tb[1], tu[0], tu[1], p, s);
     default: return launch<COSMOT_EPI_EULER>(ta, tb[0], tb[1], tu[0], tu[1], p, s);

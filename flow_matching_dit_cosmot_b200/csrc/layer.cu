@@ -7,7 +7,7 @@
 //   1 routed RMSNorm            h -> a                      (g1 of each set)
 //   2 routed QKV GEMM + mRoPE    a -> qkv
 //   3 MoT attention              qkv -> o
-//   4 routed O GEMM + residual   o, h -> h1
+//   4 routed O GEMM + residual   o, h -> h1                 (h1 in float32)
 //   5 routed RMSNorm             h1 -> a                     (g2)
 //   6 routed gate/up + SiLU*mul  a -> u
 //   7 routed down + residual     u, h1 -> h_out
@@ -82,7 +82,7 @@ WsLayout ws_layout(const cosmot_dims& d, const cosmot_seq_desc& s) {
   w.qkv = off; off += align256(rows * qkv_cols * 2);
   w.a = off;   off += align256(rows * d.d_model * 2);
   w.o = off;   off += align256(rows * q_cols * 2);
-  w.h1 = off;  off += align256(rows * d.d_model * 2);
+  w.h1 = off;  off += align256(rows * d.d_model * 4);  // float32: the residual stream between the two halves
   w.u = off;   off += align256(rows * d.ffn * 2);
   w.total = off;
   return w;
@@ -190,16 +190,18 @@ cosmot_status layer_body(const cosmot_dims& D, const cosmot_layer_weights* w, co
                             static_cast<uint16_t*>(o) + c0 * qc, qc, stream);
   if (st != COSMOT_OK) return st;
   if ((st = M.mark(3)) != COSMOT_OK) return st;
-  // 4. output projection + residual
+  // 4. output projection + residual; h1 stays in float32 (it is read twice more:
+  // by the pre-FFN norm and as the residual of the down projection)
   e = cosmot_epilogue{};
   e.kind = COSMOT_EPI_RESIDUAL;
+  e.flags = COSMOT_EPI_OUT_F32;
   e.res = x_in;
   e.ld_res = d;
   st = cosmot_routed_linear(o, qc, qc, segs, ns, R.wo, G.wo, nullptr, nullptr, d, h1, d, &e, stream);
   if (st != COSMOT_OK) return st;
   if ((st = M.mark(4)) != COSMOT_OK) return st;
   // 5. pre-FFN norm
-  st = cosmot_rmsnorm_routed(h1, d, segs, ns, R.g2, G.g2, d, D.eps, a, d, stream);
+  st = rmsnorm_routed(h1, true, d, segs, ns, R.g2, G.g2, d, D.eps, a, d, stream);
   if (st != COSMOT_OK) return st;
   if ((st = M.mark(5)) != COSMOT_OK) return st;
   // 6. gate/up with SiLU * mul
@@ -211,6 +213,7 @@ cosmot_status layer_body(const cosmot_dims& D, const cosmot_layer_weights* w, co
   // 7. down projection + residual
   e = cosmot_epilogue{};
   e.kind = COSMOT_EPI_RESIDUAL;
+  e.flags = COSMOT_EPI_RES_F32;
   e.res = h1;
   e.ld_res = d;
   st = cosmot_routed_linear(u, F, F, segs, ns, R.wd, G.wd, nullptr, nullptr, d, x_out, d, &e, stream);
@@ -220,10 +223,12 @@ cosmot_status layer_body(const cosmot_dims& D, const cosmot_layer_weights* w, co
 
 // Steps 8-9: final norm of the first nz noisy rows of h_last, velocity head,
 // Euler step (or the guided step) into the same rows of `state`.
+// io (or null): the float32 state and velocity output of the noisy rows, packed
+// [batch][nz] (unguided steps only).
 cosmot_status layer_head(const cosmot_dims& D, const cosmot_layer_weights* w, const cosmot_seq_desc& S,
                          const WsLayout& L, uint8_t* ws, const void* h_last, void* state, double sigma,
                          double sigma_next, cosmot_stream_t stream, const StageMarks& M, const double* guidance,
-                         int64_t nz) {
+                         int64_t nz, const cosmot_step_io* io = nullptr) {
   cosmot_status st;
   const int64_t N = (int64_t)S.n_ar + S.n_clean + S.n_noisy;
   const int64_t d = D.d_model;
@@ -270,19 +275,37 @@ cosmot_status layer_head(const cosmot_dims& D, const cosmot_layer_weights* w, co
   e.x = state;
   e.ld_x = d;
   e.dsigma = (float)(sigma_next - sigma);
+  if (io) {  // the velocity GEMM's input rows are the packed noisy rows b * nz + i
+    e.x_state = io->x_state;
+    e.ld_state = io->ld_state;
+    e.state_from_x = io->state_from_h;
+    e.vel = io->vel;
+    e.ld_vel = io->ld_vel;
+  }
   st = cosmot_routed_linear(a, d, d, vs, B, w->wvel, w->wvel, nullptr, nullptr, d, hb, d, &e, stream);
   if (st != COSMOT_OK) return st;
   return M.mark(9);
 }
 
+cosmot_status check_io(const cosmot_step_io* io, const cosmot_dims& D, const double* guidance) {
+  if (!io) return COSMOT_OK;
+  if (guidance) return COSMOT_ERR_UNSUPPORTED;
+  if (io->x_state && (!aligned16(io->x_state) || io->ld_state < D.d_model || io->ld_state % 8))
+    return COSMOT_ERR_INVALID_ARG;
+  if (io->vel && (!aligned16(io->vel) || io->ld_vel < D.d_model || io->ld_vel % 8)) return COSMOT_ERR_INVALID_ARG;
+  return COSMOT_OK;
+}
+
 cosmot_status layer_forward_impl(const cosmot_dims* dims, const cosmot_layer_weights* w, const cosmot_seq_desc* seq,
                                  void* h, void* h_out, double sigma, double sigma_next, void* workspace,
                                  size_t workspace_bytes, cosmot_stream_t stream, const cudaEvent_t* events,
-                                 const double* guidance = nullptr) {
+                                 const double* guidance = nullptr, const cosmot_step_io* io = nullptr) {
   const StageMarks M{events, reinterpret_cast<cudaStream_t>(stream)};
   cosmot_status st = check_dims(dims);
   if (st != COSMOT_OK) return st;
   st = check_seq(seq);
+  if (st != COSMOT_OK) return st;
+  st = check_io(io, *dims, guidance);
   if (st != COSMOT_OK) return st;
   if (!w || !h || !h_out || !workspace) return COSMOT_ERR_INVALID_ARG;
   if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return COSMOT_ERR_INVALID_ARG;
@@ -291,7 +314,7 @@ cosmot_status layer_forward_impl(const cosmot_dims* dims, const cosmot_layer_wei
   uint8_t* ws = static_cast<uint8_t*>(workspace);
   st = layer_body(*dims, w, *seq, L, ws, h, h_out, nullptr, stream, M);
   if (st != COSMOT_OK) return st;
-  return layer_head(*dims, w, *seq, L, ws, h_out, h, sigma, sigma_next, stream, M, guidance, seq->n_noisy);
+  return layer_head(*dims, w, *seq, L, ws, h_out, h, sigma, sigma_next, stream, M, guidance, seq->n_noisy, io);
 }
 
 // Stack workspace: one layer's working set, a second hidden-state buffer for
@@ -362,9 +385,11 @@ cosmot_status stack_bodies(const cosmot_dims* dims, const cosmot_layer_weights* 
 cosmot_status stack_forward_impl(const cosmot_dims* dims, const cosmot_layer_weights* layers, int32_t n_layers,
                                  const cosmot_seq_desc* seq, void* h, void* h_out, double sigma, double sigma_next,
                                  void* workspace, size_t workspace_bytes, cosmot_stream_t stream,
-                                 const cudaEvent_t* events) {
+                                 const cudaEvent_t* events, const cosmot_step_io* io = nullptr) {
   StackWs W;
   cosmot_status st = stack_check(dims, layers, n_layers, seq, h, h_out, workspace, workspace_bytes, &W);
+  if (st != COSMOT_OK) return st;
+  st = check_io(io, *dims, nullptr);
   if (st != COSMOT_OK) return st;
   uint8_t* ws = static_cast<uint8_t*>(workspace);
   st = stack_bodies(dims, layers, n_layers, seq, W, ws, h, h_out, stream, events);
@@ -372,7 +397,7 @@ cosmot_status stack_forward_impl(const cosmot_dims* dims, const cosmot_layer_wei
   // the head's marks 8 and 9 land at events[8 n_layers] and [8 n_layers + 1]
   const StageMarks MH{events ? events + 8 * (n_layers - 1) : nullptr, reinterpret_cast<cudaStream_t>(stream)};
   return layer_head(*dims, &layers[n_layers - 1], *seq, W.layer, ws, h_out, h, sigma, sigma_next, stream, MH,
-                    nullptr, seq->n_noisy);
+                    nullptr, seq->n_noisy, io);
 }
 
 // ---------------------------------------------------------------- row shards
@@ -451,11 +476,12 @@ cosmot_status shard_post(const cosmot_dims* dims, const cosmot_layer_weights* w,
   const cosmot_set_weights& G = w->set[1];
   cosmot_epilogue e{};
   e.kind = COSMOT_EPI_RESIDUAL;
+  e.flags = COSMOT_EPI_OUT_F32;  // h1 in float32, as in layer_body
   e.res = h_local;
   e.ld_res = d;
   st = cosmot_routed_linear(o_local, qc, qc, segs, ns, R.wo, G.wo, nullptr, nullptr, d, ws + L.h1, d, &e, stream);
   if (st != COSMOT_OK) return st;
-  st = cosmot_rmsnorm_routed(ws + L.h1, d, segs, ns, R.g2, G.g2, d, D.eps, ws + L.a, d, stream);
+  st = rmsnorm_routed(ws + L.h1, true, d, segs, ns, R.g2, G.g2, d, D.eps, ws + L.a, d, stream);
   if (st != COSMOT_OK) return st;
   e = cosmot_epilogue{};
   e.kind = COSMOT_EPI_SILU_MUL;
@@ -463,6 +489,7 @@ cosmot_status shard_post(const cosmot_dims* dims, const cosmot_layer_weights* w,
   if (st != COSMOT_OK) return st;
   e = cosmot_epilogue{};
   e.kind = COSMOT_EPI_RESIDUAL;
+  e.flags = COSMOT_EPI_RES_F32;
   e.res = ws + L.h1;
   e.ld_res = d;
   st = cosmot_routed_linear(ws + L.u, F, F, segs, ns, R.wd, G.wd, nullptr, nullptr, d, h_out_local, d, &e, stream);
@@ -550,6 +577,14 @@ cosmot_status cosmot_layer_forward(const cosmot_dims* dims, const cosmot_layer_w
                                     nullptr);
 }
 
+cosmot_status cosmot_layer_forward_io(const cosmot_dims* dims, const cosmot_layer_weights* w,
+                                      const cosmot_seq_desc* seq, void* h, void* h_out, double sigma,
+                                      double sigma_next, const cosmot_step_io* io, void* workspace,
+                                      size_t workspace_bytes, cosmot_stream_t stream) {
+  return cosmot::layer_forward_impl(dims, w, seq, h, h_out, sigma, sigma_next, workspace, workspace_bytes, stream,
+                                    nullptr, nullptr, io);
+}
+
 cosmot_status cosmot_layer_forward_cfg(const cosmot_dims* dims, const cosmot_layer_weights* w,
                                        const cosmot_seq_desc* seq, void* h, void* h_out, double sigma,
                                        double sigma_next, double guidance, void* workspace, size_t workspace_bytes,
@@ -619,6 +654,14 @@ cosmot_status cosmot_stack_forward(const cosmot_dims* dims, const cosmot_layer_w
                                     workspace_bytes, stream, nullptr);
 }
 
+cosmot_status cosmot_stack_forward_io(const cosmot_dims* dims, const cosmot_layer_weights* layers, int32_t n_layers,
+                                      const cosmot_seq_desc* seq, void* h, void* h_out, double sigma,
+                                      double sigma_next, const cosmot_step_io* io, void* workspace,
+                                      size_t workspace_bytes, cosmot_stream_t stream) {
+  return cosmot::stack_forward_impl(dims, layers, n_layers, seq, h, h_out, sigma, sigma_next, workspace,
+                                    workspace_bytes, stream, nullptr, io);
+}
+
 cosmot_status cosmot_policy_step(const cosmot_dims* dims, const cosmot_layer_weights* layers, int32_t n_layers,
                                  const cosmot_seq_desc* seq, const cosmot_action_desc* act, void* h, void* h_out,
                                  double sigma, double sigma_next, const double* guidance, void* workspace,
@@ -673,20 +716,21 @@ cosmot_status cosmot_copy_columns(const void* src, int64_t ld_src, void* dst, in
 cosmot_status cosmot_stack_forward_timed(const cosmot_dims* dims, const cosmot_layer_weights* layers,
                                          int32_t n_layers, const cosmot_seq_desc* seq, void* h, void* h_out,
                                          double sigma, double sigma_next, void* workspace, size_t workspace_bytes,
-                                         cosmot_stream_t stream, void* const* stage_events, int32_t n_events) {
+                                         cosmot_stream_t stream, void* const* stage_events, int32_t n_events,
+                                         const cosmot_step_io* io) {
   if (!stage_events || n_layers < 1 || n_layers > cosmot::kMaxLayers || n_events != 8 * n_layers + 2)
     return COSMOT_ERR_INVALID_ARG;
   for (int i = 0; i < n_events; ++i)
     if (!stage_events[i]) return COSMOT_ERR_INVALID_ARG;
   return cosmot::stack_forward_impl(dims, layers, n_layers, seq, h, h_out, sigma, sigma_next, workspace,
-                                    workspace_bytes, stream, reinterpret_cast<const cudaEvent_t*>(stage_events));
+                                    workspace_bytes, stream, reinterpret_cast<const cudaEvent_t*>(stage_events), io);
 }
 
 cosmot_status cosmot_layer_forward_timed(const cosmot_dims* dims, const cosmot_layer_weights* w,
                                          const cosmot_seq_desc* seq, void* h, void* h_out, double sigma,
                                          double sigma_next, void* workspace, size_t workspace_bytes,
                                          cosmot_stream_t stream, void* const* stage_events, int32_t n_events,
-                                         const double* guidance) {
+                                         const double* guidance, const cosmot_step_io* io) {
   if (!stage_events || n_events != COSMOT_LAYER_STAGES + 1) return COSMOT_ERR_INVALID_ARG;
   for (int i = 0; i < n_events; ++i)
     if (!stage_events[i]) return COSMOT_ERR_INVALID_ARG;
@@ -696,7 +740,7 @@ cosmot_status cosmot_layer_forward_timed(const cosmot_dims* dims, const cosmot_l
       return COSMOT_ERR_UNSUPPORTED;
   }
   return cosmot::layer_forward_impl(dims, w, seq, h, h_out, sigma, sigma_next, workspace, workspace_bytes, stream,
-                                    reinterpret_cast<const cudaEvent_t*>(stage_events), guidance);
+                                    reinterpret_cast<const cudaEvent_t*>(stage_events), guidance, io);
 }
 
 }  // extern "C"

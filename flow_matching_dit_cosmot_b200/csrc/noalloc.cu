@@ -9,10 +9,17 @@
 // workspace from a fixed array compiled into the library instead.
 //
 // The array is a file-scope __device__ variable: every GPU that loads this
-// library holds kNoAllocScratchBytes for it until the process exits.  In host
-// code its name only stands in for the symbol and is not a device address, so
-// the address is looked up with cudaGetSymbolAddress, once per device, with
-// that device current, the first time the entry point runs on it.
+// library's device code holds kNoAllocScratchBytes for it until the process
+// exits.  The CUDA driver reserves it when it loads this file's module on a
+// device.  Under the default lazy module loading that happens at the first
+// cudaGetSymbolAddress below, i.e. inside the first call on each device (with
+// CUDA_MODULE_LOADING=EAGER, at context creation instead), so a caller with a
+// deadline makes one warm-up call before its loop.  In host code the array's
+// name only stands in for the symbol and is not a device address, so the
+// address is looked up with cudaGetSymbolAddress, once per device, with that
+// device current, the first time the entry point runs on it.  The cached
+// address belongs to the device's current primary context: after a
+// cudaDeviceReset the entry point must not be called again in that process.
 #include <mutex>
 
 #include "cosmot_internal.h"
@@ -22,7 +29,7 @@ namespace {
 
 // COSMOT_NOALLOC_SCRATCH_BYTES (64 MiB): enough for one full-width (d_model
 // 4096, FFN 14336) DROID policy step (703 tokens, batch 1), which needs about
-// 55 MB of workspace.
+// 61 MB of workspace.
 constexpr size_t kNoAllocScratchBytes = COSMOT_NOALLOC_SCRATCH_BYTES;
 
 static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];

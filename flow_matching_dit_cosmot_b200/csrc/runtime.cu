@@ -113,7 +113,7 @@ const char* cosmot_status_string(cosmot_status s) {
   }
 }
 
-int32_t cosmot_version(void) { return 100; }
+int32_t cosmot_version(void) { return 200; }
 
 cosmot_status cosmot_get_device_status(cosmot_stream_t stream, cosmot_status* out, int32_t* where_out) {
   if (!out) return COSMOT_ERR_INVALID_ARG;

@@ -166,8 +166,13 @@ enum {
   COSMOT_EPI_RESIDUAL = 1,  /* out = bf16(acc + res); res may alias out */
   COSMOT_EPI_SILU_MUL = 2,  /* out[:, j] = bf16(silu(a.Wg_j) * (a.Wu_j)); W = gate, W_up = up */
   COSMOT_EPI_MROPE = 3,     /* QKV projection: heads in columns [0, rope_cols) rotated by mRoPE */
-  COSMOT_EPI_EULER = 4      /* out = bf16(x + dsigma * acc); x may alias out */
+  COSMOT_EPI_EULER = 4      /* out = bf16(x + dsigma * acc); x may alias out; see x_state below */
 };
+
+/* cosmot_epilogue.flags (RESIDUAL only): float32 instead of bf16 for the
+ * output and/or the residual, so that a residual stream can stay in float32. */
+#define COSMOT_EPI_OUT_F32 1
+#define COSMOT_EPI_RES_F32 2
 
 typedef struct {
   int32_t kind;
@@ -181,6 +186,16 @@ typedef struct {
   int64_t ld_x;
   float dsigma;            /* EULER: sigma_next - sigma */
   float reserved;
+  /* EULER, optional float32 sampler state: x_state [rows, ld_state] float32,
+   * indexed by INPUT row.  When non-NULL, x is read from x_state (or from `x`
+   * when state_from_x = 1), x' = x + dsigma * acc is written back to x_state
+   * in float32, and bf16(x') still goes to `out`. */
+  float* x_state;
+  int64_t ld_state;
+  void* vel;               /* EULER, optional: [rows, ld_vel] bf16, indexed by input row, receives bf16(acc) */
+  int64_t ld_vel;
+  int32_t state_from_x;
+  int32_t flags;           /* COSMOT_EPI_OUT_F32 | COSMOT_EPI_RES_F32 (RESIDUAL only), else 0 */
 } cosmot_epilogue;
 
 /*
@@ -195,6 +210,8 @@ typedef struct {
  *   out    device bf16 [*, n_out], ld_out
  * Requires k % 8 == 0, n_out % 8 == 0, ld_a/ld_out % 8 == 0; MROPE needs
  * head_dim in {64, 128} and rope_cols a multiple of head_dim; 1 <= n_segs <= 64.
+ * With COSMOT_EPI_OUT_F32 (RESIDUAL) `out` is float32 [*, ld_out]; with
+ * COSMOT_EPI_RES_F32 `res` is float32 [*, ld_res]; both 16-byte aligned.
  */
 COSMOT_API cosmot_status cosmot_routed_linear(const void* a, int64_t ld_a, int64_t k, const cosmot_segment* segs,
                                    int32_t n_segs, const void* w0, const void* w1, const void* w0_up,
@@ -360,6 +377,42 @@ COSMOT_API cosmot_status cosmot_layer_forward(const cosmot_dims* dims, const cos
                                    cosmot_stream_t stream);
 
 /*
+ * Sampler state and diagnostic outputs of one step (cosmot_layer_forward_io).
+ * "Cosmos 3 方法原理全解" §7.2: the sampler integrates x_next = x + (sigma_next -
+ * sigma) v over all steps; the layer reads x as its bf16 DM input rows, but the
+ * running state need not be rounded to bf16 after every step.
+ *   x_state       NULL, or device float32 [batch][n_noisy][ld_state]: the state
+ *                 of the noisy rows, kept in float32 between steps.  The Euler
+ *                 step reads x from here (from the bf16 noisy rows of h instead
+ *                 when state_from_h = 1, as the first step of a sampling does),
+ *                 writes x' here in float32, and writes bf16(x') into the noisy
+ *                 rows of h, which the next step's layer reads as its input.
+ *   vel           NULL, or device bf16 [batch][n_noisy][ld_vel]: receives the
+ *                 velocity v = RMSNorm(h2; gfin) Wvel^T of the noisy rows (the
+ *                 step itself uses v's fp32 accumulator, not this copy).
+ *   ld_state, ld_vel: row pitches in elements, >= d_model, multiples of 8
+ *                 (x_state and vel 16-byte aligned).
+ */
+typedef struct {
+  float* x_state;
+  int64_t ld_state;
+  void* vel;
+  int64_t ld_vel;
+  int32_t state_from_h;
+  int32_t reserved;
+} cosmot_step_io;
+
+/*
+ * cosmot_layer_forward with the optional state and outputs of `io` (NULL = the
+ * plain cosmot_layer_forward).  Unguided steps only; everything else, including
+ * n_cached, as cosmot_layer_forward.
+ */
+COSMOT_API cosmot_status cosmot_layer_forward_io(const cosmot_dims* dims, const cosmot_layer_weights* w,
+                                                 const cosmot_seq_desc* seq, void* h, void* h_out, double sigma,
+                                                 double sigma_next, const cosmot_step_io* io, void* workspace,
+                                                 size_t workspace_bytes, cosmot_stream_t stream);
+
+/*
  * One guided sampler step ("Cosmos 3 方法原理全解" §7.2-7.3): seq->batch holds
  * (conditioned, baseline) pairs, sequences 2p and 2p+1, with equal layouts and
  * equal DM rows (the state x) but different AR rows (the prompt and the
@@ -376,6 +429,9 @@ COSMOT_API cosmot_status cosmot_layer_forward_cfg(const cosmot_dims* dims, const
                                                   size_t workspace_bytes, cosmot_stream_t stream);
 
 /*
+ * Streaming key/value cache update ("NVIDIA 发布 Cosmos 3 系列四个开放权重世界模型",
+ * "流式生成如何工作": each finished block's keys and values stay in the cache for
+ * the blocks that follow; "Cosmos 3 方法原理全解" §3 for the projection).
  * Commit K/V into the workspace's cache: rows [seq.n_cached, N) of every sequence
  * of h go through the pre-attention RMSNorm and the QKV projection with mRoPE
  * (positions of those rows from seq.rope_cs), and the resulting QKV rows are
@@ -418,6 +474,12 @@ COSMOT_API cosmot_status cosmot_stack_forward(const cosmot_dims* dims, const cos
                                               int32_t n_layers, const cosmot_seq_desc* seq, void* h, void* h_out,
                                               double sigma, double sigma_next, void* workspace,
                                               size_t workspace_bytes, cosmot_stream_t stream);
+/* cosmot_stack_forward with the optional float32 state and velocity output of
+ * cosmot_step_io (see cosmot_layer_forward_io); io = NULL is the plain call. */
+COSMOT_API cosmot_status cosmot_stack_forward_io(const cosmot_dims* dims, const cosmot_layer_weights* layers,
+                                                 int32_t n_layers, const cosmot_seq_desc* seq, void* h, void* h_out,
+                                                 double sigma, double sigma_next, const cosmot_step_io* io,
+                                                 void* workspace, size_t workspace_bytes, cosmot_stream_t stream);
 
 /*
  * Sampler noise levels with the flow shift ("Cosmos 3 方法原理全解" §6.3:
@@ -538,13 +600,15 @@ COSMOT_API cosmot_status cosmot_copy_columns(const void* src, int64_t ld_src, vo
  * i (COSMOT_STAGE_NORM1 .. COSMOT_STAGE_DOWN_RESIDUAL) and events[8l + 7]
  * after its last one (where the final-norm stage starts); events[8 n_layers]
  * is recorded before the velocity stage and events[8 n_layers + 1] after it.
- * The computation is identical to cosmot_stack_forward.
+ * The computation is identical to cosmot_stack_forward_io with `io` (NULL:
+ * cosmot_stack_forward).
  */
 COSMOT_API cosmot_status cosmot_stack_forward_timed(const cosmot_dims* dims, const cosmot_layer_weights* layers,
                                                     int32_t n_layers, const cosmot_seq_desc* seq, void* h,
                                                     void* h_out, double sigma, double sigma_next, void* workspace,
                                                     size_t workspace_bytes, cosmot_stream_t stream,
-                                                    void* const* stage_events, int32_t n_events);
+                                                    void* const* stage_events, int32_t n_events,
+                                                    const cosmot_step_io* io);
 
 /*
  * cosmot_layer_forward without a caller workspace, for callers that may not
@@ -554,8 +618,14 @@ COSMOT_API cosmot_status cosmot_stack_forward_timed(const cosmot_dims* dims, con
  * have no counterpart; this is a deployment convenience of this library.
  *
  * The workspace is a fixed array of COSMOT_NOALLOC_SCRATCH_BYTES compiled into
- * the library; every GPU that loads the library keeps it until the process
- * exits.  Inputs, outputs and semantics are those of cosmot_layer_forward.
+ * the library; every GPU that loads the library's device code keeps it until
+ * the process exits.  Inputs, outputs and semantics are those of
+ * cosmot_layer_forward.
+ *   - The CUDA driver reserves the array when it loads the module that holds
+ *     it.  With the default lazy module loading that is inside the first call
+ *     on each device (with CUDA_MODULE_LOADING=EAGER, at context creation), so
+ *     make one warm-up call on every device before the deadline loop; later
+ *     calls reserve nothing.
  *   - Sizes whose cosmot_layer_workspace_size exceeds the limit return
  *     COSMOT_ERR_WORKSPACE before any launch (64 MiB covers a full-width DROID
  *     policy step, 703 tokens at d_model 4096, batch 1).
@@ -568,8 +638,11 @@ COSMOT_API cosmot_status cosmot_stack_forward_timed(const cosmot_dims* dims, con
  *     on one stream.
  *   - The first call on each device looks up the array's device address
  *     (cudaGetSymbolAddress, with that device current); make that first call
- *     before any stream capture.
- * No device memory is allocated or freed on any path.
+ *     before any stream capture.  The address is kept for the life of the
+ *     process: after cudaDeviceReset on a device, do not call this entry point
+ *     on that device again.
+ * The library itself calls no allocator on any path (no cudaMalloc or
+ * cudaFree); the only reservation is the driver's, at module load, above.
  */
 #define COSMOT_NOALLOC_SCRATCH_BYTES ((size_t)64 << 20)
 COSMOT_API cosmot_status cosmot_layer_forward_noalloc(const cosmot_dims* dims, const cosmot_layer_weights* w,
@@ -596,15 +669,17 @@ enum {
  * after the last one, so cudaEventElapsedTime between consecutive events is the
  * device time of one stage.  The events are cudaEvent_t handles created by the
  * caller on the current device; n_events must be COSMOT_LAYER_STAGES + 1.  With
- * guidance == NULL the computation is identical to cosmot_layer_forward; with
- * a guidance weight it is that of cosmot_layer_forward_cfg (the last stage then
- * covers the velocity GEMM and the guided Euler step).
+ * guidance == NULL the computation is identical to cosmot_layer_forward_io with
+ * `io` (which may be NULL); with a guidance weight it is that of
+ * cosmot_layer_forward_cfg (the last stage then covers the velocity GEMM and the
+ * guided Euler step), and io must be NULL.
  */
 COSMOT_API cosmot_status cosmot_layer_forward_timed(const cosmot_dims* dims, const cosmot_layer_weights* w,
                                                     const cosmot_seq_desc* seq, void* h, void* h_out, double sigma,
                                                     double sigma_next, void* workspace, size_t workspace_bytes,
                                                     cosmot_stream_t stream, void* const* stage_events,
-                                                    int32_t n_events, const double* guidance);
+                                                    int32_t n_events, const double* guidance,
+                                                    const cosmot_step_io* io);
 
 #ifdef __cplusplus
 }

@@ -161,8 +161,9 @@ def layer_forward(dims, W: LayerWeights, h, region, pos, chunk, sigma, sigma_nex
     (already rotated) that sit between the AR keys and this sequence's DM keys
     in key order, as a streaming key/value cache does.
 
-    Returns a dict with h2 [len(rows), d], x_new [len(rows), d] (NaN on AR
-    rows), vel [len(rows), d] (NaN except on noisy rows) and the row indices.
+    Returns a dict with h2 [len(rows), d], the attention half h1 [len(rows), d],
+    x_new [len(rows), d] (NaN on AR rows), vel [len(rows), d] (NaN except on
+    noisy rows) and the row indices.
     With head=False the velocity head and the Euler step are left out (x_new
     and vel all NaN): a layer inside a stack.
     """
@@ -219,7 +220,7 @@ def layer_forward(dims, W: LayerWeights, h, region, pos, chunk, sigma, sigma_nex
     x_new = np.full_like(h2, np.nan)
     vel = np.full_like(h2, np.nan)
     if not head:
-        return {"rows": rows, "h2": h2, "x_new": x_new, "vel": vel}
+        return {"rows": rows, "h1": h1, "h2": h2, "x_new": x_new, "vel": vel}
     reg_r = region[rows]
     clean = reg_r == REGION_CLEAN
     noisy = reg_r == REGION_NOISY
@@ -227,7 +228,7 @@ def layer_forward(dims, W: LayerWeights, h, region, pos, chunk, sigma, sigma_nex
     if noisy.any():
         vel[noisy] = rms_norm(h2[noisy], W.gfin, dims.eps) @ W.wvel.T
         x_new[noisy] = euler_step(hr[noisy], vel[noisy], sigma, sigma_next)
-    return {"rows": rows, "h2": h2, "x_new": x_new, "vel": vel}
+    return {"rows": rows, "h1": h1, "h2": h2, "x_new": x_new, "vel": vel}
 
 
 def euler_step(x, v, sigma, sigma_next):

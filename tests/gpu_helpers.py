@@ -52,3 +52,24 @@ def sample_rows(n: int, seg_bounds, k: int, seed: int = 0) -> np.ndarray:
         if e > b:
             rows.update([b, e - 1])
     return np.array(sorted(rows), dtype=np.int64)
+
+
+def layer_parity(what, ref, noisy, dsigma, h_out=None, x_new=None, vel=None, x_f32=False, depth=1):
+    """The parity checks of one layer call against the oracle's outputs `ref`
+    (layer_forward's dict, rows already selected to match the arrays given):
+    h_out against h2 (its rounding term propagates through the FFN branch
+    h2 - h1), and on the `noisy` rows the velocity against v and the state
+    against x' = x + dsigma v.  `x_new` and `vel` hold the noisy rows only;
+    `x_f32`: the state is the float32 sampler state (no bf16 half-ulp)."""
+    from tolerance import SIGMA_H_OUT, SIGMA_VEL, assert_close, rms
+    if h_out is not None:
+        assert_close(h_out, ref["h2"], f"{what} h_out", sigma=SIGMA_H_OUT, branch_rms=rms(ref["h2"] - ref["h1"]),
+                     depth=depth)
+    if not np.asarray(noisy).any():
+        return
+    v = ref["vel"][noisy]
+    if vel is not None:
+        assert_close(vel, v, f"{what} velocity", sigma=SIGMA_VEL, branch_rms=rms(v), depth=depth)
+    if x_new is not None:
+        assert_close(x_new, ref["x_new"][noisy], f"{what} x'", sigma=SIGMA_VEL, branch_rms=abs(dsigma) * rms(v),
+                     depth=depth, out_bf16=not x_f32)

@@ -102,7 +102,7 @@ def test_layer_workspace_and_validation():
     seq = A.L.SeqDesc(258, 0, 18720, 1, 0, 0, 16, 0)
     n = A.L.cosmot_layer_workspace_size(dims, seq)
     rows = 18978
-    want = rows * (4096 + 12288 + 4096 + 4096 + 14336) * 2
+    want = rows * (4096 + 12288 + 4096 + 2 * 4096 + 14336) * 2  # h1 is float32
     assert want <= n <= want + 5 * 256
     # the layer rejects a short workspace and bad dims without launching
     lib = A.L.lib()
@@ -252,7 +252,7 @@ def test_ctypes_structs_and_constants_match_the_header(tmp_path):
     structs = {"cosmot_layout_spec": L.LayoutSpec, "cosmot_segment": L.Segment, "cosmot_epilogue": L.Epilogue,
                "cosmot_attn_desc": L.AttnDesc, "cosmot_dims": L.Dims, "cosmot_set_weights": L.SetWeights,
                "cosmot_layer_weights": L.LayerWeights, "cosmot_seq_desc": L.SeqDesc,
-               "cosmot_action_desc": L.ActionDesc}
+               "cosmot_action_desc": L.ActionDesc, "cosmot_step_io": L.StepIO}
     consts = [n for n in dir(L) if re.fullmatch(r"COSMOT_[A-Z_]+", n)]
     lines = ["#include <stdio.h>", "#include <stddef.h>", '#include "cosmot.h"', "int main(void) {"]
     for cname, cls in structs.items():

@@ -21,7 +21,7 @@ if not torch.cuda.is_available():  # pragma: no cover
 
 from flow_matching_dit_cosmot_b200 import api as A  # noqa: E402
 from flow_matching_dit_cosmot_b200 import _lib as L  # noqa: E402
-from gpu_helpers import assert_device_ok, bits, device_weights, dims as cdims, layout_spec, to_dev, to_f64  # noqa
+from gpu_helpers import assert_device_ok, bits, device_weights, dims as cdims, layer_parity, layout_spec, to_dev, to_f64  # noqa
 
 DIMS = ModelDims(d_model=256, n_heads=4, n_kv_heads=2, head_dim=64, ffn=512, rope_sections=(8, 12, 12))
 
@@ -41,13 +41,9 @@ def _layer_case(spec, seed=4100):
     assert_device_ok()
     ref = olayer.layer_forward(DIMS, olayer.weights_from_bits(DIMS, w), synth.bf16_to_f64(h), lay.region, lay.pos,
                                lay.chunk, 0.8, 0.6)
-    assert_close(to_f64(h_out[0]), ref["h2"], "h_out", rounded_inputs=3)
     noisy = lay.region == olayout.REGION_NOISY
+    layer_parity("edge", ref, noisy, -0.2, h_out=to_f64(h_out[0]), x_new=to_f64(hd_[0])[noisy])
     np.testing.assert_array_equal(bits(hd_[0])[~noisy], h[~noisy])
-    if noisy.any():
-        vel = ref["vel"][noisy]
-        assert_close(to_f64(hd_[0])[noisy], ref["x_new"][noisy], "x'", rounded_inputs=2,
-                     branch_rms=0.2 * float(np.sqrt(np.mean(vel ** 2))))
     return lay
 
 

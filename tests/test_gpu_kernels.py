@@ -13,7 +13,7 @@ from oracle import layer as olayer
 from oracle import layout as olayout
 from oracle import mask as omask
 from oracle import rope as orope
-from tolerance import assert_close
+from tolerance import SIGMA_ATTN, assert_close, rms
 
 pytestmark = pytest.mark.gpu
 
@@ -163,6 +163,48 @@ def test_routed_linear_residual():
     assert_close(to_f64(out), acc + synth.bf16_to_f64(res), "gemm+residual")
 
 
+@pytest.mark.parametrize("flags", ["out_f32", "res_f32", "both"])
+def test_routed_linear_residual_float32(flags):
+    """The residual epilogue with a float32 output (the layer's h1) and/or a
+    float32 residual (h1 read back by the down projection): fp32 values are
+    stored and read without rounding."""
+    m_split, m_total, k, n_out = 77, 400, 512, 264
+    a, w0, w1, segs, acc = _gemm_case(m_split, m_total, k, n_out, seed=2)
+    fl = {"out_f32": L.COSMOT_EPI_OUT_F32, "res_f32": L.COSMOT_EPI_RES_F32,
+          "both": L.COSMOT_EPI_OUT_F32 | L.COSMOT_EPI_RES_F32}[flags]
+    rng = np.random.default_rng(21)
+    res32 = rng.standard_normal((m_total, n_out)).astype(np.float32)  # values a bf16 cannot hold
+    res16 = _bf16((m_total, n_out), 22)
+    use_f32_res = bool(fl & L.COSMOT_EPI_RES_F32)
+    rd = torch.from_numpy(res32).cuda() if use_f32_res else to_dev(res16)
+    out = torch.empty((m_total, n_out), dtype=torch.float32 if fl & L.COSMOT_EPI_OUT_F32 else torch.bfloat16,
+                      device="cuda")
+    ad, w0d, w1d = to_dev(a), to_dev(w0), to_dev(w1)
+    e = L.Epilogue(kind=L.COSMOT_EPI_RESIDUAL, res=A.ptr(rd), ld_res=n_out, flags=fl)
+    L.cosmot_routed_linear(A.ptr(ad), k, k, segs, A.ptr(w0d), A.ptr(w1d), n_out, A.ptr(out), n_out, e,
+                           stream=A.stream_handle())
+    torch.cuda.synchronize()
+    assert_device_ok()
+    ref = acc + (res32.astype(np.float64) if use_f32_res else synth.bf16_to_f64(res16))
+    got = out.double().cpu().numpy()
+    if fl & L.COSMOT_EPI_OUT_F32:  # fp32 accumulation and one fp32 add: far inside the bf16 bounds
+        assert np.abs(got - ref).max() < 1e-4, np.abs(got - ref).max()
+    else:
+        assert_close(got, ref, "gemm+float32 residual")
+
+
+def test_routed_linear_rejects_float32_flags_off_the_residual_epilogue():
+    a = torch.zeros((16, 64), dtype=torch.bfloat16, device="cuda")
+    e = L.Epilogue(kind=L.COSMOT_EPI_NONE, flags=L.COSMOT_EPI_OUT_F32)
+    code = L.cosmot_routed_linear(A.ptr(a), 64, 64, [(0, 16, 0, 0)], A.ptr(a), A.ptr(a), 16, A.ptr(a), 64, e,
+                                  stream=A.stream_handle(), check=False)
+    assert code == L.COSMOT_ERR_INVALID_ARG
+    e = L.Epilogue(kind=L.COSMOT_EPI_RESIDUAL, res=A.ptr(a), ld_res=64, flags=4)
+    code = L.cosmot_routed_linear(A.ptr(a), 64, 64, [(0, 16, 0, 0)], A.ptr(a), A.ptr(a), 16, A.ptr(a), 64, e,
+                                  stream=A.stream_handle(), check=False)
+    assert code == L.COSMOT_ERR_INVALID_ARG
+
+
 def test_routed_linear_silu_mul():
     m_split, m_total, k, f = 150, 450, 256, 384
     a = _bf16((m_total, k), 30)
@@ -228,6 +270,37 @@ def test_routed_linear_euler_in_place():
     v = synth.bf16_to_f64(a) @ synth.bf16_to_f64(w).T
     ref = olayer.euler_step(synth.bf16_to_f64(x)[150:450], v, 0.8, 0.7)
     assert_close(got[150:450], ref, "gemm+euler")
+    np.testing.assert_array_equal(bits(xd)[:150], x[:150])
+    np.testing.assert_array_equal(bits(xd)[450:], x[450:])
+
+
+def test_routed_linear_euler_float32_state_and_velocity():
+    """The Euler epilogue with a float32 state (indexed by input row) and the
+    velocity written out: the first call reads x from the bf16 rows
+    (state_from_x), the second from the float32 state it left; both write the
+    bf16 copy into the output rows."""
+    n_rows, k, c, xrows = 300, 256, 256, 500
+    a = _bf16((n_rows, k), 53)
+    w = _bf16((c, k), 54, std=0.06)
+    x = _bf16((xrows, c), 55)
+    xd, ad, wd = to_dev(x), to_dev(a), to_dev(w)
+    x32 = torch.full((n_rows, c), float("nan"), dtype=torch.float32, device="cuda")
+    vel = torch.full((n_rows, c), float("nan"), dtype=torch.bfloat16, device="cuda")
+    segs = [(0, n_rows, 150, 1)]
+    v = synth.bf16_to_f64(a) @ synth.bf16_to_f64(w).T
+    ref = synth.bf16_to_f64(x)[150:450]
+    for step, (s0, s1) in enumerate(((0.8, 0.7), (0.7, 0.55))):
+        e = L.Epilogue(kind=L.COSMOT_EPI_EULER, x=A.ptr(xd), ld_x=c, dsigma=float(np.float32(s1 - s0)),
+                       x_state=A.ptr(x32), ld_state=c, vel=A.ptr(vel), ld_vel=c, state_from_x=1 if step == 0 else 0)
+        L.cosmot_routed_linear(A.ptr(ad), k, k, segs, A.ptr(wd), A.ptr(wd), c, A.ptr(xd), c, e,
+                               stream=A.stream_handle())
+        torch.cuda.synchronize()
+        assert_device_ok()
+        ref = olayer.euler_step(ref, v, s0, s1)
+        got32 = x32.double().cpu().numpy()
+        assert np.abs(got32 - ref).max() < 1e-4, np.abs(got32 - ref).max()  # no bf16 rounding of the state
+        np.testing.assert_array_equal(bits(xd)[150:450], bits(x32.to(torch.bfloat16)))
+        assert_close(to_f64(vel), v, "velocity output")
     np.testing.assert_array_equal(bits(xd)[:150], x[:150])
     np.testing.assert_array_equal(bits(xd)[450:], x[450:])
 
@@ -331,14 +404,14 @@ def test_attention_of_constant_values_is_one():
 @pytest.mark.parametrize("hd", [128, 64])
 def test_attention_full_mask(hd):
     got, ref = _attn_case(n_keys=700, n_ar=130, n_q=700, q_off=0, H=4, Hkv=2, hd=hd, mode="full")
-    assert_close(got, ref, f"attention hd{hd}", rounded_inputs=1)
+    assert_close(got, ref, f"attention hd{hd}", sigma=SIGMA_ATTN, branch_rms=rms(ref))
 
 
 def test_attention_causal_ar_only_and_tiny():
     got, ref = _attn_case(n_keys=300, n_ar=300, n_q=300, q_off=0, H=2, Hkv=2, hd=128, mode="full", seed=1)
-    assert_close(got, ref, "causal", rounded_inputs=1)
+    assert_close(got, ref, "causal", sigma=SIGMA_ATTN, branch_rms=rms(ref))
     got, ref = _attn_case(n_keys=3, n_ar=2, n_q=3, q_off=0, H=1, Hkv=1, hd=128, mode="full", seed=2)
-    assert_close(got, ref, "tiny", rounded_inputs=1)
+    assert_close(got, ref, "tiny", sigma=SIGMA_ATTN, branch_rms=rms(ref))
 
 
 def test_attention_block_causal_and_batch():
@@ -346,7 +419,7 @@ def test_attention_block_causal_and_batch():
     ch = np.full(n_keys, -1, np.int32)
     ch[n_ar:] = (np.arange(n_keys - n_ar) // 89)  # chunks not aligned to 128-key tiles
     got, ref = _attn_case(n_keys, n_ar, n_keys, 0, H=4, Hkv=4, hd=128, mode="block_causal", chunk=ch, batch=2, seed=3)
-    assert_close(got, ref, "block causal", rounded_inputs=1)
+    assert_close(got, ref, "block causal", sigma=SIGMA_ATTN, branch_rms=rms(ref))
 
 
 def test_attention_block_causal_hd64_gqa():
@@ -356,7 +429,7 @@ def test_attention_block_causal_hd64_gqa():
     ch = np.full(n_keys, -1, np.int32)
     ch[n_ar:] = np.arange(n_keys - n_ar) // 200
     got, ref = _attn_case(n_keys, n_ar, n_keys, 0, H=4, Hkv=2, hd=64, mode="block_causal", chunk=ch, batch=2, seed=5)
-    assert_close(got, ref, "block causal hd64", rounded_inputs=1)
+    assert_close(got, ref, "block causal hd64", sigma=SIGMA_ATTN, branch_rms=rms(ref))
 
 
 def test_attention_query_suffix_streaming():
@@ -365,4 +438,4 @@ def test_attention_query_suffix_streaming():
     ch = np.full(n_keys, -1, np.int32)
     ch[n_ar:] = np.arange(n_keys - n_ar) // 250
     got, ref = _attn_case(n_keys, n_ar, 250, n_keys - 250, H=2, Hkv=1, hd=128, mode="block_causal", chunk=ch, seed=4)
-    assert_close(got, ref, "stream", rounded_inputs=1)
+    assert_close(got, ref, "stream", sigma=SIGMA_ATTN, branch_rms=rms(ref))

@@ -7,7 +7,6 @@ import synth
 from oracle import layer as olayer
 from oracle import layout as olayout
 from synth import LayoutSpec, ModelDims, VideoSpec
-from tolerance import assert_close
 
 pytestmark = pytest.mark.gpu
 
@@ -17,7 +16,7 @@ if not torch.cuda.is_available():  # pragma: no cover
 
 from flow_matching_dit_cosmot_b200 import api as A  # noqa: E402
 from flow_matching_dit_cosmot_b200 import _lib as L  # noqa: E402
-from gpu_helpers import assert_device_ok, bits, device_weights, dims as cdims, layout_spec, to_dev, to_f64  # noqa
+from gpu_helpers import assert_device_ok, bits, device_weights, dims as cdims, layer_parity, layout_spec, to_dev, to_f64  # noqa
 
 
 class LayerRun:
@@ -44,6 +43,19 @@ class LayerRun:
         assert_device_ok()
         return h, h_out
 
+    def gpu_io(self, sigma=0.8, sigma_next=0.7):
+        """cosmot_layer_forward_io: the float32 state (taken from h on this first
+        step) and the velocity of the noisy rows as extra outputs."""
+        h = to_dev(self.h)
+        h_out = torch.empty_like(h)
+        nz = self.lay.n_noisy
+        x32 = torch.full((self.batch, nz, self.dims.d_model), float("nan"), dtype=torch.float32, device="cuda")
+        vel = torch.full((self.batch, nz, self.dims.d_model), float("nan"), dtype=torch.bfloat16, device="cuda")
+        self.layer.forward(h, h_out, sigma, sigma_next, self.seq, x_state=x32, state_from_h=True, vel=vel)
+        torch.cuda.synchronize()
+        assert_device_ok()
+        return h, h_out, x32, vel
+
     def oracle(self, b=0, sigma=0.8, sigma_next=0.7, h_bits=None):
         W = olayer.weights_from_bits(self.dims, self.w)
         h = synth.bf16_to_f64((self.h if h_bits is None else h_bits)[b])
@@ -52,15 +64,23 @@ class LayerRun:
 
 
 def _check(run, h_dev, hout_dev, sigma=0.8, sigma_next=0.7):
+    """Plain entry point: h_out and the bf16 state in h against the oracle.
+    The io entry point on the same inputs: identical h_out and h bits, and its
+    float32 state and velocity against the oracle."""
     lay = run.lay
     noisy = lay.region == olayout.REGION_NOISY
+    h_io, hout_io, x32, vel = run.gpu_io(sigma, sigma_next)
+    np.testing.assert_array_equal(bits(hout_io), bits(hout_dev))
+    np.testing.assert_array_equal(bits(h_io), bits(h_dev))
     for b in range(run.batch):
         ref = run.oracle(b, sigma, sigma_next)
-        assert_close(to_f64(hout_dev[b]), ref["h2"], f"h_out[{b}]", rounded_inputs=3)
+        ds = sigma_next - sigma
+        layer_parity(f"[{b}]", ref, noisy, ds, h_out=to_f64(hout_dev[b]), x_new=to_f64(h_dev[b])[noisy])
         if noisy.any():
-            vel = ref["vel"][noisy]
-            br = abs(sigma_next - sigma) * float(np.sqrt(np.mean(vel ** 2)))
-            assert_close(to_f64(h_dev[b])[noisy], ref["x_new"][noisy], f"x'[{b}]", rounded_inputs=2, branch_rms=br)
+            layer_parity(f"io [{b}]", ref, noisy, ds, x_new=x32[b].double().cpu().numpy(), vel=to_f64(vel[b]),
+                         x_f32=True)
+            # the bf16 copy in h is the float32 state rounded to nearest even
+            np.testing.assert_array_equal(bits(h_io[b])[noisy], bits(x32[b].to(torch.bfloat16)))
         # AR and clean rows of h are never written (clean DM tokens pass through bit-exact)
         np.testing.assert_array_equal(bits(h_dev[b])[~noisy], run.h[b][~noisy])
 

@@ -2,15 +2,18 @@
 
 P ranks are emulated in one process: each shard runs its phases through the
 library and the two exchanges are done by copying between the shards'
-buffers (the ranks never wait on one another).  Every output element is
-computed with the same arithmetic as the single-GPU layer, so the result must
-be bit-identical to cosmot_layer_forward.
+buffers (the ranks never wait on one another).  The reassembled result is
+checked against the fp64 oracle's layer (h_out and x' of every row), and,
+since every output element is computed with the same arithmetic as the
+single-GPU layer, it must also be bit-identical to cosmot_layer_forward.
 """
 
 import numpy as np
 import pytest
 
 import synth
+from oracle import layer as olayer
+from oracle import layout as olayout
 from synth import LayoutSpec, ModelDims, VideoSpec
 
 pytestmark = pytest.mark.gpu
@@ -22,7 +25,8 @@ if not torch.cuda.is_available():  # pragma: no cover
 from flow_matching_dit_cosmot_b200 import api as A  # noqa: E402
 from flow_matching_dit_cosmot_b200 import _lib as L  # noqa: E402
 from flow_matching_dit_cosmot_b200.ulysses import UlyssesShard, emulate  # noqa: E402
-from gpu_helpers import assert_device_ok, bits, device_weights, dims as cdims, layout_spec, to_dev  # noqa: E402
+from gpu_helpers import (assert_device_ok, bits, device_weights, dims as cdims, layer_parity, layout_spec,  # noqa: E402
+                         to_dev, to_f64)
 
 DIMS = ModelDims(d_model=512, n_heads=8, n_kv_heads=4, head_dim=64, ffn=1024, rope_sections=(8, 12, 12))
 
@@ -32,7 +36,6 @@ DIMS = ModelDims(d_model=512, n_heads=8, n_kv_heads=4, head_dim=64, ffn=1024, ro
 def test_emulated_ranks_equal_the_single_gpu_layer(p, name, mode):
     spec = {"droid": synth.preset("droid").layout,
             "unaligned": LayoutSpec(n_text=20, video=VideoSpec(2, 5, 13, 24, 2, 3))}[name]
-    from oracle import layout as olayout
     lay = olayout.build_layout(spec)
     n = lay.n_tokens
     w = synth.make_weights(DIMS, 4400)
@@ -52,6 +55,14 @@ def test_emulated_ranks_equal_the_single_gpu_layer(p, name, mode):
     emulate(shards, h_loc, out_loc, 0.8, 0.6)
     torch.cuda.synchronize()
     assert_device_ok()
+    # the shards' rows put back together, against the oracle ("Cosmos 3 方法原理全解" §3, §7.2)
+    got_h = np.concatenate([to_f64(x) for x in h_loc])
+    got_out = np.concatenate([to_f64(o) for o in out_loc])
+    ref = olayer.layer_forward(DIMS, olayer.weights_from_bits(DIMS, w), synth.bf16_to_f64(h), lay.region, lay.pos,
+                               lay.chunk, 0.8, 0.6, mode)
+    noisy = lay.region == olayout.REGION_NOISY
+    layer_parity(f"ulysses P={p} {name}", ref, noisy, 0.6 - 0.8, h_out=got_out, x_new=got_h[noisy])
+    np.testing.assert_array_equal(bits(torch.cat(h_loc))[~noisy], h[~noisy])
     for sh, x, o in zip(shards, h_loc, out_loc):
         np.testing.assert_array_equal(bits(x), bits(h_ref[0, sh.row0:sh.row1]))
         np.testing.assert_array_equal(bits(o), bits(out_ref[0, sh.row0:sh.row1]))
