@@ -932,16 +932,23 @@ def run_micro(args, wl):
         print(json.dumps(line), flush=True)
         return
     if args.micro == "attention":
+        n_q, q_off = T, 0
+        if wl.stream is not None and not args.tokens:
+            # a streaming step: the newest block's rows are the queries; every
+            # key (AR, the cached blocks, the block itself) is visible to them
+            n_q = wl.layout.n_noisy
+            T = wl.layout.n_ar + (wl.stream.cached_blocks + 1) * n_q
+            q_off = T - n_q
         qkv = rnd(T, qkvc)
-        o = torch.empty((T, H * hd), dtype=torch.bfloat16, device=dev)
-        desc = L.AttnDesc(n_q=T, q_key_offset=0, n_keys=T, n_ar=n_ar, n_heads=H, n_kv_heads=Hkv, head_dim=hd,
+        o = torch.empty((n_q, H * hd), dtype=torch.bfloat16, device=dev)
+        desc = L.AttnDesc(n_q=n_q, q_key_offset=q_off, n_keys=T, n_ar=n_ar, n_heads=H, n_kv_heads=Hkv, head_dim=hd,
                           mask_mode=L.COSMOT_MASK_FULL, batch=1)
         base = qkv.data_ptr()
 
         def launch():
-            L.cosmot_mot_attention(desc, base, qkvc, base + 2 * H * hd, base + 2 * (H + Hkv) * hd, qkvc,
-                                   o.data_ptr(), H * hd, sh)
-        pairs = n_ar * (n_ar + 1) // 2 + (T - n_ar) * T
+            L.cosmot_mot_attention(desc, base + q_off * qkvc * 2, qkvc, base + 2 * H * hd, base + 2 * (H + Hkv) * hd,
+                                   qkvc, o.data_ptr(), H * hd, sh)
+        pairs = (n_ar * (n_ar + 1) // 2 + (T - n_ar) * T) if q_off == 0 else n_q * T
         work, unit, peak = 4 * pairs * H * hd, "TFLOP/s", float(peaks["bf16_tflops"])
     elif args.micro == "gemm":
         a = rnd(T, d)

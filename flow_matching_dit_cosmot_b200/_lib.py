@@ -13,6 +13,7 @@ import os
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libcosmot.so")
+LIB_DEBUG_PATH = os.path.join(_HERE, "libcosmot_debug.so")  # the same ABI, with device-side store checks
 
 COSMOT_OK = 0
 COSMOT_ERR_INVALID_ARG = 1
@@ -20,6 +21,7 @@ COSMOT_ERR_UNSUPPORTED = 2
 COSMOT_ERR_CUDA = 3
 COSMOT_ERR_TIMEOUT = 4
 COSMOT_ERR_WORKSPACE = 5
+COSMOT_ERR_BOUNDS = 6
 
 COSMOT_EPI_NONE = 0
 COSMOT_EPI_RESIDUAL = 1
@@ -33,6 +35,7 @@ COSMOT_MASK_FULL = 0
 COSMOT_MASK_BLOCK_CAUSAL = 1
 COSMOT_ATTN_NO_TILE_SKIP = 1
 COSMOT_SITE_SELFTEST = 900
+COSMOT_SITE_SELFTEST_BOUNDS = 901
 
 c_i32, c_i64, c_f32, c_f64, c_vp = ctypes.c_int32, ctypes.c_int64, ctypes.c_float, ctypes.c_double, ctypes.c_void_p
 
@@ -104,6 +107,8 @@ SIGNATURES = {
     "cosmot_version": (c_i32, []),
     "cosmot_get_device_status": (c_i32, [c_vp, _P(c_i32), _P(c_i32)]),
     "cosmot_selftest_wait_timeout": (c_i32, [c_vp]),
+    "cosmot_debug_checks": (c_i32, []),
+    "cosmot_selftest_bounds_check": (c_i32, [c_vp]),
     "cosmot_layout_counts": (c_i32, [_P(LayoutSpec), _P(c_i32), _P(c_i32), _P(c_i32), _P(c_i32)]),
     "cosmot_build_layout": (c_i32, [_P(LayoutSpec), c_vp, c_vp, c_vp, c_vp]),
     "cosmot_mrope_table": (c_i32, [c_vp, c_i64, c_i32, _P(c_i32), c_f64, c_vp, c_vp]),
@@ -156,21 +161,38 @@ STAGE_NAMES = ("norm1", "qkv_mrope", "attention", "oproj_residual", "norm2", "ga
                "norm_final", "velocity_euler")
 
 _lib = None
+_lib_debug = None
+
+
+def load(path: str) -> ctypes.CDLL:
+    """Loads one build of the library and declares every entry's signature."""
+    if not os.path.exists(path):
+        raise ImportError(f"{os.path.basename(path)} not built at {path}; run "
+                          f"`python -m flow_matching_dit_cosmot_b200.build`")
+    L = ctypes.CDLL(path)
+    for name, (res, args) in SIGNATURES.items():
+        f = getattr(L, name)
+        f.restype = res
+        f.argtypes = args
+    return L
 
 
 def lib() -> ctypes.CDLL:
     """Loads libcosmot.so (built in-tree by flow_matching_dit_cosmot_b200.build)."""
     global _lib
     if _lib is None:
-        if not os.path.exists(LIB_PATH):
-            raise ImportError(f"libcosmot.so not built at {LIB_PATH}; run `python -m flow_matching_dit_cosmot_b200.build`")
-        L = ctypes.CDLL(LIB_PATH)
-        for name, (res, args) in SIGNATURES.items():
-            f = getattr(L, name)
-            f.restype = res
-            f.argtypes = args
-        _lib = L
+        _lib = load(LIB_PATH)
     return _lib
+
+
+def lib_debug() -> ctypes.CDLL:
+    """Loads libcosmot_debug.so: the debug build, whose kernels check the index
+    of every global store and latch COSMOT_ERR_BOUNDS instead of writing out of
+    place.  Call its entries directly (same names and signatures)."""
+    global _lib_debug
+    if _lib_debug is None:
+        _lib_debug = load(LIB_DEBUG_PATH)
+    return _lib_debug
 
 
 class CosmotError(RuntimeError):

@@ -4,7 +4,9 @@
 
 Each .cu under csrc/ compiles to an object in _build/ (in parallel), then the
 objects link into flow_matching_dit_cosmot_b200/libcosmot.so.  Objects are
-rebuilt when their source or any header changed.
+rebuilt when their source or any header changed.  The same sources compiled
+with COSMOT_DEBUG_CHECKS (device-side store index checks that latch
+COSMOT_ERR_BOUNDS) link into libcosmot_debug.so beside it.
 """
 
 from __future__ import annotations
@@ -21,6 +23,7 @@ CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 BUILD = os.path.join(ROOT, "_build")
 LIB = os.path.join(PKG, "libcosmot.so")
+LIB_DEBUG = os.path.join(PKG, "libcosmot_debug.so")
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
 
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
@@ -40,9 +43,9 @@ def _stale(obj, src, deps):
     return any(os.path.getmtime(p) > t for p in [src] + deps)
 
 
-def _compile(src, verbose=False, ptxas_verbose=False):
-    obj = os.path.join(BUILD, os.path.basename(src) + ".o")
-    cmd = [NVCC, *ARCH, *FLAGS, "-c", src, "-o", obj]
+def _compile(src, verbose=False, ptxas_verbose=False, debug=False):
+    obj = os.path.join(BUILD, ("debug_" if debug else "") + os.path.basename(src) + ".o")
+    cmd = [NVCC, *ARCH, *FLAGS, *(["-DCOSMOT_DEBUG_CHECKS=1"] if debug else []), "-c", src, "-o", obj]
     if ptxas_verbose:
         cmd += ["-Xptxas", "-v"]
     if verbose:
@@ -57,19 +60,25 @@ def build(verbose: bool = False, force: bool = False, ptxas_verbose: bool = Fals
     os.makedirs(BUILD, exist_ok=True)
     srcs = sorted(glob.glob(os.path.join(CSRC, "*.cu")))
     deps = _headers()
-    todo = [s for s in srcs if force or ptxas_verbose or _stale(os.path.join(BUILD, os.path.basename(s) + ".o"), s, deps)]
-    with cf.ThreadPoolExecutor(max_workers=min(8, max(1, len(todo)))) as ex:
-        for obj, err in ex.map(lambda s: _compile(s, verbose, ptxas_verbose), todo):
+    jobs = []
+    for debug in (False, True):
+        for s in srcs:
+            obj = os.path.join(BUILD, ("debug_" if debug else "") + os.path.basename(s) + ".o")
+            if force or (ptxas_verbose and not debug) or _stale(obj, s, deps):
+                jobs.append((s, debug))
+    with cf.ThreadPoolExecutor(max_workers=min(16, max(1, len(jobs)))) as ex:
+        for obj, err in ex.map(lambda j: _compile(j[0], verbose, ptxas_verbose and not j[1], j[1]), jobs):
             if ptxas_verbose and err:
                 print(err)
-    objs = [os.path.join(BUILD, os.path.basename(s) + ".o") for s in srcs]
-    if force or todo or not os.path.exists(LIB) or any(os.path.getmtime(o) > os.path.getmtime(LIB) for o in objs):
-        cmd = [NVCC, *ARCH, "-shared", "-o", LIB, *objs]
-        if verbose:
-            print(" ".join(cmd), flush=True)
-        r = subprocess.run(cmd, capture_output=True, text=True)
-        if r.returncode != 0:
-            raise RuntimeError(f"link failed:\n{r.stdout}\n{r.stderr}")
+    for lib, prefix in ((LIB, ""), (LIB_DEBUG, "debug_")):
+        objs = [os.path.join(BUILD, prefix + os.path.basename(s) + ".o") for s in srcs]
+        if force or jobs or not os.path.exists(lib) or any(os.path.getmtime(o) > os.path.getmtime(lib) for o in objs):
+            cmd = [NVCC, *ARCH, "-shared", "-o", lib, *objs]
+            if verbose:
+                print(" ".join(cmd), flush=True)
+            r = subprocess.run(cmd, capture_output=True, text=True)
+            if r.returncode != 0:
+                raise RuntimeError(f"link failed:\n{r.stdout}\n{r.stderr}")
     return LIB
 
 

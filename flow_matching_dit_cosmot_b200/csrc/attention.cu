@@ -554,7 +554,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         uint32_t ov[32];
         tmem_ld32(o_addr + 32 * c, ov);
         tmem_ld_wait();
-        if (valid) {
+        if (valid && dcheck(qi < p.n_q && w.h < p.n_heads && w.b < p.batch, p.status, kWhereAttnStore)) {
 #pragma unroll
           for (int q4 = 0; q4 < 4; ++q4) {
             uint4 v4;

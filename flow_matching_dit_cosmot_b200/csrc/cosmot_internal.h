@@ -20,7 +20,13 @@ enum Where : int {
   kWhereAttnMma = 201,
   kWhereAttnSoftmax = 202,
   kWhereAttnDrain = 203,
+  // debug-build store checks (COSMOT_ERR_BOUNDS)
+  kWhereGemmStore = 104,
+  kWhereAttnStore = 204,
+  kWhereNormStore = 300,
+  kWhereEulerStore = 301,
   kWhereSelftest = COSMOT_SITE_SELFTEST,
+  kWhereSelftestBounds = COSMOT_SITE_SELFTEST_BOUNDS,
 };
 
 // Encodes a 2D bf16 tensor map: `rows` x `cols` elements with row pitch

@@ -17,6 +17,7 @@ struct SegTable {
   int64_t row_begin[kMaxSegs];
   int64_t out_row[kMaxSegs];
   int64_t prefix[kMaxSegs + 1];  // flattened row index where each segment starts
+  int64_t out_extent;            // output rows the segments address (debug store checks)
   int32_t set[kMaxSegs];
   int32_t n;
 };
@@ -24,6 +25,7 @@ struct SegTable {
 bool fill_segs(const cosmot_segment* segs, int32_t n, SegTable* t) {
   if (!segs || n < 1 || n > kMaxSegs) return false;
   t->n = n;
+  t->out_extent = 0;
   int64_t acc = 0;
   for (int i = 0; i < n; ++i) {
     if (segs[i].row_begin < 0 || segs[i].row_end < segs[i].row_begin || segs[i].out_row < 0) return false;
@@ -33,6 +35,8 @@ bool fill_segs(const cosmot_segment* segs, int32_t n, SegTable* t) {
     t->set[i] = segs[i].weight_set;
     t->prefix[i] = acc;
     acc += segs[i].row_end - segs[i].row_begin;
+    const int64_t end = segs[i].out_row + (segs[i].row_end - segs[i].row_begin);
+    if (end > t->out_extent) t->out_extent = end;
   }
   t->prefix[n] = acc;
   return true;
@@ -53,7 +57,8 @@ template <int kVecPerLane>
 __global__ void __launch_bounds__(256) rmsnorm_f32in_kernel(const float* __restrict__ h, int64_t ld_h,
                                                             const SegTable segs, const __nv_bfloat16* __restrict__ g0,
                                                             const __nv_bfloat16* __restrict__ g1, int32_t d, float eps,
-                                                            __nv_bfloat16* __restrict__ out, int64_t ld_out) {
+                                                            __nv_bfloat16* __restrict__ out, int64_t ld_out,
+                                                            int* status) {
   const int lane = threadIdx.x & 31;
   const int64_t warps_total = (int64_t)gridDim.x * (blockDim.x >> 5);
   const int nvec = d >> 3;
@@ -80,6 +85,7 @@ __global__ void __launch_bounds__(256) rmsnorm_f32in_kernel(const float* __restr
 #pragma unroll
     for (int off = 16; off > 0; off >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, off);
     const float rstd = rsqrtf(ss / (float)d + eps);
+    if (!dcheck(o >= 0 && o < segs.out_extent, status, kWhereNormStore)) continue;
     uint4* dst = reinterpret_cast<uint4*>(out + o * ld_out);
     const uint4* gv = reinterpret_cast<const uint4*>(g);
 #pragma unroll
@@ -103,11 +109,93 @@ __global__ void __launch_bounds__(256) rmsnorm_f32in_kernel(const float* __restr
   }
 }
 
+// Wide rows (d >= 1024): one 128-thread block per row, up to kVecPerThread
+// 16-byte vectors of 8 elements per thread held in registers across both
+// passes (float32 rows as two float4 per vector), so a row is read once.  Small
+// blocks keep up to 16 rows in flight per SM; the sum of squares is reduced by
+// warp shuffles and a two-slot shared-memory exchange (one barrier per row).
+constexpr int kNormBlock = 128;
+
+template <typename TIn, int kVecPerThread>
+__global__ void __launch_bounds__(kNormBlock) rmsnorm_block_kernel(const TIn* __restrict__ h, int64_t ld_h,
+                                                                  const SegTable segs,
+                                                                  const __nv_bfloat16* __restrict__ g0,
+                                                                  const __nv_bfloat16* __restrict__ g1, int32_t d,
+                                                                  float eps, __nv_bfloat16* __restrict__ out,
+                                                                  int64_t ld_out, int* status) {
+  constexpr bool kF32 = sizeof(TIn) == 4;
+  __shared__ float part[2][kNormBlock / 32];
+  const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+  const int nvec = d >> 3;
+  int slot = 0;
+  for (int64_t gr = blockIdx.x; gr < segs.prefix[segs.n]; gr += gridDim.x, slot ^= 1) {
+    int s = 0;
+    while (s + 1 < segs.n && gr >= segs.prefix[s + 1]) ++s;
+    const int64_t local = gr - segs.prefix[s];
+    const TIn* src = h + (segs.row_begin[s] + local) * ld_h;
+    float f[kVecPerThread][8];
+    float ss = 0.f;
+#pragma unroll
+    for (int j = 0; j < kVecPerThread; ++j) {
+      const int c = threadIdx.x + kNormBlock * j;
+      if (c < nvec) {
+        if (kF32) {
+          const float4 a = *reinterpret_cast<const float4*>(reinterpret_cast<const float*>(src) + 8 * c);
+          const float4 b = *reinterpret_cast<const float4*>(reinterpret_cast<const float*>(src) + 8 * c + 4);
+          f[j][0] = a.x; f[j][1] = a.y; f[j][2] = a.z; f[j][3] = a.w;
+          f[j][4] = b.x; f[j][5] = b.y; f[j][6] = b.z; f[j][7] = b.w;
+        } else {
+          const uint4 v = *reinterpret_cast<const uint4*>(reinterpret_cast<const __nv_bfloat16*>(src) + 8 * c);
+          const uint32_t* u = reinterpret_cast<const uint32_t*>(&v);
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            const float2 x = unpack_bf16x2(u[q]);
+            f[j][2 * q] = x.x;
+            f[j][2 * q + 1] = x.y;
+          }
+        }
+#pragma unroll
+        for (int q = 0; q < 8; ++q) ss = fmaf(f[j][q], f[j][q], ss);
+      }
+    }
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, off);
+    if (lane == 0) part[slot][wid] = ss;
+    __syncthreads();  // also orders this row's reads of part[slot] before its reuse two rows later
+    float tot = 0.f;
+#pragma unroll
+    for (int i = 0; i < kNormBlock / 32; ++i) tot += part[slot][i];
+    const float rstd = rsqrtf(tot / (float)d + eps);
+    const __nv_bfloat16* g = segs.set[s] ? g1 : g0;
+    const int64_t orow = segs.out_row[s] + local;
+    const bool store_ok = dcheck(orow >= 0 && orow < segs.out_extent, status, kWhereNormStore);
+    uint4* dst = reinterpret_cast<uint4*>(out + orow * ld_out);
+    const uint4* gv = reinterpret_cast<const uint4*>(g);
+#pragma unroll
+    for (int j = 0; j < kVecPerThread; ++j) {
+      const int c = threadIdx.x + kNormBlock * j;
+      if (c < nvec && store_ok) {
+        const uint4 gg = __ldg(gv + c);
+        const uint32_t* gu = reinterpret_cast<const uint32_t*>(&gg);
+        uint4 res;
+        uint32_t* ru = reinterpret_cast<uint32_t*>(&res);
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          const float2 wq = unpack_bf16x2(gu[q]);
+          ru[q] = pack_bf16x2(f[j][2 * q] * rstd * wq.x, f[j][2 * q + 1] * rstd * wq.y);
+        }
+        dst[c] = res;
+      }
+    }
+  }
+}
+
 template <int kVecPerLane>
 __global__ void __launch_bounds__(256) rmsnorm_kernel(const __nv_bfloat16* __restrict__ h, int64_t ld_h,
                                                       const SegTable segs, const __nv_bfloat16* __restrict__ g0,
                                                       const __nv_bfloat16* __restrict__ g1, int32_t d, float eps,
-                                                      __nv_bfloat16* __restrict__ out, int64_t ld_out) {
+                                                      __nv_bfloat16* __restrict__ out, int64_t ld_out,
+                                                      int* status) {
   const int lane = threadIdx.x & 31;
   const int64_t warps_total = (int64_t)gridDim.x * (blockDim.x >> 5);
   const int nvec = d >> 3;
@@ -139,6 +227,7 @@ __global__ void __launch_bounds__(256) rmsnorm_kernel(const __nv_bfloat16* __res
 #pragma unroll
     for (int off = 16; off > 0; off >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, off);
     const float rstd = rsqrtf(ss / (float)d + eps);
+    if (!dcheck(o >= 0 && o < segs.out_extent, status, kWhereNormStore)) continue;
     uint4* dst = reinterpret_cast<uint4*>(out + o * ld_out);
     const uint4* gv = reinterpret_cast<const uint4*>(g);
 #pragma unroll
@@ -210,12 +299,14 @@ __global__ void __launch_bounds__(256) mrope_kernel(__nv_bfloat16* __restrict__ 
 // ---------------------------------------------------------------- Euler
 __global__ void __launch_bounds__(256) euler_kernel(__nv_bfloat16* __restrict__ x, int64_t ld_x,
                                                     const __nv_bfloat16* __restrict__ v, int64_t ld_v,
-                                                    int64_t row_begin, int64_t n_rows, int64_t n_cols, float dsigma) {
+                                                    int64_t row_begin, int64_t n_rows, int64_t n_cols, float dsigma,
+                                                    int* status) {
   const int64_t vec_per_row = n_cols >> 3;
   const int64_t total = n_rows * vec_per_row;
   for (int64_t e = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; e < total; e += (int64_t)gridDim.x * blockDim.x) {
     const int64_t r = row_begin + e / vec_per_row;
     const int64_t c = (e % vec_per_row) << 3;
+    if (!dcheck(r < row_begin + n_rows && c + 8 <= n_cols, status, kWhereEulerStore)) continue;
     uint4* xp = reinterpret_cast<uint4*>(x + r * ld_x + c);
     uint4 xv = *xp;
     uint4 vv = __ldg(reinterpret_cast<const uint4*>(v + r * ld_v + c));
@@ -286,7 +377,7 @@ cosmot_status rmsnorm_routed(const void* h, bool h_f32, int64_t ld_h, const cosm
     const void* g = t.set[i] ? g1 : g0;
     if (!g || !aligned16(g)) return COSMOT_ERR_INVALID_ARG;
   }
-  if (d > 8 * 32 * 24) return COSMOT_ERR_UNSUPPORTED;  // d <= 6144 with 24 vectors per lane
+  if (d > 8 * kNormBlock * 6) return COSMOT_ERR_UNSUPPORTED;  // d <= 6144: 6 vectors per thread of a block
   const int64_t rows = t.prefix[t.n];
   if (rows == 0) return COSMOT_OK;
   const int threads = 256;
@@ -296,23 +387,34 @@ cosmot_status rmsnorm_routed(const void* h, bool h_f32, int64_t ld_h, const cosm
   const auto* gp0 = static_cast<const __nv_bfloat16*>(g0);
   const auto* gp1 = static_cast<const __nv_bfloat16*>(g1);
   auto* op = static_cast<__nv_bfloat16*>(out);
-  const int vpl = (int)((d / 8 + 31) / 32);
-  if (h_f32) {
-    const auto* hf = static_cast<const float*>(h);
-    if (vpl <= 4)
-      rmsnorm_f32in_kernel<4><<<grid, threads, 0, s>>>(hf, ld_h, t, gp0, gp1, (int32_t)d, eps, op, ld_out);
-    else if (vpl <= 16)
-      rmsnorm_f32in_kernel<16><<<grid, threads, 0, s>>>(hf, ld_h, t, gp0, gp1, (int32_t)d, eps, op, ld_out);
-    else
-      rmsnorm_f32in_kernel<24><<<grid, threads, 0, s>>>(hf, ld_h, t, gp0, gp1, (int32_t)d, eps, op, ld_out);
+  int* st = device_status_ptr();
+  if (!st) return COSMOT_ERR_CUDA;
+  if (d >= 1024) {  // one block per row
+    const int64_t cap = (int64_t)num_sms() * 16;
+    const unsigned bgrid = (unsigned)(rows < cap ? rows : cap);
+    const int vpt = (int)((d / 8 + kNormBlock - 1) / kNormBlock);
+    if (h_f32) {
+      const auto* hf = static_cast<const float*>(h);
+      if (vpt <= 4)
+        rmsnorm_block_kernel<float, 4><<<bgrid, kNormBlock, 0, s>>>(hf, ld_h, t, gp0, gp1, (int32_t)d, eps, op, ld_out, st);
+      else
+        rmsnorm_block_kernel<float, 6><<<bgrid, kNormBlock, 0, s>>>(hf, ld_h, t, gp0, gp1, (int32_t)d, eps, op, ld_out, st);
+    } else {
+      if (vpt <= 4)
+        rmsnorm_block_kernel<__nv_bfloat16, 4><<<bgrid, kNormBlock, 0, s>>>(hp, ld_h, t, gp0, gp1, (int32_t)d, eps, op,
+                                                                           ld_out, st);
+      else
+        rmsnorm_block_kernel<__nv_bfloat16, 6><<<bgrid, kNormBlock, 0, s>>>(hp, ld_h, t, gp0, gp1, (int32_t)d, eps, op,
+                                                                           ld_out, st);
+    }
     return launch_status();
   }
-  if (vpl <= 4)
-    rmsnorm_kernel<4><<<grid, threads, 0, s>>>(hp, ld_h, t, gp0, gp1, (int32_t)d, eps, op, ld_out);
-  else if (vpl <= 16)
-    rmsnorm_kernel<16><<<grid, threads, 0, s>>>(hp, ld_h, t, gp0, gp1, (int32_t)d, eps, op, ld_out);
+  // narrow rows (d < 1024): one warp per row, at most 4 vectors per lane
+  if (h_f32)
+    rmsnorm_f32in_kernel<4><<<grid, threads, 0, s>>>(static_cast<const float*>(h), ld_h, t, gp0, gp1, (int32_t)d, eps,
+                                                     op, ld_out, st);
   else
-    rmsnorm_kernel<24><<<grid, threads, 0, s>>>(hp, ld_h, t, gp0, gp1, (int32_t)d, eps, op, ld_out);
+    rmsnorm_kernel<4><<<grid, threads, 0, s>>>(hp, ld_h, t, gp0, gp1, (int32_t)d, eps, op, ld_out, st);
   return launch_status();
 }
 
@@ -357,9 +459,11 @@ cosmot_status cosmot_flow_euler_step(void* x, int64_t ld_x, const void* v, int64
   if (items == 0) return COSMOT_OK;
   const float dsigma = (float)(sigma_next - sigma);
   const int threads = 256;
+  int* st = device_status_ptr();
+  if (!st) return COSMOT_ERR_CUDA;
   euler_kernel<<<grid_for(items, threads), threads, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
       static_cast<__nv_bfloat16*>(x), ld_x, static_cast<const __nv_bfloat16*>(v), ld_v, row_begin,
-      row_end - row_begin, n_cols, dsigma);
+      row_end - row_begin, n_cols, dsigma, st);
   return launch_status();
 }
 

@@ -73,6 +73,8 @@ struct Params {
   int64_t ld_vel;
   __nv_bfloat16* out;     // float32 storage with COSMOT_EPI_OUT_F32
   int64_t ld_out;
+  int64_t out_rows;       // output rows the segments address (debug store checks)
+  int64_t a_rows;         // input rows the segments address (x_state / vel rows)
   int* status;
 };
 
@@ -325,7 +327,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           tmem_ld32(tacc + BN / 2 + 32 * c, u);
           tmem_ld_wait();
           const int32_t col0 = col_base + 32 * c;
-          if (valid && col0 < p.n_out) {
+          if (valid && col0 < p.n_out && dcheck(orow >= 0 && orow < p.out_rows, p.status, kWhereGemmStore)) {
 #pragma unroll
             for (int j = 0; j < 32; ++j) {
               const float g = __uint_as_float(v[j]);
@@ -351,7 +353,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             tmem_ld32(tacc + hb * hd + i0, v);
             tmem_ld32(tacc + hb * hd + half + i0, u);
             tmem_ld_wait();
-            if (valid && hcol < p.n_out) {
+            if (valid && hcol < p.n_out && dcheck(orow >= 0 && orow < p.out_rows, p.status, kWhereGemmStore)) {
               float lo[32], hi[32];
               if (rotate) {
 #pragma unroll
@@ -383,7 +385,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           tmem_ld32(tacc + 32 * c, v);
           tmem_ld_wait();
           const int32_t col0 = tl.n * BN + 32 * c;
-          if (valid && col0 < p.n_out) {
+          if (valid && col0 < p.n_out && dcheck(orow >= 0 && orow < p.out_rows, p.status, kWhereGemmStore)) {
             if (EPI == COSMOT_EPI_RESIDUAL) {
               float rs[32];
               if (FL & COSMOT_EPI_RES_F32)
@@ -395,15 +397,16 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             } else if (EPI == COSMOT_EPI_EULER) {
               // x' = x + dsigma * v in fp32; x from the fp32 state when there is one
               const int64_t arow = tl.a_row0 + r;
+              const bool arow_ok = dcheck(arow >= 0 && arow < p.a_rows, p.status, kWhereGemmStore);
               float xs[32];
-              if (p.xs && !p.xs_from_x)
+              if (p.xs && !p.xs_from_x && arow_ok)
                 load_row32_f32(p.xs + arow * p.ld_xs + col0, col0, p.n_out, xs);
               else
                 load_row32(p.x + orow * p.ld_x + col0, col0, p.n_out, xs);
 #pragma unroll
               for (int j = 0; j < 32; ++j) f[j] = fmaf(p.dsigma, __uint_as_float(v[j]), xs[j]);
-              if (p.xs) store_row32_f32(p.xs + arow * p.ld_xs + col0, col0, p.n_out, f);
-              if (p.vel) {
+              if (p.xs && arow_ok) store_row32_f32(p.xs + arow * p.ld_xs + col0, col0, p.n_out, f);
+              if (p.vel && arow_ok) {
                 float vv[32];
 #pragma unroll
                 for (int j = 0; j < 32; ++j) vv[j] = __uint_as_float(v[j]);
@@ -495,6 +498,11 @@ extern "C" cosmot_status cosmot_routed_linear(const void* a, int64_t ld_a, int64
   }
   p.mtile_prefix[n_segs] = mt;
   p.num_m_tiles = mt;
+  for (int i = 0; i < n_segs; ++i) {
+    const int64_t end = segs[i].out_row + (segs[i].row_end - segs[i].row_begin);
+    if (end > p.out_rows) p.out_rows = end;
+  }
+  p.a_rows = max_row;
   if (mt == 0) return COSMOT_OK;
   if (max_row > INT32_MAX) return COSMOT_ERR_UNSUPPORTED;
   const bool silu = kind == COSMOT_EPI_SILU_MUL;

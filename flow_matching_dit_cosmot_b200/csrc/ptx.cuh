@@ -33,6 +33,23 @@ __device__ __forceinline__ uint64_t globaltimer_ns() {
   return t;
 }
 
+// Debug builds (COSMOT_DEBUG_CHECKS: libcosmot_debug.so) check the index of
+// every global store against the extent the host derived for it; a failed
+// check latches COSMOT_ERR_BOUNDS with its site and the store is skipped, so
+// nothing is written out of place and nothing traps.  Release builds compile
+// the checks away.
+__device__ __forceinline__ bool dcheck(bool ok, int* status, int where) {
+#if defined(COSMOT_DEBUG_CHECKS)
+  if (!ok) latch_status(status, COSMOT_ERR_BOUNDS, where);
+  return ok;
+#else
+  (void)ok;
+  (void)status;
+  (void)where;
+  return true;
+#endif
+}
+
 // One second: far above any legitimate wait in these kernels (the longest
 // mainloop of a tile is well under a millisecond), far below a watchdog.
 constexpr uint64_t kWaitLimitNs = 1000000000ull;

@@ -90,9 +90,38 @@ __global__ void __launch_bounds__(64) selftest_timeout_kernel(int* status) {
   __syncthreads();
 }
 
+// Test-only: a checked store one past its stated extent (index 1 of extent 1
+// into a two-element array, so the store would stay in bounds even unchecked).
+__device__ int g_selftest_bounds_target[2];
+
+__global__ void selftest_bounds_kernel(int* status) {
+  const int extent = 1, index = 1;
+  if (dcheck(index < extent, status, kWhereSelftestBounds)) g_selftest_bounds_target[index] = 1;
+}
+
 }  // namespace cosmot
 
 extern "C" {
+
+int32_t cosmot_debug_checks(void) {
+#if defined(COSMOT_DEBUG_CHECKS)
+  return 1;
+#else
+  return 0;
+#endif
+}
+
+cosmot_status cosmot_selftest_bounds_check(cosmot_stream_t stream) {
+#if defined(COSMOT_DEBUG_CHECKS)
+  int* st = cosmot::device_status_ptr();
+  if (!st) return COSMOT_ERR_CUDA;
+  cosmot::selftest_bounds_kernel<<<1, 1, 0, reinterpret_cast<cudaStream_t>(stream)>>>(st);
+  return cosmot::launch_status();
+#else
+  (void)stream;
+  return COSMOT_ERR_UNSUPPORTED;
+#endif
+}
 
 cosmot_status cosmot_selftest_wait_timeout(cosmot_stream_t stream) {
   int* st = cosmot::device_status_ptr();
@@ -109,6 +138,7 @@ const char* cosmot_status_string(cosmot_status s) {
     case COSMOT_ERR_CUDA: return "COSMOT_ERR_CUDA";
     case COSMOT_ERR_TIMEOUT: return "COSMOT_ERR_TIMEOUT";
     case COSMOT_ERR_WORKSPACE: return "COSMOT_ERR_WORKSPACE";
+    case COSMOT_ERR_BOUNDS: return "COSMOT_ERR_BOUNDS";
     default: return "COSMOT_ERR_UNKNOWN";
   }
 }

@@ -56,7 +56,8 @@ enum {
   COSMOT_ERR_UNSUPPORTED = 2,
   COSMOT_ERR_CUDA = 3,
   COSMOT_ERR_TIMEOUT = 4,
-  COSMOT_ERR_WORKSPACE = 5
+  COSMOT_ERR_WORKSPACE = 5,
+  COSMOT_ERR_BOUNDS = 6     /* debug build only: a device-side store index check failed (store skipped) */
 };
 
 /* Human-readable name of a status code (static string, never NULL). */
@@ -74,6 +75,28 @@ COSMOT_API cosmot_status cosmot_get_device_status(cosmot_stream_t stream, cosmot
 
 /* Site code that cosmot_selftest_wait_timeout latches with its timeout. */
 #define COSMOT_SITE_SELFTEST 900
+/* Site code that cosmot_selftest_bounds_check latches (debug build). */
+#define COSMOT_SITE_SELFTEST_BOUNDS 901
+
+/*
+ * 1 in the debug build of the library (libcosmot_debug.so, compiled with
+ * COSMOT_DEBUG_CHECKS), 0 in the release build.  The debug build checks the
+ * index of every global store its kernels make (GEMM, attention, norm and
+ * Euler outputs) against the extent the host side derived for that output; a
+ * failed check latches COSMOT_ERR_BOUNDS with the kernel's site code into the
+ * device status word and skips the store (no trap).  Results are otherwise
+ * identical to the release build's.
+ */
+COSMOT_API int32_t cosmot_debug_checks(void);
+
+/*
+ * Test-only check of the debug build's store checks: one thread makes a
+ * checked store whose index is one past the extent it states (the index still
+ * lies inside the kernel's own buffer), so the check fails, latches
+ * COSMOT_ERR_BOUNDS at COSMOT_SITE_SELFTEST_BOUNDS and skips the store.  The
+ * release build returns COSMOT_ERR_UNSUPPORTED and launches nothing.
+ */
+COSMOT_API cosmot_status cosmot_selftest_bounds_check(cosmot_stream_t stream);
 
 /*
  * Test-only check of the failure path.  One CTA whose consumer thread waits on

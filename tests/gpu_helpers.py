@@ -73,3 +73,24 @@ def layer_parity(what, ref, noisy, dsigma, h_out=None, x_new=None, vel=None, x_f
     if x_new is not None:
         assert_close(x_new, ref["x_new"][noisy], f"{what} x'", sigma=SIGMA_VEL, branch_rms=abs(dsigma) * rms(v),
                      depth=depth, out_bf16=not x_f32)
+
+
+CANARY = 0x7BAD  # a bf16 NaN pattern no kernel writes
+
+
+class Guarded:
+    """A contiguous bf16 buffer with `guard` canary elements before and after
+    it, so a test can check that a call wrote nothing outside its output."""
+
+    def __init__(self, data: torch.Tensor, guard: int = 4096):
+        n = data.numel()
+        self.raw = torch.full((n + 2 * guard,), CANARY, dtype=torch.int16, device=data.device)
+        self.guard = guard
+        self.t = self.raw[guard:guard + n].view(torch.bfloat16).view(data.shape)
+        self.t.copy_(data)
+
+    def assert_canaries(self, what: str = ""):
+        g = self.guard
+        raw = self.raw.cpu().numpy()
+        bad = int((raw[:g] != CANARY).sum() + (raw[-g:] != CANARY).sum())
+        assert bad == 0, f"{what}: {bad} guard elements around the buffer were overwritten"

@@ -29,20 +29,28 @@ def test_header_declares_the_hot_path_entry_points():
         assert n in names
 
 
-def test_library_exports_every_declared_symbol():
+@pytest.mark.parametrize("debug", [False, True])
+def test_library_exports_every_declared_symbol(debug):
+    """Both builds (release, and the debug build with device-side store
+    checks) export every entry the header declares."""
     from flow_matching_dit_cosmot_b200 import _lib as L
-    L.lib()
-    out = subprocess.run(["nm", "-D", "--defined-only", L.LIB_PATH], capture_output=True, text=True, check=True).stdout
+    lib = L.lib_debug() if debug else L.lib()
+    path = L.LIB_DEBUG_PATH if debug else L.LIB_PATH
+    out = subprocess.run(["nm", "-D", "--defined-only", path], capture_output=True, text=True, check=True).stdout
     exported = set(re.findall(r"\sT\s(cosmot_\w+)", out))
     missing = [n for n in _declared() if n not in exported]
     assert not missing, missing
     assert set(_declared()) == set(L.SIGNATURES), "binding and header disagree"
+    assert lib.cosmot_debug_checks() == (1 if debug else 0)
+    if not debug:  # host-only: the release build has no store checks to exercise
+        assert lib.cosmot_selftest_bounds_check(None) == L.COSMOT_ERR_UNSUPPORTED
 
 
 def test_status_strings_and_version():
     from flow_matching_dit_cosmot_b200 import _lib as L
     assert L.status_string(0) == "COSMOT_OK"
     assert L.status_string(4) == "COSMOT_ERR_TIMEOUT"
+    assert L.status_string(6) == "COSMOT_ERR_BOUNDS"
     assert L.status_string(99) == "COSMOT_ERR_UNKNOWN"
     assert L.cosmot_version() >= 100
 

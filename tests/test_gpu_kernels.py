@@ -23,7 +23,7 @@ if not torch.cuda.is_available():  # pragma: no cover
 
 from flow_matching_dit_cosmot_b200 import api as A  # noqa: E402
 from flow_matching_dit_cosmot_b200 import _lib as L  # noqa: E402
-from gpu_helpers import assert_device_ok, bits, layout_spec, to_dev, to_f64  # noqa: E402
+from gpu_helpers import Guarded, assert_device_ok, bits, layout_spec, to_dev, to_f64  # noqa: E402
 from synth import LayoutSpec, VideoSpec  # noqa: E402
 
 
@@ -98,7 +98,8 @@ def test_rmsnorm_routed(d):
     g0 = synth.normal_bf16((d,), 4, 1, std=0.02, mean=1.0)
     g1 = synth.normal_bf16((d,), 5, 1, std=0.02, mean=1.0)
     hd_, g0d, g1d = to_dev(h), to_dev(g0), to_dev(g1)
-    out = torch.zeros((rows + 7, d), dtype=torch.bfloat16, device="cuda")
+    og = Guarded(torch.zeros((rows + 7, d), dtype=torch.bfloat16, device="cuda"))
+    out = og.t
     segs = [(0, 37, 7, 0), (37, 300, 44, 1)]  # output rows shifted by 7
     L.cosmot_rmsnorm_routed(A.ptr(hd_), d, segs, A.ptr(g0d), A.ptr(g1d), d, 1e-6, A.ptr(out), d,
                             A.stream_handle())
@@ -108,6 +109,7 @@ def test_rmsnorm_routed(d):
                           olayer.rms_norm(h64[37:], synth.bf16_to_f64(g1), 1e-6)])
     assert_close(got, ref, "rmsnorm")
     assert np.all(bits(out)[:7] == 0)
+    og.assert_canaries("rmsnorm output")
 
 
 # ---------------------------------------------------------------- routed GEMM
@@ -126,12 +128,14 @@ def _gemm_case(m_split, m_total, k, n_out, seed=0):
                                                      (258, 1000, 4096, 512)])
 def test_routed_linear_plain(m_split, m_total, k, n_out):
     a, w0, w1, segs, acc = _gemm_case(m_split, m_total, k, n_out)
-    out = torch.empty((m_total, n_out), dtype=torch.bfloat16, device="cuda")
+    og = Guarded(torch.empty((m_total, n_out), dtype=torch.bfloat16, device="cuda"))
+    out = og.t
     ad, w0d, w1d = to_dev(a), to_dev(w0), to_dev(w1)
     L.cosmot_routed_linear(A.ptr(ad), k, k, segs, A.ptr(w0d), A.ptr(w1d), n_out, A.ptr(out), n_out,
                            stream=A.stream_handle())
     assert_close(to_f64(out), acc, "gemm")
     assert_device_ok()
+    og.assert_canaries("gemm output")
 
 
 def test_routed_linear_equal_sets_equal_single_segment():
@@ -365,7 +369,8 @@ def _attn_case(n_keys, n_ar, n_q, q_off, H, Hkv, hd, mode, chunk=None, batch=1, 
         vv = synth.bf16_to_f64(v[b * n_keys:(b + 1) * n_keys]).reshape(n_keys, Hkv, hd)
         ref.append(olayer.attention(qq, kk, vv, allow, 1.0 / np.sqrt(hd)).reshape(n_q, H * hd))
     qd, kd, vd = to_dev(q), to_dev(k), to_dev(v)
-    o = torch.full((batch * n_q, H * hd), float("nan"), dtype=torch.bfloat16, device="cuda")
+    og = Guarded(torch.full((batch * n_q, H * hd), float("nan"), dtype=torch.bfloat16, device="cuda"))
+    o = og.t
     chd = torch.from_numpy(ch).cuda()
     d = L.AttnDesc(n_q=n_q, q_key_offset=q_off, n_keys=n_keys, n_ar=n_ar, n_heads=H, n_kv_heads=Hkv, head_dim=hd,
                    mask_mode=L.COSMOT_MASK_FULL if mode == "full" else L.COSMOT_MASK_BLOCK_CAUSAL,
@@ -373,6 +378,7 @@ def _attn_case(n_keys, n_ar, n_q, q_off, H, Hkv, hd, mode, chunk=None, batch=1, 
     L.cosmot_mot_attention(d, A.ptr(qd), H * hd, A.ptr(kd), A.ptr(vd), Hkv * hd, A.ptr(o), H * hd, A.stream_handle())
     got = to_f64(o)
     assert_device_ok()
+    og.assert_canaries("attention output")
     return got, np.concatenate(ref)
 
 

@@ -16,7 +16,8 @@ if not torch.cuda.is_available():  # pragma: no cover
 
 from flow_matching_dit_cosmot_b200 import api as A  # noqa: E402
 from flow_matching_dit_cosmot_b200 import _lib as L  # noqa: E402
-from gpu_helpers import assert_device_ok, bits, device_weights, dims as cdims, layer_parity, layout_spec, to_dev, to_f64  # noqa
+from gpu_helpers import (Guarded, assert_device_ok, bits, device_weights, dims as cdims, layer_parity,  # noqa: E402
+                         layout_spec, to_dev, to_f64)
 
 
 class LayerRun:
@@ -36,12 +37,15 @@ class LayerRun:
                                        self.dlay.chunk, L.COSMOT_MASK_FULL if mode == "full" else L.COSMOT_MASK_BLOCK_CAUSAL)
 
     def gpu(self, h_bits=None, sigma=0.8, sigma_next=0.7):
-        h = to_dev(self.h if h_bits is None else h_bits)
-        h_out = torch.empty_like(h)
-        self.layer.forward(h, h_out, sigma, sigma_next, self.seq)
+        # both buffers sit between canary guard bands: nothing outside them may change
+        h = Guarded(to_dev(self.h if h_bits is None else h_bits))
+        h_out = Guarded(torch.empty_like(h.t))
+        self.layer.forward(h.t, h_out.t, sigma, sigma_next, self.seq)
         torch.cuda.synchronize()
         assert_device_ok()
-        return h, h_out
+        h.assert_canaries("h")
+        h_out.assert_canaries("h_out")
+        return h.t, h_out.t
 
     def gpu_io(self, sigma=0.8, sigma_next=0.7):
         """cosmot_layer_forward_io: the float32 state (taken from h on this first
