@@ -591,6 +591,12 @@ def run_native(args, wl):
 
     h_src = h.clone() if kind == "sampler" else None
     launches_per_step = 2 + n_stage * len(calls) + (2 if kind == "stream" else 0)
+    if kind == "stream" and n_layers == 1:  # a key-split attention adds its merge kernel to every call
+        sd = L.AttnDesc(n_q=lay.n_noisy, q_key_offset=N - lay.n_noisy, n_keys=N, n_ar=lay.n_ar, n_heads=dims_s.n_heads,
+                        n_kv_heads=dims_s.n_kv_heads, head_dim=dims_s.head_dim, mask_mode=mode, batch=B,
+                        flags=L.COSMOT_ATTN_NO_TILE_SKIP)
+        if L.cosmot_attention_kv_split(sd) > 1:
+            launches_per_step += len(calls)
     if n_layers > 1:  # 7 kernels per layer body, 2 for the head (the AR K/V copies are memcpys)
         launches_per_step = 2 + (7 * n_layers + 2) * len(calls)
         if ca:  # the action embedding and the action head; the guided head adds one kernel per pair
@@ -931,6 +937,7 @@ def run_micro(args, wl):
         line["euler_standalone_floor_ms"] = round(6 * nz * d / hbm * 1e3, 4)
         print(json.dumps(line), flush=True)
         return
+    kv_split = 1
     if args.micro == "attention":
         n_q, q_off = T, 0
         if wl.stream is not None and not args.tokens:
@@ -944,10 +951,21 @@ def run_micro(args, wl):
         desc = L.AttnDesc(n_q=n_q, q_key_offset=q_off, n_keys=T, n_ar=n_ar, n_heads=H, n_kv_heads=Hkv, head_dim=hd,
                           mask_mode=L.COSMOT_MASK_FULL, batch=1)
         base = qkv.data_ptr()
+        # the key split the layer would take for this shape (1 = none)
+        kv_split = L.cosmot_attention_kv_split(desc) if q_off else 1
+        split_ws = torch.empty((max(1, L.cosmot_attention_split_workspace(desc, kv_split)),), dtype=torch.uint8,
+                               device=dev)
 
-        def launch():
+        def launch_plain():
             L.cosmot_mot_attention(desc, base + q_off * qkvc * 2, qkvc, base + 2 * H * hd, base + 2 * (H + Hkv) * hd,
                                    qkvc, o.data_ptr(), H * hd, sh)
+
+        def launch():
+            if kv_split == 1:
+                return launch_plain()
+            L.cosmot_mot_attention_split(desc, base + q_off * qkvc * 2, qkvc, base + 2 * H * hd,
+                                         base + 2 * (H + Hkv) * hd, qkvc, o.data_ptr(), H * hd, kv_split,
+                                         split_ws.data_ptr(), split_ws.numel(), sh)
         pairs = (n_ar * (n_ar + 1) // 2 + (T - n_ar) * T) if q_off == 0 else n_q * T
         work, unit, peak = 4 * pairs * H * hd, "TFLOP/s", float(peaks["bf16_tflops"])
     elif args.micro == "gemm":
@@ -989,11 +1007,16 @@ def run_micro(args, wl):
     ms, med = time_launch(launch)
     scale = 1e12 if unit == "TFLOP/s" else 1e9
     achieved = work / (ms / 1e3) / scale
+    extra = {}
+    if args.micro == "attention" and kv_split > 1:
+        ms_plain, _ = time_launch(launch_plain)
+        extra = {"kv_split": kv_split, "ms_unsplit": ms_plain,
+                 "achieved_unsplit": round(work / (ms_plain / 1e3) / scale, 1)}
     print(json.dumps({"micro": args.micro, "workload": wl.name, "tokens": T, "ms": ms, "median_ms": med,
                       "achieved": round(achieved, 1),
                       "unit": unit, "peak": peak, "frac": round(achieved / peak, 3),
                       "peak_source": f"{peak_src} burst", "algorithmic_per_launch": work,
-                      "steps": args.steps, "warmup": args.warmup}), flush=True)
+                      "steps": args.steps, "warmup": args.warmup, **extra}), flush=True)
 
 
 def main():

@@ -118,6 +118,10 @@ SIGNATURES = {
     "cosmot_mrope_apply": (c_i32, [c_vp, c_i64, c_i32, c_vp, c_i64, c_i32, c_i64, c_i32, c_vp, c_vp]),
     "cosmot_mot_attention": (c_i32, [_P(AttnDesc), c_vp, c_i64, c_vp, c_vp, c_i64, c_vp, c_i64, c_vp]),
     "cosmot_mot_mask_export": (c_i32, [_P(AttnDesc), c_vp, c_vp, c_vp]),
+    "cosmot_mot_attention_split": (c_i32, [_P(AttnDesc), c_vp, c_i64, c_vp, c_vp, c_i64, c_vp, c_i64, c_i32, c_vp,
+                                           ctypes.c_size_t, c_vp]),
+    "cosmot_attention_split_workspace": (c_i32, [_P(AttnDesc), c_i32, _P(ctypes.c_size_t)]),
+    "cosmot_attention_kv_split": (c_i32, [_P(AttnDesc)]),
     "cosmot_flow_euler_step": (c_i32, [c_vp, c_i64, c_vp, c_i64, c_i64, c_i64, c_i64, c_f64, c_f64, c_vp]),
     "cosmot_flow_cfg_euler_step": (c_i32, [c_vp, c_vp, c_i64, c_vp, c_vp, c_i64, c_i64, c_i64, c_f64, c_f64, c_f64,
                                            c_vp]),
@@ -283,6 +287,22 @@ def cosmot_mot_attention(desc: AttnDesc, q: int, ld_q: int, k: int, v: int, ld_k
                          stream: int = 0, check=True):
     return _call("cosmot_mot_attention", ctypes.byref(desc), c_vp(q), ld_q, c_vp(k), c_vp(v), ld_kv, c_vp(o), ld_o,
                  c_vp(stream), check=check)
+
+
+def cosmot_mot_attention_split(desc: AttnDesc, q: int, ld_q: int, k: int, v: int, ld_kv: int, o: int, ld_o: int,
+                               kv_split: int, workspace: int, workspace_bytes: int, stream: int = 0, check=True):
+    return _call("cosmot_mot_attention_split", ctypes.byref(desc), c_vp(q), ld_q, c_vp(k), c_vp(v), ld_kv, c_vp(o),
+                 ld_o, kv_split, c_vp(workspace or None), workspace_bytes, c_vp(stream), check=check)
+
+
+def cosmot_attention_split_workspace(desc: AttnDesc, kv_split: int) -> int:
+    n = ctypes.c_size_t(0)
+    _call("cosmot_attention_split_workspace", ctypes.byref(desc), kv_split, ctypes.byref(n))
+    return n.value
+
+
+def cosmot_attention_kv_split(desc: AttnDesc) -> int:
+    return lib().cosmot_attention_kv_split(ctypes.byref(desc))
 
 
 def cosmot_mot_mask_export(desc: AttnDesc, tile_codes: int, visible: int = 0, stream: int = 0, check=True):

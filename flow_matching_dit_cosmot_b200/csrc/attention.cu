@@ -71,6 +71,7 @@ constexpr float kRescaleThreshold = 8.0f;  // log2 units
 // visit list is a bitmask in shared memory (one bit per 128-key tile).
 constexpr int kMaxVisitWords = 2048;
 constexpr int64_t kMaxVisitTiles = (int64_t)kMaxVisitWords * 32;
+constexpr int32_t kMaxKvSplit = 8;
 
 template <int HD>
 struct Cfg {
@@ -96,6 +97,12 @@ struct Params {
   const int32_t* chunk;
   __nv_bfloat16* o;
   int64_t ld_o;
+  // Key split of the DM items (kv_split > 1): split s of an item visits key
+  // tiles [s n_kt / kv_split, (s + 1) n_kt / kv_split) and writes its O / l in
+  // float32 with its running max and sum; attn_merge_kernel combines the splits.
+  int32_t kv_split;
+  float* part_o;    // [kv_split][batch][n_q][n_heads * HD]
+  float2* part_ml;  // [kv_split][batch][n_q][n_heads]: (running max, sum)
   int* status;
 };
 
@@ -104,17 +111,22 @@ struct Work {
   bool is_ar;
   int64_t row0;     // first query row of tile 0
   int64_t seg_end;  // query rows >= seg_end are not in this segment
-  int32_t n_kt;     // key tiles to visit
+  int32_t n_kt;     // key tiles of the item (before any key split)
+  int32_t split;    // key split of a DM item (0 when unsplit)
+  int32_t kt0, kt1; // key tiles [kt0, kt1) this CTA visits
 };
 
 __device__ __forceinline__ Work decode_work(const Params& p) {
   Work w;
   int64_t bid = blockIdx.x;
-  const int64_t items_dm = (int64_t)p.batch * p.n_heads * p.dm_pairs;
+  const int64_t items_dm = (int64_t)p.batch * p.n_heads * p.dm_pairs * p.kv_split;
   int32_t pairs;
+  w.split = 0;
   if (bid < items_dm) {
     w.is_ar = false;
     pairs = p.dm_pairs;
+    w.split = (int32_t)(bid % p.kv_split);
+    bid /= p.kv_split;
   } else {
     bid -= items_dm;
     w.is_ar = true;
@@ -136,6 +148,8 @@ __device__ __forceinline__ Work decode_work(const Params& p) {
     w.seg_end = p.n_q;
     w.n_kt = (int32_t)((p.n_keys + BKV - 1) / BKV);
   }
+  w.kt0 = (int32_t)((int64_t)w.split * w.n_kt / p.kv_split);
+  w.kt1 = w.is_ar ? w.n_kt : (int32_t)((int64_t)(w.split + 1) * w.n_kt / p.kv_split);
   return w;
 }
 
@@ -294,6 +308,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   tc_fence_after();
   const uint32_t tmem_base = *reinterpret_cast<volatile uint32_t*>(tmem_slot);
   const int32_t n_kt = w.n_kt;
+  const int32_t kt_begin = w.kt0, kt_end = w.kt1;  // this CTA's key tiles
   if (use_visit) {
     // Nothing to skip (a streaming block sees every cached key): walk the
     // tiles plainly.  Every thread reads the same words, so this stays uniform.
@@ -320,8 +335,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       const int kvrow = (int)(w.b * p.kv_bstride);
       // Load L = 2j (K) and 2j + 1 (V) of the j-th visited key tile.
       bool ok = true;
-      for (int32_t kt = next_visit(visit, use_visit, 0, n_kt), L = 0; kt < n_kt && ok;
-           kt = next_visit(visit, use_visit, kt + 1, n_kt)) {
+      for (int32_t kt = next_visit(visit, use_visit, kt_begin, kt_end), L = 0; kt < kt_end && ok;
+           kt = next_visit(visit, use_visit, kt + 1, kt_end)) {
         for (int kv = 0; kv < 2; ++kv, ++L) {
           const int slot = L % SLOTS;
           const uint32_t par = (L / SLOTS) & 1;
@@ -387,11 +402,11 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         umma_commit(bar_kv_empty + 8 * 0);
       }
       // j counts visited key tiles; kt is the j-th one.
-      int32_t kt = next_visit(visit, use_visit, 0, n_kt);
-      for (int j = 0; kt < n_kt && ok; ++j) {
-        const int32_t kt_next = next_visit(visit, use_visit, kt + 1, n_kt);
+      int32_t kt = next_visit(visit, use_visit, kt_begin, kt_end);
+      for (int j = 0; kt < kt_end && ok; ++j) {
+        const int32_t kt_next = next_visit(visit, use_visit, kt + 1, kt_end);
         const int LV = 2 * j + 1, LK = 2 * j + 2;
-        const bool has_next = kt_next < n_kt;
+        const bool has_next = kt_next < kt_end;
         const uint32_t par = j & 1;
         // Order of the softmax events in steady state: tile 0 half, tile 0
         // full, tile 1 half, tile 1 full (tile 1 runs about half a block later).
@@ -450,8 +465,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     bool ok = true;
     // j counts visited key tiles (it sets the barrier phases); kt is the j-th.
     int j = 0;
-    for (int32_t kt = next_visit(visit, use_visit, 0, n_kt); kt < n_kt;
-         kt = next_visit(visit, use_visit, kt + 1, n_kt), ++j) {
+    for (int32_t kt = next_visit(visit, use_visit, kt_begin, kt_end); kt < kt_end;
+         kt = next_visit(visit, use_visit, kt + 1, kt_end), ++j) {
       const int64_t kbase = (int64_t)kt * BKV;
       // Block-causal rows need element masks only where the tile holds a DM
       // key of a later chunk.  The warp reads the tile's 128 chunk ids (AR keys
@@ -548,6 +563,26 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     if (ok && __all_sync(0xffffffffu, mbar_wait(bar_o_done + 8 * t, 0, p.status, kWhereAttnSoftmax))) {
       tc_fence_after();
       const float inv_l = l > 0.f ? 1.0f / l : 0.f;
+      if (p.kv_split > 1 && !w.is_ar) {
+        // one key split of the row: O / l in float32 with (running max, sum)
+        const int64_t prow = ((int64_t)w.split * p.batch + w.b) * p.n_q + qi;
+        float* pdst = p.part_o + prow * ((int64_t)p.n_heads * HD) + (int64_t)w.h * HD;
+        const bool store = valid && dcheck(qi < p.n_q && w.split < p.kv_split, p.status, kWhereAttnStore);
+        if (store) p.part_ml[prow * p.n_heads + w.h] = make_float2(m, l);
+#pragma unroll 1
+        for (int c = 0; c < HD / 32; ++c) {
+          uint32_t ov[32];
+          tmem_ld32(o_addr + 32 * c, ov);
+          tmem_ld_wait();
+          if (store) {
+#pragma unroll
+            for (int q4 = 0; q4 < 8; ++q4)
+              *reinterpret_cast<float4*>(pdst + 32 * c + 4 * q4) =
+                  make_float4(__uint_as_float(ov[4 * q4]) * inv_l, __uint_as_float(ov[4 * q4 + 1]) * inv_l,
+                              __uint_as_float(ov[4 * q4 + 2]) * inv_l, __uint_as_float(ov[4 * q4 + 3]) * inv_l);
+          }
+        }
+      } else {
       __nv_bfloat16* dst = p.o + (w.b * p.o_bstride + qi) * p.ld_o + (int64_t)w.h * HD;
 #pragma unroll 1
       for (int c = 0; c < HD / 32; ++c) {
@@ -565,6 +600,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             *reinterpret_cast<uint4*>(dst + 32 * c + 8 * q4) = v4;
           }
         }
+      }
       }
     }
   }
@@ -607,7 +643,7 @@ namespace attn {
 
 // Descriptor checks and kernel parameters shared by the attention entry point
 // and the mask export.
-cosmot_status make_params(const cosmot_attn_desc* d, Params& p, int64_t& grid) {
+cosmot_status make_params(const cosmot_attn_desc* d, Params& p, int64_t& grid, int32_t kv_split = 1) {
   if (!d) return COSMOT_ERR_INVALID_ARG;
   const int hd = d->head_dim;
   if (hd != 64 && hd != 128) return COSMOT_ERR_UNSUPPORTED;
@@ -646,7 +682,8 @@ cosmot_status make_params(const cosmot_attn_desc* d, Params& p, int64_t& grid) {
   p.skip = d->mask_mode == COSMOT_MASK_BLOCK_CAUSAL && !(d->flags & COSMOT_ATTN_NO_TILE_SKIP);
   p.status = device_status_ptr();
   if (!p.status) return COSMOT_ERR_CUDA;
-  grid = (int64_t)d->batch * d->n_heads * (p.ar_pairs + p.dm_pairs);
+  p.kv_split = kv_split;
+  grid = (int64_t)d->batch * d->n_heads * (p.ar_pairs + (int64_t)p.dm_pairs * kv_split);
   if (grid > INT32_MAX) return COSMOT_ERR_UNSUPPORTED;
   return COSMOT_OK;
 }
@@ -692,20 +729,111 @@ __global__ void __launch_bounds__(2 * BQ) mask_export_kernel(const __grid_consta
 }  // namespace attn
 }  // namespace cosmot
 
-extern "C" cosmot_status cosmot_mot_attention(const cosmot_attn_desc* d, const void* q, int64_t ld_q, const void* k,
-                                              const void* v, int64_t ld_kv, void* o, int64_t ld_o,
-                                              cosmot_stream_t stream) {
-  using namespace cosmot;
+namespace cosmot {
+namespace attn {
+
+// Combines the key splits of every (sequence, query row, head): with M the
+// largest running max, weights w_s = l_s 2^(m_s - M) and O = sum_s w_s O_s /
+// sum_s w_s, summed in split order (deterministic).  One warp per row and head,
+// each lane HD/32 columns; a row no split saw (every w_s = 0) outputs 0.
+template <int HD>
+__global__ void __launch_bounds__(256) attn_merge_kernel(const Params p) {
+  const int64_t warp = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const int lane = threadIdx.x & 31;
+  const int64_t total = (int64_t)p.batch * (p.n_q - p.n_q_ar) * p.n_heads;
+  if (warp >= total) return;
+  const int32_t h = (int32_t)(warp % p.n_heads);
+  const int64_t rb = warp / p.n_heads;              // (sequence, DM query row)
+  const int32_t b = (int32_t)(rb / (p.n_q - p.n_q_ar));
+  const int64_t qi = p.n_q_ar + rb % (p.n_q - p.n_q_ar);
+  float mmax = -INFINITY;
+  for (int s = 0; s < p.kv_split; ++s) {
+    const float2 ml = p.part_ml[(((int64_t)s * p.batch + b) * p.n_q + qi) * p.n_heads + h];
+    if (ml.y > 0.f) mmax = fmaxf(mmax, ml.x);
+  }
+  constexpr int C = HD / 32;
+  float acc[C];
+#pragma unroll
+  for (int c = 0; c < C; ++c) acc[c] = 0.f;
+  float wsum = 0.f;
+  for (int s = 0; s < p.kv_split; ++s) {
+    const int64_t prow = ((int64_t)s * p.batch + b) * p.n_q + qi;
+    const float2 ml = p.part_ml[prow * p.n_heads + h];
+    if (!(ml.y > 0.f)) continue;
+    const float wgt = ml.y * ex2_approx(ml.x - mmax);
+    wsum += wgt;
+    const float* src = p.part_o + prow * ((int64_t)p.n_heads * HD) + (int64_t)h * HD + lane * C;
+#pragma unroll
+    for (int c = 0; c < C; ++c) acc[c] = fmaf(wgt, src[c], acc[c]);
+  }
+  const float inv = wsum > 0.f ? 1.0f / wsum : 0.f;
+  if (!dcheck(qi < p.n_q && b < p.batch, p.status, kWhereAttnStore)) return;
+  __nv_bfloat16* dst = p.o + (b * p.o_bstride + qi) * p.ld_o + (int64_t)h * HD + lane * C;
+#pragma unroll
+  for (int c = 0; c < C; c += 2) *reinterpret_cast<uint32_t*>(dst + c) = pack_bf16x2(acc[c] * inv, acc[c + 1] * inv);
+}
+
+// Bytes of the float32 partials of a key-split attention call.
+size_t split_workspace_bytes(const cosmot_attn_desc* d, int32_t kv_split) {
+  const int64_t rows = (int64_t)d->batch * d->n_q;
+  return (size_t)kv_split * rows * d->n_heads * (size_t)d->head_dim * 4 + 256 +
+         (size_t)kv_split * rows * d->n_heads * 8;
+}
+
+}  // namespace attn
+
+int32_t attention_kv_split(int64_t dm_items, int64_t n_keys) {
+  const int64_t n_kt = (n_keys + 127) / 128;
+  const int64_t sms = num_sms();
+  if (dm_items <= 0) return 1;
+  auto eff = [&](int64_t s) {
+    const int64_t u = dm_items * s;
+    return (double)u / (double)(((u + sms - 1) / sms) * sms);
+  };
+  int32_t best = 1;
+  for (int32_t s = 2; s <= 4 && s * 8 <= n_kt; ++s)
+    if (eff(s) > eff(best) + 0.05) best = s;
+  return best;
+}
+
+}  // namespace cosmot
+
+extern "C" cosmot_status cosmot_attention_split_workspace(const cosmot_attn_desc* d, int32_t kv_split, size_t* bytes) {
   using namespace cosmot::attn;
+  if (!d || !bytes || kv_split < 1 || kv_split > kMaxKvSplit || d->batch < 1 || d->n_q < 0 || d->n_heads < 1 ||
+      (d->head_dim != 64 && d->head_dim != 128))
+    return COSMOT_ERR_INVALID_ARG;
+  *bytes = kv_split == 1 ? 0 : split_workspace_bytes(d, kv_split);
+  return COSMOT_OK;
+}
+
+namespace cosmot {
+namespace attn {
+
+cosmot_status attention_impl(const cosmot_attn_desc* d, const void* q, int64_t ld_q, const void* k, const void* v,
+                             int64_t ld_kv, void* o, int64_t ld_o, int32_t kv_split, void* workspace,
+                             size_t workspace_bytes, cosmot_stream_t stream) {
   if (!d || !q || !k || !v || !o) return COSMOT_ERR_INVALID_ARG;
+  if (kv_split < 1 || kv_split > kMaxKvSplit) return COSMOT_ERR_INVALID_ARG;
   Params p;
   int64_t grid = 0;
-  cosmot_status st = make_params(d, p, grid);
+  cosmot_status st = make_params(d, p, grid, kv_split);
   if (st != COSMOT_OK) return st;
   const int hd = d->head_dim;
   const int64_t qcols = (int64_t)d->n_heads * hd, kvcols = (int64_t)d->n_kv_heads * hd;
   if (ld_q < qcols || ld_kv < kvcols || ld_o < qcols || ld_q % 8 || ld_kv % 8 || ld_o % 8) return COSMOT_ERR_INVALID_ARG;
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o)) return COSMOT_ERR_INVALID_ARG;
+  if (kv_split > 1) {
+    // every split must visit at least one key tile: no tile skipping, and at
+    // least kv_split key tiles
+    if (p.skip) return COSMOT_ERR_UNSUPPORTED;
+    if ((d->n_keys + BKV - 1) / BKV < kv_split) return COSMOT_ERR_INVALID_ARG;
+    if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u)) return COSMOT_ERR_INVALID_ARG;
+    if (workspace_bytes < split_workspace_bytes(d, kv_split)) return COSMOT_ERR_WORKSPACE;
+    const size_t o_bytes = ((size_t)kv_split * d->batch * d->n_q * d->n_heads * (size_t)hd * 4 + 255) & ~size_t(255);
+    p.part_o = static_cast<float*>(workspace);
+    p.part_ml = reinterpret_cast<float2*>(static_cast<uint8_t*>(workspace) + o_bytes);
+  }
   if (d->n_q == 0) return COSMOT_OK;
   p.o = static_cast<__nv_bfloat16*>(o);
   p.ld_o = ld_o;
@@ -725,8 +853,42 @@ extern "C" cosmot_status cosmot_mot_attention(const cosmot_attn_desc* d, const v
   if (p.skip)
     return hd == 128 ? launch<128, true>(tq, tk, tv, p, (unsigned)grid, s)
                      : launch<64, true>(tq, tk, tv, p, (unsigned)grid, s);
-  return hd == 128 ? launch<128, false>(tq, tk, tv, p, (unsigned)grid, s)
-                   : launch<64, false>(tq, tk, tv, p, (unsigned)grid, s);
+  st = hd == 128 ? launch<128, false>(tq, tk, tv, p, (unsigned)grid, s)
+                 : launch<64, false>(tq, tk, tv, p, (unsigned)grid, s);
+  if (st != COSMOT_OK || kv_split == 1 || d->n_q == p.n_q_ar) return st;
+  const int64_t warps = (int64_t)d->batch * (d->n_q - p.n_q_ar) * d->n_heads;
+  const unsigned mgrid = (unsigned)((warps + 7) / 8);
+  if (hd == 128)
+    attn_merge_kernel<128><<<mgrid, 256, 0, s>>>(p);
+  else
+    attn_merge_kernel<64><<<mgrid, 256, 0, s>>>(p);
+  return launch_status();
+}
+
+}  // namespace attn
+}  // namespace cosmot
+
+extern "C" cosmot_status cosmot_mot_attention(const cosmot_attn_desc* d, const void* q, int64_t ld_q, const void* k,
+                                              const void* v, int64_t ld_kv, void* o, int64_t ld_o,
+                                              cosmot_stream_t stream) {
+  return cosmot::attn::attention_impl(d, q, ld_q, k, v, ld_kv, o, ld_o, 1, nullptr, 0, stream);
+}
+
+extern "C" cosmot_status cosmot_mot_attention_split(const cosmot_attn_desc* d, const void* q, int64_t ld_q,
+                                                    const void* k, const void* v, int64_t ld_kv, void* o,
+                                                    int64_t ld_o, int32_t kv_split, void* workspace,
+                                                    size_t workspace_bytes, cosmot_stream_t stream) {
+  return cosmot::attn::attention_impl(d, q, ld_q, k, v, ld_kv, o, ld_o, kv_split, workspace, workspace_bytes,
+                                      stream);
+}
+
+extern "C" int32_t cosmot_attention_kv_split(const cosmot_attn_desc* d) {
+  if (!d || d->batch < 1 || d->n_heads < 1 || d->n_q < 0 || d->n_keys < 1) return 1;
+  if (d->mask_mode == COSMOT_MASK_BLOCK_CAUSAL && !(d->flags & COSMOT_ATTN_NO_TILE_SKIP)) return 1;
+  const int64_t nqar0 = d->n_ar - d->q_key_offset;
+  const int64_t nqar = nqar0 < 0 ? 0 : (nqar0 > d->n_q ? d->n_q : nqar0);
+  const int64_t dm_pairs = ((d->n_q - nqar + 127) / 128 + 1) / 2;
+  return cosmot::attention_kv_split((int64_t)d->batch * d->n_heads * dm_pairs, d->n_keys);
 }
 
 extern "C" cosmot_status cosmot_mot_mask_export(const cosmot_attn_desc* d, uint8_t* tile_codes, uint8_t* visible,

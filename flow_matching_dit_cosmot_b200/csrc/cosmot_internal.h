@@ -50,6 +50,10 @@ cosmot_status rmsnorm_routed(const void* h, bool h_f32, int64_t ld_h, const cosm
                              const void* g0, const void* g1, int64_t d, float eps, void* out, int64_t ld_out,
                              cosmot_stream_t stream);
 
+// Key split of an attention call with dm_items DM work items (sequences x
+// heads x query-tile pairs) over n_keys keys (see cosmot_attention_kv_split).
+int32_t attention_kv_split(int64_t dm_items, int64_t n_keys);
+
 // Per-device address of the status word that kernels latch failures into.
 int* device_status_ptr();
 

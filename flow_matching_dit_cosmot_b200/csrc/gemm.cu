@@ -33,18 +33,26 @@ namespace cosmot {
 namespace gemm {
 
 constexpr int BM = 128;
-constexpr int BN = 256;
 constexpr int BK = 64;  // 64 bf16 = 128 bytes = one swizzle row
 constexpr int STAGES = 4;
 constexpr int A_BYTES = BM * BK * 2;
-constexpr int B_BYTES = BN * BK * 2;
-constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
 constexpr int NUM_THREADS = 192;
 constexpr int TMEM_COLS = 512;
 constexpr int kMaxSegs = 64;
 constexpr int kGroupM = 16;
-constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 256 + 1024;
-constexpr uint32_t IDESC = idesc_bf16_f32(BM, BN, false, false);
+
+// Tile width BN: 256 by default; 160 where a call has too few output tiles to
+// fill the SMs with 256-wide ones (a few hundred rows against a 4096-wide
+// output: 5 row tiles x 16 column tiles = 80 tiles for 148 SMs become 5 x 26
+// = 130).  Any multiple of 32 up to 256 is a valid tcgen05 N for M = 128.
+template <int BN>
+struct Tiles {
+  static_assert(BN % 32 == 0 && BN >= 32 && BN <= 256, "tile width");
+  static constexpr int B_BYTES = BN * BK * 2;
+  static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+  static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 256 + 1024;
+  static constexpr uint32_t IDESC = idesc_bf16_f32(BM, BN, false, false);
+};
 
 struct Params {
   int64_t row_begin[kMaxSegs];
@@ -161,12 +169,17 @@ __device__ __forceinline__ void load_row32(const __nv_bfloat16* src, int32_t col
   }
 }
 
-// FL: COSMOT_EPI_OUT_F32 / COSMOT_EPI_RES_F32 bits of the RESIDUAL epilogue.
-template <int EPI, int FL>
+// FL: COSMOT_EPI_OUT_F32 / COSMOT_EPI_RES_F32 bits of the RESIDUAL epilogue;
+// BN: the tile width.
+template <int EPI, int FL, int BN>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
     routed_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUtensorMap tmap_b0,
                        const __grid_constant__ CUtensorMap tmap_b1, const __grid_constant__ CUtensorMap tmap_u0,
                        const __grid_constant__ CUtensorMap tmap_u1, const __grid_constant__ Params p) {
+  using T = Tiles<BN>;
+  constexpr int B_BYTES = T::B_BYTES;
+  constexpr int STAGE_BYTES = T::STAGE_BYTES;
+  constexpr uint32_t IDESC = T::IDESC;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const uint32_t sbase = smem_u32(smem);
@@ -349,6 +362,13 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           const bool rotate = hcol < p.rope_cols;
 #pragma unroll 1
           for (int i0 = 0; i0 < half; i0 += 32) {
+            // the row's (cos, sin) of pairs i0 .. i0 + 31, requested before the
+            // accumulator loads so that their latency overlaps
+            float4 csv[16];
+            if (valid && rotate) {
+#pragma unroll
+              for (int j = 0; j < 16; ++j) csv[j] = __ldg(reinterpret_cast<const float4*>(cs_row + i0 + 2 * j));
+            }
             uint32_t u[32];
             tmem_ld32(tacc + hb * hd + i0, v);
             tmem_ld32(tacc + hb * hd + half + i0, u);
@@ -358,7 +378,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
               if (rotate) {
 #pragma unroll
                 for (int j = 0; j < 32; j += 2) {
-                  const float4 cs = __ldg(reinterpret_cast<const float4*>(cs_row + i0 + j));
+                  const float4 cs = csv[j >> 1];
                   const float a0 = __uint_as_float(v[j]), a1 = __uint_as_float(v[j + 1]);
                   const float b0 = __uint_as_float(u[j]), b1 = __uint_as_float(u[j + 1]);
                   lo[j] = a0 * cs.x - b0 * cs.y;
@@ -434,9 +454,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   if (warp == 1) tmem_dealloc(tmem_base, TMEM_COLS);
 }
 
-template <int EPI, int FL = 0>
+template <int EPI, int FL = 0, int BN = 256>
 cosmot_status launch(const CUtensorMap& ta, const CUtensorMap& tb0, const CUtensorMap& tb1, const CUtensorMap& tu0,
                      const CUtensorMap& tu1, const Params& p, cudaStream_t s) {
+  constexpr int SMEM_BYTES = Tiles<BN>::SMEM_BYTES;
   static std::mutex mu;
   static uint64_t done_mask = 0;  // devices whose smem limit was raised
   int dev = 0;
@@ -444,7 +465,8 @@ cosmot_status launch(const CUtensorMap& ta, const CUtensorMap& tb0, const CUtens
   {
     std::lock_guard<std::mutex> lk(mu);
     if (dev >= 64 || !(done_mask & (1ull << dev))) {
-      if (cudaFuncSetAttribute(routed_gemm_kernel<EPI, FL>, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES) !=
+      if (cudaFuncSetAttribute(routed_gemm_kernel<EPI, FL, BN>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               SMEM_BYTES) !=
           cudaSuccess)
         return COSMOT_ERR_CUDA;
       if (dev < 64) done_mask |= 1ull << dev;
@@ -452,7 +474,7 @@ cosmot_status launch(const CUtensorMap& ta, const CUtensorMap& tb0, const CUtens
   }
   int grid = num_sms();
   if (p.num_tiles < grid) grid = p.num_tiles;
-  routed_gemm_kernel<EPI, FL><<<grid, NUM_THREADS, SMEM_BYTES, s>>>(ta, tb0, tb1, tu0, tu1, p);
+  routed_gemm_kernel<EPI, FL, BN><<<grid, NUM_THREADS, SMEM_BYTES, s>>>(ta, tb0, tb1, tu0, tu1, p);
   return launch_status();
 }
 
@@ -506,7 +528,19 @@ extern "C" cosmot_status cosmot_routed_linear(const void* a, int64_t ld_a, int64
   if (mt == 0) return COSMOT_OK;
   if (max_row > INT32_MAX) return COSMOT_ERR_UNSUPPORTED;
   const bool silu = kind == COSMOT_EPI_SILU_MUL;
-  p.num_n_tiles = (int32_t)((n_out + (silu ? BN / 2 : BN) - 1) / (silu ? BN / 2 : BN));
+  // Tile width: 160 instead of 256 when that keeps clearly more SMs busy over
+  // the waves of tiles (mRoPE needs whole heads in a tile, SiLU*mul a gate and
+  // an up half: both keep 256).
+  int bn = 256;
+  if (kind == COSMOT_EPI_NONE || kind == COSMOT_EPI_RESIDUAL || kind == COSMOT_EPI_EULER) {
+    const int64_t sms = num_sms();
+    auto eff = [&](int64_t w) {
+      const int64_t t = (int64_t)mt * ((n_out + w - 1) / w);
+      return (double)t / (double)(((t + sms - 1) / sms) * sms);
+    };
+    if (eff(160) > eff(256) + 0.1) bn = 160;
+  }
+  p.num_n_tiles = (int32_t)((n_out + (silu ? bn / 2 : bn) - 1) / (silu ? bn / 2 : bn));
   if ((int64_t)p.num_m_tiles * p.num_n_tiles > INT32_MAX) return COSMOT_ERR_UNSUPPORTED;
   p.num_tiles = p.num_m_tiles * p.num_n_tiles;
   p.num_kb = (int32_t)((k + BK - 1) / BK);
@@ -554,7 +588,7 @@ extern "C" cosmot_status cosmot_routed_linear(const void* a, int64_t ld_a, int64
   if (st != COSMOT_OK) return st;
   const void* wb[2] = {w0, w1};
   const void* wu[2] = {w0_up, w1_up};
-  const uint32_t brows = silu ? BN / 2 : BN;
+  const uint32_t brows = silu ? bn / 2 : bn;
   for (int s = 0; s < 2; ++s) {
     const int src = uses[s] ? s : (uses[0] ? 0 : 1);  // an unused set reuses a valid map
     if (!wb[src]) return COSMOT_ERR_INVALID_ARG;
@@ -569,6 +603,23 @@ extern "C" cosmot_status cosmot_routed_linear(const void* a, int64_t ld_a, int64
     }
   }
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (bn == 160) {
+    switch (kind) {
+      case COSMOT_EPI_NONE: return launch<COSMOT_EPI_NONE, 0, 160>(ta, tb[0], tb[1], tu[0], tu[1], p, s);
+      case COSMOT_EPI_EULER: return launch<COSMOT_EPI_EULER, 0, 160>(ta, tb[0], tb[1], tu[0], tu[1], p, s);
+      default:
+        switch (flags) {
+          case COSMOT_EPI_OUT_F32:
+            return launch<COSMOT_EPI_RESIDUAL, COSMOT_EPI_OUT_F32, 160>(ta, tb[0], tb[1], tu[0], tu[1], p, s);
+          case COSMOT_EPI_RES_F32:
+            return launch<COSMOT_EPI_RESIDUAL, COSMOT_EPI_RES_F32, 160>(ta, tb[0], tb[1], tu[0], tu[1], p, s);
+          case COSMOT_EPI_OUT_F32 | COSMOT_EPI_RES_F32:
+            return launch<COSMOT_EPI_RESIDUAL, COSMOT_EPI_OUT_F32 | COSMOT_EPI_RES_F32, 160>(ta, tb[0], tb[1], tu[0],
+                                                                                          tu[1], p, s);
+          default: return launch<COSMOT_EPI_RESIDUAL, 0, 160>(ta, tb[0], tb[1], tu[0], tu[1], p, s);
+        }
+    }
+  }
   switch (kind) {
     case COSMOT_EPI_NONE: return launch<COSMOT_EPI_NONE>(ta, tb[0], tb[1], tu[0], tu[1], p, s);
     case COSMOT_EPI_RESIDUAL:

@@ -29,7 +29,8 @@ namespace {
 constexpr int kMaxBatch = 32;
 
 struct WsLayout {
-  size_t a, qkv, o, h1, u, total;
+  size_t a, qkv, o, h1, u, part, part_bytes, total;
+  int32_t kv_split;  // key split of a streaming-style call (queries = the noisy rows)
 };
 
 size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
@@ -72,6 +73,25 @@ int make_segments(const cosmot_seq_desc& S, int64_t lo, int64_t out_shift, cosmo
   return ns;
 }
 
+// The attention of a call that computes only the noisy rows of each sequence.
+cosmot_attn_desc stream_attn_desc(const cosmot_dims& d, const cosmot_seq_desc& s) {
+  const int64_t N = (int64_t)s.n_ar + s.n_clean + s.n_noisy;
+  cosmot_attn_desc ad{};
+  ad.n_q = s.n_noisy;
+  ad.q_key_offset = N - s.n_noisy;
+  ad.n_keys = N;
+  ad.n_ar = s.n_ar;
+  ad.n_heads = d.n_heads;
+  ad.n_kv_heads = d.n_kv_heads;
+  ad.head_dim = d.head_dim;
+  ad.mask_mode = s.mask_mode;
+  ad.chunk = s.chunk;
+  ad.batch = s.batch;
+  ad.flags = COSMOT_ATTN_NO_TILE_SKIP;
+  ad.q_batch_stride = ad.kv_batch_stride = ad.o_batch_stride = N;
+  return ad;
+}
+
 WsLayout ws_layout(const cosmot_dims& d, const cosmot_seq_desc& s) {
   const size_t rows = (size_t)s.batch * (size_t)(s.n_ar + s.n_clean + s.n_noisy);
   const size_t qkv_cols = (size_t)(d.n_heads + 2 * d.n_kv_heads) * d.head_dim;
@@ -84,6 +104,15 @@ WsLayout ws_layout(const cosmot_dims& d, const cosmot_seq_desc& s) {
   w.o = off;   off += align256(rows * q_cols * 2);
   w.h1 = off;  off += align256(rows * d.d_model * 4);  // float32: the residual stream between the two halves
   w.u = off;   off += align256(rows * d.ffn * 2);
+  // A call whose queries are the noisy rows alone (a streaming step: the AR
+  // rows and the cache are the n_cached prefix) may split its keys across
+  // CTAs to fill the SMs; its float32 partials live here.
+  cosmot_attn_desc ad = stream_attn_desc(d, s);
+  w.kv_split = s.n_noisy > 0 ? cosmot_attention_kv_split(&ad) : 1;
+  w.part_bytes = 0;
+  if (w.kv_split > 1) cosmot_attention_split_workspace(&ad, w.kv_split, &w.part_bytes);
+  w.part = off;
+  off += align256(w.part_bytes);
   w.total = off;
   return w;
 }
@@ -183,11 +212,17 @@ cosmot_status layer_body(const cosmot_dims& D, const cosmot_layer_weights* w, co
   ad.batch = B;
   // A streaming step's queries are its newest block; its cache holds earlier
   // chunks only, so no key tile is hidden from every query.
-  if (c0 >= (int64_t)S.n_ar + S.n_clean && S.n_noisy > 0) ad.flags = COSMOT_ATTN_NO_TILE_SKIP;
+  const bool noisy_only = c0 == (int64_t)S.n_ar + S.n_clean && S.n_noisy > 0;
+  if (noisy_only) ad.flags = COSMOT_ATTN_NO_TILE_SKIP;
   ad.q_batch_stride = ad.kv_batch_stride = ad.o_batch_stride = N;
   uint16_t* qkvp = static_cast<uint16_t*>(qkv);
-  st = cosmot_mot_attention(&ad, qkvp + c0 * qkvc, qkvc, qkvp + qc, qkvp + qc + kvc, qkvc,
-                            static_cast<uint16_t*>(o) + c0 * qc, qc, stream);
+  if (noisy_only && L.kv_split > 1)  // few query tiles: split the keys to fill the SMs
+    st = cosmot_mot_attention_split(&ad, qkvp + c0 * qkvc, qkvc, qkvp + qc, qkvp + qc + kvc, qkvc,
+                                    static_cast<uint16_t*>(o) + c0 * qc, qc, L.kv_split, ws + L.part, L.part_bytes,
+                                    stream);
+  else
+    st = cosmot_mot_attention(&ad, qkvp + c0 * qkvc, qkvc, qkvp + qc, qkvp + qc + kvc, qkvc,
+                              static_cast<uint16_t*>(o) + c0 * qc, qc, stream);
   if (st != COSMOT_OK) return st;
   if ((st = M.mark(3)) != COSMOT_OK) return st;
   // 4. output projection + residual; h1 stays in float32 (it is read twice more:

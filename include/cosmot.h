@@ -292,6 +292,33 @@ COSMOT_API cosmot_status cosmot_mot_attention(const cosmot_attn_desc* desc, cons
                                    const void* v, int64_t ld_kv, void* o, int64_t ld_o, cosmot_stream_t stream);
 
 /*
+ * cosmot_mot_attention with the keys of every DM query item split kv_split
+ * ways (1..8) across CTAs: split s of an item visits key tiles [s n_kt /
+ * kv_split, (s + 1) n_kt / kv_split) of n_kt = ceil(n_keys / 128), writes its
+ * O / l in float32 to the workspace with its running max m_s and sum l_s, and
+ * a second kernel combines them in split order: O = sum_s w_s O_s / sum_s w_s,
+ * w_s = l_s 2^(m_s - max m).  Fills the SMs when a call has few query tiles (a
+ * streaming step's single block); AR query items are not split.  Results equal
+ * cosmot_mot_attention's up to the summation order of the softmax sums.
+ * Requires no tile skipping (FULL mask, or COSMOT_ATTN_NO_TILE_SKIP) and
+ * kv_split <= n_kt (else UNSUPPORTED / INVALID_ARG); workspace: device, 256-byte
+ * aligned, cosmot_attention_split_workspace bytes (WORKSPACE if shorter).
+ */
+COSMOT_API cosmot_status cosmot_mot_attention_split(const cosmot_attn_desc* desc, const void* q, int64_t ld_q,
+                                                    const void* k, const void* v, int64_t ld_kv, void* o,
+                                                    int64_t ld_o, int32_t kv_split, void* workspace,
+                                                    size_t workspace_bytes, cosmot_stream_t stream);
+/* Workspace bytes of cosmot_mot_attention_split (0 for kv_split = 1); host only. */
+COSMOT_API cosmot_status cosmot_attention_split_workspace(const cosmot_attn_desc* desc, int32_t kv_split,
+                                                          size_t* bytes);
+/* The key split the layer uses for this call shape: among 1..4 (with at least
+ * 8 key tiles a split), the one that keeps the SMs busiest over the waves of
+ * DM work items, taken only when it beats no split by more than 5 points.  It
+ * depends on the batch, heads, DM query tiles, key count and the device's SM
+ * count only. */
+COSMOT_API int32_t cosmot_attention_kv_split(const cosmot_attn_desc* desc);
+
+/*
  * Debug export of the masking decisions cosmot_mot_attention takes for the
  * same descriptor (sequence 0; they depend on neither the sequence nor the
  * head).  The pages define the mask only element by element (the §3 equations);

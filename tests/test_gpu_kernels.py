@@ -354,7 +354,7 @@ def test_euler_sampler_lands_on_x0():
 
 # ---------------------------------------------------------------- attention
 
-def _attn_case(n_keys, n_ar, n_q, q_off, H, Hkv, hd, mode, chunk=None, batch=1, seed=0):
+def _attn_case(n_keys, n_ar, n_q, q_off, H, Hkv, hd, mode, chunk=None, batch=1, seed=0, kv_split=1):
     rng_seed = 80 + seed
     q = _bf16((batch * n_q, H * hd), rng_seed)
     k = _bf16((batch * n_keys, Hkv * hd), rng_seed + 1)
@@ -374,8 +374,15 @@ def _attn_case(n_keys, n_ar, n_q, q_off, H, Hkv, hd, mode, chunk=None, batch=1, 
     chd = torch.from_numpy(ch).cuda()
     d = L.AttnDesc(n_q=n_q, q_key_offset=q_off, n_keys=n_keys, n_ar=n_ar, n_heads=H, n_kv_heads=Hkv, head_dim=hd,
                    mask_mode=L.COSMOT_MASK_FULL if mode == "full" else L.COSMOT_MASK_BLOCK_CAUSAL,
-                   chunk=A.ptr(chd), batch=batch, q_batch_stride=n_q, kv_batch_stride=n_keys, o_batch_stride=n_q)
-    L.cosmot_mot_attention(d, A.ptr(qd), H * hd, A.ptr(kd), A.ptr(vd), Hkv * hd, A.ptr(o), H * hd, A.stream_handle())
+                   chunk=A.ptr(chd), batch=batch, q_batch_stride=n_q, kv_batch_stride=n_keys, o_batch_stride=n_q,
+                   flags=L.COSMOT_ATTN_NO_TILE_SKIP if kv_split > 1 else 0)
+    if kv_split > 1:
+        ws = torch.full((L.cosmot_attention_split_workspace(d, kv_split),), 255, dtype=torch.uint8, device="cuda")
+        L.cosmot_mot_attention_split(d, A.ptr(qd), H * hd, A.ptr(kd), A.ptr(vd), Hkv * hd, A.ptr(o), H * hd, kv_split,
+                                     A.ptr(ws), ws.numel(), A.stream_handle())
+    else:
+        L.cosmot_mot_attention(d, A.ptr(qd), H * hd, A.ptr(kd), A.ptr(vd), Hkv * hd, A.ptr(o), H * hd,
+                               A.stream_handle())
     got = to_f64(o)
     assert_device_ok()
     og.assert_canaries("attention output")
@@ -445,3 +452,84 @@ def test_attention_query_suffix_streaming():
     ch[n_ar:] = np.arange(n_keys - n_ar) // 250
     got, ref = _attn_case(n_keys, n_ar, 250, n_keys - 250, H=2, Hkv=1, hd=128, mode="block_causal", chunk=ch, seed=4)
     assert_close(got, ref, "stream", sigma=SIGMA_ATTN, branch_rms=rms(ref))
+
+
+@pytest.mark.parametrize("kv_split", [2, 3])
+@pytest.mark.parametrize("case", ["full_with_ar", "suffix_block_causal", "hd64_gqa_batch2"])
+def test_attention_key_split(kv_split, case):
+    """The keys of every DM query item split across CTAs, the float32 partials
+    combined by the merge kernel: against the oracle, and close to the unsplit
+    kernel (only the order of the softmax sums differs).  AR query rows are
+    never split."""
+    if case == "full_with_ar":
+        args = dict(n_keys=1100, n_ar=130, n_q=1100, q_off=0, H=4, Hkv=2, hd=128, mode="full")
+    elif case == "suffix_block_causal":
+        n_keys, n_ar = 66 + 3 * 250 + 250, 66
+        ch = np.full(n_keys, -1, np.int32)
+        ch[n_ar:] = np.arange(n_keys - n_ar) // 250
+        args = dict(n_keys=n_keys, n_ar=n_ar, n_q=250, q_off=n_keys - 250, H=2, Hkv=1, hd=128, mode="block_causal",
+                    chunk=ch)
+    else:
+        args = dict(n_keys=900, n_ar=40, n_q=900, q_off=0, H=4, Hkv=2, hd=64, mode="full", batch=2)
+    got, ref = _attn_case(**args, seed=7, kv_split=kv_split)
+    assert_close(got, ref, f"attention split {kv_split} {case}", sigma=SIGMA_ATTN, branch_rms=rms(ref))
+    plain, _ = _attn_case(**args, seed=7)
+    assert np.abs(got - plain).max() <= 2.0 ** -7 * np.abs(plain).max() + 1e-3
+    n_ar_q = max(0, min(args["n_q"], args["n_ar"] - args["q_off"]))
+    if n_ar_q:  # AR rows take the unsplit path: identical bits
+        rows = np.concatenate([np.arange(b * args["n_q"], b * args["n_q"] + n_ar_q) for b in range(args.get("batch", 1))])
+        np.testing.assert_array_equal(got[rows], plain[rows])
+
+
+def test_attention_key_split_argument_errors():
+    n, H, hd = 600, 2, 128
+    qkv = torch.zeros((n, 3 * H * hd), dtype=torch.bfloat16, device="cuda")
+    o = torch.zeros((n, H * hd), dtype=torch.bfloat16, device="cuda")
+    ch = torch.zeros((n,), dtype=torch.int32, device="cuda")
+    base = qkv.data_ptr()
+    ws = torch.zeros((1 << 24,), dtype=torch.uint8, device="cuda")
+    f = L.cosmot_mot_attention_split
+
+    def call(d, split, nbytes=ws.numel()):
+        return f(d, base, 3 * H * hd, base + 2 * H * hd, base + 4 * H * hd, 3 * H * hd, o.data_ptr(), H * hd, split,
+                 ws.data_ptr(), nbytes, A.stream_handle(), check=False)
+    full = L.AttnDesc(n_q=n, q_key_offset=0, n_keys=n, n_ar=10, n_heads=H, n_kv_heads=H, head_dim=hd, batch=1)
+    assert call(full, 6) == L.COSMOT_ERR_INVALID_ARG  # 5 key tiles cannot be split 6 ways
+    assert call(full, 9) == L.COSMOT_ERR_INVALID_ARG
+    assert call(full, 2, nbytes=1024) == L.COSMOT_ERR_WORKSPACE
+    skip = L.AttnDesc(n_q=n, q_key_offset=0, n_keys=n, n_ar=10, n_heads=H, n_kv_heads=H, head_dim=hd, batch=1,
+                      mask_mode=L.COSMOT_MASK_BLOCK_CAUSAL, chunk=ch.data_ptr())
+    assert call(skip, 2) == L.COSMOT_ERR_UNSUPPORTED  # tile skipping and key splits do not mix
+    torch.cuda.synchronize()
+    assert_device_ok()
+
+
+def test_routed_linear_narrow_tiles_on_few_rows():
+    """573 rows against a 4,096-wide output (a DROID denoising step at Nano
+    widths) give 80 tiles 256 wide for 148 SMs, so the projection takes
+    160-wide tiles (130 of them, the last one 96 columns wide).  Against the
+    oracle, and bit-identical to the same rows computed inside a larger call
+    that keeps 256-wide tiles: the tile width changes how many columns a CTA
+    computes, never how one output element is accumulated."""
+    k, n_out, m_small, m_big = 512, 4096, 573, 5000
+    a = _bf16((m_big, k), 60)
+    w0 = _bf16((n_out, k), 61, std=1.0 / np.sqrt(k))
+    w1 = _bf16((n_out, k), 62, std=1.0 / np.sqrt(k))
+    res = _bf16((m_big, n_out), 63)
+    ad, w0d, w1d, rd = to_dev(a), to_dev(w0), to_dev(w1), to_dev(res)
+    outs = {}
+    split = 128  # one AR row tile, then the DM rows: 5 row tiles for 573 rows
+    for m in (m_small, m_big):
+        segs = [(0, split, 0, 0), (split, m, split, 1)]
+        og = Guarded(torch.empty((m, n_out), dtype=torch.bfloat16, device="cuda"))
+        e = L.Epilogue(kind=L.COSMOT_EPI_RESIDUAL, res=A.ptr(rd), ld_res=n_out)
+        L.cosmot_routed_linear(A.ptr(ad), k, k, segs, A.ptr(w0d), A.ptr(w1d), n_out, A.ptr(og.t), n_out, e,
+                               stream=A.stream_handle())
+        torch.cuda.synchronize()
+        assert_device_ok()
+        og.assert_canaries(f"gemm {m} rows")
+        outs[m] = og.t
+    a64, r64 = synth.bf16_to_f64(a[:m_small]), synth.bf16_to_f64(res[:m_small])
+    ref = np.concatenate([a64[:split] @ synth.bf16_to_f64(w0).T, a64[split:] @ synth.bf16_to_f64(w1).T]) + r64
+    assert_close(to_f64(outs[m_small]), ref, "gemm 160-wide tiles")
+    np.testing.assert_array_equal(bits(outs[m_small]), bits(outs[m_big][:m_small]))

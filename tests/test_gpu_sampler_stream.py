@@ -153,3 +153,46 @@ def test_streaming_rollout_with_kv_ring(mode):
                      out_bf16=False)
         # each side commits the K/V of its own final x
         olayer.stream_commit(dims, W, st, x, lb)
+
+
+def test_streaming_block_with_key_split():
+    """A streaming block whose attention the layer splits by keys (few query
+    tiles against a long cache: 8 heads x 4 query-tile pairs = 32 work items
+    on the SMs, 33 key tiles): four denoising steps against the oracle."""
+    dims = ModelDims(d_model=1024, n_heads=8, n_kv_heads=8, head_dim=128, ffn=2048, rope_sections=(16, 24, 24))
+    video = VideoSpec(4, 16, 16, 24, 0, 1)  # 1,024 tokens per block
+    n_text, hist, sig = 8, 3, (1.0, 0.75, 0.5, 0.25, 0.0)
+    T = video.tokens_per_step
+    n_ar = n_text + 2
+    w = synth.make_weights(dims, 1005)
+    layer = A.MoTLayer(cdims(A, dims), device_weights(w))
+    h_ar = synth.make_activations(n_ar, dims.d_model, 2005)
+    hist_x = [synth.make_activations(T, dims.d_model, 2105 + i) for i in range(hist)]
+    noise = synth.make_activations(T, dims.d_model, 2205)
+    dl = A.build_layout(_virtual_spec(n_text, video, hist, 0))
+    cs = A.mrope_table(dl.pos, dims.head_dim, dims.rope_sections)
+    mode = L.COSMOT_MASK_BLOCK_CAUSAL
+    seq0 = layer.seq_desc(dl.n_ar, dl.n_clean, dl.n_noisy, 1, cs, dl.chunk, mask_mode=mode)
+    seq = layer.seq_desc(dl.n_ar, dl.n_clean, dl.n_noisy, 1, cs, dl.chunk, mask_mode=mode, n_cached=n_ar + hist * T)
+    N = n_ar + hist * T + T
+    ad = L.AttnDesc(n_q=T, q_key_offset=N - T, n_keys=N, n_ar=n_ar, n_heads=8, n_kv_heads=8, head_dim=128,
+                    mask_mode=mode, chunk=A.ptr(dl.chunk), batch=1, flags=L.COSMOT_ATTN_NO_TILE_SKIP)
+    assert L.cosmot_attention_kv_split(ad) > 1  # the layer takes the split path here
+    h = to_dev(np.concatenate([h_ar] + hist_x + [noise]))
+    ws = torch.empty(layer.workspace_bytes(seq0), dtype=torch.uint8, device="cuda")
+    layer.commit_kv(h, seq0, 0, workspace=ws)
+    h_out = torch.empty_like(h)
+    x32 = torch.empty((1, T, dims.d_model), dtype=torch.float32, device="cuda")
+    for k, (s0, s1) in enumerate(zip(sig[:-1], sig[1:])):
+        layer.forward(h, h_out, s0, s1, seq, workspace=ws, x_state=x32, state_from_h=(k == 0))
+    torch.cuda.synchronize()
+    assert_device_ok()
+    W = olayer.weights_from_bits(dims, w)
+    spec_blk = LayoutSpec(n_text=n_text, video=video)
+    st = olayer.StreamState(slots=hist)
+    for i in range(hist):
+        olayer.stream_commit(dims, W, st, synth.bf16_to_f64(hist_x[i]), olayout.build_layout(spec_blk, tau_offset=i))
+    lb = olayout.build_layout(spec_blk, tau_offset=hist)
+    x, last = olayer.stream_block(dims, W, st, synth.bf16_to_f64(h_ar), synth.bf16_to_f64(noise), lb, sig)
+    assert_close(x32[0].double().cpu().numpy(), x, "split-key block", sigma=SIGMA_VEL,
+                 branch_rms=abs(sig[-1] - sig[-2]) * rms(last["vel"]), out_bf16=False)
