@@ -366,3 +366,42 @@ def test_readme_c_example_compiles_against_the_header(tmp_path):
     r = subprocess.run([cc, "-std=c11", "-fsyntax-only", "-Wall", "-Werror", "-I", os.path.join(root, "include"),
                         "-I", cuda_inc, str(src)], capture_output=True, text=True)
     assert r.returncode == 0, r.stderr
+
+
+def test_attention_key_split_choice_and_workspace():
+    """Host-only: the key split the layer takes for a call shape (148 SMs
+    assumed without a device) and the workspace it needs.  A streaming step
+    (1,560 query rows, 32 heads, 14,106 keys: 224 work items, 1.5 waves)
+    splits 3 ways; the 480p layer (2,368 items, exactly 16 waves) does not;
+    block-causal calls that may skip key tiles never split."""
+    from flow_matching_dit_cosmot_b200 import _lib as L
+
+    def desc(n_q, n_keys, n_ar, heads=32, batch=1, mode=0, flags=L.COSMOT_ATTN_NO_TILE_SKIP):
+        return L.AttnDesc(n_q=n_q, q_key_offset=n_keys - n_q, n_keys=n_keys, n_ar=n_ar, n_heads=heads,
+                          n_kv_heads=heads, head_dim=128, mask_mode=mode, batch=batch, flags=flags)
+
+    stream = desc(1560, 66 + 9 * 1560, 66)
+    assert L.cosmot_attention_kv_split(stream) == 3
+    assert L.cosmot_attention_kv_split(desc(18720, 18978, 258)) == 1
+    assert L.cosmot_attention_kv_split(desc(1560, 66 + 9 * 1560, 66, mode=L.COSMOT_MASK_BLOCK_CAUSAL, flags=0)) == 1
+    assert L.cosmot_attention_kv_split(desc(392, 703, 130)) == 1  # 6 key tiles: too few to split
+    n = L.cosmot_attention_split_workspace(stream, 3)
+    assert n >= 3 * 1560 * 32 * 128 * 4 + 3 * 1560 * 32 * 8
+    assert L.cosmot_attention_split_workspace(stream, 1) == 0
+
+
+def test_streaming_workspace_holds_the_key_split_partials():
+    """The layer workspace of a streaming layout reserves the key split's
+    float32 partials (the split runs when a step's queries are the block's
+    noisy rows); the 480p layout reserves none."""
+    from flow_matching_dit_cosmot_b200 import api as A
+    dm = synth.preset("stream").dims
+    dims = A.make_dims(dm.d_model, dm.n_heads, dm.n_kv_heads, dm.head_dim, dm.ffn, dm.rope_sections)
+    n_ar, hist, T = 66, 8 * 1560, 1560
+    base = A.L.SeqDesc(n_ar, hist, T, 1, 1, 0, 16, 16)
+    rows = n_ar + hist + T
+    layer_only = rows * (4096 + 12288 + 4096 + 2 * 4096 + 14336) * 2
+    got = A.L.cosmot_layer_workspace_size(dims, base)
+    assert got >= layer_only + 3 * T * 4096 * 4
+    t2v = A.L.SeqDesc(258, 0, 18720, 1, 0, 0, 16, 0)
+    assert A.L.cosmot_layer_workspace_size(dims, t2v) <= 18978 * (4096 + 12288 + 4096 + 2 * 4096 + 14336) * 2 + 6 * 256

@@ -101,3 +101,38 @@ def test_routed_linear_with_an_empty_segment():
     a64, w064, w164 = (synth.bf16_to_f64(x) for x in (a, w0, w1))
     ref = np.concatenate([a64[:90] @ w064.T, a64[90:] @ w164.T])
     assert_close(to_f64(out), ref, "gemm with an empty segment")
+
+
+def test_layer_at_the_largest_batch():
+    """32 sequences, the largest batch one call takes (64 row segments in
+    every routed launch): every sequence's outputs equal those of the same
+    sequence run alone, bit for bit, and the first and last match the oracle."""
+    spec = LayoutSpec(n_text=5, video=VideoSpec(1, 3, 4, 24, 1, 1))
+    lay = olayout.build_layout(spec)
+    B = 32
+    w = synth.make_weights(DIMS, 4700)
+    h = np.stack([synth.make_activations(lay.n_tokens, DIMS.d_model, 4701 + b) for b in range(B)])
+    dlay = A.build_layout(layout_spec(A, spec))
+    cs = A.mrope_table(dlay.pos, DIMS.head_dim, DIMS.rope_sections)
+    layer = A.MoTLayer(cdims(A, DIMS), device_weights(w))
+    hd_, h_out = to_dev(h), torch.empty((B, lay.n_tokens, DIMS.d_model), dtype=torch.bfloat16, device="cuda")
+    layer.forward(hd_, h_out, 0.8, 0.6, layer.seq_desc(lay.n_ar, lay.n_clean, lay.n_noisy, B, cs, dlay.chunk))
+    torch.cuda.synchronize()
+    assert_device_ok()
+    W = olayer.weights_from_bits(DIMS, w)
+    noisy = lay.region == olayout.REGION_NOISY
+    for b in range(B):
+        one, one_out = to_dev(h[b:b + 1]), torch.empty((1, lay.n_tokens, DIMS.d_model), dtype=torch.bfloat16,
+                                                       device="cuda")
+        layer.forward(one, one_out, 0.8, 0.6, layer.seq_desc(lay.n_ar, lay.n_clean, lay.n_noisy, 1, cs, dlay.chunk))
+        torch.cuda.synchronize()
+        np.testing.assert_array_equal(bits(h_out[b]), bits(one_out[0]))
+        np.testing.assert_array_equal(bits(hd_[b]), bits(one[0]))
+        if b in (0, B - 1):
+            ref = olayer.layer_forward(DIMS, W, synth.bf16_to_f64(h[b]), lay.region, lay.pos, lay.chunk, 0.8, 0.6)
+            layer_parity(f"batch {B} [{b}]", ref, noisy, -0.2, h_out=to_f64(h_out[b]), x_new=to_f64(hd_[b])[noisy])
+    bad = layer.seq_desc(lay.n_ar, lay.n_clean, lay.n_noisy, B + 1, cs, dlay.chunk)
+    ws = torch.empty((1 << 20,), dtype=torch.uint8, device="cuda")
+    code = L.cosmot_layer_forward(layer.dims, layer.cw, bad, hd_.data_ptr(), h_out.data_ptr(), 0.8, 0.6,
+                                  ws.data_ptr(), ws.numel(), A.stream_handle(), check=False)
+    assert code == L.COSMOT_ERR_UNSUPPORTED
