@@ -44,8 +44,8 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # only while that code is unchanged.
 NCU_TRAFFIC = {
     # one attention launch at the 480p shape (18,978 rows x 32 heads):
-    # dram__bytes_read.sum 474,648,832 + dram__bytes_write.sum 136,260,608
-    "t2v480:attention": {"bytes_per_launch": 610909440, "src_sha": "abea48bb2bacaadf"},
+    # dram__bytes_read.sum 474,230,528 + dram__bytes_write.sum 135,390,976
+    "t2v480:attention": {"bytes_per_launch": 609621504, "src_sha": "f1dd4a7f66d5deda"},
 }
 
 

@@ -104,11 +104,11 @@ WsLayout ws_layout(const cosmot_dims& d, const cosmot_seq_desc& s) {
   w.o = off;   off += align256(rows * q_cols * 2);
   w.h1 = off;  off += align256(rows * d.d_model * 4);  // float32: the residual stream between the two halves
   w.u = off;   off += align256(rows * d.ffn * 2);
-  // A call whose queries are the noisy rows alone (a streaming step: the AR
-  // rows and the cache are the n_cached prefix) may split its keys across
-  // CTAs to fill the SMs; its float32 partials live here.
+  // A call whose queries are the noisy rows alone behind a cached prefix of
+  // AR and clean rows (a streaming step: the AR rows and the cache) may split
+  // its keys across CTAs to fill the SMs; its float32 partials live here.
   cosmot_attn_desc ad = stream_attn_desc(d, s);
-  w.kv_split = s.n_noisy > 0 ? cosmot_attention_kv_split(&ad) : 1;
+  w.kv_split = s.n_noisy > 0 && s.n_clean > 0 ? cosmot_attention_kv_split(&ad) : 1;
   w.part_bytes = 0;
   if (w.kv_split > 1) cosmot_attention_split_workspace(&ad, w.kv_split, &w.part_bytes);
   w.part = off;
@@ -216,7 +216,11 @@ cosmot_status layer_body(const cosmot_dims& D, const cosmot_layer_weights* w, co
   if (noisy_only) ad.flags = COSMOT_ATTN_NO_TILE_SKIP;
   ad.q_batch_stride = ad.kv_batch_stride = ad.o_batch_stride = N;
   uint16_t* qkvp = static_cast<uint16_t*>(qkv);
-  if (noisy_only && L.kv_split > 1)  // few query tiles: split the keys to fill the SMs
+  // Few query tiles against a long cache (a streaming step: the cached prefix
+  // holds clean or history rows): split the keys to fill the SMs.  A sampler
+  // step that caches only the AR rows never splits, so it stays bit-identical
+  // to a full recompute.
+  if (noisy_only && S.n_clean > 0 && L.kv_split > 1)
     st = cosmot_mot_attention_split(&ad, qkvp + c0 * qkvc, qkvc, qkvp + qc, qkvp + qc + kvc, qkvc,
                                     static_cast<uint16_t*>(o) + c0 * qc, qc, L.kv_split, ws + L.part, L.part_bytes,
                                     stream);

@@ -196,3 +196,25 @@ def test_streaming_block_with_key_split():
     x, last = olayer.stream_block(dims, W, st, synth.bf16_to_f64(h_ar), synth.bf16_to_f64(noise), lb, sig)
     assert_close(x32[0].double().cpu().numpy(), x, "split-key block", sigma=SIGMA_VEL,
                  branch_rms=abs(sig[-1] - sig[-2]) * rms(last["vel"]), out_bf16=False)
+
+
+def test_sampler_without_clean_rows_stays_bit_identical():
+    """A text-to-video-like layout (no clean rows) whose noisy-only attention
+    would be worth a key split (8 heads x 8 query-tile pairs against 17 key
+    tiles): the sampler's later steps reuse only the AR rows, never split, and
+    stay bit-identical to a full recompute."""
+    dims = ModelDims(d_model=1024, n_heads=8, n_kv_heads=8, head_dim=128, ffn=2048, rope_sections=(16, 24, 24))
+    spec = LayoutSpec(n_text=30, video=VideoSpec(1, 16, 16, 24, 0, 8))  # 32 AR + 2,048 noisy
+    lay = olayout.build_layout(spec)
+    w = synth.make_weights(dims, 1006)
+    h0 = synth.make_activations(lay.n_tokens, dims.d_model, 2006)[None]
+    dlay = A.build_layout(layout_spec(A, spec))
+    cs = A.mrope_table(dlay.pos, dims.head_dim, dims.rope_sections)
+    layer = A.MoTLayer(cdims(A, dims), device_weights(w))
+    sig = (1.0, 0.8, 0.6)
+    h_c, out_c, st_c, _ = _run_sampler(layer, dlay, cs, h0, sig, 1, cached=True, f32_state=True)
+    h_f, out_f, st_f, _ = _run_sampler(layer, dlay, cs, h0, sig, 1, cached=False, f32_state=True)
+    np.testing.assert_array_equal(bits(h_c), bits(h_f))
+    np.testing.assert_array_equal(bits(out_c)[0, lay.n_ar:], bits(out_f)[0, lay.n_ar:])
+    for a, b_ in zip(st_c, st_f):
+        np.testing.assert_array_equal(a.cpu().numpy(), b_.cpu().numpy())
