@@ -7,7 +7,8 @@
 //     acc[128 x 256] = A[rows, K] . W_set[cols, K]^T
 // on the tensor cores with the fp32 accumulator in tensor memory.
 //
-// Structure (one persistent CTA per SM, 192 threads):
+// Structure (one persistent CTA per SM, 192 threads; for most calls a pair of
+// CTAs per 256-row tile, see Tiles below):
 //   warp 0      TMA producer: A tile 128x64 and B tile 256x64 (bf16, 128-byte
 //               swizzle) per k-block into a 4-stage shared-memory ring.
 //   warp 1      owns TMEM (512 columns = two 128x256 fp32 accumulators) and
@@ -34,7 +35,6 @@ namespace gemm {
 
 constexpr int BM = 128;
 constexpr int BK = 64;  // 64 bf16 = 128 bytes = one swizzle row
-constexpr int STAGES = 4;
 constexpr int A_BYTES = BM * BK * 2;
 constexpr int NUM_THREADS = 192;
 constexpr int TMEM_COLS = 512;
@@ -45,13 +45,23 @@ constexpr int kGroupM = 16;
 // fill the SMs with 256-wide ones (a few hundred rows against a 4096-wide
 // output: 5 row tiles x 16 column tiles = 80 tiles for 148 SMs become 5 x 26
 // = 130).  Any multiple of 32 up to 256 is a valid tcgen05 N for M = 128.
-template <int BN>
+//
+// CG = 2: a cluster of two CTAs computes a 256-row tile with
+// tcgen05.mma.cta_group::2 (M = 256): each CTA loads its own 128 A rows and
+// half of the B rows (the gate or the up half for SiLU*mul), so a CTA moves
+// 32 KB per k-block instead of 48 KB for the same work, and six stages fit.
+// The even CTA's full barrier counts both CTAs' bytes; its MMA thread commits
+// to both CTAs' barriers; both epilogues release an accumulator on the even
+// CTA's barrier.  Single-CTA tiles (CG = 1) stay for calls with few rows.
+template <int BN, int CG = 1>
 struct Tiles {
   static_assert(BN % 32 == 0 && BN >= 32 && BN <= 256, "tile width");
-  static constexpr int B_BYTES = BN * BK * 2;
+  static_assert(CG == 1 || (CG == 2 && BN == 256), "pair tiles are 256 x 256");
+  static constexpr int STAGES = CG == 2 ? 6 : 4;
+  static constexpr int B_BYTES = BN * BK * 2 / CG;  // this CTA's B rows
   static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
   static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 256 + 1024;
-  static constexpr uint32_t IDESC = idesc_bf16_f32(BM, BN, false, false);
+  static constexpr uint32_t IDESC = idesc_bf16_f32(BM * CG, BN, false, false);
 };
 
 struct Params {
@@ -90,10 +100,12 @@ struct Tile {
   int32_t set;
   int32_t n;          // column tile
   int64_t a_row0;     // first A row
-  int32_t rows;       // valid rows (<= BM)
+  int32_t rows;       // valid rows (<= the tile's rows)
   int64_t out_row0;   // output row of a_row0
 };
 
+// TM: rows of a tile (128, or 256 for a pair of CTAs).
+template <int TM>
 __device__ __forceinline__ Tile decode_tile(const Params& p, int32_t t) {
   const int32_t per_group = p.group_m * p.num_n_tiles;
   const int32_t g = t / per_group;
@@ -107,9 +119,9 @@ __device__ __forceinline__ Tile decode_tile(const Params& p, int32_t t) {
   int s = 0;
   while (s + 1 < p.n_segs && m >= p.mtile_prefix[s + 1]) ++s;
   tl.set = p.set[s];
-  tl.a_row0 = p.row_begin[s] + (int64_t)(m - p.mtile_prefix[s]) * BM;
+  tl.a_row0 = p.row_begin[s] + (int64_t)(m - p.mtile_prefix[s]) * TM;
   const int64_t left = p.row_end[s] - tl.a_row0;
-  tl.rows = (int32_t)(left < BM ? left : BM);
+  tl.rows = (int32_t)(left < TM ? left : TM);
   tl.out_row0 = p.out_row[s] + (tl.a_row0 - p.row_begin[s]);
   return tl;
 }
@@ -170,16 +182,18 @@ __device__ __forceinline__ void load_row32(const __nv_bfloat16* src, int32_t col
 }
 
 // FL: COSMOT_EPI_OUT_F32 / COSMOT_EPI_RES_F32 bits of the RESIDUAL epilogue;
-// BN: the tile width.
-template <int EPI, int FL, int BN>
+// BN: the tile width; CG: CTAs per tile (2: launched as clusters of two).
+template <int EPI, int FL, int BN, int CG>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
     routed_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUtensorMap tmap_b0,
                        const __grid_constant__ CUtensorMap tmap_b1, const __grid_constant__ CUtensorMap tmap_u0,
                        const __grid_constant__ CUtensorMap tmap_u1, const __grid_constant__ Params p) {
-  using T = Tiles<BN>;
+  using T = Tiles<BN, CG>;
+  constexpr int STAGES = T::STAGES;
   constexpr int B_BYTES = T::B_BYTES;
   constexpr int STAGE_BYTES = T::STAGE_BYTES;
   constexpr uint32_t IDESC = T::IDESC;
+  constexpr int TM = BM * CG;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const uint32_t sbase = smem_u32(smem);
@@ -193,6 +207,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
+  // Pair tiles: `rank` 0 (even CTA) issues the MMAs; tile work is walked per pair.
+  const uint32_t rank = CG == 2 ? cluster_ctarank() : 0u;
+  const int32_t unit = CG == 2 ? (int32_t)(blockIdx.x >> 1) : (int32_t)blockIdx.x;
+  const int32_t units = CG == 2 ? (int32_t)(gridDim.x >> 1) : (int32_t)gridDim.x;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
@@ -201,17 +219,24 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(bar_tfull + 8 * b, 1);
-      mbar_init(bar_tempty + 8 * b, 4 * 32);
+      // one arrive per epilogue thread; pairs: one per epilogue warp of both CTAs
+      mbar_init(bar_tempty + 8 * b, CG == 2 ? 8 : 4 * 32);
     }
     mbar_init(bar_drain, 1);
     fence_barrier_init();
   }
   if (warp == 1) {
-    tmem_alloc(smem_u32(tmem_slot), TMEM_COLS);
-    tmem_relinquish();
+    if constexpr (CG == 2) {
+      tmem_alloc_pair(smem_u32(tmem_slot), TMEM_COLS);
+      tmem_relinquish_pair();
+    } else {
+      tmem_alloc(smem_u32(tmem_slot), TMEM_COLS);
+      tmem_relinquish();
+    }
   }
   tc_fence_before();
   __syncthreads();
+  if constexpr (CG == 2) cluster_sync();  // both CTAs' barriers exist before either signals the other
   tc_fence_after();
   const uint32_t tmem_base = *reinterpret_cast<volatile uint32_t*>(tmem_slot);
 
@@ -229,8 +254,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       uint32_t phase = 0;
       uint32_t armed_mask = 0, armed_parity = 0;
       bool ok = true;
-      for (int32_t t = blockIdx.x; t < p.num_tiles && ok; t += gridDim.x) {
-        const Tile tl = decode_tile(p, t);
+      for (int32_t t = unit; t < p.num_tiles && ok; t += units) {
+        const Tile tl = decode_tile<TM>(p, t);
         const CUtensorMap* mb = tl.set ? &tmap_b1 : &tmap_b0;
         const CUtensorMap* mu = tl.set ? &tmap_u1 : &tmap_u0;
         for (int kb = 0; kb < p.num_kb; ++kb) {
@@ -241,13 +266,24 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           const uint32_t fb = bar_full + 8 * stage;
           const uint32_t sa = sbase + stage * STAGE_BYTES;
           const uint32_t sb = sa + A_BYTES;
-          mbar_arrive_expect_tx(fb, STAGE_BYTES);
-          tma_load_2d(sa, &tmap_a, fb, kb * BK, (int)tl.a_row0);
-          if (EPI == COSMOT_EPI_SILU_MUL) {
-            tma_load_2d(sb, mb, fb, kb * BK, tl.n * (BN / 2));
-            tma_load_2d(sb + B_BYTES / 2, mu, fb, kb * BK, tl.n * (BN / 2));
+          if constexpr (CG == 2) {
+            // both CTAs' bytes complete on the even CTA's barrier, which only it arms
+            const uint32_t fb0 = mapa_shared(fb, 0);
+            if (rank == 0) mbar_arrive_expect_tx(fb, 2 * STAGE_BYTES);
+            tma_load_2d_pair(sa, &tmap_a, fb0, kb * BK, (int)(tl.a_row0 + (int64_t)rank * BM));
+            if (EPI == COSMOT_EPI_SILU_MUL)
+              tma_load_2d_pair(sb, rank ? mu : mb, fb0, kb * BK, tl.n * (BN / 2));
+            else
+              tma_load_2d_pair(sb, mb, fb0, kb * BK, tl.n * BN + (int)rank * (BN / 2));
           } else {
-            tma_load_2d(sb, mb, fb, kb * BK, tl.n * BN);
+            mbar_arrive_expect_tx(fb, STAGE_BYTES);
+            tma_load_2d(sa, &tmap_a, fb, kb * BK, (int)tl.a_row0);
+            if (EPI == COSMOT_EPI_SILU_MUL) {
+              tma_load_2d(sb, mb, fb, kb * BK, tl.n * (BN / 2));
+              tma_load_2d(sb + B_BYTES / 2, mu, fb, kb * BK, tl.n * (BN / 2));
+            } else {
+              tma_load_2d(sb, mb, fb, kb * BK, tl.n * BN);
+            }
           }
           armed_mask |= 1u << stage;
           armed_parity = (armed_parity & ~(1u << stage)) | (phase << stage);
@@ -258,8 +294,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         }
       }
       // No bulk copy may still be writing shared memory when the CTA exits.
+      // Pairs: the even CTA's barriers count the odd CTA's copies too, and the
+      // odd CTA leaves only after the closing cluster barrier.
       for (int s = 0; s < STAGES; ++s)
-        if (armed_mask & (1u << s)) {
+        if (rank == 0 && (armed_mask & (1u << s))) {
           const uint32_t par = (armed_parity >> s) & 1u;
           const uint64_t t0 = globaltimer_ns();
           while (!mbar_try_wait(bar_full + 8 * s, par) && globaltimer_ns() - t0 < kWaitLimitNs) {
@@ -269,12 +307,12 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     __syncwarp();
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
-    if (lane == 0) {
+    if (lane == 0 && rank == 0) {
       int stage = 0;
       uint32_t phase = 0;
       bool ok = true;
       uint32_t local = 0;
-      for (int32_t t = blockIdx.x; t < p.num_tiles && ok; t += gridDim.x, ++local) {
+      for (int32_t t = unit; t < p.num_tiles && ok; t += units, ++local) {
         const uint32_t buf = local & 1;
         const uint32_t use = local >> 1;
         if (!mbar_wait(bar_tempty + 8 * buf, (use & 1) ^ 1, p.status, kWhereGemmMma)) break;
@@ -292,19 +330,31 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           for (int k = 0; k < BK / 16; ++k) {
             const uint64_t ad = sw128_desc(sa + 32 * k, 16, 1024);
             const uint64_t bd = sw128_desc(sb + 32 * k, 16, 1024);
-            umma_ss(d_tmem, ad, bd, IDESC, (kb | k) != 0 ? 1u : 0u);
+            if constexpr (CG == 2)
+              umma_ss_pair(d_tmem, ad, bd, IDESC, (kb | k) != 0 ? 1u : 0u);
+            else
+              umma_ss(d_tmem, ad, bd, IDESC, (kb | k) != 0 ? 1u : 0u);
           }
-          umma_commit(bar_empty + 8 * stage);
+          if constexpr (CG == 2)
+            umma_commit_pair_mc(bar_empty + 8 * stage, 3);
+          else
+            umma_commit(bar_empty + 8 * stage);
           if (++stage == STAGES) {
             stage = 0;
             phase ^= 1;
           }
         }
         if (!ok) break;
-        umma_commit(bar_tfull + 8 * buf);
+        if constexpr (CG == 2)
+          umma_commit_pair_mc(bar_tfull + 8 * buf, 3);
+        else
+          umma_commit(bar_tfull + 8 * buf);
       }
       // Wait until every MMA issued above has completed before TMEM is freed.
-      umma_commit(bar_drain);
+      if constexpr (CG == 2)
+        umma_commit_pair_mc(bar_drain, 1);
+      else
+        umma_commit(bar_drain);
       const uint64_t t0 = globaltimer_ns();
       while (!mbar_try_wait(bar_drain, 0)) {
         if (globaltimer_ns() - t0 > kWaitLimitNs) {
@@ -319,15 +369,16 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     const int lane_base = (warp & 3) * 32;  // TMEM lanes this warp may access
     const int r = lane_base + lane;          // row within the tile
     uint32_t local = 0;
-    for (int32_t t = blockIdx.x; t < p.num_tiles; t += gridDim.x, ++local) {
+    for (int32_t t = unit; t < p.num_tiles; t += units, ++local) {
       const uint32_t buf = local & 1;
       const uint32_t use = local >> 1;
       // Warp-uniform: the tcgen05.ld below is .sync.aligned.
       if (!__all_sync(0xffffffffu, mbar_wait(bar_tfull + 8 * buf, use & 1, p.status, kWhereGemmEpilogue))) break;
       tc_fence_after();
-      const Tile tl = decode_tile(p, t);
-      const bool valid = r < tl.rows;
-      const int64_t orow = tl.out_row0 + r;
+      const Tile tl = decode_tile<TM>(p, t);
+      const int rr = (int)rank * BM + r;  // row within the (pair's) tile
+      const bool valid = rr < tl.rows;
+      const int64_t orow = tl.out_row0 + rr;
       const uint32_t tacc = tmem_base + ((uint32_t)lane_base << 16) + buf * BN;
       uint32_t v[32];
       float f[32];
@@ -353,7 +404,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       } else if (EPI == COSMOT_EPI_MROPE) {
         const int hd = p.head_dim;
         const int half = hd >> 1;
-        const int64_t arow = tl.a_row0 + r;  // positions follow the input row
+        const int64_t arow = tl.a_row0 + rr;  // positions follow the input row
         const int64_t trow = p.rope_period > 0 ? arow % p.rope_period : arow;
         const float2* cs_row = p.rope_cs + trow * half;
 #pragma unroll 1
@@ -416,7 +467,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
               for (int j = 0; j < 32; ++j) f[j] = __uint_as_float(v[j]) + rs[j];
             } else if (EPI == COSMOT_EPI_EULER) {
               // x' = x + dsigma * v in fp32; x from the fp32 state when there is one
-              const int64_t arow = tl.a_row0 + r;
+              const int64_t arow = tl.a_row0 + rr;
               const bool arow_ok = dcheck(arow >= 0 && arow < p.a_rows, p.status, kWhereGemmStore);
               float xs[32];
               if (p.xs && !p.xs_from_x && arow_ok)
@@ -444,20 +495,65 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         }
       }
       tc_fence_before();
-      mbar_arrive(bar_tempty + 8 * buf);
+      if constexpr (CG == 2) {
+        __syncwarp();
+        if (lane == 0) mbar_arrive_cluster(mapa_shared(bar_tempty + 8 * buf, 0));
+      } else {
+        mbar_arrive(bar_tempty + 8 * buf);
+      }
     }
   }
 
   tc_fence_before();
   __syncthreads();
+  if constexpr (CG == 2) cluster_sync();  // the pair's MMAs have drained; neither CTA's memory is in use
   tc_fence_after();
-  if (warp == 1) tmem_dealloc(tmem_base, TMEM_COLS);
+  if (warp == 1) {
+    if constexpr (CG == 2)
+      tmem_dealloc_pair(tmem_base, TMEM_COLS);
+    else
+      tmem_dealloc(tmem_base, TMEM_COLS);
+  }
 }
 
-template <int EPI, int FL = 0, int BN = 256>
+// Clusters of two this kernel keeps resident at once on the current device
+// (0 if it cannot run as pairs).
+int resident_pairs() {
+  static std::mutex mu;
+  static int cached[64] = {0};
+  static uint64_t done_mask = 0;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 0;
+  std::lock_guard<std::mutex> lk(mu);
+  if (!(done_mask & (1ull << dev))) {
+    auto kern = routed_gemm_kernel<COSMOT_EPI_NONE, 0, 256, 2>;  // every pair instance has this footprint
+    int n = 0;
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Tiles<256, 2>::SMEM_BYTES) ==
+        cudaSuccess) {
+      cudaLaunchConfig_t cfg{};
+      cudaLaunchAttribute attr[1];
+      attr[0].id = cudaLaunchAttributeClusterDimension;
+      attr[0].val.clusterDim.x = 2;
+      attr[0].val.clusterDim.y = 1;
+      attr[0].val.clusterDim.z = 1;
+      cfg.gridDim = dim3(2 * 74, 1, 1);
+      cfg.blockDim = dim3(NUM_THREADS, 1, 1);
+      cfg.dynamicSmemBytes = Tiles<256, 2>::SMEM_BYTES;
+      cfg.attrs = attr;
+      cfg.numAttrs = 1;
+      if (cudaOccupancyMaxActiveClusters(&n, kern, &cfg) != cudaSuccess) n = 0;
+    }
+    (void)cudaGetLastError();
+    cached[dev] = n;
+    done_mask |= 1ull << dev;
+  }
+  return cached[dev];
+}
+
+template <int EPI, int FL = 0, int BN = 256, int CG = 1>
 cosmot_status launch(const CUtensorMap& ta, const CUtensorMap& tb0, const CUtensorMap& tb1, const CUtensorMap& tu0,
                      const CUtensorMap& tu1, const Params& p, cudaStream_t s) {
-  constexpr int SMEM_BYTES = Tiles<BN>::SMEM_BYTES;
+  constexpr int SMEM_BYTES = Tiles<BN, CG>::SMEM_BYTES;
   static std::mutex mu;
   static uint64_t done_mask = 0;  // devices whose smem limit was raised
   int dev = 0;
@@ -465,16 +561,36 @@ cosmot_status launch(const CUtensorMap& ta, const CUtensorMap& tb0, const CUtens
   {
     std::lock_guard<std::mutex> lk(mu);
     if (dev >= 64 || !(done_mask & (1ull << dev))) {
-      if (cudaFuncSetAttribute(routed_gemm_kernel<EPI, FL, BN>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+      if (cudaFuncSetAttribute(routed_gemm_kernel<EPI, FL, BN, CG>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                SMEM_BYTES) !=
           cudaSuccess)
         return COSMOT_ERR_CUDA;
       if (dev < 64) done_mask |= 1ull << dev;
     }
   }
+  if constexpr (CG == 2) {
+    int pairs = resident_pairs();
+    if (pairs < 1) return COSMOT_ERR_CUDA;
+    if (p.num_tiles < pairs) pairs = p.num_tiles;
+    cudaLaunchConfig_t cfg{};
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.gridDim = dim3(2 * pairs, 1, 1);
+    cfg.blockDim = dim3(NUM_THREADS, 1, 1);
+    cfg.dynamicSmemBytes = SMEM_BYTES;
+    cfg.stream = s;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    if (cudaLaunchKernelEx(&cfg, routed_gemm_kernel<EPI, FL, BN, CG>, ta, tb0, tb1, tu0, tu1, p) != cudaSuccess)
+      return COSMOT_ERR_CUDA;
+    return launch_status();
+  }
   int grid = num_sms();
   if (p.num_tiles < grid) grid = p.num_tiles;
-  routed_gemm_kernel<EPI, FL, BN><<<grid, NUM_THREADS, SMEM_BYTES, s>>>(ta, tb0, tb1, tu0, tu1, p);
+  routed_gemm_kernel<EPI, FL, BN, CG><<<grid, NUM_THREADS, SMEM_BYTES, s>>>(ta, tb0, tb1, tu0, tu1, p);
   return launch_status();
 }
 
@@ -502,30 +618,34 @@ extern "C" cosmot_status cosmot_routed_linear(const void* a, int64_t ld_a, int64
   p.n_segs = n_segs;
   bool uses[2] = {false, false};
   int64_t max_row = 0;
-  int32_t mt = 0;
   for (int i = 0; i < n_segs; ++i) {
     const cosmot_segment& s = segs[i];
     if (s.row_begin < 0 || s.row_end < s.row_begin || s.out_row < 0 || (s.weight_set != 0 && s.weight_set != 1))
       return COSMOT_ERR_INVALID_ARG;
+    if (s.row_end - s.row_begin > INT32_MAX / 4) return COSMOT_ERR_UNSUPPORTED;
     p.row_begin[i] = s.row_begin;
     p.row_end[i] = s.row_end;
     p.out_row[i] = s.out_row;
     p.set[i] = s.weight_set;
-    p.mtile_prefix[i] = mt;
-    const int64_t tiles = (s.row_end - s.row_begin + BM - 1) / BM;
-    if ((int64_t)mt + tiles > INT32_MAX / 4) return COSMOT_ERR_UNSUPPORTED;
-    mt += (int32_t)tiles;
     if (s.row_end > s.row_begin) uses[s.weight_set] = true;
     if (s.row_end > max_row) max_row = s.row_end;
   }
-  p.mtile_prefix[n_segs] = mt;
-  p.num_m_tiles = mt;
+  // row tiles of `tm` rows over all segments (a tile never straddles two)
+  auto count_mtiles = [&](int64_t tm) {
+    int64_t n = 0;
+    for (int i = 0; i < n_segs; ++i) n += (segs[i].row_end - segs[i].row_begin + tm - 1) / tm;
+    return n;
+  };
+  const int64_t mt1 = count_mtiles(BM);
+  if (mt1 > INT32_MAX / 4) return COSMOT_ERR_UNSUPPORTED;
+  const int32_t mt = (int32_t)mt1;
   for (int i = 0; i < n_segs; ++i) {
     const int64_t end = segs[i].out_row + (segs[i].row_end - segs[i].row_begin);
     if (end > p.out_rows) p.out_rows = end;
   }
   p.a_rows = max_row;
   if (mt == 0) return COSMOT_OK;
+  const int64_t sms = num_sms();
   if (max_row > INT32_MAX) return COSMOT_ERR_UNSUPPORTED;
   const bool silu = kind == COSMOT_EPI_SILU_MUL;
   // Tile width: 160 instead of 256 when that keeps clearly more SMs busy over
@@ -533,7 +653,6 @@ extern "C" cosmot_status cosmot_routed_linear(const void* a, int64_t ld_a, int64
   // an up half: both keep 256).
   int bn = 256;
   if (kind == COSMOT_EPI_NONE || kind == COSMOT_EPI_RESIDUAL || kind == COSMOT_EPI_EULER) {
-    const int64_t sms = num_sms();
     auto eff = [&](int64_t w) {
       const int64_t t = (int64_t)mt * ((n_out + w - 1) / w);
       return (double)t / (double)(((t + sms - 1) / sms) * sms);
@@ -541,11 +660,32 @@ extern "C" cosmot_status cosmot_routed_linear(const void* a, int64_t ld_a, int64
     if (eff(160) > eff(256) + 0.1) bn = 160;
   }
   p.num_n_tiles = (int32_t)((n_out + (silu ? bn / 2 : bn) - 1) / (silu ? bn / 2 : bn));
+  // CTA pairs (256-row tiles, half the B bytes a CTA) unless they need more
+  // than 10 % more rounds over the SMs than single-CTA tiles: a pair's round
+  // is the shorter one (the single-CTA main loop waits on its loads ~20 % of
+  // the time; measured on the 480p layer, pairs took QKV from 1.49 to 1.38 ms
+  // and the O projection from 0.57 to 0.50 ms).
+  int cg = 1;
+  if (bn == 256) {
+    const int64_t pairs = resident_pairs();
+    if (pairs > 0) {
+      const int64_t t1 = mt1 * p.num_n_tiles, t2 = count_mtiles(2 * BM) * p.num_n_tiles;
+      if ((t2 + pairs - 1) / pairs * 10 <= (t1 + sms - 1) / sms * 11) cg = 2;
+    }
+  }
+  const int64_t tm = (int64_t)BM * cg;
+  int32_t mtc = 0;
+  for (int i = 0; i < n_segs; ++i) {
+    p.mtile_prefix[i] = mtc;
+    mtc += (int32_t)((segs[i].row_end - segs[i].row_begin + tm - 1) / tm);
+  }
+  p.mtile_prefix[n_segs] = mtc;
+  p.num_m_tiles = mtc;
   if ((int64_t)p.num_m_tiles * p.num_n_tiles > INT32_MAX) return COSMOT_ERR_UNSUPPORTED;
   p.num_tiles = p.num_m_tiles * p.num_n_tiles;
   p.num_kb = (int32_t)((k + BK - 1) / BK);
   p.n_out = (int32_t)n_out;
-  p.group_m = kGroupM;
+  p.group_m = kGroupM / cg;
   p.out = static_cast<__nv_bfloat16*>(out);
   p.ld_out = ld_out;
   p.status = device_status_ptr();
@@ -588,7 +728,9 @@ extern "C" cosmot_status cosmot_routed_linear(const void* a, int64_t ld_a, int64
   if (st != COSMOT_OK) return st;
   const void* wb[2] = {w0, w1};
   const void* wu[2] = {w0_up, w1_up};
-  const uint32_t brows = silu ? bn / 2 : bn;
+  // a CTA's B box: the tile's columns, the gate or up half for SiLU*mul, and
+  // for a pair of CTAs one half of either
+  const uint32_t brows = cg == 2 ? 128u : (silu ? bn / 2 : bn);
   for (int s = 0; s < 2; ++s) {
     const int src = uses[s] ? s : (uses[0] ? 0 : 1);  // an unused set reuses a valid map
     if (!wb[src]) return COSMOT_ERR_INVALID_ARG;
@@ -603,6 +745,25 @@ extern "C" cosmot_status cosmot_routed_linear(const void* a, int64_t ld_a, int64
     }
   }
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (cg == 2) {
+    switch (kind) {
+      case COSMOT_EPI_NONE: return launch<COSMOT_EPI_NONE, 0, 256, 2>(ta, tb[0], tb[1], tu[0], tu[1], p, s);
+      case COSMOT_EPI_SILU_MUL: return launch<COSMOT_EPI_SILU_MUL, 0, 256, 2>(ta, tb[0], tb[1], tu[0], tu[1], p, s);
+      case COSMOT_EPI_MROPE: return launch<COSMOT_EPI_MROPE, 0, 256, 2>(ta, tb[0], tb[1], tu[0], tu[1], p, s);
+      case COSMOT_EPI_EULER: return launch<COSMOT_EPI_EULER, 0, 256, 2>(ta, tb[0], tb[1], tu[0], tu[1], p, s);
+      default:
+        switch (flags) {
+          case COSMOT_EPI_OUT_F32:
+            return launch<COSMOT_EPI_RESIDUAL, COSMOT_EPI_OUT_F32, 256, 2>(ta, tb[0], tb[1], tu[0], tu[1], p, s);
+          case COSMOT_EPI_RES_F32:
+            return launch<COSMOT_EPI_RESIDUAL, COSMOT_EPI_RES_F32, 256, 2>(ta, tb[0], tb[1], tu[0], tu[1], p, s);
+          case COSMOT_EPI_OUT_F32 | COSMOT_EPI_RES_F32:
+            return launch<COSMOT_EPI_RESIDUAL, COSMOT_EPI_OUT_F32 | COSMOT_EPI_RES_F32, 256, 2>(ta, tb[0], tb[1], tu[0],
+                                                                                              tu[1], p, s);
+          default: return launch<COSMOT_EPI_RESIDUAL, 0, 256, 2>(ta, tb[0], tb[1], tu[0], tu[1], p, s);
+        }
+    }
+  }
   if (bn == 160) {
     switch (kind) {
       case COSMOT_EPI_NONE: return launch<COSMOT_EPI_NONE, 0, 160>(ta, tb[0], tb[1], tu[0], tu[1], p, s);

@@ -138,6 +138,30 @@ def test_routed_linear_plain(m_split, m_total, k, n_out):
     og.assert_canaries("gemm output")
 
 
+def test_routed_linear_pair_and_single_tiles_agree_bit_for_bit():
+    """Most calls run 256-row tiles on a pair of CTAs (tcgen05.mma.cta_group::2);
+    a call whose pairs would need clearly more rounds over the SMs runs
+    128-row tiles on single CTAs.  On 148 SMs, 4736 rows x 1024 columns are
+    148 single tiles (one round) but 76 pair tiles (two rounds over 74
+    pairs): single CTAs; the same rows x 256 columns fit in one round either
+    way: pairs.  Every element is the same K-ordered fp32 sum in both, so the
+    shared columns agree to the bit, and both meet the reference."""
+    m_total, k = 4736, 256
+    a, w0, w1, segs, acc = _gemm_case(300, m_total, k, 1024, seed=7)
+    ad, w0d, w1d = to_dev(a), to_dev(w0), to_dev(w1)
+    wide = torch.empty((m_total, 1024), dtype=torch.bfloat16, device="cuda")
+    narrow = torch.empty((m_total, 256), dtype=torch.bfloat16, device="cuda")
+    L.cosmot_routed_linear(A.ptr(ad), k, k, segs, A.ptr(w0d), A.ptr(w1d), 1024, A.ptr(wide), 1024,
+                           stream=A.stream_handle())
+    L.cosmot_routed_linear(A.ptr(ad), k, k, segs, A.ptr(w0d), A.ptr(w1d), 256, A.ptr(narrow), 256,
+                           stream=A.stream_handle())
+    torch.cuda.synchronize()
+    assert_device_ok()
+    assert_close(to_f64(wide), acc, "gemm, single-CTA tiles")
+    assert_close(to_f64(narrow), acc[:, :256], "gemm, pair tiles")
+    np.testing.assert_array_equal(bits(narrow), bits(wide[:, :256]))
+
+
 def test_routed_linear_equal_sets_equal_single_segment():
     """With both weight sets holding the same matrix (in separate buffers) the
     routed projection is bit-identical to one segment over all rows: routing
