@@ -196,7 +196,68 @@ class ClockSampler:
                 return line.strip()
         return None
 
+    # NVML clock-event reason bits (nvml.h: clocksEventReason*); read only
+    _NVML_REASONS = (("sw_power_cap", 0x4), ("hw_slowdown", 0x8), ("sw_thermal_slowdown", 0x20),
+                     ("hw_thermal_slowdown", 0x40))
+
+    def _nvml_start(self):
+        """Samples SM clock and clock-event reasons every 10 ms through NVML in a
+        thread (nvidia-smi's 200 ms loop gives a timed region of a few hundred
+        ms only two or three samples).  Returns False if NVML is unavailable."""
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+        except Exception:
+            return False
+        handle = None
+        try:
+            count = pynvml.nvmlDeviceGetCount()
+            if self.uuid is None and count != 1:
+                return False  # NVML indices ignore CUDA_VISIBLE_DEVICES: match by UUID or not at all
+            for i in range(count):
+                h = pynvml.nvmlDeviceGetHandleByIndex(i)
+                u = pynvml.nvmlDeviceGetUUID(h)
+                u = u.decode() if isinstance(u, bytes) else u
+                if self.uuid is None or u.lower() == self.uuid.lower():
+                    handle = h
+                    break
+        except Exception:
+            handle = None
+        if handle is None:
+            return False
+        import threading
+        self._nvml, self._h, self._samples, self._stop = pynvml, handle, [], threading.Event()
+
+        def loop():
+            while not self._stop.is_set():
+                try:
+                    sm = self._nvml.nvmlDeviceGetClockInfo(self._h, self._nvml.NVML_CLOCK_SM)
+                    smax = self._nvml.nvmlDeviceGetMaxClockInfo(self._h, self._nvml.NVML_CLOCK_SM)
+                    get = getattr(self._nvml, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
+                        self._nvml.nvmlDeviceGetCurrentClocksThrottleReasons
+                    rs = get(self._h)
+                    self._samples.append((sm, smax, rs))
+                except Exception:
+                    pass
+                self._stop.wait(0.01)
+
+        self._thread = threading.Thread(target=loop, daemon=True)
+        self._thread.start()
+        return True
+
+    def _nvml_stop(self):
+        self._stop.set()
+        self._thread.join(timeout=5)
+        sm = [x[0] for x in self._samples]
+        smax = [x[1] for x in self._samples]
+        reasons = {nm for _, _, rs in self._samples for nm, bit in self._NVML_REASONS if rs & bit}
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(smax) if smax else None,
+                "reasons": sorted(reasons), "samples": len(sm), "source": "NVML, every 10 ms"}
+
     def start(self):
+        self.nvml = self._nvml_start()
+        if self.nvml:
+            return
         cmd = ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits", "-lms", "200"]
         if self.uuid:
             cmd += ["-i", self.uuid]
@@ -207,6 +268,8 @@ class ClockSampler:
             self.proc = None
 
     def stop(self):
+        if getattr(self, "nvml", False):
+            return self._nvml_stop()
         if self.proc is None:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
         self.proc.terminate()
