@@ -604,41 +604,43 @@ def run_native(args, wl):
     tokens_per_step = {"layer": B * N, "sampler": B * N * len(calls), "stream": B * lay.n_noisy * len(calls)}[kind]
 
     step_no = [0]
+    hcur = [h]  # the input buffer a step runs on (the pipelined end-to-end loop alternates two)
 
     def step(stage_evs=None, commit_evs=None):
         b = step_no[0]
         step_no[0] += 1
+        hp = hcur[0].data_ptr()
         L.cosmot_build_layout(spec_for(b), pos.data_ptr(), chunk.data_ptr(), 0, sh)
         L.cosmot_mrope_table(pos.data_ptr(), N, dims_s.head_dim, dims_s.rope_sections, dims_s.rope_base,
                              cs.data_ptr(), sh)
         for i, (c, s0, s1) in enumerate(calls):
             if ca:
-                L.cosmot_policy_step(dims, stack.cw, seqs[c], act_desc(s0, s1), h.data_ptr(), h_out.data_ptr(), s0,
+                L.cosmot_policy_step(dims, stack.cw, seqs[c], act_desc(s0, s1), hp, h_out.data_ptr(), s0,
                                      s1, wl.guidance, ws.data_ptr(), ws.numel(), sh,
                                      [e.cuda_event for e in stage_evs[i]] if stage_evs is not None else None)
             elif stack is not None:
                 if stage_evs is not None:
-                    L.cosmot_stack_forward_timed(dims, stack.cw, seqs[c], h.data_ptr(), h_out.data_ptr(), s0, s1,
+                    L.cosmot_stack_forward_timed(dims, stack.cw, seqs[c], hp, h_out.data_ptr(), s0, s1,
                                                  ws.data_ptr(), ws.numel(), sh, [e.cuda_event for e in stage_evs[i]],
                                                  step_ios[i])
                 else:
-                    L.cosmot_stack_forward_io(dims, stack.cw, seqs[c], h.data_ptr(), h_out.data_ptr(), s0, s1,
+                    L.cosmot_stack_forward_io(dims, stack.cw, seqs[c], hp, h_out.data_ptr(), s0, s1,
                                               step_ios[i], ws.data_ptr(), ws.numel(), sh)
             elif stage_evs is not None:
-                L.cosmot_layer_forward_timed(dims, layer.cw, seqs[c], h.data_ptr(), h_out.data_ptr(), s0, s1,
+                L.cosmot_layer_forward_timed(dims, layer.cw, seqs[c], hp, h_out.data_ptr(), s0, s1,
                                              ws.data_ptr(), ws.numel(), sh, [e.cuda_event for e in stage_evs[i]],
                                              wl.guidance, step_ios[i])
             elif guided:
-                L.cosmot_layer_forward_cfg(dims, layer.cw, seqs[c], h.data_ptr(), h_out.data_ptr(), s0, s1,
+                L.cosmot_layer_forward_cfg(dims, layer.cw, seqs[c], hp, h_out.data_ptr(), s0, s1,
                                            wl.guidance, ws.data_ptr(), ws.numel(), sh)
             else:
-                L.cosmot_layer_forward_io(dims, layer.cw, seqs[c], h.data_ptr(), h_out.data_ptr(), s0, s1,
+                L.cosmot_layer_forward_io(dims, layer.cw, seqs[c], hp, h_out.data_ptr(), s0, s1,
                                           step_ios[i], ws.data_ptr(), ws.numel(), sh)
         if kind == "stream":
             if commit_evs is not None:
                 commit_evs[0].record(stream)
             slot = b % wl.stream.cached_blocks
-            L.cosmot_layer_commit_kv(dims, layer.cw, commit_seq, h.data_ptr(),
+            L.cosmot_layer_commit_kv(dims, layer.cw, commit_seq, hp,
                                      lay.n_ar + slot * lay.n_noisy, ws.data_ptr(), ws.numel(), sh)
             if commit_evs is not None:
                 commit_evs[1].record(stream)
@@ -760,13 +762,24 @@ def run_native(args, wl):
         serial_ms = reduce_max(sum(e_s[i].elapsed_time(e_e[i]) for i in range(args.steps)), dev)
 
         # (b) pipelined, as a serving loop runs it: a copy stream uploads step
-        # i+1's inputs into device staging buffers and downloads step i-1's
-        # result while step i computes; every step's copies are inside the
-        # timed region (one event pair around all K steps, L2 flushed before
-        # each step's compute).
+        # i+1's inputs and downloads step i-1's result while step i computes;
+        # every step's copies are inside the timed region (one event pair
+        # around all K steps, L2 flushed before each step's compute).  Without
+        # an action state the step's own input buffer alternates between two
+        # (the uploads land in it and the result is read from it: no device
+        # copy on the compute stream); a policy step stages its inputs.
         cstream = torch.cuda.Stream(dev)
-        st_in = [[torch.empty_like(dst) for dst, _ in ins] for _ in range(2)]
-        st_out = [[torch.empty_like(src) for _, src in outs] for _ in range(2)]
+        direct = not ca
+        h_alt = h.clone() if direct else None
+
+        def same_view(v, base):  # view v of h, taken of the other buffer
+            return base.as_strided(v.size(), v.stride(), v.storage_offset())
+        if direct:
+            st_in = [[dst for dst, _ in ins], [same_view(dst, h_alt) for dst, _ in ins]]
+            st_out = [[src for _, src in outs], [same_view(src, h_alt) for _, src in outs]]
+        else:
+            st_in = [[torch.empty_like(dst) for dst, _ in ins] for _ in range(2)]
+            st_out = [[torch.empty_like(src) for _, src in outs] for _ in range(2)]
         h_out_pin = [[torch.empty_like(dst).pin_memory() for dst, _ in outs] for _ in range(2)]
         K = args.steps
         ev = {k: [torch.cuda.Event() for _ in range(K)] for k in ("in", "used", "out", "down")}
@@ -776,8 +789,8 @@ def run_native(args, wl):
 
         def upload(i):
             with torch.cuda.stream(cstream):
-                if i >= 2:
-                    cstream.wait_event(ev["used"][i - 2])  # the slot's previous contents consumed
+                if i >= 2:  # the slot's previous contents consumed (and, direct, its result downloaded)
+                    cstream.wait_event(ev["down" if direct else "used"][i - 2])
                 for stg, (_, src) in zip(st_in[i % 2], ins):
                     stg.copy_(src, non_blocking=True)
                 ev["in"][i].record(cstream)
@@ -789,14 +802,18 @@ def run_native(args, wl):
                 upload(i + 1)
             stream.wait_event(ev["in"][i])
             flush.zero_()
-            for stg, (dst, _) in zip(st_in[i % 2], ins):
-                dst.copy_(stg, non_blocking=True)
+            if direct:
+                hcur[0] = h if i % 2 == 0 else h_alt
+            else:
+                for stg, (dst, _) in zip(st_in[i % 2], ins):
+                    dst.copy_(stg, non_blocking=True)
             ev["used"][i].record(stream)
             step()
-            if i >= 2:
-                stream.wait_event(ev["down"][i - 2])  # the output slot's previous download done
-            for stg, (_, src) in zip(st_out[i % 2], outs):
-                stg.copy_(src, non_blocking=True)
+            if not direct:
+                if i >= 2:
+                    stream.wait_event(ev["down"][i - 2])  # the output slot's previous download done
+                for stg, (_, src) in zip(st_out[i % 2], outs):
+                    stg.copy_(src, non_blocking=True)
             ev["out"][i].record(stream)
             with torch.cuda.stream(cstream):
                 cstream.wait_event(ev["out"][i])
@@ -806,12 +823,14 @@ def run_native(args, wl):
         stream.wait_event(ev["down"][K - 1])
         p_e.record(stream)
         torch.cuda.synchronize()
+        hcur[0] = h
         e2e_ms = reduce_max(p_s.elapsed_time(p_e), dev)
         e2e = {"value": job_throughput(tokens_per_step, args.steps, world, e2e_ms), "unit": UNIT,
                "h2d_bytes_per_step": int(sum(src.numel() * 2 for _, src in ins)),
                "d2h_bytes_per_step": int(sum(dst.numel() * 2 for dst, _ in outs)),
                "ms_per_step": e2e_ms / args.steps,
-               "mode": "pipelined: a second stream uploads step i+1 and downloads step i-1 while step i computes",
+               "mode": "pipelined: a second stream uploads step i+1 and downloads step i-1 while step i computes"
+                       + ("; the step's input buffer alternates between two" if direct else "; inputs staged"),
                "serial": {"value": job_throughput(tokens_per_step, args.steps, world, serial_ms),
                           "ms_per_step": serial_ms / args.steps},
                "path": "cosmot_build_layout + cosmot_mrope_table + "
