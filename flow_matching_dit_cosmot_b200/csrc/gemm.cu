@@ -56,7 +56,7 @@ constexpr int kGroupM = 16;
 template <int BN, int CG = 1>
 struct Tiles {
   static_assert(BN % 32 == 0 && BN >= 32 && BN <= 256, "tile width");
-  static_assert(CG == 1 || (CG == 2 && BN == 256), "pair tiles are 256 x 256");
+  static_assert(CG == 1 || (CG == 2 && (BN == 256 || BN == 224)), "pair tiles are 256 x 256 or 256 x 224");
   static constexpr int STAGES = CG == 2 ? 6 : 4;
   static constexpr int B_BYTES = BN * BK * 2 / CG;  // this CTA's B rows
   static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
@@ -646,6 +646,7 @@ extern "C" cosmot_status cosmot_routed_linear(const void* a, int64_t ld_a, int64
   p.a_rows = max_row;
   if (mt == 0) return COSMOT_OK;
   const int64_t sms = num_sms();
+  auto rounds = [](int64_t tiles, int64_t slots) { return (tiles + slots - 1) / slots; };
   if (max_row > INT32_MAX) return COSMOT_ERR_UNSUPPORTED;
   const bool silu = kind == COSMOT_EPI_SILU_MUL;
   // Tile width: 160 instead of 256 when that keeps clearly more SMs busy over
@@ -660,17 +661,36 @@ extern "C" cosmot_status cosmot_routed_linear(const void* a, int64_t ld_a, int64
     if (eff(160) > eff(256) + 0.1) bn = 160;
   }
   p.num_n_tiles = (int32_t)((n_out + (silu ? bn / 2 : bn) - 1) / (silu ? bn / 2 : bn));
-  // CTA pairs (256-row tiles, half the B bytes a CTA) unless they need more
-  // than 10 % more rounds over the SMs than single-CTA tiles: a pair's round
-  // is the shorter one (the single-CTA main loop waits on its loads ~20 % of
-  // the time; measured on the 480p layer, pairs took QKV from 1.49 to 1.38 ms
-  // and the O projection from 0.57 to 0.50 ms).
+  // CTA pairs (256-row tiles, half the B bytes a CTA) when their rounds over
+  // the SMs, times the tile width, cost no more than single-CTA tiles' with a
+  // 20 % surcharge for the single-CTA main loop's load waits (a clock64
+  // trace: 20-25 % of each tile against 12 % for pairs).  Pairs are 256 or
+  // 224 columns wide (224 fills the last round better at a few thousand
+  // rows; mRoPE and SiLU*mul keep 256).  On the 480p layer pairs took QKV
+  // from 1.49 to 1.38 ms and the O projection from 0.57 to 0.50 ms.
   int cg = 1;
-  if (bn == 256) {
+  {
     const int64_t pairs = resident_pairs();
     if (pairs > 0) {
-      const int64_t t1 = mt1 * p.num_n_tiles, t2 = count_mtiles(2 * BM) * p.num_n_tiles;
-      if ((t2 + pairs - 1) / pairs * 10 <= (t1 + sms - 1) / sms * 11) cg = 2;
+      const int64_t cost1 = rounds(mt1 * p.num_n_tiles, sms) * bn * 6;  // x 5, plus the 20 %
+      const int64_t mt2 = count_mtiles(2 * BM);
+      const bool narrow_ok = kind == COSMOT_EPI_NONE || kind == COSMOT_EPI_RESIDUAL || kind == COSMOT_EPI_EULER;
+      int best = 0;
+      int64_t best_cost = cost1;
+      for (int w : {256, 224}) {
+        if (w != 256 && !narrow_ok) continue;
+        const int64_t cols = silu ? w / 2 : w;
+        const int64_t cost = rounds(mt2 * ((n_out + cols - 1) / cols), pairs) * w * 5;
+        if (cost <= best_cost) {
+          best_cost = cost;
+          best = w;
+        }
+      }
+      if (best) {
+        cg = 2;
+        bn = best;
+        p.num_n_tiles = (int32_t)((n_out + (silu ? bn / 2 : bn) - 1) / (silu ? bn / 2 : bn));
+      }
     }
   }
   const int64_t tm = (int64_t)BM * cg;
@@ -730,7 +750,7 @@ extern "C" cosmot_status cosmot_routed_linear(const void* a, int64_t ld_a, int64
   const void* wu[2] = {w0_up, w1_up};
   // a CTA's B box: the tile's columns, the gate or up half for SiLU*mul, and
   // for a pair of CTAs one half of either
-  const uint32_t brows = cg == 2 ? 128u : (silu ? bn / 2 : bn);
+  const uint32_t brows = cg == 2 ? (uint32_t)bn / 2 : (silu ? bn / 2 : bn);
   for (int s = 0; s < 2; ++s) {
     const int src = uses[s] ? s : (uses[0] ? 0 : 1);  // an unused set reuses a valid map
     if (!wb[src]) return COSMOT_ERR_INVALID_ARG;
@@ -745,6 +765,23 @@ extern "C" cosmot_status cosmot_routed_linear(const void* a, int64_t ld_a, int64
     }
   }
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (cg == 2 && bn == 224) {
+    switch (kind) {
+      case COSMOT_EPI_NONE: return launch<COSMOT_EPI_NONE, 0, 224, 2>(ta, tb[0], tb[1], tu[0], tu[1], p, s);
+      case COSMOT_EPI_EULER: return launch<COSMOT_EPI_EULER, 0, 224, 2>(ta, tb[0], tb[1], tu[0], tu[1], p, s);
+      default:
+        switch (flags) {
+          case COSMOT_EPI_OUT_F32:
+            return launch<COSMOT_EPI_RESIDUAL, COSMOT_EPI_OUT_F32, 224, 2>(ta, tb[0], tb[1], tu[0], tu[1], p, s);
+          case COSMOT_EPI_RES_F32:
+            return launch<COSMOT_EPI_RESIDUAL, COSMOT_EPI_RES_F32, 224, 2>(ta, tb[0], tb[1], tu[0], tu[1], p, s);
+          case COSMOT_EPI_OUT_F32 | COSMOT_EPI_RES_F32:
+            return launch<COSMOT_EPI_RESIDUAL, COSMOT_EPI_OUT_F32 | COSMOT_EPI_RES_F32, 224, 2>(ta, tb[0], tb[1], tu[0],
+                                                                                              tu[1], p, s);
+          default: return launch<COSMOT_EPI_RESIDUAL, 0, 224, 2>(ta, tb[0], tb[1], tu[0], tu[1], p, s);
+        }
+    }
+  }
   if (cg == 2) {
     switch (kind) {
       case COSMOT_EPI_NONE: return launch<COSMOT_EPI_NONE, 0, 256, 2>(ta, tb[0], tb[1], tu[0], tu[1], p, s);

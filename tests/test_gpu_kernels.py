@@ -162,6 +162,29 @@ def test_routed_linear_pair_and_single_tiles_agree_bit_for_bit():
     np.testing.assert_array_equal(bits(narrow), bits(wide[:, :256]))
 
 
+def test_routed_linear_224_wide_pair_tiles():
+    """A few thousand rows against a 4096-wide output (a streaming step's O,
+    down and velocity projections) run 256 x 224 pair tiles: 1,560 rows are
+    7 pair row tiles, and 19 column tiles of 224 fill the second of two
+    rounds over 74 pairs better than 16 of 256.  Residual epilogue with a
+    float32 output, two segments, against the reference."""
+    m_total, k, n_out = 1560, 256, 4096
+    a, w0, w1, segs, acc = _gemm_case(60, m_total, k, n_out, seed=8)
+    rng = np.random.default_rng(23)
+    res = rng.standard_normal((m_total, n_out)).astype(np.float32)
+    out = torch.full((m_total, n_out), float("nan"), dtype=torch.float32, device="cuda")
+    ad, w0d, w1d, rd = to_dev(a), to_dev(w0), to_dev(w1), torch.from_numpy(res).cuda()
+    e = L.Epilogue(kind=L.COSMOT_EPI_RESIDUAL, res=A.ptr(rd), ld_res=n_out,
+                   flags=L.COSMOT_EPI_OUT_F32 | L.COSMOT_EPI_RES_F32)
+    L.cosmot_routed_linear(A.ptr(ad), k, k, segs, A.ptr(w0d), A.ptr(w1d), n_out, A.ptr(out), n_out, e,
+                           stream=A.stream_handle())
+    torch.cuda.synchronize()
+    assert_device_ok()
+    got = out.double().cpu().numpy()
+    # fp32 accumulation and one fp32 add: far inside the bf16 bounds
+    assert np.abs(got - (acc + res.astype(np.float64))).max() < 1e-4
+
+
 def test_routed_linear_equal_sets_equal_single_segment():
     """With both weight sets holding the same matrix (in separate buffers) the
     routed projection is bit-identical to one segment over all rows: routing
