@@ -230,7 +230,8 @@ __device__ __forceinline__ void umma_commit_pair_mc(uint32_t bar, uint16_t cta_m
                : "memory");
 }
 // A tile load of one CTA of the pair whose completion is counted on the even
-// CTA's barrier (`bar_cluster`, a shared::cluster address).  No multicast.
+// CTA's barrier (`bar_cluster`, a shared::cluster address); the data lands in
+// this CTA's own shared memory only.
 __device__ __forceinline__ void tma_load_2d_pair(uint32_t dst, const CUtensorMap* map, uint32_t bar_cluster, int c0,
                                                  int c1) {
   asm volatile(
