@@ -46,13 +46,14 @@ constexpr int kGroupM = 16;
 // output: 5 row tiles x 16 column tiles = 80 tiles for 148 SMs become 5 x 26
 // = 130).  Any multiple of 32 up to 256 is a valid tcgen05 N for M = 128.
 //
-// CG = 2: a cluster of two CTAs computes a 256-row tile with
-// tcgen05.mma.cta_group::2 (M = 256): each CTA loads its own 128 A rows and
-// half of the B rows (the gate or the up half for SiLU*mul), so a CTA moves
-// 32 KB per k-block instead of 48 KB for the same work, and six stages fit.
-// The even CTA's full barrier counts both CTAs' bytes; its MMA thread commits
-// to both CTAs' barriers; both epilogues release an accumulator on the even
-// CTA's barrier.  Single-CTA tiles (CG = 1) stay for calls with few rows.
+// CG = 2: a cluster of two CTAs computes a 256-row tile, 256 (or 224) columns
+// wide, with tcgen05.mma.cta_group::2 (M = 256): each CTA loads its own 128 A
+// rows and half of the B rows (the gate or the up half for SiLU*mul), so a
+// CTA moves 32 KB per k-block instead of 48 KB for the same work, and six
+// stages fit.  The even CTA's full barrier counts both CTAs' bytes; its MMA
+// thread commits to both CTAs' barriers; both epilogues release an
+// accumulator on the even CTA's barrier.  The tile plan (cosmot_routed_linear)
+// keeps single-CTA tiles (CG = 1) for calls with a few hundred rows.
 template <int BN, int CG = 1>
 struct Tiles {
   static_assert(BN % 32 == 0 && BN >= 32 && BN <= 256, "tile width");
