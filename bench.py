@@ -248,6 +248,10 @@ class ClockSampler:
     def _nvml_stop(self):
         self._stop.set()
         self._thread.join(timeout=5)
+        try:
+            self._nvml.nvmlShutdown()
+        except Exception:
+            pass
         sm = [x[0] for x in self._samples]
         smax = [x[1] for x in self._samples]
         reasons = {nm for _, _, rs in self._samples for nm, bit in self._NVML_REASONS if rs & bit}
