@@ -45,6 +45,9 @@ constexpr int kGroupM = 16;
 // fill the SMs with 256-wide ones (a few hundred rows against a 4096-wide
 // output: 5 row tiles x 16 column tiles = 80 tiles for 148 SMs become 5 x 26
 // = 130).  Any multiple of 32 up to 256 is a valid tcgen05 N for M = 128.
+// Such calls read their weights cold, once, and wait on the loads, so tiles
+// up to 160 wide keep six stages in flight (216 KB) where 256-wide ones fit
+// four.
 //
 // CG = 2: a cluster of two CTAs computes a 256-row tile, 256 (or 224) columns
 // wide, with tcgen05.mma.cta_group::2 (M = 256): each CTA loads its own 128 A
@@ -58,10 +61,11 @@ template <int BN, int CG = 1>
 struct Tiles {
   static_assert(BN % 32 == 0 && BN >= 32 && BN <= 256, "tile width");
   static_assert(CG == 1 || (CG == 2 && (BN == 256 || BN == 224)), "pair tiles are 256 x 256 or 256 x 224");
-  static constexpr int STAGES = CG == 2 ? 6 : 4;
+  static constexpr int STAGES = CG == 2 || BN <= 160 ? 6 : 4;
   static constexpr int B_BYTES = BN * BK * 2 / CG;  // this CTA's B rows
   static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
   static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 256 + 1024;
+  static_assert(SMEM_BYTES <= 227 * 1024, "shared memory per CTA");
   static constexpr uint32_t IDESC = idesc_bf16_f32(BM * CG, BN, false, false);
 };
 
