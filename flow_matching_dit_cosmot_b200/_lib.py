@@ -389,7 +389,7 @@ def cosmot_action_head(h_last: int, ld_h: int, segs, g_fin: int, eps: float, w_o
 def cosmot_policy_step(dims: Dims, layers, seq: SeqDesc, act: ActionDesc, h: int, h_out: int, sigma: float,
                        sigma_next: float, guidance, workspace: int, workspace_bytes: int, stream: int = 0,
                        events=None, check=True):
-    """`events`: None, or 8 * len(layers) + 2 raw cudaEvent_t handles (ints)."""
+    """`events`: None, or 8 * len(layers) + 2 raw cudaEvent_t handles (ints; None skips that boundary)."""
     if not isinstance(layers, ctypes.Array):
         layers = (LayerWeights * len(layers))(*layers)
     g = ctypes.byref(c_f64(guidance)) if guidance is not None else None
@@ -452,7 +452,7 @@ def cosmot_stack_forward_io(dims: Dims, layers, seq: SeqDesc, h: int, h_out: int
 def cosmot_stack_forward_timed(dims: Dims, layers, seq: SeqDesc, h: int, h_out: int, sigma: float,
                                sigma_next: float, workspace: int, workspace_bytes: int, stream: int, events,
                                io: StepIO | None = None, check=True):
-    """`events`: 8 * len(layers) + 2 raw cudaEvent_t handles (ints)."""
+    """`events`: 8 * len(layers) + 2 raw cudaEvent_t handles (ints; None skips that boundary)."""
     if not isinstance(layers, ctypes.Array):
         layers = (LayerWeights * len(layers))(*layers)
     arr = (c_vp * len(events))(*[c_vp(e) for e in events])
@@ -471,7 +471,7 @@ def cosmot_layer_forward_noalloc(dims: Dims, w: LayerWeights, seq: SeqDesc, h: i
 def cosmot_layer_forward_timed(dims: Dims, w: LayerWeights, seq: SeqDesc, h: int, h_out: int, sigma: float,
                                sigma_next: float, workspace: int, workspace_bytes: int, stream: int, events,
                                guidance: float | None = None, io: StepIO | None = None, check=True):
-    """`events`: COSMOT_LAYER_STAGES + 1 raw cudaEvent_t handles (ints); `guidance`
+    """`events`: COSMOT_LAYER_STAGES + 1 raw cudaEvent_t handles (ints; None skips that boundary); `guidance`
     selects the guided step of cosmot_layer_forward_cfg; `io` the float32 state
     and velocity output of cosmot_layer_forward_io."""
     arr = (c_vp * len(events))(*[c_vp(e) for e in events])

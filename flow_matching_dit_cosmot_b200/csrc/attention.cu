@@ -278,6 +278,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     tmem_alloc(smem_u32(tmem_slot), TMEM_COLS);
     tmem_relinquish();
   }
+  // Up to here the CTA touched only its own shared and tensor memory and the
+  // kernel parameters, so this prologue may overlap the previous kernel.
+  pdl_trigger();
+  pdl_wait();
   bool use_visit = kSkip && skips_tiles(p, w);  // CTA-uniform
   if (use_visit) {
     // A tile is visited iff one of its keys is visible to the item's latest
@@ -631,7 +635,9 @@ cosmot_status launch(const CUtensorMap& tq, const CUtensorMap& tk, const CUtenso
       if (dev < 64) done_mask |= 1ull << dev;
     }
   }
-  mot_attention_kernel<HD, kSkip><<<grid, NUM_THREADS, Cfg<HD>::SMEM_BYTES, s>>>(tq, tk, tv, p);
+  if (launch_pdl(mot_attention_kernel<HD, kSkip>, dim3(grid), dim3(NUM_THREADS), Cfg<HD>::SMEM_BYTES, s, nullptr, tq,
+                 tk, tv, p) != cudaSuccess)
+    return COSMOT_ERR_CUDA;
   return launch_status();
 }
 
@@ -738,6 +744,8 @@ namespace attn {
 // each lane HD/32 columns; a row no split saw (every w_s = 0) outputs 0.
 template <int HD>
 __global__ void __launch_bounds__(256) attn_merge_kernel(const Params p) {
+  pdl_trigger();
+  pdl_wait();
   const int64_t warp = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   const int lane = threadIdx.x & 31;
   const int64_t total = (int64_t)p.batch * (p.n_q - p.n_q_ar) * p.n_heads;
@@ -858,10 +866,9 @@ cosmot_status attention_impl(const cosmot_attn_desc* d, const void* q, int64_t l
   if (st != COSMOT_OK || kv_split == 1 || d->n_q == p.n_q_ar) return st;
   const int64_t warps = (int64_t)d->batch * (d->n_q - p.n_q_ar) * d->n_heads;
   const unsigned mgrid = (unsigned)((warps + 7) / 8);
-  if (hd == 128)
-    attn_merge_kernel<128><<<mgrid, 256, 0, s>>>(p);
-  else
-    attn_merge_kernel<64><<<mgrid, 256, 0, s>>>(p);
+  const cudaError_t e = hd == 128 ? launch_pdl(attn_merge_kernel<128>, dim3(mgrid), dim3(256), 0, s, nullptr, p)
+                                  : launch_pdl(attn_merge_kernel<64>, dim3(mgrid), dim3(256), 0, s, nullptr, p);
+  if (e != cudaSuccess) return COSMOT_ERR_CUDA;
   return launch_status();
 }
 

@@ -44,6 +44,30 @@ inline cosmot_status launch_status() {
 
 int num_sms();
 
+// Launches a kernel with programmatic stream serialization: it may be
+// scheduled while the previous kernel of the stream drains, so its prologue
+// (barrier setup, tensor-memory allocation, descriptor prefetch) overlaps that
+// kernel's last wave.  The kernel must execute pdl_wait (ptx.cuh) in every
+// thread before touching memory an earlier kernel writes or reads, and before
+// it exits.  `extra` adds one more launch attribute (a cluster shape).
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s,
+                              const cudaLaunchAttribute* extra, Args&&... args) {
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  unsigned n = 1;
+  if (extra != nullptr) attr[n++] = *extra;
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cfg.attrs = attr;
+  cfg.numAttrs = n;
+  return cudaLaunchKernelEx(&cfg, kern, static_cast<Args&&>(args)...);
+}
+
 // cosmot_rmsnorm_routed with a float32 input when h_f32 (the layer's h1, the
 // residual stream between the attention and FFN halves, is kept in float32).
 cosmot_status rmsnorm_routed(const void* h, bool h_f32, int64_t ld_h, const cosmot_segment* segs, int32_t n_segs,

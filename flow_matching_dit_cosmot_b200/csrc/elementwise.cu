@@ -59,6 +59,8 @@ __global__ void __launch_bounds__(256) rmsnorm_f32in_kernel(const float* __restr
                                                             const __nv_bfloat16* __restrict__ g1, int32_t d, float eps,
                                                             __nv_bfloat16* __restrict__ out, int64_t ld_out,
                                                             int* status) {
+  pdl_trigger();
+  pdl_wait();
   const int lane = threadIdx.x & 31;
   const int64_t warps_total = (int64_t)gridDim.x * (blockDim.x >> 5);
   const int nvec = d >> 3;
@@ -123,6 +125,8 @@ __global__ void __launch_bounds__(kNormBlock) rmsnorm_block_kernel(const TIn* __
                                                                   const __nv_bfloat16* __restrict__ g1, int32_t d,
                                                                   float eps, __nv_bfloat16* __restrict__ out,
                                                                   int64_t ld_out, int* status) {
+  pdl_trigger();
+  pdl_wait();
   constexpr bool kF32 = sizeof(TIn) == 4;
   __shared__ float part[2][kNormBlock / 32];
   const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
@@ -196,6 +200,8 @@ __global__ void __launch_bounds__(256) rmsnorm_kernel(const __nv_bfloat16* __res
                                                       const __nv_bfloat16* __restrict__ g1, int32_t d, float eps,
                                                       __nv_bfloat16* __restrict__ out, int64_t ld_out,
                                                       int* status) {
+  pdl_trigger();
+  pdl_wait();
   const int lane = threadIdx.x & 31;
   const int64_t warps_total = (int64_t)gridDim.x * (blockDim.x >> 5);
   const int nvec = d >> 3;
@@ -258,6 +264,8 @@ __global__ void __launch_bounds__(256) mrope_kernel(__nv_bfloat16* __restrict__ 
                                                     __nv_bfloat16* __restrict__ k, int64_t ld_k, int32_t n_k_heads,
                                                     int64_t n_rows, int32_t head_dim,
                                                     const float2* __restrict__ cs) {
+  pdl_trigger();
+  pdl_wait();
   const int32_t half = head_dim >> 1;
   const int32_t groups = half >> 3;
   const int32_t per_row = (n_q_heads + n_k_heads) * groups;
@@ -301,6 +309,8 @@ __global__ void __launch_bounds__(256) euler_kernel(__nv_bfloat16* __restrict__ 
                                                     const __nv_bfloat16* __restrict__ v, int64_t ld_v,
                                                     int64_t row_begin, int64_t n_rows, int64_t n_cols, float dsigma,
                                                     int* status) {
+  pdl_trigger();
+  pdl_wait();
   const int64_t vec_per_row = n_cols >> 3;
   const int64_t total = n_rows * vec_per_row;
   for (int64_t e = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; e < total; e += (int64_t)gridDim.x * blockDim.x) {
@@ -330,6 +340,8 @@ __global__ void __launch_bounds__(256) cfg_euler_kernel(__nv_bfloat16* x_cond, _
                                                         const __nv_bfloat16* __restrict__ v_cond,
                                                         const __nv_bfloat16* __restrict__ v_base, int64_t ld_v,
                                                         int64_t n_rows, int64_t n_cols, float dsigma, float w) {
+  pdl_trigger();
+  pdl_wait();
   const int64_t vec_per_row = n_cols >> 3;
   const int64_t total = n_rows * vec_per_row;
   for (int64_t e = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; e < total; e += (int64_t)gridDim.x * blockDim.x) {
@@ -396,25 +408,25 @@ cosmot_status rmsnorm_routed(const void* h, bool h_f32, int64_t ld_h, const cosm
     if (h_f32) {
       const auto* hf = static_cast<const float*>(h);
       if (vpt <= 4)
-        rmsnorm_block_kernel<float, 4><<<bgrid, kNormBlock, 0, s>>>(hf, ld_h, t, gp0, gp1, (int32_t)d, eps, op, ld_out, st);
+        (void)launch_pdl(rmsnorm_block_kernel<float, 4>, dim3(bgrid), dim3(kNormBlock), 0, s, nullptr, hf, ld_h, t, gp0, gp1, (int32_t)d, eps, op, ld_out, st);
       else
-        rmsnorm_block_kernel<float, 6><<<bgrid, kNormBlock, 0, s>>>(hf, ld_h, t, gp0, gp1, (int32_t)d, eps, op, ld_out, st);
+        (void)launch_pdl(rmsnorm_block_kernel<float, 6>, dim3(bgrid), dim3(kNormBlock), 0, s, nullptr, hf, ld_h, t, gp0, gp1, (int32_t)d, eps, op, ld_out, st);
     } else {
       if (vpt <= 4)
-        rmsnorm_block_kernel<__nv_bfloat16, 4><<<bgrid, kNormBlock, 0, s>>>(hp, ld_h, t, gp0, gp1, (int32_t)d, eps, op,
+        (void)launch_pdl(rmsnorm_block_kernel<__nv_bfloat16, 4>, dim3(bgrid), dim3(kNormBlock), 0, s, nullptr, hp, ld_h, t, gp0, gp1, (int32_t)d, eps, op,
                                                                            ld_out, st);
       else
-        rmsnorm_block_kernel<__nv_bfloat16, 6><<<bgrid, kNormBlock, 0, s>>>(hp, ld_h, t, gp0, gp1, (int32_t)d, eps, op,
+        (void)launch_pdl(rmsnorm_block_kernel<__nv_bfloat16, 6>, dim3(bgrid), dim3(kNormBlock), 0, s, nullptr, hp, ld_h, t, gp0, gp1, (int32_t)d, eps, op,
                                                                            ld_out, st);
     }
     return launch_status();
   }
   // narrow rows (d < 1024): one warp per row, at most 4 vectors per lane
   if (h_f32)
-    rmsnorm_f32in_kernel<4><<<grid, threads, 0, s>>>(static_cast<const float*>(h), ld_h, t, gp0, gp1, (int32_t)d, eps,
+    (void)launch_pdl(rmsnorm_f32in_kernel<4>, dim3(grid), dim3(threads), 0, s, nullptr, static_cast<const float*>(h), ld_h, t, gp0, gp1, (int32_t)d, eps,
                                                      op, ld_out, st);
   else
-    rmsnorm_kernel<4><<<grid, threads, 0, s>>>(hp, ld_h, t, gp0, gp1, (int32_t)d, eps, op, ld_out, st);
+    (void)launch_pdl(rmsnorm_kernel<4>, dim3(grid), dim3(threads), 0, s, nullptr, hp, ld_h, t, gp0, gp1, (int32_t)d, eps, op, ld_out, st);
   return launch_status();
 }
 
@@ -442,7 +454,7 @@ cosmot_status cosmot_mrope_apply(void* q, int64_t ld_q, int32_t n_q_heads, void*
   const int64_t items = n_rows * (n_q_heads + n_k_heads) * (head_dim / 16);
   if (items == 0) return COSMOT_OK;
   const int threads = 256;
-  mrope_kernel<<<grid_for(items, threads), threads, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
+  (void)launch_pdl(mrope_kernel, dim3(grid_for(items, threads)), dim3(threads), 0, reinterpret_cast<cudaStream_t>(stream), nullptr, 
       static_cast<__nv_bfloat16*>(q), ld_q, n_q_heads, static_cast<__nv_bfloat16*>(k), ld_k, n_k_heads, n_rows,
       head_dim, reinterpret_cast<const float2*>(cs));
   return launch_status();
@@ -461,7 +473,7 @@ cosmot_status cosmot_flow_euler_step(void* x, int64_t ld_x, const void* v, int64
   const int threads = 256;
   int* st = device_status_ptr();
   if (!st) return COSMOT_ERR_CUDA;
-  euler_kernel<<<grid_for(items, threads), threads, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
+  (void)launch_pdl(euler_kernel, dim3(grid_for(items, threads)), dim3(threads), 0, reinterpret_cast<cudaStream_t>(stream), nullptr, 
       static_cast<__nv_bfloat16*>(x), ld_x, static_cast<const __nv_bfloat16*>(v), ld_v, row_begin,
       row_end - row_begin, n_cols, dsigma, st);
   return launch_status();
@@ -477,7 +489,7 @@ cosmot_status cosmot_flow_cfg_euler_step(void* x_cond, void* x_base, int64_t ld_
   const int64_t items = n_rows * (n_cols / 8);
   if (items == 0) return COSMOT_OK;
   const int threads = 256;
-  cfg_euler_kernel<<<grid_for(items, threads), threads, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
+  (void)launch_pdl(cfg_euler_kernel, dim3(grid_for(items, threads)), dim3(threads), 0, reinterpret_cast<cudaStream_t>(stream), nullptr, 
       static_cast<__nv_bfloat16*>(x_cond), static_cast<__nv_bfloat16*>(x_base), ld_x,
       static_cast<const __nv_bfloat16*>(v_cond), static_cast<const __nv_bfloat16*>(v_base), ld_v, n_rows, n_cols,
       (float)(sigma_next - sigma), (float)guidance);

@@ -244,17 +244,23 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   if constexpr (CG == 2) cluster_sync();  // both CTAs' barriers exist before either signals the other
   tc_fence_after();
   const uint32_t tmem_base = *reinterpret_cast<volatile uint32_t*>(tmem_slot);
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_desc(&tmap_a);
+    tma_prefetch_desc(&tmap_b0);
+    tma_prefetch_desc(&tmap_b1);
+    if (EPI == COSMOT_EPI_SILU_MUL) {
+      tma_prefetch_desc(&tmap_u0);
+      tma_prefetch_desc(&tmap_u1);
+    }
+  }
+  // Up to here the CTA touched only its own shared and tensor memory and the
+  // kernel parameters, so this prologue may overlap the previous kernel.
+  pdl_trigger();
+  pdl_wait();
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
-      tma_prefetch_desc(&tmap_a);
-      tma_prefetch_desc(&tmap_b0);
-      tma_prefetch_desc(&tmap_b1);
-      if (EPI == COSMOT_EPI_SILU_MUL) {
-        tma_prefetch_desc(&tmap_u0);
-        tma_prefetch_desc(&tmap_u1);
-      }
       int stage = 0;
       uint32_t phase = 0;
       uint32_t armed_mask = 0, armed_parity = 0;
@@ -577,25 +583,21 @@ cosmot_status launch(const CUtensorMap& ta, const CUtensorMap& tb0, const CUtens
     int pairs = resident_pairs();
     if (pairs < 1) return COSMOT_ERR_CUDA;
     if (p.num_tiles < pairs) pairs = p.num_tiles;
-    cudaLaunchConfig_t cfg{};
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = 2;
-    attr[0].val.clusterDim.y = 1;
-    attr[0].val.clusterDim.z = 1;
-    cfg.gridDim = dim3(2 * pairs, 1, 1);
-    cfg.blockDim = dim3(NUM_THREADS, 1, 1);
-    cfg.dynamicSmemBytes = SMEM_BYTES;
-    cfg.stream = s;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    if (cudaLaunchKernelEx(&cfg, routed_gemm_kernel<EPI, FL, BN, CG>, ta, tb0, tb1, tu0, tu1, p) != cudaSuccess)
+    cudaLaunchAttribute cluster;
+    cluster.id = cudaLaunchAttributeClusterDimension;
+    cluster.val.clusterDim.x = 2;
+    cluster.val.clusterDim.y = 1;
+    cluster.val.clusterDim.z = 1;
+    if (launch_pdl(routed_gemm_kernel<EPI, FL, BN, CG>, dim3(2 * pairs), dim3(NUM_THREADS), SMEM_BYTES, s, &cluster, ta,
+                   tb0, tb1, tu0, tu1, p) != cudaSuccess)
       return COSMOT_ERR_CUDA;
     return launch_status();
   }
   int grid = num_sms();
   if (p.num_tiles < grid) grid = p.num_tiles;
-  routed_gemm_kernel<EPI, FL, BN, CG><<<grid, NUM_THREADS, SMEM_BYTES, s>>>(ta, tb0, tb1, tu0, tu1, p);
+  if (launch_pdl(routed_gemm_kernel<EPI, FL, BN, CG>, dim3(grid), dim3(NUM_THREADS), SMEM_BYTES, s, nullptr, ta, tb0,
+                 tb1, tu0, tu1, p) != cudaSuccess)
+    return COSMOT_ERR_CUDA;
   return launch_status();
 }
 

@@ -138,12 +138,14 @@ cosmot_status cosmot_layer_workspace_size(const cosmot_dims* dims, const cosmot_
 namespace cosmot {
 namespace {
 
-// Records ev[i] (when given) on the stream just before stage i starts.
+// Records ev[i] (when the array and the entry are given) on the stream just
+// before stage i starts.  A NULL entry leaves that boundary unmarked, so the
+// kernels on either side keep their programmatic (overlapped) launch.
 struct StageMarks {
   const cudaEvent_t* ev;
   cudaStream_t s;
   cosmot_status mark(int i) const {
-    if (!ev) return COSMOT_OK;
+    if (!ev || !ev[i]) return COSMOT_OK;
     return cudaEventRecord(ev[i], s) == cudaSuccess ? COSMOT_OK : COSMOT_ERR_CUDA;
   }
 };
@@ -706,11 +708,8 @@ cosmot_status cosmot_policy_step(const cosmot_dims* dims, const cosmot_layer_wei
                                  double sigma, double sigma_next, const double* guidance, void* workspace,
                                  size_t workspace_bytes, cosmot_stream_t stream, void* const* stage_events,
                                  int32_t n_events) {
-  if (stage_events) {
-    if (n_layers < 1 || n_layers > cosmot::kMaxLayers || n_events != 8 * n_layers + 2) return COSMOT_ERR_INVALID_ARG;
-    for (int i = 0; i < n_events; ++i)
-      if (!stage_events[i]) return COSMOT_ERR_INVALID_ARG;
-  }
+  if (stage_events && (n_layers < 1 || n_layers > cosmot::kMaxLayers || n_events != 8 * n_layers + 2))
+    return COSMOT_ERR_INVALID_ARG;
   return cosmot::policy_step_impl(dims, layers, n_layers, seq, act, h, h_out, sigma, sigma_next, guidance, workspace,
                                   workspace_bytes, stream, reinterpret_cast<const cudaEvent_t*>(stage_events));
 }
@@ -759,8 +758,6 @@ cosmot_status cosmot_stack_forward_timed(const cosmot_dims* dims, const cosmot_l
                                          const cosmot_step_io* io) {
   if (!stage_events || n_layers < 1 || n_layers > cosmot::kMaxLayers || n_events != 8 * n_layers + 2)
     return COSMOT_ERR_INVALID_ARG;
-  for (int i = 0; i < n_events; ++i)
-    if (!stage_events[i]) return COSMOT_ERR_INVALID_ARG;
   return cosmot::stack_forward_impl(dims, layers, n_layers, seq, h, h_out, sigma, sigma_next, workspace,
                                     workspace_bytes, stream, reinterpret_cast<const cudaEvent_t*>(stage_events), io);
 }
@@ -771,8 +768,6 @@ cosmot_status cosmot_layer_forward_timed(const cosmot_dims* dims, const cosmot_l
                                          cosmot_stream_t stream, void* const* stage_events, int32_t n_events,
                                          const double* guidance, const cosmot_step_io* io) {
   if (!stage_events || n_events != COSMOT_LAYER_STAGES + 1) return COSMOT_ERR_INVALID_ARG;
-  for (int i = 0; i < n_events; ++i)
-    if (!stage_events[i]) return COSMOT_ERR_INVALID_ARG;
   if (guidance) {
     if (!seq || !dims || seq->batch < 2 || seq->batch % 2) return COSMOT_ERR_INVALID_ARG;
     if ((int64_t)dims->ffn * (seq->n_ar + seq->n_clean + seq->n_noisy) < (int64_t)dims->d_model * seq->n_noisy)

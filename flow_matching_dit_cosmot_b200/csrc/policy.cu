@@ -58,6 +58,8 @@ __global__ void __launch_bounds__(256) action_embed_kernel(const __nv_bfloat16* 
                                                            const ActSegs segs,
                                                            const __nv_bfloat16* __restrict__ w_in, int32_t ca,
                                                            int32_t d, __nv_bfloat16* __restrict__ h, int64_t ld_h) {
+  pdl_trigger();
+  pdl_wait();
   const int chunks = d >> 3;
   const int64_t total = segs.prefix[segs.n] * chunks;
   for (int64_t e = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; e < total; e += (int64_t)gridDim.x * blockDim.x) {
@@ -142,6 +144,8 @@ __global__ void __launch_bounds__(256) action_head_kernel(const __nv_bfloat16* _
                                                           float eps, const __nv_bfloat16* __restrict__ w_out,
                                                           int32_t ca, int32_t d, __nv_bfloat16* x, int64_t ld_x,
                                                           float dsigma, int32_t guided, float w) {
+  pdl_trigger();
+  pdl_wait();
   const int lane = threadIdx.x & 31;
   const int64_t warps_total = (int64_t)gridDim.x * (blockDim.x >> 5);
   // guided: one item per row of the even (conditioned) segments
@@ -211,7 +215,7 @@ cosmot_status cosmot_action_embed(const void* x, int64_t ld_x, const cosmot_segm
   if (!fill_act_segs(segs, n_segs, &t)) return COSMOT_ERR_INVALID_ARG;
   if (t.prefix[t.n] == 0) return COSMOT_OK;
   const int64_t items = t.prefix[t.n] * (d_model / 8);
-  action_embed_kernel<<<grid_cap(items, 256), 256, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
+  (void)launch_pdl(action_embed_kernel, dim3(grid_cap(items, 256)), dim3(256), 0, reinterpret_cast<cudaStream_t>(stream), nullptr, 
       static_cast<const __nv_bfloat16*>(x), ld_x, t, static_cast<const __nv_bfloat16*>(w_in), action_dim, d_model,
       static_cast<__nv_bfloat16*>(h), ld_h);
   return launch_status();
@@ -236,7 +240,7 @@ cosmot_status cosmot_action_head(const void* h_last, int64_t ld_h, const cosmot_
   }
   const int64_t items = guidance ? t.prefix[t.n] / 2 : t.prefix[t.n];
   if (items == 0) return COSMOT_OK;
-  action_head_kernel<<<grid_cap(items, 8), 256, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
+  (void)launch_pdl(action_head_kernel, dim3(grid_cap(items, 8)), dim3(256), 0, reinterpret_cast<cudaStream_t>(stream), nullptr, 
       static_cast<const __nv_bfloat16*>(h_last), ld_h, t, static_cast<const __nv_bfloat16*>(g_fin), eps,
       static_cast<const __nv_bfloat16*>(w_out), action_dim, d_model, static_cast<__nv_bfloat16*>(x), ld_x,
       (float)(sigma_next - sigma), guidance ? 1 : 0, guidance ? (float)*guidance : 0.f);

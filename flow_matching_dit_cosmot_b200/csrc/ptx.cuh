@@ -27,6 +27,20 @@ __device__ __forceinline__ bool device_failed(const int* status) {
   return *((const volatile int*)status) != 0;
 }
 
+// --------------------------------------------------------------------------
+// Programmatic dependent launch (kernels started through launch_pdl).
+// pdl_trigger lets the next kernel of the stream be scheduled once every CTA
+// of this grid has issued it; pdl_wait blocks the thread until the previous
+// kernel of the stream has completed and its memory operations are visible.
+// A kernel started through launch_pdl executes pdl_wait in every thread
+// before it reads or writes global memory that an earlier kernel touches and
+// before it exits, so that completion stays ordered along the stream.  In a
+// kernel launched without the attribute both are no-ops.
+// --------------------------------------------------------------------------
+__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
 __device__ __forceinline__ uint64_t globaltimer_ns() {
   uint64_t t;
   asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));

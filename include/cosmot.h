@@ -598,7 +598,7 @@ typedef struct {
  * cosmot_stack_forward; INVALID_ARG also for a bad action descriptor.
  * stage_events: NULL, or n_events = 8 * n_layers + 2 CUDA events recorded as
  * for cosmot_stack_forward_timed (the action head falls in the final-norm
- * stage); the computation is the same either way.
+ * stage; NULL entries are skipped); the computation is the same either way.
  */
 COSMOT_API cosmot_status cosmot_policy_step(const cosmot_dims* dims, const cosmot_layer_weights* layers,
                                             int32_t n_layers, const cosmot_seq_desc* seq,
@@ -650,8 +650,10 @@ COSMOT_API cosmot_status cosmot_copy_columns(const void* src, int64_t ld_src, vo
  * i (COSMOT_STAGE_NORM1 .. COSMOT_STAGE_DOWN_RESIDUAL) and events[8l + 7]
  * after its last one (where the final-norm stage starts); events[8 n_layers]
  * is recorded before the velocity stage and events[8 n_layers + 1] after it.
- * The computation is identical to cosmot_stack_forward_io with `io` (NULL:
- * cosmot_stack_forward).
+ * A NULL entry is skipped: that boundary is not marked, and the kernels on
+ * either side keep overlapping their launch (a caller timing one stage passes
+ * only the events around it).  The computation is identical to
+ * cosmot_stack_forward_io with `io` (NULL: cosmot_stack_forward).
  */
 COSMOT_API cosmot_status cosmot_stack_forward_timed(const cosmot_dims* dims, const cosmot_layer_weights* layers,
                                                     int32_t n_layers, const cosmot_seq_desc* seq, void* h,
@@ -718,7 +720,10 @@ enum {
  * is recorded on `stream` just before stage i and stage_events[COSMOT_LAYER_STAGES]
  * after the last one, so cudaEventElapsedTime between consecutive events is the
  * device time of one stage.  The events are cudaEvent_t handles created by the
- * caller on the current device; n_events must be COSMOT_LAYER_STAGES + 1.  With
+ * caller on the current device; n_events must be COSMOT_LAYER_STAGES + 1, and a
+ * NULL entry is skipped (that boundary is not marked, so the kernels on either
+ * side keep overlapping their launch: a caller timing one stage passes only the
+ * two events around it).  With
  * guidance == NULL the computation is identical to cosmot_layer_forward_io with
  * `io` (which may be NULL); with a guidance weight it is that of
  * cosmot_layer_forward_cfg (the last stage then covers the velocity GEMM and the

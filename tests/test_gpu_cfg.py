@@ -115,3 +115,35 @@ def test_guided_timed_entry_matches():
     assert_device_ok()
     np.testing.assert_array_equal(bits(ha), bits(hb))
     np.testing.assert_array_equal(bits(oa), bits(ob))
+
+
+def test_timed_entry_with_sparse_events_matches():
+    """The stage-timed entry given only the two events around the attention
+    stage (the other boundaries NULL and unmarked) computes exactly the plain
+    layer step, and the given pair times the stage."""
+    spec = synth.preset("droid").layout
+    lay = olayout.build_layout(spec)
+    n, d = lay.n_tokens, MEDIUM.d_model
+    w = synth.make_weights(MEDIUM, 1011)
+    h = synth.make_activations(n, d, 2810)[None]
+    dlay = A.build_layout(layout_spec(A, spec))
+    cs = A.mrope_table(dlay.pos, MEDIUM.head_dim, MEDIUM.rope_sections)
+    layer = A.MoTLayer(cdims(A, MEDIUM), device_weights(w))
+    seq = layer.seq_desc(dlay.n_ar, dlay.n_clean, dlay.n_noisy, 1, cs, dlay.chunk)
+    ha, hb = to_dev(h), to_dev(h)
+    oa, ob = torch.empty_like(ha), torch.empty_like(hb)
+    layer.forward(ha, oa, 1.0, 0.9, seq)
+    ws = layer.workspace(seq, ha.device)
+    attention = 2  # stage index of the attention
+    evs = [torch.cuda.Event(enable_timing=True) if k in (attention, attention + 1) else None
+           for k in range(L.COSMOT_LAYER_STAGES + 1)]
+    for e in evs:
+        if e is not None:
+            e.record()
+    L.cosmot_layer_forward_timed(layer.dims, layer.cw, seq, hb.data_ptr(), ob.data_ptr(), 1.0, 0.9, ws.data_ptr(),
+                                 ws.numel(), A.stream_handle(), [e.cuda_event if e is not None else None for e in evs])
+    torch.cuda.synchronize()
+    assert_device_ok()
+    np.testing.assert_array_equal(bits(ha), bits(hb))
+    np.testing.assert_array_equal(bits(oa), bits(ob))
+    assert evs[attention].elapsed_time(evs[attention + 1]) > 0

@@ -141,3 +141,30 @@ def test_stack_timed_entry_matches():
     np.testing.assert_array_equal(bits(ha), bits(hb))
     np.testing.assert_array_equal(bits(oa), bits(ob))
     assert all(evs[i].elapsed_time(evs[i + 1]) >= 0 for i in range(len(evs) - 1))
+
+
+def test_stack_timed_entry_with_sparse_events_matches():
+    """Given only the two events around one stage of every layer (the others
+    NULL, which leaves those boundaries unmarked), the stage-timed stack entry
+    still computes exactly what the plain one does, and each given pair times
+    its stage."""
+    run = StackRun(GQA, synth.preset("droid").layout, 2)
+    ha, hb = to_dev(run.h), to_dev(run.h)
+    oa, ob = torch.empty_like(ha), torch.empty_like(hb)
+    run.stack.forward(ha, oa, 1.0, 0.9, run.seq())
+    ws = torch.empty_like(run.stack.workspace(run.seq()))
+    gate_up = 5  # stage index of the gate/up projection inside a layer
+    keep = {8 * lyr + gate_up + e for lyr in range(2) for e in (0, 1)}
+    evs = [torch.cuda.Event(enable_timing=True) if k in keep else None for k in range(8 * 2 + 2)]
+    for e in evs:
+        if e is not None:
+            e.record()
+    L.cosmot_stack_forward_timed(run.stack.dims, run.stack.cw, run.seq(), hb.data_ptr(), ob.data_ptr(), 1.0, 0.9,
+                                 ws.data_ptr(), ws.numel(), A.stream_handle(),
+                                 [e.cuda_event if e is not None else None for e in evs])
+    torch.cuda.synchronize()
+    assert_device_ok()
+    np.testing.assert_array_equal(bits(ha), bits(hb))
+    np.testing.assert_array_equal(bits(oa), bits(ob))
+    for lyr in range(2):
+        assert evs[8 * lyr + gate_up].elapsed_time(evs[8 * lyr + gate_up + 1]) > 0
