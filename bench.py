@@ -44,8 +44,8 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # only while that code is unchanged.
 NCU_TRAFFIC = {
     # one attention launch at the 480p shape (18,978 rows x 32 heads):
-    # dram__bytes_read.sum 474,230,528 + dram__bytes_write.sum 135,390,976
-    "t2v480:attention": {"bytes_per_launch": 609621504, "src_sha": "f1dd4a7f66d5deda"},
+    # dram__bytes_read.sum 475,295,232 + dram__bytes_write.sum 135,822,848
+    "t2v480:attention": {"bytes_per_launch": 611118080, "src_sha": "5ebc251138102a27"},
 }
 
 
