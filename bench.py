@@ -477,6 +477,40 @@ def src_sha(name):
     return code_sha(open(p, encoding="utf-8").read()) if os.path.exists(p) else None
 
 
+def stage_spans(n_layers, n_stage):
+    """(stage, k) pairs: that stage of one layer call runs from event k to event k + 1.
+
+    The event layout of the stage-timed entry points: one layer has an event
+    before each of its n_stage stages and one after the last; a stack of
+    n_layers records 8 l + i before stage i (< 7) of layer l, 8 l + 7 after
+    that layer's last one (where the final-norm stage starts), 8 n_layers
+    before the velocity stage and 8 n_layers + 1 after it.
+    """
+    if n_layers > 1:
+        return [(j, 8 * lyr + j) for lyr in range(n_layers) for j in range(7)] + [(7, 8 * n_layers - 1),
+                                                                                  (8, 8 * n_layers)]
+    return [(j, j) for j in range(n_stage)]
+
+
+def dominant_marks(n_layers, n_stage, dom):
+    """Event indices a timed step records: the two boundaries of stage `dom` in every layer."""
+    return {k + e for j, k in stage_spans(n_layers, n_stage) if j == dom for e in (0, 1)}
+
+
+def stage_times(per_step_evs, n_layers, n_stage, steps):
+    """Mean device ms per step of every stage, from the events recorded at its two
+    boundaries (None: that boundary was not recorded)."""
+    import numpy as np
+    out = np.zeros(n_stage)
+    spans = stage_spans(n_layers, n_stage)
+    for per_call in per_step_evs:
+        for evs in per_call:
+            for j, k in spans:
+                if evs[k] is not None and evs[k + 1] is not None:
+                    out[j] += evs[k].elapsed_time(evs[k + 1])
+    return out / steps
+
+
 def run_native(args, wl):
     import torch
     import torch.distributed as dist
@@ -689,21 +723,6 @@ def run_native(args, wl):
     if st:
         raise RuntimeError(f"device status {L.status_string(st)} at {where}")
 
-    def stage_times(per_step_evs):
-        """Mean device ms per step of every stage, from the events recorded at its two boundaries."""
-        out = np.zeros(n_stage)
-        for per_call in per_step_evs:
-            for evs in per_call:
-                if n_layers > 1:
-                    spans = [(j, 8 * lyr + j) for lyr in range(n_layers) for j in range(7)]
-                    spans += [(7, 8 * n_layers - 1), (8, 8 * n_layers)]
-                else:
-                    spans = [(j, j) for j in range(n_stage)]
-                for j, k in spans:
-                    if evs[k] is not None and evs[k + 1] is not None:
-                        out[j] += evs[k].elapsed_time(evs[k + 1])
-        return out / args.steps
-
     # Instrumented steps, outside the timed region: an event at every stage
     # boundary gives the stage table and picks the dominant stage.  Each event
     # between two kernels also ends their overlapped launch, so these steps run
@@ -717,15 +736,11 @@ def run_native(args, wl):
         step(stage_evs[i], commit_evs[i])
         prof_ends[i].record(stream)
     torch.cuda.synchronize()
-    stage_ms = stage_times(stage_evs)
+    stage_ms = stage_times(stage_evs, n_layers, n_stage, args.steps)
     prof_ms_step = sum(prof_starts[i].elapsed_time(prof_ends[i]) for i in range(args.steps)) / args.steps
     commit_ms = (sum(e[0].elapsed_time(e[1]) for e in commit_evs) / args.steps) if kind == "stream" else 0.0
     dom = max(range(n_stage), key=lambda j: stage_ms[j])
-    if n_layers > 1:
-        dom_keep = ({k for lyr in range(n_layers) for k in (8 * lyr + dom, 8 * lyr + dom + 1)} if dom < 7 else
-                    {8 * n_layers - 1, 8 * n_layers} if dom == 7 else {8 * n_layers, 8 * n_layers + 1})
-    else:
-        dom_keep = {dom, dom + 1}
+    dom_keep = dominant_marks(n_layers, n_stage, dom)
 
     def dom_events():
         """A timed step's events: only the two around the dominant stage (in every layer)."""
@@ -762,7 +777,7 @@ def run_native(args, wl):
     step_ms = [starts[i].elapsed_time(ends[i]) for i in range(args.steps)]
     total_ms = sum(step_ms)
     median_ms = statistics.median(step_ms)
-    dom_ms = stage_times(dom_evs)[dom]  # the dominant stage inside the timed steps
+    dom_ms = stage_times(dom_evs, n_layers, n_stage, args.steps)[dom]  # the dominant stage inside the timed steps
 
     # ---------------------------------------------------------------- end to end (host buffers)
     e2e = None
