@@ -635,10 +635,8 @@ cosmot_status launch(const CUtensorMap& tq, const CUtensorMap& tk, const CUtenso
       if (dev < 64) done_mask |= 1ull << dev;
     }
   }
-  if (launch_pdl(mot_attention_kernel<HD, kSkip>, dim3(grid), dim3(NUM_THREADS), Cfg<HD>::SMEM_BYTES, s, nullptr, tq,
-                 tk, tv, p) != cudaSuccess)
-    return COSMOT_ERR_CUDA;
-  return launch_status();
+  return launch_status(launch_pdl(mot_attention_kernel<HD, kSkip>, dim3(grid), dim3(NUM_THREADS), Cfg<HD>::SMEM_BYTES,
+                                  s, nullptr, tq, tk, tv, p));
 }
 
 }  // namespace attn
@@ -868,8 +866,7 @@ cosmot_status attention_impl(const cosmot_attn_desc* d, const void* q, int64_t l
   const unsigned mgrid = (unsigned)((warps + 7) / 8);
   const cudaError_t e = hd == 128 ? launch_pdl(attn_merge_kernel<128>, dim3(mgrid), dim3(256), 0, s, nullptr, p)
                                   : launch_pdl(attn_merge_kernel<64>, dim3(mgrid), dim3(256), 0, s, nullptr, p);
-  if (e != cudaSuccess) return COSMOT_ERR_CUDA;
-  return launch_status();
+  return launch_status(e);
 }
 
 }  // namespace attn

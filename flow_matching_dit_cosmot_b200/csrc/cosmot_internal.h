@@ -42,6 +42,14 @@ inline cosmot_status launch_status() {
   return e == cudaSuccess ? COSMOT_OK : COSMOT_ERR_CUDA;
 }
 
+// The status of a launch call's own return code and of the runtime's last
+// error, which is read (and so cleared) either way: a failed launch leaves
+// nothing behind for the next call's check.
+inline cosmot_status launch_status(cudaError_t launched) {
+  const cudaError_t last = cudaGetLastError();
+  return launched == cudaSuccess && last == cudaSuccess ? COSMOT_OK : COSMOT_ERR_CUDA;
+}
+
 int num_sms();
 
 // Launches a kernel with programmatic stream serialization: it may be

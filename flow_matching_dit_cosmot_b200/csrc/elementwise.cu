@@ -401,6 +401,7 @@ cosmot_status rmsnorm_routed(const void* h, bool h_f32, int64_t ld_h, const cosm
   auto* op = static_cast<__nv_bfloat16*>(out);
   int* st = device_status_ptr();
   if (!st) return COSMOT_ERR_CUDA;
+  cudaError_t e;
   if (d >= 1024) {  // one block per row
     const int64_t cap = (int64_t)num_sms() * 16;
     const unsigned bgrid = (unsigned)(rows < cap ? rows : cap);
@@ -408,29 +409,29 @@ cosmot_status rmsnorm_routed(const void* h, bool h_f32, int64_t ld_h, const cosm
     if (h_f32) {
       const auto* hf = static_cast<const float*>(h);
       if (vpt <= 4)
-        (void)launch_pdl(rmsnorm_block_kernel<float, 4>, dim3(bgrid), dim3(kNormBlock), 0, s, nullptr, hf, ld_h, t,
+        e = launch_pdl(rmsnorm_block_kernel<float, 4>, dim3(bgrid), dim3(kNormBlock), 0, s, nullptr, hf, ld_h, t,
                          gp0, gp1, (int32_t)d, eps, op, ld_out, st);
       else
-        (void)launch_pdl(rmsnorm_block_kernel<float, 6>, dim3(bgrid), dim3(kNormBlock), 0, s, nullptr, hf, ld_h, t,
+        e = launch_pdl(rmsnorm_block_kernel<float, 6>, dim3(bgrid), dim3(kNormBlock), 0, s, nullptr, hf, ld_h, t,
                          gp0, gp1, (int32_t)d, eps, op, ld_out, st);
     } else {
       if (vpt <= 4)
-        (void)launch_pdl(rmsnorm_block_kernel<__nv_bfloat16, 4>, dim3(bgrid), dim3(kNormBlock), 0, s, nullptr, hp,
+        e = launch_pdl(rmsnorm_block_kernel<__nv_bfloat16, 4>, dim3(bgrid), dim3(kNormBlock), 0, s, nullptr, hp,
                          ld_h, t, gp0, gp1, (int32_t)d, eps, op, ld_out, st);
       else
-        (void)launch_pdl(rmsnorm_block_kernel<__nv_bfloat16, 6>, dim3(bgrid), dim3(kNormBlock), 0, s, nullptr, hp,
+        e = launch_pdl(rmsnorm_block_kernel<__nv_bfloat16, 6>, dim3(bgrid), dim3(kNormBlock), 0, s, nullptr, hp,
                          ld_h, t, gp0, gp1, (int32_t)d, eps, op, ld_out, st);
     }
-    return launch_status();
+    return launch_status(e);
   }
   // narrow rows (d < 1024): one warp per row, at most 4 vectors per lane
   if (h_f32)
-    (void)launch_pdl(rmsnorm_f32in_kernel<4>, dim3(grid), dim3(threads), 0, s, nullptr, static_cast<const float*>(h),
+    e = launch_pdl(rmsnorm_f32in_kernel<4>, dim3(grid), dim3(threads), 0, s, nullptr, static_cast<const float*>(h),
                      ld_h, t, gp0, gp1, (int32_t)d, eps, op, ld_out, st);
   else
-    (void)launch_pdl(rmsnorm_kernel<4>, dim3(grid), dim3(threads), 0, s, nullptr, hp, ld_h, t, gp0, gp1, (int32_t)d,
+    e = launch_pdl(rmsnorm_kernel<4>, dim3(grid), dim3(threads), 0, s, nullptr, hp, ld_h, t, gp0, gp1, (int32_t)d,
                      eps, op, ld_out, st);
-  return launch_status();
+  return launch_status(e);
 }
 
 }  // namespace cosmot
@@ -457,11 +458,10 @@ cosmot_status cosmot_mrope_apply(void* q, int64_t ld_q, int32_t n_q_heads, void*
   const int64_t items = n_rows * (n_q_heads + n_k_heads) * (head_dim / 16);
   if (items == 0) return COSMOT_OK;
   const int threads = 256;
-  (void)launch_pdl(mrope_kernel, dim3(grid_for(items, threads)), dim3(threads), 0,
-                   reinterpret_cast<cudaStream_t>(stream), nullptr, static_cast<__nv_bfloat16*>(q), ld_q, n_q_heads,
-                   static_cast<__nv_bfloat16*>(k), ld_k, n_k_heads, n_rows, head_dim,
-                   reinterpret_cast<const float2*>(cs));
-  return launch_status();
+  return launch_status(launch_pdl(mrope_kernel, dim3(grid_for(items, threads)), dim3(threads), 0,
+                                  reinterpret_cast<cudaStream_t>(stream), nullptr, static_cast<__nv_bfloat16*>(q), ld_q,
+                                  n_q_heads, static_cast<__nv_bfloat16*>(k), ld_k, n_k_heads, n_rows, head_dim,
+                                  reinterpret_cast<const float2*>(cs)));
 }
 
 cosmot_status cosmot_flow_euler_step(void* x, int64_t ld_x, const void* v, int64_t ld_v, int64_t row_begin,
@@ -477,10 +477,10 @@ cosmot_status cosmot_flow_euler_step(void* x, int64_t ld_x, const void* v, int64
   const int threads = 256;
   int* st = device_status_ptr();
   if (!st) return COSMOT_ERR_CUDA;
-  (void)launch_pdl(euler_kernel, dim3(grid_for(items, threads)), dim3(threads), 0,
-                   reinterpret_cast<cudaStream_t>(stream), nullptr, static_cast<__nv_bfloat16*>(x), ld_x,
-                   static_cast<const __nv_bfloat16*>(v), ld_v, row_begin, row_end - row_begin, n_cols, dsigma, st);
-  return launch_status();
+  return launch_status(launch_pdl(euler_kernel, dim3(grid_for(items, threads)), dim3(threads), 0,
+                                  reinterpret_cast<cudaStream_t>(stream), nullptr, static_cast<__nv_bfloat16*>(x), ld_x,
+                                  static_cast<const __nv_bfloat16*>(v), ld_v, row_begin, row_end - row_begin, n_cols,
+                                  dsigma, st));
 }
 
 cosmot_status cosmot_flow_cfg_euler_step(void* x_cond, void* x_base, int64_t ld_x, const void* v_cond,
@@ -493,12 +493,11 @@ cosmot_status cosmot_flow_cfg_euler_step(void* x_cond, void* x_base, int64_t ld_
   const int64_t items = n_rows * (n_cols / 8);
   if (items == 0) return COSMOT_OK;
   const int threads = 256;
-  (void)launch_pdl(cfg_euler_kernel, dim3(grid_for(items, threads)), dim3(threads), 0,
-                   reinterpret_cast<cudaStream_t>(stream), nullptr, static_cast<__nv_bfloat16*>(x_cond),
-                   static_cast<__nv_bfloat16*>(x_base), ld_x, static_cast<const __nv_bfloat16*>(v_cond),
-                   static_cast<const __nv_bfloat16*>(v_base), ld_v, n_rows, n_cols, (float)(sigma_next - sigma),
-                   (float)guidance);
-  return launch_status();
+  return launch_status(launch_pdl(cfg_euler_kernel, dim3(grid_for(items, threads)), dim3(threads), 0,
+                                  reinterpret_cast<cudaStream_t>(stream), nullptr, static_cast<__nv_bfloat16*>(x_cond),
+                                  static_cast<__nv_bfloat16*>(x_base), ld_x, static_cast<const __nv_bfloat16*>(v_cond),
+                                  static_cast<const __nv_bfloat16*>(v_base), ld_v, n_rows, n_cols,
+                                  (float)(sigma_next - sigma), (float)guidance));
 }
 
 }  // extern "C"

@@ -588,17 +588,13 @@ cosmot_status launch(const CUtensorMap& ta, const CUtensorMap& tb0, const CUtens
     cluster.val.clusterDim.x = 2;
     cluster.val.clusterDim.y = 1;
     cluster.val.clusterDim.z = 1;
-    if (launch_pdl(routed_gemm_kernel<EPI, FL, BN, CG>, dim3(2 * pairs), dim3(NUM_THREADS), SMEM_BYTES, s, &cluster, ta,
-                   tb0, tb1, tu0, tu1, p) != cudaSuccess)
-      return COSMOT_ERR_CUDA;
-    return launch_status();
+    return launch_status(launch_pdl(routed_gemm_kernel<EPI, FL, BN, CG>, dim3(2 * pairs), dim3(NUM_THREADS), SMEM_BYTES,
+                                    s, &cluster, ta, tb0, tb1, tu0, tu1, p));
   }
   int grid = num_sms();
   if (p.num_tiles < grid) grid = p.num_tiles;
-  if (launch_pdl(routed_gemm_kernel<EPI, FL, BN, CG>, dim3(grid), dim3(NUM_THREADS), SMEM_BYTES, s, nullptr, ta, tb0,
-                 tb1, tu0, tu1, p) != cudaSuccess)
-    return COSMOT_ERR_CUDA;
-  return launch_status();
+  return launch_status(launch_pdl(routed_gemm_kernel<EPI, FL, BN, CG>, dim3(grid), dim3(NUM_THREADS), SMEM_BYTES, s,
+                                  nullptr, ta, tb0, tb1, tu0, tu1, p));
 }
 
 }  // namespace gemm

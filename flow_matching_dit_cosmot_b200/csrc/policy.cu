@@ -215,11 +215,10 @@ cosmot_status cosmot_action_embed(const void* x, int64_t ld_x, const cosmot_segm
   if (!fill_act_segs(segs, n_segs, &t)) return COSMOT_ERR_INVALID_ARG;
   if (t.prefix[t.n] == 0) return COSMOT_OK;
   const int64_t items = t.prefix[t.n] * (d_model / 8);
-  (void)launch_pdl(action_embed_kernel, dim3(grid_cap(items, 256)), dim3(256), 0,
-                   reinterpret_cast<cudaStream_t>(stream), nullptr, static_cast<const __nv_bfloat16*>(x), ld_x, t,
-                   static_cast<const __nv_bfloat16*>(w_in), action_dim, d_model, static_cast<__nv_bfloat16*>(h),
-                   ld_h);
-  return launch_status();
+  return launch_status(launch_pdl(action_embed_kernel, dim3(grid_cap(items, 256)), dim3(256), 0,
+                                  reinterpret_cast<cudaStream_t>(stream), nullptr, static_cast<const __nv_bfloat16*>(x),
+                                  ld_x, t, static_cast<const __nv_bfloat16*>(w_in), action_dim, d_model,
+                                  static_cast<__nv_bfloat16*>(h), ld_h));
 }
 
 cosmot_status cosmot_action_head(const void* h_last, int64_t ld_h, const cosmot_segment* segs, int32_t n_segs,
@@ -241,12 +240,13 @@ cosmot_status cosmot_action_head(const void* h_last, int64_t ld_h, const cosmot_
   }
   const int64_t items = guidance ? t.prefix[t.n] / 2 : t.prefix[t.n];
   if (items == 0) return COSMOT_OK;
-  (void)launch_pdl(action_head_kernel, dim3(grid_cap(items, 8)), dim3(256), 0, reinterpret_cast<cudaStream_t>(stream),
-                   nullptr, static_cast<const __nv_bfloat16*>(h_last), ld_h, t,
-                   static_cast<const __nv_bfloat16*>(g_fin), eps, static_cast<const __nv_bfloat16*>(w_out), action_dim,
-                   d_model, static_cast<__nv_bfloat16*>(x), ld_x, (float)(sigma_next - sigma), guidance ? 1 : 0,
-                   guidance ? (float)*guidance : 0.f);
-  return launch_status();
+  return launch_status(launch_pdl(action_head_kernel, dim3(grid_cap(items, 8)), dim3(256), 0,
+                                  reinterpret_cast<cudaStream_t>(stream), nullptr,
+                                  static_cast<const __nv_bfloat16*>(h_last), ld_h, t,
+                                  static_cast<const __nv_bfloat16*>(g_fin), eps,
+                                  static_cast<const __nv_bfloat16*>(w_out), action_dim, d_model,
+                                  static_cast<__nv_bfloat16*>(x), ld_x, (float)(sigma_next - sigma), guidance ? 1 : 0,
+                                  guidance ? (float)*guidance : 0.f));
 }
 
 }  // extern "C"
